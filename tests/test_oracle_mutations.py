@@ -1,0 +1,159 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check a pin catches each.
+
+Every mutant below is a one-line slip someone could make while writing the
+oracle: a wrong nibble order, a dropped bias, a wrong group index, a
+transposed operand, a missing renormalisation, and so on.  For each, at least
+one pin in ``oracle_pins`` must fail; otherwise the pins would not be strong
+enough to trust the oracle.
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+from tests import oracle_pins as P
+
+
+def _msb_first_unpack(words, bits):
+    words = np.asarray(words, dtype=np.uint32)
+    per = 32 // bits
+    mask = np.uint32((1 << bits) - 1)
+    shifts = (np.arange(per, dtype=np.uint32)[::-1] * np.uint32(bits))
+    codes = (words[..., :, None] >> shifts) & mask
+    return codes.reshape(*words.shape[:-1], words.shape[-1] * per).astype(np.uint8)
+
+
+def _dequant_no_bias(words, sb, bits):
+    q = O.unpack_codes(words, bits).astype(np.float64)
+    s, b = O.unpack_scale_bias(sb)
+    return q * np.repeat(s, 64, axis=-1)
+
+
+def _dequant_group32(words, sb, bits):
+    q = O.unpack_codes(words, bits).astype(np.float64)
+    s, b = O.unpack_scale_bias(sb)
+    k = q.shape[-1]
+    gi = np.minimum(np.arange(k) // 32, s.shape[-1] - 1)
+    return q * s[..., gi] + b[..., gi]
+
+
+def _dequant_swapped_sb(words, sb, bits):
+    q = O.unpack_codes(words, bits).astype(np.float64)
+    s, b = O.unpack_scale_bias(sb)
+    return q * np.repeat(b, 64, axis=-1) + np.repeat(s, 64, axis=-1)
+
+
+def _dequant_centered(words, sb, bits):
+    # symmetric-code slip: (q - 2^(b-1)) * s + b
+    q = O.unpack_codes(words, bits).astype(np.float64) - (1 << (bits - 1))
+    s, b = O.unpack_scale_bias(sb)
+    return q * np.repeat(s, 64, axis=-1) + np.repeat(b, 64, axis=-1)
+
+
+def _forward_transposed_down(blob, hidden, inter, bits, x):
+    wg, wu, wd = O.expert_matrices(blob, hidden, inter, bits)
+    a = O.silu(wg @ x) * (wu @ x)
+    # slip: use the down matrix as if it were stored [I][H]
+    return wd.reshape(inter, hidden).T @ a
+
+
+def _forward_swapped_gate_up(blob, hidden, inter, bits, x):
+    wg, wu, wd = O.expert_matrices(blob, hidden, inter, bits)
+    return wd @ (O.silu(wu @ x) * (wg @ x))
+
+
+def _silu_wrong(z):
+    z = np.asarray(z, dtype=np.float64)
+    return z * O.sigmoid(-z)
+
+
+def _top_k_ascending(logits, k):
+    return np.argsort(np.asarray(logits), kind="stable")[:k].astype(np.int32)
+
+
+def _top_k_ties_high(logits, k):
+    l = np.asarray(logits, dtype=np.float64)
+    order = np.lexsort((-np.arange(l.size), -l))
+    return order[:k].astype(np.int32)
+
+
+def _route_no_renorm(w_router_bf16, w_sgate_bf16, x, top_k):
+    r = ORIG_ROUTE(w_router_bf16, w_sgate_bf16, x, top_k)
+    r["w"] = r["p"][r["idx"]]
+    return r
+
+
+def _route_sg_no_sigmoid(w_router_bf16, w_sgate_bf16, x, top_k):
+    r = ORIG_ROUTE(w_router_bf16, w_sgate_bf16, x, top_k)
+    if w_sgate_bf16 is not None:
+        r["sg"] = float(O.bf16_to_f64(w_sgate_bf16) @ np.asarray(x, dtype=np.float64))
+    return r
+
+
+def _layer_no_residual(w_router_bf16, w_sgate_bf16, get_blob, shared_blob, x, residual, *a, **kw):
+    return ORIG_LAYER(w_router_bf16, w_sgate_bf16, get_blob, shared_blob, x,
+                      np.zeros_like(np.asarray(residual, dtype=np.float64)), *a, **kw)
+
+
+def _expert_bytes_bf16_once(hidden, inter, bits, group=64):
+    # slip: one 2-byte scale per group and no bias
+    return 3 * hidden * inter * bits // 8 + 3 * hidden * inter // group * 2
+
+
+def _quantize_bias_max(w, bits):
+    codes, sb = ORIG_QUANT(w, bits)
+    g = np.asarray(w, dtype=np.float32).reshape(w.shape[0], -1, 64)
+    mx_bits = O.f32_to_bf16_bits(g.max(-1))
+    return codes, (sb & np.uint32(0xFFFF)) | (mx_bits.astype(np.uint32) << np.uint32(16))
+
+
+def _quantize_floor(w, bits):
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    n, kdim = w.shape
+    g = w.reshape(n, kdim // 64, 64)
+    mn, mx = g.min(-1), g.max(-1)
+    s32 = (mx - mn).astype(np.float32) / np.float32((1 << bits) - 1)
+    sbits = O.f32_to_bf16_bits(s32)
+    bbits = O.f32_to_bf16_bits(mn)
+    s_f = (sbits.astype(np.uint32) << 16).view(np.float32)
+    b_f = (bbits.astype(np.uint32) << 16).view(np.float32)
+    q = np.clip(np.floor((g - b_f[..., None]) / s_f[..., None]), 0, (1 << bits) - 1).astype(np.uint32)
+    return O.pack_codes(q.reshape(n, kdim), bits), sbits.astype(np.uint32) | (bbits.astype(np.uint32) << 16)
+
+
+ORIG_ROUTE = O.route
+ORIG_LAYER = O.layer_decode
+ORIG_QUANT = O.quantize_matrix
+
+MUTANTS = {
+    "msb_first_packing": ("unpack_codes", _msb_first_unpack),
+    "dropped_bias": ("dequantize", _dequant_no_bias),
+    "group_index_32": ("dequantize", _dequant_group32),
+    "scale_bias_swapped": ("dequantize", _dequant_swapped_sb),
+    "centered_codes": ("dequantize", _dequant_centered),
+    "transposed_down": ("expert_forward", _forward_transposed_down),
+    "gate_up_swapped": ("expert_forward", _forward_swapped_gate_up),
+    "silu_sign": ("silu", _silu_wrong),
+    "topk_ascending": ("top_k_order", _top_k_ascending),
+    "topk_ties_high_index": ("top_k_order", _top_k_ties_high),
+    "no_renormalisation": ("route", _route_no_renorm),
+    "shared_gate_no_sigmoid": ("route", _route_sg_no_sigmoid),
+    "no_residual": ("layer_decode", _layer_no_residual),
+    "expert_bytes_wrong": ("expert_bytes", _expert_bytes_bf16_once),
+    "quantizer_bias_is_max": ("quantize_matrix", _quantize_bias_max),
+    "quantizer_floor": ("quantize_matrix", _quantize_floor),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(O, attr, fn)
+    failed = []
+    for pin in P.ALL_PINS:
+        try:
+            pin(O)
+        except AssertionError:
+            failed.append(pin.__name__)
+        except Exception as e:  # a crash also counts as caught
+            failed.append(f"{pin.__name__}:{type(e).__name__}")
+    assert failed, f"mutant {name} survived every pin"

@@ -1,0 +1,374 @@
+"""Benchmark: single-token MoE layer decode on B200 through the C-ABI engine.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fmoe|reference] [--config full4|full2|tiny]
+
+One step = one token decoded through one full MoE layer (router GEMV over 512
+experts, softmax/top-4/renormalise, 4 routed + 1 shared 4-bit experts, fused
+combine) with the weights resident in HBM.  The default workload is the
+full-size 4-bit layer: hidden 4096, expert intermediate 1024, 512 experts,
+group 64 (3.6 GB of experts per layer, 39.6 MB read per decode).
+
+Timing: W untimed warm-up steps; then K steps, each bracketed by CUDA events
+on the launching stream, with L2 flushed before every step (a 256 MiB write
+outside the event pair) so that the router and shared expert are re-read from
+HBM each time; tokens rotate through a pool of 64 pre-drawn inputs so the
+routed experts change every step.  A barrier and a device synchronise bracket
+the timed region; the value is the total over all ranks divided by the
+slowest rank's time.  With --gpus N > 1 (torchrun) every rank decodes its own
+replica of the layer: the path has no data-path exchange.
+
+The JSON line also carries: the roofline of the layer kernel (algorithmic bytes
+per launch / measured launch time vs the measured HBM copy bandwidth), an
+end-to-end figure through the same C-ABI call with host buffers (pinned host
+-> device copy of x and residual, decode, device -> host copy of out inside
+the event pair), the SM clocks sampled during the timed region, and the CPU
+oracle timed on a bounded sample as a baseline.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth as S  # noqa: E402
+
+CONFIGS = {
+    "full4": dict(workload="full_h4096_i1024_e512_k4_shared_4bit", hidden=4096, inter=1024, experts=512,
+                  top_k=4, bits=4, shared_bits=4),
+    "full2": dict(workload="full_h4096_i1024_e512_k4_routed2bit_shared4bit", hidden=4096, inter=1024,
+                  experts=512, top_k=4, bits=2, shared_bits=4),
+    "tiny": dict(workload="tiny_h512_i128_e16_k4_shared_4bit", hidden=512, inter=128, experts=16, top_k=4,
+                 bits=4, shared_bits=4),
+}
+METRIC = "MoE layer decodes/s (batch 1)"
+UNIT = "decodes/s"
+SEED = 2026
+POOL = 64
+FLUSH_BYTES = 256 << 20
+
+
+def expert_bytes(h, i, b):
+    return 3 * h * i * b // 8 + 3 * h * i // 64 * 4
+
+
+def algorithmic_bytes(cfg) -> dict:
+    """Bytes one decode must read or write at least (each weight once)."""
+    h, i, e, k = cfg["hidden"], cfg["inter"], cfg["experts"], cfg["top_k"]
+    experts = k * expert_bytes(h, i, cfg["bits"]) + expert_bytes(h, i, cfg["shared_bits"])
+    router = e * h * 2 + h * 2
+    vectors = 3 * h * 4  # x, residual in; out
+    return dict(experts=experts, router=router, vectors=vectors, total=experts + router + vectors)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_quantized_expert_router_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(cfg_name: str):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current kernel source."""
+    p = os.path.join(ROOT, "profiles", f"layer_kernel_{cfg_name}.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("source_hash") != source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smmax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smmax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smmax) if smmax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle leg (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(cfg, budget_s: float, max_tokens: int = 1000) -> dict:
+    """Time the oracle (as it stands) on a bounded sample of the same workload."""
+    import oracle as O
+    h, i, e, k = cfg["hidden"], cfg["inter"], cfg["experts"], cfg["top_k"]
+    w_router = S.router_bf16(SEED, 0, e, h)
+    w_sg = S.sgate_bf16(SEED, 0, h)
+
+    def blob(ex, bits):
+        return O.assemble_blob(S.expert_parts(SEED, 0, ex, h, i, bits), h, i, bits)
+
+    shared = blob(S.SHARED_EXPERT_ID, cfg["shared_bits"])
+    xs = S.token_x(SEED, 0, 0, POOL, h)
+    res = S.token_residual(SEED, 0, 0, POOL, h)
+    # expert blobs are input preparation, drawn before the clock starts
+    pre = {}
+    for t in range(min(POOL, 8)):
+        for ex in O.route(w_router, w_sg, xs[t], k)["idx"]:
+            if int(ex) not in pre:
+                pre[int(ex)] = blob(int(ex), cfg["bits"])
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        t = n % min(POOL, 8)
+        O.layer_decode(w_router, w_sg, lambda ex: pre[ex], shared, xs[t], res[t], k, h, i, cfg["bits"],
+                       cfg["shared_bits"])
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= max_tokens:
+            break
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    return dict(value=n / el, unit=UNIT, cores=cores, kind="oracle", seconds=el, tokens=n,
+                sample=f"{n} single-token decodes of the {cfg['workload']} layer (fp64 numpy oracle, "
+                       f"expert blobs pre-drawn), {el:.1f} s")
+
+
+def run_reference(args, cfg, rank, world):
+    if rank != 0:
+        return
+    steps, warm = args.steps, args.warmup
+    # bounded: the whole reference run stays within a few minutes
+    per_step_budget = max(0.5, min(20.0, 120.0 / max(1, steps + warm)))
+    for _ in range(warm):
+        oracle_sample(cfg, per_step_budget * 0.2, max_tokens=1)
+    t_total, n_total = 0.0, 0
+    last = None
+    for _ in range(steps):
+        r = oracle_sample(cfg, per_step_budget, max_tokens=2)
+        t_total += r["seconds"]
+        n_total += r["tokens"]
+        last = r
+    value = n_total / t_total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
+        "warmup": warm, "ms_per_step": 1000.0 * t_total / n_total, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {**{k: v for k, v in cfg.items()}, "batch": 1, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": last["cores"], "kind": "oracle",
+                         "sample": f"{n_total} decodes over {steps} steps"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU leg
+# ---------------------------------------------------------------------------
+
+def run_fmoe(args, cfg, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import bit_quantized_expert_router_b200 as F
+    import synth.gpu as SG
+    from bit_quantized_expert_router_b200 import build as B
+
+    if rank == 0 or not os.path.exists(F.LIB_PATH):
+        B.build_engine()
+        SG.build()
+    if world > 1:
+        dist.barrier()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    h, i, e, k = cfg["hidden"], cfg["inter"], cfg["experts"], cfg["top_k"]
+    t = SG.make_layer(SEED + rank, 0, h, i, e, cfg["bits"], cfg["shared_bits"], F.blob_offsets, F.expert_bytes,
+                      dev)
+    L = F.Layer(t["w_router"], t["w_sgate"], t["experts"], t["shared"], h, i, k, cfg["bits"],
+                cfg["shared_bits"])
+    xs = torch.from_numpy(S.token_x(SEED + rank, 0, 0, POOL, h)).to(dev)
+    rs = torch.from_numpy(S.token_residual(SEED + rank, 0, 0, POOL, h)).to(dev)
+    out = torch.empty(POOL, h, dtype=torch.float32, device=dev)
+    ws = L.workspace(1)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(j):
+        L.decode(xs[j % POOL], rs[j % POOL], out=out[j % POOL], ws=ws)
+
+    for j in range(args.warmup):
+        flush.fill_(j & 0xFF)
+        step(j)
+    torch.cuda.synchronize()
+    if F.get_status():
+        raise RuntimeError("device status word set during warm-up")
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.1)
+    for j in range(K):
+        flush.fill_((j + 1) & 0xFF)
+        ev[j][0].record(stream)
+        step(j)
+        ev[j][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    times_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = float(sum(times_ms))
+    status = F.get_status()
+
+    # end to end through the same call with host buffers
+    xh = torch.from_numpy(S.token_x(SEED + rank, 0, 1, POOL, h)).pin_memory()
+    rh = torch.from_numpy(S.token_residual(SEED + rank, 0, 1, POOL, h)).pin_memory()
+    oh = torch.empty(POOL, h, dtype=torch.float32).pin_memory()
+    xd = torch.empty(h, dtype=torch.float32, device=dev)
+    rd = torch.empty(h, dtype=torch.float32, device=dev)
+    od = torch.empty(h, dtype=torch.float32, device=dev)
+    K2 = min(K, 1000)
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K2)]
+    for j in range(K2 + 3):
+        flush.fill_(j & 0xFF)
+        if j >= 3:
+            ev2[j - 3][0].record(stream)
+        xd.copy_(xh[j % POOL], non_blocking=True)
+        rd.copy_(rh[j % POOL], non_blocking=True)
+        L.decode(xd, rd, out=od, ws=ws)
+        oh[j % POOL].copy_(od, non_blocking=True)
+        if j >= 3:
+            ev2[j - 3][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in ev2)
+
+    # max over ranks
+    tt = torch.tensor([total_ms, e2e_ms / K2 * K], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    total_ms_max, e2e_ms_max = float(tt[0]), float(tt[1])
+
+    if rank == 0:
+        ab = algorithmic_bytes(cfg)
+        peak, peak_kind = peaks()
+        avg_launch_s = total_ms / 1000.0 / K
+        achieved = ab["total"] / avg_launch_s / 1e9
+        value = world * K / (total_ms_max / 1000.0)
+        line = {
+            "impl": "fmoe", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": total_ms_max / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u4/bf16 weights, f32 compute", "data": "synthetic",
+            "config": {**cfg, "batch": 1, "group": 64, "l2": "flushed before every timed step (256 MiB write)",
+                       "input_pool": POOL, "parallelism": f"replicas x{world}"},
+            "us_per_decode": 1000.0 * total_ms_max / K,
+            "p50_us": 1000.0 * statistics.median(times_ms), "p99_us": 1000.0 * float(np.percentile(times_ms, 99)),
+            "expert_gbs": ab["experts"] / avg_launch_s / 1e9,
+            "expert_frac_of_hbm": ab["experts"] / avg_launch_s / 1e9 / peak,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": profiled_traffic(args.config),
+                         "kernel": "layer_kernel", "algorithmic_bytes_per_launch": ab["total"]},
+            "e2e": {"value": world * K / (e2e_ms_max / 1000.0), "unit": UNIT, "h2d_bytes_per_step": 2 * h * 4,
+                    "d2h_bytes_per_step": h * 4},
+            "gpu_launches": K,
+            "clocks": clk,
+            "device_status": status,
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_sample(cfg, args.cpu_seconds)
+            line["cpu_baseline"].pop("seconds", None)
+            line["cpu_baseline"].pop("tokens", None)
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["fmoe", "reference"], default="fmoe")
+    ap.add_argument("--config", choices=sorted(CONFIGS), default="full4")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = CONFIGS[args.config]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, cfg, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_fmoe(args, cfg, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,258 @@
+"""Python binding of libfmoe.so (the single-token quantised MoE layer on B200).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current stream.  If the
+shared library is missing the import of any entry point fails loudly; there is
+no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libfmoe.so")
+
+FMOE_OK, FMOE_EINVAL, FMOE_ENOMEM, FMOE_ECUDA, FMOE_EDEVICE = range(5)
+GROUP = 64
+MAX_TOKENS = 16
+MAX_TOPK = 8
+
+EXPORTED = [
+    "fmoe_expert_bytes", "fmoe_blob_offsets", "fmoe_quantize_expert", "fmoe_route_workspace_bytes",
+    "fmoe_route", "fmoe_expert_workspace_bytes", "fmoe_expert_forward", "fmoe_workspace_bytes",
+    "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status", "fmoe_strerror",
+]
+
+
+class FmoeError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {strerror(code)} (code {code})")
+
+
+class FmoeLayerC(ctypes.Structure):
+    """Mirror of the C struct fmoe_layer."""
+    _fields_ = [
+        ("w_router", ctypes.c_void_p), ("w_sgate", ctypes.c_void_p), ("experts", ctypes.c_void_p),
+        ("expert_stride", ctypes.c_int64), ("shared", ctypes.c_void_p), ("hidden", ctypes.c_int),
+        ("inter", ctypes.c_int), ("n_experts", ctypes.c_int), ("top_k", ctypes.c_int),
+        ("bits", ctypes.c_int), ("shared_bits", ctypes.c_int), ("group", ctypes.c_int),
+    ]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfmoe.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                           "`python -m bit_quantized_expert_router_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.fmoe_expert_bytes.argtypes = [i, i, i]
+    L.fmoe_expert_bytes.restype = sz
+    L.fmoe_blob_offsets.argtypes = [i, i, i, ctypes.POINTER(ctypes.c_int64)]
+    L.fmoe_quantize_expert.argtypes = [vp, vp, vp, i, i, i, i, vp, sz, vp]
+    L.fmoe_route_workspace_bytes.argtypes = [i, i]
+    L.fmoe_route_workspace_bytes.restype = sz
+    L.fmoe_route.argtypes = [vp, vp, vp, i, i, i, i, vp, vp, vp, vp, vp, sz, vp]
+    L.fmoe_expert_workspace_bytes.argtypes = [i, i]
+    L.fmoe_expert_workspace_bytes.restype = sz
+    L.fmoe_expert_forward.argtypes = [vp, i, i, i, vp, vp, vp, sz, vp]
+    L.fmoe_workspace_bytes.argtypes = [ctypes.POINTER(FmoeLayerC), i]
+    L.fmoe_workspace_bytes.restype = sz
+    L.fmoe_workspace_init.argtypes = [vp, sz, vp]
+    L.fmoe_layer_decode.argtypes = [ctypes.POINTER(FmoeLayerC), vp, vp, vp, i, vp, sz, vp, vp, vp]
+    L.fmoe_get_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
+    L.fmoe_strerror.argtypes = [i]
+    L.fmoe_strerror.restype = ctypes.c_char_p
+    for name in ("fmoe_blob_offsets", "fmoe_quantize_expert", "fmoe_route", "fmoe_expert_forward",
+                 "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status"):
+        getattr(L, name).restype = i
+    _lib = L
+    return L
+
+
+def strerror(code: int) -> str:
+    return lib().fmoe_strerror(code).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != FMOE_OK:
+        raise FmoeError(rc, what)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _dev_tensor(t: torch.Tensor, dtype, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+# ---------------------------------------------------------------------------
+
+def expert_bytes(hidden: int, inter: int, bits: int) -> int:
+    return int(lib().fmoe_expert_bytes(hidden, inter, bits))
+
+
+def blob_offsets(hidden: int, inter: int, bits: int) -> list[int]:
+    off = (ctypes.c_int64 * 6)()
+    _check(lib().fmoe_blob_offsets(hidden, inter, bits, off), "fmoe_blob_offsets")
+    return list(off)
+
+
+def workspace_init(ws: torch.Tensor, stream=None):
+    _check(lib().fmoe_workspace_init(ws.data_ptr(), ws.numel() * ws.element_size(), _stream(stream)),
+           "fmoe_workspace_init")
+
+
+def _alloc_ws(nbytes: int, device) -> torch.Tensor:
+    return torch.zeros(max(256, (nbytes + 255) // 256 * 256), dtype=torch.uint8, device=device)
+
+
+def quantize_expert(w_gate: torch.Tensor, w_up: torch.Tensor, w_down: torch.Tensor, bits: int,
+                    out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Quantise fp32 (gate [I][H], up [I][H], down [H][I]) into a packed blob (uint8)."""
+    for t, n in ((w_gate, "w_gate"), (w_up, "w_up"), (w_down, "w_down")):
+        _dev_tensor(t, torch.float32, n)
+    inter, hidden = w_gate.shape
+    nbytes = expert_bytes(hidden, inter, bits)
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=w_gate.device)
+    _check(lib().fmoe_quantize_expert(w_gate.data_ptr(), w_up.data_ptr(), w_down.data_ptr(), hidden, inter,
+                                      bits, GROUP, out.data_ptr(), out.numel(), _stream(stream)),
+           "fmoe_quantize_expert")
+    return out
+
+
+def route(w_router: torch.Tensor, w_sgate: torch.Tensor | None, x: torch.Tensor, top_k: int,
+          want_logits: bool = False, stream=None):
+    """Router for T tokens: returns (idx int32 [T][K], w fp32 [T][K], sgate fp32 [T], logits|None)."""
+    _dev_tensor(w_router, torch.int16, "w_router")
+    if w_sgate is not None:
+        _dev_tensor(w_sgate, torch.int16, "w_sgate")
+    _dev_tensor(x, torch.float32, "x")
+    x2 = x.view(-1, x.shape[-1])
+    T, H = x2.shape
+    E = w_router.shape[0]
+    dev = x.device
+    idx = torch.empty(T, top_k, dtype=torch.int32, device=dev)
+    w = torch.empty(T, top_k, dtype=torch.float32, device=dev)
+    sg = torch.empty(T, dtype=torch.float32, device=dev)
+    logits = torch.empty(T, E, dtype=torch.float32, device=dev) if want_logits else None
+    nws = int(lib().fmoe_route_workspace_bytes(T, E))
+    ws = _alloc_ws(nws, dev)
+    _check(lib().fmoe_route(w_router.data_ptr(), _ptr(w_sgate), x2.data_ptr(), T, H, E, top_k, idx.data_ptr(),
+                            w.data_ptr(), sg.data_ptr(), _ptr(logits), ws.data_ptr(), ws.numel(),
+                            _stream(stream)), "fmoe_route")
+    return idx, w, sg, logits
+
+
+def expert_workspace(hidden: int, inter: int, device) -> torch.Tensor:
+    return _alloc_ws(int(lib().fmoe_expert_workspace_bytes(hidden, inter)), device)
+
+
+def expert_forward(blob: torch.Tensor, hidden: int, inter: int, bits: int, x: torch.Tensor,
+                   out: torch.Tensor | None = None, ws: torch.Tensor | None = None, stream=None):
+    """One expert for one token: y = Wd (silu(Wg x) * (Wu x))."""
+    _dev_tensor(blob, torch.uint8, "blob")
+    _dev_tensor(x, torch.float32, "x")
+    if out is None:
+        out = torch.empty(hidden, dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = expert_workspace(hidden, inter, x.device)
+    _check(lib().fmoe_expert_forward(blob.data_ptr(), hidden, inter, bits, x.data_ptr(), out.data_ptr(),
+                                     ws.data_ptr(), ws.numel(), _stream(stream)), "fmoe_expert_forward")
+    return out
+
+
+@dataclass
+class Layer:
+    """Device-resident weights of one MoE layer (all tensors on one GPU).
+
+    experts: uint8 [E][stride] packed routed experts; shared: uint8 blob or None;
+    w_router: int16 [E][H] bf16 bits; w_sgate: int16 [H] bf16 bits or None.
+    """
+    w_router: torch.Tensor
+    w_sgate: torch.Tensor | None
+    experts: torch.Tensor
+    shared: torch.Tensor | None
+    hidden: int
+    inter: int
+    top_k: int
+    bits: int = 4
+    shared_bits: int = 4
+
+    def __post_init__(self):
+        _dev_tensor(self.w_router, torch.int16, "w_router")
+        if self.w_sgate is not None:
+            _dev_tensor(self.w_sgate, torch.int16, "w_sgate")
+        _dev_tensor(self.experts, torch.uint8, "experts")
+        if self.shared is not None:
+            _dev_tensor(self.shared, torch.uint8, "shared")
+        self.n_experts = self.w_router.shape[0]
+        self.c = FmoeLayerC(
+            w_router=self.w_router.data_ptr(), w_sgate=_ptr(self.w_sgate), experts=self.experts.data_ptr(),
+            expert_stride=self.experts.stride(0) if self.experts.dim() == 2 else expert_bytes(
+                self.hidden, self.inter, self.bits),
+            shared=_ptr(self.shared), hidden=self.hidden, inter=self.inter, n_experts=self.n_experts,
+            top_k=self.top_k, bits=self.bits, shared_bits=self.shared_bits, group=GROUP)
+        self._ws = None
+
+    def workspace_bytes(self, T: int = 1) -> int:
+        return int(lib().fmoe_workspace_bytes(ctypes.byref(self.c), T))
+
+    def workspace(self, T: int = 1) -> torch.Tensor:
+        if self._ws is None or self._ws.numel() < self.workspace_bytes(T):
+            self._ws = _alloc_ws(self.workspace_bytes(T), self.experts.device)
+        return self._ws
+
+    def decode(self, x: torch.Tensor, residual: torch.Tensor | None = None, out: torch.Tensor | None = None,
+               idx_out: torch.Tensor | None = None, w_out: torch.Tensor | None = None,
+               ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """out[t] = residual[t] + sum_k w[t,k] E_idx(x[t]) + sgate[t] E_shared(x[t]), T = x rows."""
+        _dev_tensor(x, torch.float32, "x")
+        x2 = x.view(-1, self.hidden)
+        T = x2.shape[0]
+        if residual is not None:
+            _dev_tensor(residual, torch.float32, "residual")
+        if out is None:
+            out = torch.empty_like(x2)
+        if ws is None:
+            ws = self.workspace(T)
+        _check(lib().fmoe_layer_decode(ctypes.byref(self.c), x2.data_ptr(), _ptr(residual), out.data_ptr(), T,
+                                       ws.data_ptr(), ws.numel(), _ptr(idx_out), _ptr(w_out), _stream(stream)),
+               "fmoe_layer_decode")
+        return out
+
+
+def get_status(stream=None) -> int:
+    """Synchronise the stream, read and clear the device status word (0 = clean)."""
+    bits = ctypes.c_uint(0)
+    rc = lib().fmoe_get_status(_stream(stream), ctypes.byref(bits))
+    if rc not in (FMOE_OK, FMOE_EDEVICE):
+        raise FmoeError(rc, "fmoe_get_status")
+    return int(bits.value)

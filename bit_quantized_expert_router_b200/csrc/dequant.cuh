@@ -1,0 +1,139 @@
+// Packed expert format and the dequantising dot-product primitives.
+//
+// Format (the pages fix only "weight = nibble * scale + bias", see
+// "Flash-MoE: Ausführen eines 397B-Parameter-Qwen-Modells ...", section
+// "FMA-optimierter Dequant-Kernel"; the rest is this library's layout):
+//   * a matrix W[N][K] stores codes as uint32 words, row-major, element k in
+//     word k / (32/b) at bit b * (k mod 32/b), least significant bits first;
+//   * then one 32-bit word per (row, group of 64 inputs): bf16 scale in bits
+//     0..15, bf16 bias in bits 16..31;
+//   * an expert blob = [gate codes | gate sb | up codes | up sb | down codes |
+//     down sb]; gate and up are [I][H], down is [H][I].
+//
+// Evaluation.  For one row and one group G the pages rewrite
+// (q*s + b) * x as fma(q, s*x, b*x); summed over the group this is
+// s * sum_k q_k x_k + b * sum_k x_k.  The engine evaluates exactly that: the
+// code-dependent part sum_k q_k x_k with one fused multiply-add per code, and
+// the bias part with a per-vector sum of x computed once when x is staged.
+//
+// Decoding a code costs one bitwise AND.  A code q at bit position p of a word,
+// masked in place and read as an fp32 bit pattern, is the (subnormal) number
+// q * 2^(p - 149).  Staging x multiplies element k by 2^(S_v - p(k)) (exact
+// powers of two, with S_v chosen per 16-byte vector from max|x|), so every
+// product q * 2^(p-149) * x * 2^(S_v-p) equals q * x * 2^(S_v - 149) with one
+// common scale per vector, and the FMA (which keeps subnormal operands)
+// computes it with ordinary fp32 rounding.  Codes in the top byte of a word are
+// first shifted down by 8 so that every masked value stays below bit 24.
+#pragma once
+#include "common.cuh"
+
+namespace fmoe {
+
+struct BlobOff {
+  long long gc, gsb, uc, usb, dc, dsb, total;
+};
+
+__host__ __device__ inline BlobOff blob_offsets(int H, int I, int bits) {
+  const long long cb = (long long)I * H * bits / 8;
+  const long long sb = (long long)I * (H / 64) * 4;
+  BlobOff o;
+  o.gc = 0;
+  o.gsb = cb;
+  o.uc = cb + sb;
+  o.usb = o.uc + cb;
+  o.dc = o.usb + sb;
+  o.dsb = o.dc + cb;
+  o.total = o.dsb + sb;
+  return o;
+}
+
+// Bit position at which code n (0 <= n < 32/b) of a word is read.
+__host__ __device__ inline int code_bitpos(int bits, int n) {
+  if (bits == 4) return n < 6 ? 4 * n : 4 * (n - 2);
+  return n < 12 ? 2 * n : 2 * (n - 4);
+}
+
+// Eight 4-bit codes of word w against eight staged inputs (pairs xa.x, xa.y,
+// xb.x, xb.y hold inputs 0-1, 2-3, 4-5, 6-7 of the word).
+__device__ __forceinline__ void dot_word4(uint64_t& acc, uint32_t w, ulonglong2 xa, ulonglong2 xb) {
+  const uint32_t w8 = w >> 8;
+  ffma2(acc, pk_u32(w & 0xFu, w & 0xF0u), xa.x);
+  ffma2(acc, pk_u32(w & 0xF00u, w & 0xF000u), xa.y);
+  ffma2(acc, pk_u32(w & 0xF0000u, w & 0xF00000u), xb.x);
+  ffma2(acc, pk_u32(w8 & 0xF0000u, w8 & 0xF00000u), xb.y);
+}
+
+// Sixteen 2-bit codes of word w against sixteen staged inputs.
+__device__ __forceinline__ void dot_word2(uint64_t& acc, uint32_t w, ulonglong2 x0, ulonglong2 x1,
+                                          ulonglong2 x2, ulonglong2 x3) {
+  const uint32_t w8 = w >> 8;
+  ffma2(acc, pk_u32(w & 0x3u, w & 0xCu), x0.x);
+  ffma2(acc, pk_u32(w & 0x30u, w & 0xC0u), x0.y);
+  ffma2(acc, pk_u32(w & 0x300u, w & 0xC00u), x1.x);
+  ffma2(acc, pk_u32(w & 0x3000u, w & 0xC000u), x1.y);
+  ffma2(acc, pk_u32(w & 0x30000u, w & 0xC0000u), x2.x);
+  ffma2(acc, pk_u32(w & 0x300000u, w & 0xC00000u), x2.y);
+  ffma2(acc, pk_u32(w8 & 0x30000u, w8 & 0xC0000u), x3.x);
+  ffma2(acc, pk_u32(w8 & 0x300000u, w8 & 0xC00000u), x3.y);
+}
+
+// Staged input vector for `bits`-wide codes over n inputs:
+//   xs: float4 array [F4][NV] with NV = n / CPV vectors of CPV = 128/b inputs,
+//       xs[j*NV + v] = inputs 4j..4j+3 of vector v, each multiplied by
+//       2^(S_v - code_bitpos(b, (4j+c) mod (32/b)));
+//   sf: float2 per vector: {sum of the vector's inputs, 2^(149 - S_v)}.
+// The transposed [F4][NV] order makes lane-consecutive vectors hit consecutive
+// shared-memory banks.
+//
+// stage_vector: one thread per vector (loop); src is global memory read
+// through L2 (it may have been written by other CTAs of this grid).
+__device__ inline void stage_vector(const float* __restrict__ src, int n, int bits, float4* xs,
+                                    float2* sf, int tid, int nthreads) {
+  const int CPV = 128 / bits, CPW = 32 / bits, F4 = CPV / 4, NV = n / CPV;
+  for (int v = tid; v < NV; v += nthreads) {
+    const float4* s4 = reinterpret_cast<const float4*>(src + (long long)v * CPV);
+    float4 buf[16];
+    float mx = 0.f, sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j < F4) {
+        buf[j] = __ldcg(s4 + j);
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(buf[j].x), fabsf(buf[j].y)), fmaxf(fabsf(buf[j].z), fabsf(buf[j].w))));
+        sum += (buf[j].x + buf[j].y) + (buf[j].z + buf[j].w);
+      }
+    }
+    // S_v: max|x| * 2^S_v < 2^125, clamped so that 2^(149 - S_v) and
+    // 2^(S_v - p) stay finite normal floats.
+    int S = 109;
+    if (mx > 0.f) {
+      int e;
+      frexpf(mx, &e);  // mx < 2^e
+      S = 125 - e;
+      S = S < 22 ? 22 : (S > 149 + 100 ? 249 : S);
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j < F4) {
+        float4 o;
+        const int n0 = (4 * j) % CPW;
+        float* oo = &o.x;
+        const float* ii = &buf[j].x;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          int e = S - code_bitpos(bits, n0 + c);  // in [0, 249]
+          float val = ii[c];
+          if (e > 126) {
+            val *= pow2f(126);
+            e -= 126;
+          }
+          oo[c] = val * pow2f(e);
+        }
+        xs[j * NV + v] = o;
+      }
+    }
+    const int fe = 149 - S;  // in [-100, 127]
+    sf[v] = make_float2(sum, fe < -126 ? 0.f : pow2f(fe));
+  }
+}
+
+}  // namespace fmoe

@@ -1,0 +1,332 @@
+// Host side of libfmoe.so: argument validation, shared-memory planning and
+// launches.  The C ABI is declared (and documented) in include/fmoe.h.
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fmoe.h"
+#include "route_quant_kernels.cuh"
+
+using namespace fmoe;
+
+namespace {
+
+constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s bound on every device-side wait
+constexpr size_t kCounterBytes = 256;
+constexpr int kMaxNst = 4;
+
+struct DevInfo {
+  int sms = 0;
+  int max_smem = 0;
+  bool layer_attr_set = false;
+};
+DevInfo g_dev[64];
+std::mutex g_mu;
+
+int dev_info(int* dev_out, DevInfo** info) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FMOE_ECUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevInfo& d = g_dev[dev];
+  if (d.sms == 0) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FMOE_ECUDA;
+    if (cudaDeviceGetAttribute(&d.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return FMOE_ECUDA;
+  }
+  *dev_out = dev;
+  *info = &d;
+  return FMOE_OK;
+}
+
+int check_stream(fmoe_stream_t s, int dev) {
+  if (s == nullptr) return FMOE_OK;
+  int sdev = -1;
+  if (cudaStreamGetDevice(reinterpret_cast<cudaStream_t>(s), &sdev) != cudaSuccess) return FMOE_EINVAL;
+  return sdev == dev ? FMOE_OK : FMOE_EINVAL;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool shape_ok(int h, int i) {
+  return h > 0 && i > 0 && h % 64 == 0 && i % 64 == 0 && h <= FMOE_MAX_HIDDEN && i <= 8192;
+}
+bool bits_ok(int b) { return b == 2 || b == 4; }
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Shared-memory plan of the layer kernel.
+struct Plan {
+  int nst, stage_bytes, xs4_off, xs2_off, xu_off, vec_floats, sf_floats;
+  size_t smem;
+};
+
+bool plan_layer(int H, int I, int K, bool has_shared, bool layer_mode, int bits_r, int bits_s,
+                int max_smem, Plan* p) {
+  const int n_slots = K + (has_shared ? 1 : 0);
+  bool use4 = false, use2 = false;
+  int stage = 0;
+  auto use_bits = [&](int b) {
+    if (b == 4) use4 = true; else use2 = true;
+    const int cb = H * b / 8;
+    const int cap = ((H / 16 + 15) & ~15) + 16;
+    stage = std::max(stage, 2 * cb + 2 * cap);
+    stage = std::max(stage, kRC * (I * b / 8 + I / 16));
+  };
+  if (K > 0) use_bits(bits_r);
+  if (has_shared) use_bits(bits_s);
+  stage = (int)round_up(stage, 128);
+  int off = 0;
+  p->xu_off = -1;
+  if (layer_mode) { p->xu_off = off; off += H; }
+  p->xs4_off = -1;
+  p->xs2_off = -1;
+  if (use4) { p->xs4_off = off; off += H; }
+  if (use2) { p->xs2_off = off; off += H; }
+  p->vec_floats = (int)round_up((size_t)std::max(off, n_slots * I), 32);
+  p->sf_floats = (int)round_up((size_t)std::max((use4 ? H / 32 : 0) + (use2 ? H / 64 : 0), n_slots * I / 32), 16);
+  p->stage_bytes = stage;
+  const size_t fixed = (size_t)p->vec_floats * 4 + (size_t)p->sf_floats * 8;
+  const size_t budget = (size_t)max_smem - sizeof(CtaShared) - 64;
+  for (int nst = kMaxNst; nst >= 1; --nst) {
+    const size_t total = (size_t)kWarps * nst * stage + fixed + (size_t)kWarps * nst * 8;
+    if (total <= budget) {
+      p->nst = nst;
+      p->smem = total;
+      return true;
+    }
+  }
+  return false;
+}
+
+size_t layer_ws_bytes(int E, int I, int K, bool has_shared) {
+  return kCounterBytes + round_up((size_t)(E + 1) * 4, 256) + round_up((size_t)(K + 1) * I * 4, 256) +
+         (has_shared ? 0 : 0);
+}
+
+int launch_layer(const LayerArgs& args, const Plan& pl, DevInfo* info, cudaStream_t s) {
+  if (!info->layer_attr_set) {
+    if (cudaFuncSetAttribute(layer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             info->max_smem - (int)sizeof(CtaShared)) != cudaSuccess)
+      return FMOE_ECUDA;
+    info->layer_attr_set = true;
+  }
+  LayerArgs a = args;
+  void* kargs[] = {&a};
+  cudaError_t e = cudaLaunchCooperativeKernel((const void*)layer_kernel, dim3(info->sms), dim3(kThreads),
+                                              kargs, pl.smem, s);
+  return e == cudaSuccess ? FMOE_OK : FMOE_ECUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fmoe_expert_bytes(int hidden, int inter, int bits) {
+  if (!shape_ok(hidden, inter) || !bits_ok(bits)) return 0;
+  return (size_t)blob_offsets(hidden, inter, bits).total;
+}
+
+int fmoe_blob_offsets(int hidden, int inter, int bits, int64_t off[6]) {
+  if (!off || !shape_ok(hidden, inter) || !bits_ok(bits)) return FMOE_EINVAL;
+  const BlobOff o = blob_offsets(hidden, inter, bits);
+  off[0] = o.gc;
+  off[1] = o.gsb;
+  off[2] = o.uc;
+  off[3] = o.usb;
+  off[4] = o.dc;
+  off[5] = o.dsb;
+  return FMOE_OK;
+}
+
+int fmoe_quantize_expert(const float* w_gate, const float* w_up, const float* w_down, int hidden,
+                         int inter, int bits, int group, void* blob_out, size_t blob_bytes,
+                         fmoe_stream_t stream) {
+  if (!w_gate || !w_up || !w_down || !blob_out || group != FMOE_GROUP || !bits_ok(bits) ||
+      !shape_ok(hidden, inter) || !aligned(blob_out, 256))
+    return FMOE_EINVAL;
+  const BlobOff o = blob_offsets(hidden, inter, bits);
+  if (blob_bytes < (size_t)o.total) return FMOE_ENOMEM;
+  int dev;
+  DevInfo* info;
+  if (int rc = dev_info(&dev, &info)) return rc;
+  if (int rc = check_stream(stream, dev)) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* b = static_cast<char*>(blob_out);
+  struct M { const float* w; int rows, nin; long long c, sb; } m[3] = {
+      {w_gate, inter, hidden, o.gc, o.gsb}, {w_up, inter, hidden, o.uc, o.usb}, {w_down, hidden, inter, o.dc, o.dsb}};
+  for (auto& mm : m) {
+    const long long n = (long long)mm.rows * (mm.nin / 64);
+    quantize_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+        mm.w, mm.rows, mm.nin, bits, reinterpret_cast<uint32_t*>(b + mm.c), reinterpret_cast<uint32_t*>(b + mm.sb));
+    if (cudaGetLastError() != cudaSuccess) return FMOE_ECUDA;
+  }
+  return FMOE_OK;
+}
+
+size_t fmoe_route_workspace_bytes(int T, int n_experts) {
+  if (T < 1 || T > FMOE_MAX_TOKENS || n_experts < 1 || n_experts > FMOE_MAX_EXPERTS) return 0;
+  return round_up((size_t)T * (n_experts + 1) * 4, 256);
+}
+
+int fmoe_route(const uint16_t* w_router, const uint16_t* w_sgate, const float* x, int T, int hidden,
+               int n_experts, int top_k, int32_t* idx, float* w, float* sgate, float* logits_opt,
+               void* ws, size_t ws_bytes, fmoe_stream_t stream) {
+  if (!w_router || !x || !idx || !w || !ws) return FMOE_EINVAL;
+  if (T < 1 || T > FMOE_MAX_TOKENS || hidden <= 0 || hidden % 64 || hidden > FMOE_MAX_HIDDEN ||
+      n_experts < 1 || n_experts > FMOE_MAX_EXPERTS || top_k < 1 || top_k > FMOE_MAX_TOPK ||
+      top_k > n_experts)
+    return FMOE_EINVAL;
+  if (!aligned(w_router, 16) || !aligned(x, 16) || (w_sgate && !aligned(w_sgate, 16))) return FMOE_EINVAL;
+  if (ws_bytes < fmoe_route_workspace_bytes(T, n_experts)) return FMOE_ENOMEM;
+  int dev;
+  DevInfo* info;
+  if (int rc = dev_info(&dev, &info)) return rc;
+  if (int rc = check_stream(stream, dev)) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* lg = static_cast<float*>(ws);
+  const int rows = n_experts + (w_sgate ? 1 : 0);
+  router_logits_kernel<<<(rows + 7) / 8, 256, 0, s>>>(w_router, w_sgate, x, T, hidden, n_experts, lg);
+  topk_kernel<<<(T + 3) / 4, 128, 0, s>>>(lg, T, n_experts, top_k, w_sgate != nullptr, idx, w, sgate);
+  if (logits_opt) copy_logits_kernel<<<32, 256, 0, s>>>(lg, T, n_experts, logits_opt);
+  return cudaGetLastError() == cudaSuccess ? FMOE_OK : FMOE_ECUDA;
+}
+
+size_t fmoe_expert_workspace_bytes(int hidden, int inter) {
+  if (!shape_ok(hidden, inter)) return 0;
+  return kCounterBytes + round_up((size_t)inter * 4, 256);
+}
+
+int fmoe_expert_forward(const void* blob, int hidden, int inter, int bits, const float* x, float* y,
+                        void* ws, size_t ws_bytes, fmoe_stream_t stream) {
+  if (!blob || !x || !y || !ws || !bits_ok(bits) || !shape_ok(hidden, inter)) return FMOE_EINVAL;
+  if (!aligned(blob, 256) || !aligned(x, 16) || !aligned(y, 16) || !aligned(ws, 256) || x == y)
+    return FMOE_EINVAL;
+  if (ws_bytes < fmoe_expert_workspace_bytes(hidden, inter)) return FMOE_ENOMEM;
+  int dev;
+  DevInfo* info;
+  if (int rc = dev_info(&dev, &info)) return rc;
+  if (int rc = check_stream(stream, dev)) return rc;
+  Plan pl;
+  if (!plan_layer(hidden, inter, 0, true, false, bits, bits, info->max_smem, &pl)) return FMOE_EINVAL;
+  LayerArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.shared = static_cast<const char*>(blob);
+  a.x = x;
+  a.out = y;
+  char* w8 = static_cast<char*>(ws);
+  a.bar = reinterpret_cast<unsigned*>(w8);
+  a.act = reinterpret_cast<float*>(w8 + kCounterBytes);
+  a.H = hidden;
+  a.I = inter;
+  a.E = 0;
+  a.K = 0;
+  a.bits_r = bits;
+  a.bits_s = bits;
+  a.n_router = 0;
+  a.n_slots = 1;
+  a.nst = pl.nst;
+  a.stage_bytes = pl.stage_bytes;
+  a.xs4_off = pl.xs4_off;
+  a.xs2_off = pl.xs2_off;
+  a.xu_off = pl.xu_off;
+  a.vec_floats = pl.vec_floats;
+  a.sf_floats = pl.sf_floats;
+  a.timeout_ns = kTimeoutNs;
+  return launch_layer(a, pl, info, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fmoe_workspace_bytes(const fmoe_layer* L, int T) {
+  if (!L || T < 1 || T > FMOE_MAX_TOKENS) return 0;
+  return layer_ws_bytes(L->n_experts, L->inter, L->top_k, L->shared != nullptr);
+}
+
+int fmoe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream_t stream) {
+  if (!ws) return FMOE_EINVAL;
+  return cudaMemsetAsync(ws, 0, ws_bytes, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? FMOE_OK
+                                                                                                 : FMOE_ECUDA;
+}
+
+int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual, float* out, int T,
+                      void* ws, size_t ws_bytes, int32_t* idx_out_opt, float* w_out_opt,
+                      fmoe_stream_t stream) {
+  if (!L || !x || !out || !ws || !L->w_router || !L->experts) return FMOE_EINVAL;
+  const int H = L->hidden, I = L->inter, E = L->n_experts, K = L->top_k;
+  if (!shape_ok(H, I) || !bits_ok(L->bits) || (L->shared && !bits_ok(L->shared_bits)) ||
+      L->group != FMOE_GROUP || E < 1 || E > FMOE_MAX_EXPERTS || K < 1 || K > FMOE_MAX_TOPK || K > E ||
+      T < 1 || T > FMOE_MAX_TOKENS || (K + 1) * I > 10240)
+    return FMOE_EINVAL;
+  if (L->expert_stride < (int64_t)fmoe_expert_bytes(H, I, L->bits) || L->expert_stride % 256)
+    return FMOE_EINVAL;
+  if (!aligned(L->experts, 256) || (L->shared && !aligned(L->shared, 256)) || !aligned(L->w_router, 16) ||
+      (L->w_sgate && !aligned(L->w_sgate, 16)) || !aligned(x, 16) || !aligned(out, 16) ||
+      (residual && !aligned(residual, 16)) || !aligned(ws, 256) || x == out)
+    return FMOE_EINVAL;
+  if (ws_bytes < fmoe_workspace_bytes(L, T)) return FMOE_ENOMEM;
+  int dev;
+  DevInfo* info;
+  if (int rc = dev_info(&dev, &info)) return rc;
+  if (int rc = check_stream(stream, dev)) return rc;
+  const bool has_shared = L->shared != nullptr;
+  Plan pl;
+  if (!plan_layer(H, I, K, has_shared, true, L->bits, has_shared ? L->shared_bits : L->bits, info->max_smem,
+                  &pl))
+    return FMOE_EINVAL;
+  LayerArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.w_router = L->w_router;
+  a.w_sgate = L->w_sgate;
+  a.experts = static_cast<const char*>(L->experts);
+  a.expert_stride = L->expert_stride;
+  a.shared = static_cast<const char*>(L->shared);
+  char* w8 = static_cast<char*>(ws);
+  a.bar = reinterpret_cast<unsigned*>(w8);
+  a.logits = reinterpret_cast<float*>(w8 + kCounterBytes);
+  a.act = reinterpret_cast<float*>(w8 + kCounterBytes + round_up((size_t)(E + 1) * 4, 256));
+  a.H = H;
+  a.I = I;
+  a.E = E;
+  a.K = K;
+  a.bits_r = L->bits;
+  a.bits_s = has_shared ? L->shared_bits : L->bits;
+  a.n_router = E + (L->w_sgate ? 1 : 0);
+  a.n_slots = K + (has_shared ? 1 : 0);
+  a.nst = pl.nst;
+  a.stage_bytes = pl.stage_bytes;
+  a.xs4_off = pl.xs4_off;
+  a.xs2_off = pl.xs2_off;
+  a.xu_off = pl.xu_off;
+  a.vec_floats = pl.vec_floats;
+  a.sf_floats = pl.sf_floats;
+  a.timeout_ns = kTimeoutNs;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  for (int t = 0; t < T; ++t) {
+    a.x = x + (long long)t * H;
+    a.residual = residual ? residual + (long long)t * H : nullptr;
+    a.out = out + (long long)t * H;
+    a.idx_out = idx_out_opt ? idx_out_opt + (long long)t * K : nullptr;
+    a.w_out = w_out_opt ? w_out_opt + (long long)t * K : nullptr;
+    a.sg_out = nullptr;
+    if (int rc = launch_layer(a, pl, info, s)) return rc;
+  }
+  return FMOE_OK;
+}
+
+int fmoe_get_status(fmoe_stream_t stream, unsigned* bits_out) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return FMOE_ECUDA;
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_fmoe_status, sizeof(v)) != cudaSuccess) return FMOE_ECUDA;
+  if (v && cudaMemcpyToSymbol(g_fmoe_status, &zero, sizeof(zero)) != cudaSuccess) return FMOE_ECUDA;
+  if (bits_out) *bits_out = v;
+  return v ? FMOE_EDEVICE : FMOE_OK;
+}
+
+const char* fmoe_strerror(int code) {
+  switch (code) {
+    case FMOE_OK: return "ok";
+    case FMOE_EINVAL: return "invalid argument (null pointer, unsupported size or alignment)";
+    case FMOE_ENOMEM: return "caller-provided buffer or workspace too small";
+    case FMOE_ECUDA: return "CUDA runtime or launch error";
+    case FMOE_EDEVICE: return "a kernel reported an error through the device status word";
+    default: return "unknown error code";
+  }
+}
+
+}  // extern "C"

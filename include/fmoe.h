@@ -1,0 +1,191 @@
+/*
+ * fmoe — single-token quantised Mixture-of-Experts layer decode on NVIDIA B200
+ * (sm_100a).  C ABI of libfmoe.so.
+ *
+ * What the library computes is the MoE step of the Flash-MoE engine, as its
+ * pages describe it:
+ *   [P1] "397B MoE en MacBook: Motor Flash-MoE a 4,4 t/s" (aibit.im)
+ *   [P2] "Flash-MoE: Ausführen eines 397B-Parameter-Qwen-Modells auf dem
+ *        MacBook Pro mit reinem C/Metal" (openclawradar.com)
+ *   [P3] "Flash-MoE - Executando um modelo de 397 bilhões de parâmetros em um
+ *        notebook" (news.hada.io)
+ * A router projection over the experts, softmax and top-K with renormalised
+ * weights ([P2] "Pipeline-Leistung"); K routed experts plus one shared expert
+ * ([P2] "Technische Implementierung"), each a gate and an up projection, a
+ * fused SwiGLU and a down projection on affine group-quantised weights
+ * (weight = nibble * scale + bias, evaluated as fma(nibble, scale*x, bias*x):
+ * [P1] "Técnicas innovadoras" item 2, [P2] "FMA-optimierter Dequant-Kernel");
+ * and a fused end step that adds the weighted expert outputs, the residual and
+ * the sigmoid-gated shared expert ([P2] "Metal-Compute-Shader").
+ *
+ * Conventions for every entry point
+ *   - Tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or retains them past the call.
+ *   - All work is enqueued asynchronously on the caller's stream `stream`
+ *     (a cudaStream_t; NULL is the legacy default stream).  Entry points do
+ *     not synchronise, except fmoe_get_status().
+ *   - Arguments are validated on the host before anything is enqueued; an
+ *     invalid call returns an error code and enqueues nothing.
+ *   - Return values: FMOE_OK or one of the FMOE_E* codes below.
+ *
+ * Packed expert format (the pages fix only the affine form; the layout is this
+ * library's, one reading among several):
+ *   - group length 64 along a matrix's input dimension; per (row, group) one
+ *     uint32 word with the bf16 scale in bits 0..15 and the bf16 bias in bits
+ *     16..31; the dequantised weight is q * scale + bias with the unsigned
+ *     code q in [0, 2^bits - 1];
+ *   - codes: uint32 words, row-major; element k of a row is in word
+ *     k / (32/bits) at bit offset bits * (k mod 32/bits), least significant
+ *     bits first (8 nibbles or 16 two-bit codes per word);
+ *   - an expert blob is [gate codes | gate scale/bias | up codes | up
+ *     scale/bias | down codes | down scale/bias] with gate and up stored
+ *     [inter][hidden] and down stored [hidden][inter]; see fmoe_blob_offsets().
+ *   - Blobs must start on a 256-byte boundary.
+ */
+#ifndef FMOE_H
+#define FMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fmoe_stream_t; /* same type as cudaStream_t */
+
+enum {
+  FMOE_OK = 0,
+  FMOE_EINVAL = 1,  /* null pointer, unsupported size, bad alignment, wrong buffer size */
+  FMOE_ENOMEM = 2,  /* caller-provided workspace (or output buffer) too small */
+  FMOE_ECUDA = 3,   /* a CUDA runtime call or launch failed */
+  FMOE_EDEVICE = 4  /* a kernel reported an error through the device status word */
+};
+
+#define FMOE_GROUP 64        /* quantisation group length */
+#define FMOE_MAX_TOKENS 16   /* T limit of fmoe_route / fmoe_layer_decode */
+#define FMOE_MAX_TOPK 8
+#define FMOE_MAX_EXPERTS 1024
+#define FMOE_MAX_HIDDEN 8192
+
+/* Bytes of one packed expert: 3*hidden*inter*bits/8 code bytes plus 4 bytes
+ * per group of 64 weights.  ([P1] "Técnicas innovadoras" item 1 and [P2]
+ * "SSD-Experten-Streaming" give about 6.75 MB per 4-bit expert: this formula
+ * gives 6.75 MiB = 7,077,888 bytes for hidden 4096, inter 1024, bits 4.)
+ * Returns 0 for unsupported arguments (bits not 2 or 4, sizes not positive
+ * multiples of 64). */
+size_t fmoe_expert_bytes(int hidden, int inter, int bits);
+
+/* Byte offsets of the six blob sections, written to off[6] in the order gate
+ * codes, gate scale/bias, up codes, up scale/bias, down codes, down
+ * scale/bias.  Returns FMOE_EINVAL for unsupported arguments or off == NULL. */
+int fmoe_blob_offsets(int hidden, int inter, int bits, int64_t off[6]);
+
+/* Quantise one expert from fp32 weights and pack it into blob_out.
+ *   w_gate, w_up: [inter][hidden] fp32, row-major; w_down: [hidden][inter].
+ *   bits: 4 or 2; group must be 64; hidden, inter: multiples of 64.
+ *   blob_out: blob_bytes >= fmoe_expert_bytes(hidden, inter, bits), 256-byte
+ *   aligned.
+ * The pages do not describe their quantiser.  This one is affine min/max per
+ * group in IEEE fp32, in this order: s = bf16(fl(fl(max - min) / (2^b - 1))),
+ * bias = bf16(min), q = clamp(rint(fl(fl(w - bias) / s)), 0, 2^b - 1), q = 0
+ * when s == 0; bf16 rounding is to nearest even.  Deterministic and
+ * bit-reproducible.  Errors: FMOE_EINVAL, FMOE_ENOMEM (blob_bytes too small),
+ * FMOE_ECUDA. */
+int fmoe_quantize_expert(const float* w_gate, const float* w_up, const float* w_down, int hidden,
+                         int inter, int bits, int group, void* blob_out, size_t blob_bytes,
+                         fmoe_stream_t stream);
+
+/* Workspace bytes needed by fmoe_route for T tokens and n_experts experts. */
+size_t fmoe_route_workspace_bytes(int T, int n_experts);
+
+/* Router for T tokens ([P2] "Pipeline-Leistung": router projection, then
+ * softmax and top-K; [P2] "Technische Implementierung": K = 4 of 512).
+ *   w_router: [n_experts][hidden] bf16 bit patterns (uint16), row-major.
+ *   w_sgate:  [hidden] bf16 shared-gate vector, or NULL (then sgate = 1).
+ *   x:        [T][hidden] fp32.
+ *   idx:      [T][top_k] int32 out: selected experts, descending logit, lower
+ *             index first on exact ties.
+ *   w:        [T][top_k] fp32 out: softmax probabilities of the selected
+ *             experts renormalised to sum to 1.
+ *   sgate:    [T] fp32 out or NULL: sigmoid(w_sgate . x).
+ *   logits_opt: [T][n_experts] fp32 out or NULL: router logits.
+ *   ws:       device workspace, ws_bytes >= fmoe_route_workspace_bytes().
+ * Limits: 1 <= T <= 16, 1 <= top_k <= min(8, n_experts), n_experts <= 1024,
+ * hidden a multiple of 64 up to 8192.  Logits are fp32 dot products of the
+ * bf16 weights (widened exactly) with fp32 x.
+ * Errors: FMOE_EINVAL, FMOE_ENOMEM (workspace), FMOE_ECUDA. */
+int fmoe_route(const uint16_t* w_router, const uint16_t* w_sgate, const float* x, int T, int hidden,
+               int n_experts, int top_k, int32_t* idx, float* w, float* sgate, float* logits_opt,
+               void* ws, size_t ws_bytes, fmoe_stream_t stream);
+
+/* Workspace bytes needed by fmoe_expert_forward. */
+size_t fmoe_expert_workspace_bytes(int hidden, int inter);
+
+/* One expert for one token: y = Wd (silu(Wg x) * (Wu x)), where silu(z) =
+ * z * sigmoid(z) ([P2] "Metal-Compute-Shader": dequantised matrix-vector
+ * products and fused SwiGLU).
+ *   blob: one packed expert (format above), 256-byte aligned.
+ *   x: [hidden] fp32; y: [hidden] fp32 out (may not alias x).
+ *   ws: device workspace of ws_bytes >= fmoe_expert_workspace_bytes(); it
+ *   must be zero-filled before its first use (fmoe_workspace_init) and each
+ *   call leaves it ready for the next.  Calls that share a workspace must be
+ *   ordered on one stream.
+ * Limits: hidden, inter multiples of 64; hidden <= 8192; inter <= 8192;
+ * |x| below 2^100.  Errors: FMOE_EINVAL, FMOE_ENOMEM, FMOE_ECUDA. */
+int fmoe_expert_forward(const void* blob, int hidden, int inter, int bits, const float* x, float* y,
+                        void* ws, size_t ws_bytes, fmoe_stream_t stream);
+
+/* One MoE layer. */
+typedef struct {
+  const uint16_t* w_router; /* [n_experts][hidden] bf16 bits */
+  const uint16_t* w_sgate;  /* [hidden] bf16 bits, or NULL: shared expert ungated */
+  const void* experts;      /* n_experts routed blobs; blob e at experts + e * expert_stride */
+  int64_t expert_stride;    /* bytes, a multiple of 256, >= fmoe_expert_bytes(hidden, inter, bits) */
+  const void* shared;       /* shared expert blob (shared_bits wide), or NULL: no shared expert */
+  int hidden, inter, n_experts, top_k;
+  int bits;                 /* routed experts: 4 or 2 */
+  int shared_bits;          /* shared expert: 4 or 2 */
+  int group;                /* must be 64 */
+} fmoe_layer;
+
+/* Workspace bytes needed by fmoe_layer_decode for T tokens. */
+size_t fmoe_workspace_bytes(const fmoe_layer* L, int T);
+
+/* Zero-fill a workspace (enqueued on stream).  Every workspace must be
+ * zero-filled once before first use; fmoe_expert_forward and
+ * fmoe_layer_decode leave it ready for the next call. */
+int fmoe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream_t stream);
+
+/* Decode T tokens through one MoE layer:
+ *   out[t] = residual[t] + sum_k w[t][k] * E_{idx[t][k]}(x[t]) + sgate[t] * E_shared(x[t])
+ * with routing as in fmoe_route and each expert as in fmoe_expert_forward
+ * ([P2] "Metal-Compute-Shader": "MoE-Kombination + Rest + Sigmoid-Gate").
+ *   x, residual, out: [T][hidden] fp32 (residual may be NULL: zero; out may
+ *   alias residual but not x).
+ *   idx_out_opt [T][top_k] int32, w_out_opt [T][top_k] fp32: optional copies
+ *   of the routing decision.
+ *   ws: workspace of ws_bytes >= fmoe_workspace_bytes(L, T), zero-filled
+ *   before its first use; calls sharing a workspace must be stream-ordered.
+ * The whole layer runs on the GPU; the routing decision never returns to the
+ * host.  Limits: as fmoe_route and fmoe_expert_forward, plus
+ * (top_k + 1) * inter <= 10240.  Errors: FMOE_EINVAL, FMOE_ENOMEM, FMOE_ECUDA.
+ * Kernel-side problems (a time-limited wait that ran out) are reported by
+ * fmoe_get_status(). */
+int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual, float* out, int T,
+                      void* ws, size_t ws_bytes, int32_t* idx_out_opt, float* w_out_opt,
+                      fmoe_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the device status word of the
+ * current device.  Returns FMOE_OK, FMOE_EDEVICE (a kernel reported a
+ * problem; bits are in *bits_out if non-NULL) or FMOE_ECUDA. */
+int fmoe_get_status(fmoe_stream_t stream, unsigned* bits_out);
+
+/* Static, human-readable text for an error code. */
+const char* fmoe_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FMOE_H */

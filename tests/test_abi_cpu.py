@@ -1,0 +1,99 @@
+"""The C-ABI library on a machine without a GPU: it builds, loads, exports every
+declared entry point, and rejects invalid arguments on the host."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def F():
+    from bit_quantized_expert_router_b200 import build as B
+    B.build_engine()
+    import bit_quantized_expert_router_b200 as F
+    F.lib()
+    return F
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "fmoe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fmoe_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("fmoe_quantize_expert", "fmoe_route", "fmoe_expert_forward", "fmoe_layer_decode"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(F):
+    out = subprocess.run(["nm", "-D", "--defined-only", F.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (fmoe_[a-z_]+)\b", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        assert hasattr(F.lib(), n)
+    assert sorted(F.EXPORTED) == declared_functions()
+
+
+def test_layout_agrees_with_oracle(F):
+    for (h, i) in ((4096, 1024), (512, 128), (320, 192), (64, 64)):
+        for bits in (2, 4):
+            assert F.expert_bytes(h, i, bits) == O.expert_bytes(h, i, bits)
+            lay = O.blob_layout(h, i, bits)
+            assert F.blob_offsets(h, i, bits) == [lay["gate"][0], lay["gate"][1], lay["up"][0], lay["up"][1],
+                                                  lay["down"][0], lay["down"][1]]
+    assert F.expert_bytes(4096, 1024, 4) == 7_077_888
+
+
+def test_invalid_arguments_rejected_on_host(F):
+    L = F.lib()
+    assert L.fmoe_expert_bytes(4096, 1024, 3) == 0
+    assert L.fmoe_expert_bytes(100, 1024, 4) == 0
+    assert L.fmoe_expert_bytes(4096, 0, 4) == 0
+    off = (ctypes.c_int64 * 6)()
+    assert L.fmoe_blob_offsets(4096, 1024, 8, off) == F.FMOE_EINVAL
+    # null pointers
+    assert L.fmoe_expert_forward(None, 4096, 1024, 4, None, None, None, 0, None) == F.FMOE_EINVAL
+    assert L.fmoe_layer_decode(None, None, None, None, 1, None, 0, None, None, None) == F.FMOE_EINVAL
+    assert L.fmoe_route(None, None, None, 1, 4096, 512, 4, None, None, None, None, None, 0, None) == F.FMOE_EINVAL
+    assert L.fmoe_quantize_expert(None, None, None, 4096, 1024, 4, 64, None, 0, None) == F.FMOE_EINVAL
+    fake = 1 << 20  # aligned non-null stand-ins; validation fails before any use
+    base = dict(w_router=fake, w_sgate=fake, experts=fake, expert_stride=7077888 + 256 - 7077888 % 256,
+                shared=fake, hidden=4096, inter=1024, n_experts=512, top_k=4, bits=4, shared_bits=4, group=64)
+
+    def decode(T=1, ws_bytes=1 << 20, x=fake, out=fake * 2, **kw):
+        c = F.FmoeLayerC(**{**base, **kw})
+        return L.fmoe_layer_decode(ctypes.byref(c), x, None, out, T, fake, ws_bytes, None, None, None)
+
+    assert decode(bits=3) == F.FMOE_EINVAL
+    assert decode(shared_bits=8) == F.FMOE_EINVAL
+    assert decode(group=32) == F.FMOE_EINVAL
+    assert decode(hidden=4000) == F.FMOE_EINVAL
+    assert decode(inter=100) == F.FMOE_EINVAL
+    assert decode(top_k=9) == F.FMOE_EINVAL
+    assert decode(top_k=0) == F.FMOE_EINVAL
+    assert decode(n_experts=3, top_k=4) == F.FMOE_EINVAL
+    assert decode(n_experts=2048) == F.FMOE_EINVAL
+    assert decode(T=0) == F.FMOE_EINVAL
+    assert decode(T=17) == F.FMOE_EINVAL
+    assert decode(expert_stride=1000) == F.FMOE_EINVAL
+    assert decode(expert_stride=7077888 + 16) == F.FMOE_EINVAL  # not a multiple of 256
+    assert decode(experts=fake + 16) == F.FMOE_EINVAL  # blobs must be 256-byte aligned
+    assert decode(x=fake + 4) == F.FMOE_EINVAL
+    assert decode(x=fake, out=fake) == F.FMOE_EINVAL  # out may not alias x
+    assert decode(ws_bytes=16) == F.FMOE_ENOMEM
+    assert decode(inter=4096) == F.FMOE_EINVAL  # (K+1)*I above the staging limit
+    c = F.FmoeLayerC(**base)
+    assert L.fmoe_workspace_bytes(ctypes.byref(c), 1) >= 256 + 513 * 4 + 5 * 1024 * 4
+    assert L.fmoe_workspace_bytes(ctypes.byref(c), 0) == 0
+    assert L.fmoe_route_workspace_bytes(17, 512) == 0
+    for code in range(5):
+        assert len(F.strerror(code)) >= 2 and F.strerror(code) != F.strerror(99)

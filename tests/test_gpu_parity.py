@@ -1,0 +1,230 @@
+"""CUDA engine (through the C ABI) against the fp64 oracle, on seeded inputs.
+
+Integer results (packed codes, selected experts) must match bit for bit; fp32
+outputs must be within max-abs 2e-3 and relative L2 1e-4 of the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth as S
+from tests import cases as C
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def F():
+    from bit_quantized_expert_router_b200 import build as B
+    B.build_engine()
+    import synth.gpu as SG
+    SG.build()
+    import bit_quantized_expert_router_b200 as F
+    F.lib()
+    SG.lib()
+    assert torch.cuda.is_available()
+    return F
+
+
+@pytest.fixture(scope="module")
+def SG(F):
+    import synth.gpu as SG
+    return SG
+
+
+def dev():
+    return torch.device("cuda:0")
+
+
+def make_gpu_layer(F, SG, seed, layer, shape: C.Shape, with_shared=True, with_sgate=True):
+    t = SG.make_layer(seed, layer, shape.hidden, shape.inter, shape.n_experts, shape.bits, shape.shared_bits,
+                      F.blob_offsets, F.expert_bytes, dev(), with_shared, with_sgate)
+    L = F.Layer(t["w_router"], t["w_sgate"], t["experts"], t["shared"], shape.hidden, shape.inter, shape.top_k,
+                shape.bits, shape.shared_bits)
+    return L, t
+
+
+# ---------------------------------------------------------------------------
+# Generator and layout agreement
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("hidden,inter,bits", [(512, 128, 4), (4096, 1024, 4), (4096, 1024, 2), (320, 192, 2)])
+def test_device_generator_and_layout_match_host(F, SG, hidden, inter, bits):
+    assert F.expert_bytes(hidden, inter, bits) == O.expert_bytes(hidden, inter, bits)
+    lay = O.blob_layout(hidden, inter, bits)
+    assert F.blob_offsets(hidden, inter, bits) == [lay["gate"][0], lay["gate"][1], lay["up"][0], lay["up"][1],
+                                                   lay["down"][0], lay["down"][1]]
+    n = 3
+    eb = F.expert_bytes(hidden, inter, bits)
+    stride = (eb + 255) // 256 * 256
+    buf = torch.zeros(n, stride, dtype=torch.uint8, device=dev())
+    SG.fill_experts(buf, stride, F.blob_offsets(hidden, inter, bits), 5, n, hidden, inter, bits, 99, 2)
+    got = buf.cpu().numpy()
+    for e in range(n):
+        want = C.cpu_blob(99, 2, 5 + e, hidden, inter, bits)
+        assert np.array_equal(got[e, :eb], want), f"expert {5 + e}"
+
+
+# ---------------------------------------------------------------------------
+# Quantiser: bit-exact
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("hidden,inter,bits", [(512, 128, 4), (512, 128, 2), (4096, 1024, 4), (4096, 1024, 2),
+                                               (320, 192, 4)])
+def test_quantize_bit_exact(F, hidden, inter, bits):
+    wg = S.dense_matrix(3, 1, inter, hidden)
+    wu = S.dense_matrix(3, 2, inter, hidden)
+    wd = S.dense_matrix(3, 3, hidden, inter)
+    # add a constant group and an exactly-representable grid group
+    wg[0, :64] = 0.25
+    wd[1, 64:128] = np.arange(64, dtype=np.float32) % 4 * np.float32(2 ** -8) - np.float32(2 ** -6)
+    blob = F.quantize_expert(*(torch.from_numpy(m).to(dev()) for m in (wg, wu, wd)), bits)
+    want = O.quantize_expert(wg, wu, wd, bits)
+    assert np.array_equal(blob.cpu().numpy(), want)
+
+
+# ---------------------------------------------------------------------------
+# Router
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("E,H,K,T", [(16, 512, 4, 1), (512, 4096, 4, 1), (512, 4096, 4, 16), (64, 320, 8, 5),
+                                     (8, 256, 8, 3), (1024, 1024, 1, 2)])
+def test_route(F, E, H, K, T):
+    seed, layer = 21, 0
+    wr = S.router_bf16(seed, layer, E, H)
+    wsg = S.sgate_bf16(seed, layer, H)
+    x = C.parity_x(seed, layer, 0, wr, min(K, E - 1) if E > K else K, H, T) if E > K else \
+        S.token_x(seed, layer, 0, T, H)
+    idx, w, sg, logits = F.route(torch.from_numpy(wr.view(np.int16)).to(dev()),
+                                 torch.from_numpy(wsg.view(np.int16)).to(dev()), torch.from_numpy(x).to(dev()),
+                                 K, want_logits=True)
+    idx, w, sg, logits = idx.cpu().numpy(), w.cpu().numpy(), sg.cpu().numpy(), logits.cpu().numpy()
+    for t in range(T):
+        r = O.route(wr, wsg, x[t], K)
+        if E > K:
+            assert idx[t].tolist() == r["idx"].tolist()
+        else:
+            assert sorted(idx[t].tolist()) == list(range(E))
+        order = [int(np.where(r["idx"] == e)[0][0]) for e in idx[t]]
+        C.assert_close(w[t], r["w"][order], f"w token {t}", max_abs=1e-6, rel_l2=1e-6)
+        assert abs(sg[t] - r["sg"]) <= 1e-6
+        C.assert_close(logits[t], r["logits"], f"logits token {t}", max_abs=1e-4, rel_l2=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# Single expert
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("hidden,inter,bits", [(512, 128, 4), (512, 128, 2), (4096, 1024, 4), (4096, 1024, 2),
+                                               (320, 192, 4), (320, 192, 2), (64, 64, 4), (8192, 1024, 4),
+                                               (1024, 4096, 2)])
+def test_expert_forward(F, SG, hidden, inter, bits):
+    eb = F.expert_bytes(hidden, inter, bits)
+    buf = torch.zeros((eb + 255) // 256 * 256, dtype=torch.uint8, device=dev())
+    SG.fill_experts(buf, eb, F.blob_offsets(hidden, inter, bits), 0, 1, hidden, inter, bits, 7, 0, 77)
+    x = S.token_x(7, 0, 0, 1, hidden)[0]
+    y = F.expert_forward(buf, hidden, inter, bits, torch.from_numpy(x).to(dev())).cpu().numpy()
+    want = O.expert_forward(C.cpu_blob(7, 0, 77, hidden, inter, bits), hidden, inter, bits, x)
+    C.assert_close(y, want, f"expert {hidden}x{inter} {bits}-bit")
+    assert F.get_status() == 0
+
+
+def test_expert_forward_extreme_inputs(F, SG):
+    """Inputs spanning many binades (tiny, large, zeros) still match."""
+    hidden, inter, bits = 512, 128, 4
+    eb = F.expert_bytes(hidden, inter, bits)
+    buf = torch.zeros(eb, dtype=torch.uint8, device=dev())
+    SG.fill_experts(buf, eb, F.blob_offsets(hidden, inter, bits), 0, 1, hidden, inter, bits, 8, 0, 3)
+    blob = C.cpu_blob(8, 0, 3, hidden, inter, bits)
+    rng = np.random.default_rng(0)
+    for scale in (1e-20, 1e-3, 1.0, 1e4, 1e12):
+        x = (rng.standard_normal(hidden) * scale).astype(np.float32)
+        x[::7] = 0.0
+        x[3] *= 1e3
+        y = F.expert_forward(buf, hidden, inter, bits, torch.from_numpy(x).to(dev())).cpu().numpy()
+        want = O.expert_forward(blob, hidden, inter, bits, x)
+        C.assert_close(y, want, f"scale {scale}", max_abs=max(2e-3, 1e-6 * np.abs(want).max()))
+
+
+# ---------------------------------------------------------------------------
+# Whole layer
+# ---------------------------------------------------------------------------
+
+def run_layer_case(F, SG, shape, seed=5, layer=0, n_steps=2, with_shared=True, with_sgate=True):
+    L, t = make_gpu_layer(F, SG, seed, layer, shape, with_shared, with_sgate)
+    wr = S.router_bf16(seed, layer, shape.n_experts, shape.hidden)
+    for step in range(n_steps):
+        x = C.parity_x(seed, layer, step, wr, shape.top_k, shape.hidden)[0]
+        res = S.token_residual(seed, layer, step, 1, shape.hidden)[0]
+        idx = torch.empty(1, shape.top_k, dtype=torch.int32, device=dev())
+        w = torch.empty(1, shape.top_k, dtype=torch.float32, device=dev())
+        out = L.decode(torch.from_numpy(x).to(dev()), torch.from_numpy(res).to(dev()), idx_out=idx, w_out=w)
+        assert F.get_status() == 0
+        r = C.oracle_layer(seed, layer, shape, x, res, with_shared, with_sgate)
+        assert idx.cpu().numpy()[0].tolist() == r["idx"].tolist()
+        C.assert_close(w.cpu().numpy()[0], r["w"], "w", max_abs=1e-6, rel_l2=1e-6)
+        C.assert_close(out.cpu().numpy()[0], r["out"], f"{shape.name} out step {step}")
+        # the layer's own contribution (out - residual) must also be within tolerance
+        C.assert_close(out.cpu().numpy()[0] - res, r["out"] - res, f"{shape.name} delta step {step}",
+                       max_abs=2e-3, rel_l2=1e-4)
+
+
+def test_layer_tiny(F, SG):
+    run_layer_case(F, SG, C.TINY, n_steps=4)
+
+
+def test_layer_full_4bit(F, SG):
+    run_layer_case(F, SG, C.FULL4, n_steps=2)
+
+
+def test_layer_full_2bit_routed(F, SG):
+    run_layer_case(F, SG, C.FULL2, n_steps=2)
+
+
+@pytest.mark.parametrize("shape,with_shared,with_sgate", [
+    (C.Shape("ragged_h320_i192_e24_k3", 320, 192, 24, 3, 4), True, True),
+    (C.Shape("no_shared_h512_i128_e16_k4", 512, 128, 16, 4, 4), False, True),
+    (C.Shape("ungated_h512_i128_e16_k2", 512, 128, 16, 2, 2, 2), True, False),
+    (C.Shape("k1_h256_i64_e8", 256, 64, 8, 1, 4), True, True),
+    (C.Shape("k8_h1024_i1024_e64", 1024, 1024, 64, 8, 4), True, True),
+    (C.Shape("e1024_h2048_i256_k4", 2048, 256, 1024, 4, 4), True, True),
+])
+def test_layer_edge_shapes(F, SG, shape, with_shared, with_sgate):
+    run_layer_case(F, SG, shape, n_steps=2, with_shared=with_shared, with_sgate=with_sgate)
+
+
+def test_layer_all_experts_selected(F, SG):
+    """K = E: every expert is used; weights are the full softmax."""
+    shape = C.Shape("k_eq_e_h256_i64_e8", 256, 64, 8, 8, 4)
+    L, t = make_gpu_layer(F, SG, 6, 0, shape)
+    x = S.token_x(6, 0, 0, 1, 256)[0]
+    res = S.token_residual(6, 0, 0, 1, 256)[0]
+    out = L.decode(torch.from_numpy(x).to(dev()), torch.from_numpy(res).to(dev()))
+    r = C.oracle_layer(6, 0, shape, x, res)
+    C.assert_close(out.cpu().numpy()[0], r["out"], "k=e")
+
+
+def test_layer_multi_token(F, SG):
+    shape = C.TINY
+    L, t = make_gpu_layer(F, SG, 9, 1, shape)
+    wr = S.router_bf16(9, 1, shape.n_experts, shape.hidden)
+    T = 5
+    x = C.parity_x(9, 1, 0, wr, shape.top_k, shape.hidden, T)
+    res = S.token_residual(9, 1, 0, T, shape.hidden)
+    idx = torch.empty(T, shape.top_k, dtype=torch.int32, device=dev())
+    out = L.decode(torch.from_numpy(x).to(dev()), torch.from_numpy(res).to(dev()), idx_out=idx)
+    for k in range(T):
+        r = C.oracle_layer(9, 1, shape, x[k], res[k])
+        assert idx.cpu().numpy()[k].tolist() == r["idx"].tolist()
+        C.assert_close(out.cpu().numpy()[k], r["out"], f"token {k}")
+
+
+def test_layer_deterministic(F, SG):
+    L, t = make_gpu_layer(F, SG, 5, 0, C.FULL4)
+    x = torch.from_numpy(S.token_x(5, 0, 3, 1, 4096)).to(dev())
+    res = torch.from_numpy(S.token_residual(5, 0, 3, 1, 4096)).to(dev())
+    a = L.decode(x, res).clone()
+    b = L.decode(x, res).clone()
+    assert torch.equal(a, b)
+    assert F.get_status() == 0

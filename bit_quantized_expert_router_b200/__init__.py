@@ -24,14 +24,17 @@ MAX_TOPK = 8
 EXPORTED = [
     "fmoe_expert_bytes", "fmoe_blob_offsets", "fmoe_quantize_expert", "fmoe_route_workspace_bytes",
     "fmoe_route", "fmoe_expert_workspace_bytes", "fmoe_expert_forward", "fmoe_workspace_bytes",
-    "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status", "fmoe_strerror",
+    "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status", "fmoe_strerror", "fmoe_last_cuda_error",
 ]
 
 
 class FmoeError(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
-        super().__init__(f"{what}: {strerror(code)} (code {code})")
+        extra = ""
+        if code == FMOE_ECUDA:
+            extra = f", cudaError {lib().fmoe_last_cuda_error()}"
+        super().__init__(f"{what}: {strerror(code)} (code {code}{extra})")
 
 
 class FmoeLayerC(ctypes.Structure):
@@ -72,6 +75,8 @@ def lib() -> ctypes.CDLL:
     L.fmoe_workspace_init.argtypes = [vp, sz, vp]
     L.fmoe_layer_decode.argtypes = [ctypes.POINTER(FmoeLayerC), vp, vp, vp, i, vp, sz, vp, vp, vp]
     L.fmoe_get_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
+    L.fmoe_last_cuda_error.argtypes = []
+    L.fmoe_last_cuda_error.restype = i
     L.fmoe_strerror.argtypes = [i]
     L.fmoe_strerror.restype = ctypes.c_char_p
     for name in ("fmoe_blob_offsets", "fmoe_quantize_expert", "fmoe_route", "fmoe_expert_forward",

@@ -77,62 +77,77 @@ __device__ __forceinline__ void dot_word2(uint64_t& acc, uint32_t w, ulonglong2 
   ffma2(acc, pk_u32(w8 & 0x300000u, w8 & 0xC00000u), x3.y);
 }
 
-// Staged input vector for `bits`-wide codes over n inputs:
-//   xs: float4 array [F4][NV] with NV = n / CPV vectors of CPV = 128/b inputs,
-//       xs[j*NV + v] = inputs 4j..4j+3 of vector v, each multiplied by
-//       2^(S_v - code_bitpos(b, (4j+c) mod (32/b)));
+// Bit position at which code n of a word is read, for a compile-time width.
+template <int BITS>
+__device__ __forceinline__ int code_bitpos_t(int n) {
+  if (BITS == 4) return n < 6 ? 4 * n : 4 * (n - 2);
+  return n < 12 ? 2 * n : 2 * (n - 4);
+}
+
+// Staged input for BITS-wide codes over n inputs (n a multiple of 128/BITS):
+//   xs: float4 array [F4][NV] with NV = n / CPV vectors of CPV = 128/BITS
+//       inputs: xs[j*NV + v] = inputs 4j..4j+3 of vector v, input k of the
+//       vector multiplied by 2^(S_v - code_bitpos(k mod 32/BITS));
 //   sf: float2 per vector: {sum of the vector's inputs, 2^(149 - S_v)}.
-// The transposed [F4][NV] order makes lane-consecutive vectors hit consecutive
-// shared-memory banks.
+// S_v is chosen per vector from max|x| so that every staged value and every
+// product with a decoded code stays a finite normal float.  The transposed
+// [F4][NV] order makes lane-consecutive vectors hit consecutive shared-memory
+// banks in the dot-product loops.  Several same-width inputs that lie back to
+// back in memory (the routed experts' activations) can be staged in one call;
+// input s's vectors are then columns s*(n_s/CPV) ... of one [F4][NV] array.
 //
-// stage_vector: one thread per vector (loop); src is global memory read
-// through L2 (it may have been written by other CTAs of this grid).
-__device__ inline void stage_vector(const float* __restrict__ src, int n, int bits, float4* xs,
-                                    float2* sf, int tid, int nthreads) {
-  const int CPV = 128 / bits, CPW = 32 / bits, F4 = CPV / 4, NV = n / CPV;
-  for (int v = tid; v < NV; v += nthreads) {
-    const float4* s4 = reinterpret_cast<const float4*>(src + (long long)v * CPV);
-    float4 buf[16];
-    float mx = 0.f, sum = 0.f;
+// All threads of the CTA call this; thread q of each pass handles float4 j of
+// vector v (q = v*F4 + j), and the F4 lanes of a vector combine their max and
+// sum with shuffles, so a pass costs one 16-byte load per thread.  With
+// kGlobal, src is global memory read through L2 (other CTAs of the grid may
+// have written it); otherwise src is this CTA's shared memory.
+template <int BITS, bool kGlobal>
+__device__ inline void stage_inputs(const float* __restrict__ src, int n, float4* xs, float2* sf, int tid,
+                                    int nthreads) {
+  constexpr int CPV = 128 / BITS, CPW = 32 / BITS, F4 = CPV / 4;
+  const int NV = n / CPV, total = NV * F4;
+  const int lane = tid & 31;
+  for (int base = tid - lane; base < total; base += nthreads) {
+    const int q = base + lane;
+    const bool on = q < total;
+    const int v = q / F4, j = q % F4;
+    float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (on) val = kGlobal ? __ldcg(reinterpret_cast<const float4*>(src) + q) : reinterpret_cast<const float4*>(src)[q];
+    float mx = fmaxf(fmaxf(fabsf(val.x), fabsf(val.y)), fmaxf(fabsf(val.z), fabsf(val.w)));
+    float sum = (val.x + val.y) + (val.z + val.w);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if (j < F4) {
-        buf[j] = __ldcg(s4 + j);
-        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(buf[j].x), fabsf(buf[j].y)), fmaxf(fabsf(buf[j].z), fabsf(buf[j].w))));
-        sum += (buf[j].x + buf[j].y) + (buf[j].z + buf[j].w);
-      }
+    for (int o = 1; o < F4; o <<= 1) {
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      sum += __shfl_xor_sync(0xffffffffu, sum, o);
     }
-    // S_v: max|x| * 2^S_v < 2^125, clamped so that 2^(149 - S_v) and
-    // 2^(S_v - p) stay finite normal floats.
+    // max|x| * 2^S < 2^125; S in [22, 249] keeps 2^(149 - S) and 2^(S - p) finite.
     int S = 109;
     if (mx > 0.f) {
       int e;
       frexpf(mx, &e);  // mx < 2^e
       S = 125 - e;
-      S = S < 22 ? 22 : (S > 149 + 100 ? 249 : S);
+      S = S < 22 ? 22 : (S > 249 ? 249 : S);
     }
+    const float* in = &val.x;
+    float4 o;
+    float* out = &o.x;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if (j < F4) {
-        float4 o;
-        const int n0 = (4 * j) % CPW;
-        float* oo = &o.x;
-        const float* ii = &buf[j].x;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          int e = S - code_bitpos(bits, n0 + c);  // in [0, 249]
-          float val = ii[c];
-          if (e > 126) {
-            val *= pow2f(126);
-            e -= 126;
-          }
-          oo[c] = val * pow2f(e);
-        }
-        xs[j * NV + v] = o;
+    for (int c = 0; c < 4; ++c) {
+      int e = S - code_bitpos_t<BITS>((4 * j + c) % CPW);  // in [0, 249]
+      float t = in[c];
+      if (e > 126) {
+        t *= pow2f(126);
+        e -= 126;
+      }
+      out[c] = t * pow2f(e);
+    }
+    if (on) {
+      xs[j * NV + v] = o;
+      if (j == 0) {
+        const int fe = 149 - S;  // in [-100, 127]
+        sf[v] = make_float2(sum, pow2f(fe));
       }
     }
-    const int fe = 149 - S;  // in [-100, 127]
-    sf[v] = make_float2(sum, fe < -126 ? 0.f : pow2f(fe));
   }
 }
 

@@ -16,11 +16,26 @@ constexpr int kMaxNst = 4;
 
 struct DevInfo {
   int sms = 0;
-  int max_smem = 0;
-  bool layer_attr_set = false;
+  int max_smem = 0;     // opt-in dynamic shared memory available to the layer kernel
+  bool layer_attr_set[4] = {false, false, false, false};
 };
+
+using LayerFn = void (*)(LayerArgs);
+// The instantiation for (routed bits, shared bits), and its index 0..3.
+LayerFn layer_fn(int br, int bs) {
+  if (br == 4) return bs == 4 ? layer_kernel<4, 4> : layer_kernel<4, 2>;
+  return bs == 4 ? layer_kernel<2, 4> : layer_kernel<2, 2>;
+}
+int layer_fn_index(int br, int bs) { return (br == 4 ? 0 : 2) + (bs == 4 ? 0 : 1); }
 DevInfo g_dev[64];
 std::mutex g_mu;
+thread_local int g_last_cuda_error = 0;
+
+// Record a failed CUDA call for fmoe_last_cuda_error() and map it to FMOE_ECUDA.
+int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = (int)e;
+  return FMOE_ECUDA;
+}
 
 int dev_info(int* dev_out, DevInfo** info) {
   int dev = 0;
@@ -28,20 +43,37 @@ int dev_info(int* dev_out, DevInfo** info) {
   std::lock_guard<std::mutex> lk(g_mu);
   DevInfo& d = g_dev[dev];
   if (d.sms == 0) {
-    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return FMOE_ECUDA;
-    if (cudaDeviceGetAttribute(&d.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-      return FMOE_ECUDA;
+    cudaError_t e;
+    if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e);
+    int optin = 0;
+    if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+      return cuda_fail(e);
+    int static_smem = 0;
+    for (int br : {4, 2})
+      for (int bs : {4, 2}) {
+        cudaFuncAttributes fa;
+        if ((e = cudaFuncGetAttributes(&fa, layer_fn(br, bs))) != cudaSuccess) return cuda_fail(e);
+        static_smem = std::max(static_smem, (int)fa.sharedSizeBytes);
+      }
+    d.max_smem = optin - static_smem;
   }
   *dev_out = dev;
   *info = &d;
   return FMOE_OK;
 }
 
+// The stream must belong to the current device.  The check is skipped while
+// the stream is being captured into a CUDA graph (a device query there would
+// invalidate the capture); the capture's own launches are checked on replay.
 int check_stream(fmoe_stream_t s, int dev) {
   if (s == nullptr) return FMOE_OK;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(s);
+  cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(cs, &st) != cudaSuccess) return FMOE_EINVAL;
+  if (st != cudaStreamCaptureStatusNone) return FMOE_OK;
   int sdev = -1;
-  if (cudaStreamGetDevice(reinterpret_cast<cudaStream_t>(s), &sdev) != cudaSuccess) return FMOE_EINVAL;
+  if (cudaStreamGetDevice(cs, &sdev) != cudaSuccess) return FMOE_EINVAL;
   return sdev == dev ? FMOE_OK : FMOE_EINVAL;
 }
 
@@ -52,43 +84,49 @@ bool shape_ok(int h, int i) {
 bool bits_ok(int b) { return b == 2 || b == 4; }
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Shared-memory plan of the layer kernel.
+// Shared-memory plan of the layer kernel (see carve_smem in layer_kernel.cuh).
 struct Plan {
-  int nst, stage_bytes, xs4_off, xs2_off, xu_off, vec_floats, sf_floats;
+  int nst, stage_bytes, nst_c, c_stage_bytes, xs4_off, xs2_off, xu_off, vec_floats, sf_floats, ys_stride, lg_floats;
   size_t smem;
 };
 
-bool plan_layer(int H, int I, int K, bool has_shared, bool layer_mode, int bits_r, int bits_s,
-                int max_smem, Plan* p) {
+bool plan_layer(int H, int I, int K, bool has_shared, int bits_r, int bits_s, int G, int n_router, int max_smem,
+                Plan* p) {
   const int n_slots = K + (has_shared ? 1 : 0);
   bool use4 = false, use2 = false;
-  int stage = 0;
+  int stage = 0, cstage = 0;
   auto use_bits = [&](int b) {
     if (b == 4) use4 = true; else use2 = true;
     const int cb = H * b / 8;
     const int cap = ((H / 16 + 15) & ~15) + 16;
     stage = std::max(stage, 2 * cb + 2 * cap);
-    stage = std::max(stage, kRC * (I * b / 8 + I / 16));
+    cstage = std::max(cstage, kRC * (I * b / 8 + I / 16));
   };
   if (K > 0) use_bits(bits_r);
   if (has_shared) use_bits(bits_s);
-  stage = (int)round_up(stage, 128);
+  cstage = (int)round_up(cstage, 128);
+  stage = (int)round_up(std::max(stage, cstage), 128);
   int off = 0;
-  p->xu_off = -1;
-  if (layer_mode) { p->xu_off = off; off += H; }
+  p->xu_off = off;  // x, copied in by one bulk copy
+  off += H;
   p->xs4_off = -1;
   p->xs2_off = -1;
   if (use4) { p->xs4_off = off; off += H; }
   if (use2) { p->xs2_off = off; off += H; }
   p->vec_floats = (int)round_up((size_t)std::max(off, n_slots * I), 32);
   p->sf_floats = (int)round_up((size_t)std::max((use4 ? H / 32 : 0) + (use2 ? H / 64 : 0), n_slots * I / 32), 16);
+  const int nq = H / kRC;
+  p->ys_stride = kRC * ((nq + G - 1) / G);
   p->stage_bytes = stage;
-  const size_t fixed = (size_t)p->vec_floats * 4 + (size_t)p->sf_floats * 8;
-  const size_t budget = (size_t)max_smem - sizeof(CtaShared) - 64;
+  p->lg_floats = (int)round_up((size_t)n_router, 4);
+  const size_t fixed = (size_t)p->vec_floats * 4 + (size_t)p->sf_floats * 8 +
+                       round_up((size_t)n_slots * p->ys_stride * 4, 16) + (size_t)p->lg_floats * 4;
+  p->c_stage_bytes = cstage;
   for (int nst = kMaxNst; nst >= 1; --nst) {
-    const size_t total = (size_t)kWarps * nst * stage + fixed + (size_t)kWarps * nst * 8;
-    if (total <= budget) {
+    const size_t total = (size_t)kWarps * nst * stage + fixed + (size_t)kWarps * (nst + kMaxNstC) * 8;
+    if (total <= (size_t)max_smem) {
       p->nst = nst;
+      p->nst_c = std::min(kMaxNstC, nst * stage / cstage);
       p->smem = total;
       return true;
     }
@@ -96,23 +134,30 @@ bool plan_layer(int H, int I, int K, bool has_shared, bool layer_mode, int bits_
   return false;
 }
 
-size_t layer_ws_bytes(int E, int I, int K, bool has_shared) {
-  return kCounterBytes + round_up((size_t)(E + 1) * 4, 256) + round_up((size_t)(K + 1) * I * 4, 256) +
-         (has_shared ? 0 : 0);
+size_t layer_ws_bytes(int E, int I, int K) {
+  return kCounterBytes + round_up((size_t)(E + 1) * 4, 256) + round_up((size_t)(K + 1) * I * 4, 256);
+}
+
+// Fill the grid-shape-dependent fields of the kernel arguments.
+void set_offsets(LayerArgs& a, int G) {
+  const int GW = G * kWarps;
+  const int n_static = a.shared ? a.I : 0;
+  a.off_a = a.n_router % GW;
+  a.off_b = (int)(((long long)a.n_router + n_static) % GW);
 }
 
 int launch_layer(const LayerArgs& args, const Plan& pl, DevInfo* info, cudaStream_t s) {
-  if (!info->layer_attr_set) {
-    if (cudaFuncSetAttribute(layer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             info->max_smem - (int)sizeof(CtaShared)) != cudaSuccess)
-      return FMOE_ECUDA;
-    info->layer_attr_set = true;
+  const LayerFn fn = layer_fn(args.bits_r, args.bits_s);
+  const int fi = layer_fn_index(args.bits_r, args.bits_s);
+  if (!info->layer_attr_set[fi]) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, info->max_smem);
+    if (e != cudaSuccess) return cuda_fail(e);
+    info->layer_attr_set[fi] = true;
   }
   LayerArgs a = args;
   void* kargs[] = {&a};
-  cudaError_t e = cudaLaunchCooperativeKernel((const void*)layer_kernel, dim3(info->sms), dim3(kThreads),
-                                              kargs, pl.smem, s);
-  return e == cudaSuccess ? FMOE_OK : FMOE_ECUDA;
+  cudaError_t e = cudaLaunchCooperativeKernel((const void*)fn, dim3(info->sms), dim3(kThreads), kargs, pl.smem, s);
+  return e == cudaSuccess ? FMOE_OK : cuda_fail(e);
 }
 
 }  // namespace
@@ -156,7 +201,7 @@ int fmoe_quantize_expert(const float* w_gate, const float* w_up, const float* w_
     const long long n = (long long)mm.rows * (mm.nin / 64);
     quantize_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
         mm.w, mm.rows, mm.nin, bits, reinterpret_cast<uint32_t*>(b + mm.c), reinterpret_cast<uint32_t*>(b + mm.sb));
-    if (cudaGetLastError() != cudaSuccess) return FMOE_ECUDA;
+    if (cudaError_t e = cudaGetLastError()) return cuda_fail(e);
   }
   return FMOE_OK;
 }
@@ -186,7 +231,8 @@ int fmoe_route(const uint16_t* w_router, const uint16_t* w_sgate, const float* x
   router_logits_kernel<<<(rows + 7) / 8, 256, 0, s>>>(w_router, w_sgate, x, T, hidden, n_experts, lg);
   topk_kernel<<<(T + 3) / 4, 128, 0, s>>>(lg, T, n_experts, top_k, w_sgate != nullptr, idx, w, sgate);
   if (logits_opt) copy_logits_kernel<<<32, 256, 0, s>>>(lg, T, n_experts, logits_opt);
-  return cudaGetLastError() == cudaSuccess ? FMOE_OK : FMOE_ECUDA;
+  if (cudaError_t e = cudaGetLastError()) return cuda_fail(e);
+  return FMOE_OK;
 }
 
 size_t fmoe_expert_workspace_bytes(int hidden, int inter) {
@@ -205,7 +251,7 @@ int fmoe_expert_forward(const void* blob, int hidden, int inter, int bits, const
   if (int rc = dev_info(&dev, &info)) return rc;
   if (int rc = check_stream(stream, dev)) return rc;
   Plan pl;
-  if (!plan_layer(hidden, inter, 0, true, false, bits, bits, info->max_smem, &pl)) return FMOE_EINVAL;
+  if (!plan_layer(hidden, inter, 0, true, bits, bits, info->sms, 0, info->max_smem, &pl)) return FMOE_EINVAL;
   LayerArgs a;
   std::memset(&a, 0, sizeof(a));
   a.shared = static_cast<const char*>(blob);
@@ -229,19 +275,24 @@ int fmoe_expert_forward(const void* blob, int hidden, int inter, int bits, const
   a.xu_off = pl.xu_off;
   a.vec_floats = pl.vec_floats;
   a.sf_floats = pl.sf_floats;
+  a.ys_stride = pl.ys_stride;
+  a.nst_c = pl.nst_c;
+  a.c_stage_bytes = pl.c_stage_bytes;
+  a.lg_floats = pl.lg_floats;
   a.timeout_ns = kTimeoutNs;
+  set_offsets(a, info->sms);
   return launch_layer(a, pl, info, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t fmoe_workspace_bytes(const fmoe_layer* L, int T) {
   if (!L || T < 1 || T > FMOE_MAX_TOKENS) return 0;
-  return layer_ws_bytes(L->n_experts, L->inter, L->top_k, L->shared != nullptr);
+  return layer_ws_bytes(L->n_experts, L->inter, L->top_k);
 }
 
 int fmoe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream_t stream) {
   if (!ws) return FMOE_EINVAL;
-  return cudaMemsetAsync(ws, 0, ws_bytes, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? FMOE_OK
-                                                                                                 : FMOE_ECUDA;
+  if (cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, reinterpret_cast<cudaStream_t>(stream))) return cuda_fail(e);
+  return FMOE_OK;
 }
 
 int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual, float* out, int T,
@@ -265,9 +316,10 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
   if (int rc = dev_info(&dev, &info)) return rc;
   if (int rc = check_stream(stream, dev)) return rc;
   const bool has_shared = L->shared != nullptr;
+  if (E + 1 > (kWarps / 2) * info->sms) return FMOE_EINVAL;  // router rows must leave staging warps
   Plan pl;
-  if (!plan_layer(H, I, K, has_shared, true, L->bits, has_shared ? L->shared_bits : L->bits, info->max_smem,
-                  &pl))
+  if (!plan_layer(H, I, K, has_shared, L->bits, has_shared ? L->shared_bits : L->bits, info->sms,
+                  E + (L->w_sgate ? 1 : 0), info->max_smem, &pl))
     return FMOE_EINVAL;
   LayerArgs a;
   std::memset(&a, 0, sizeof(a));
@@ -295,7 +347,12 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
   a.xu_off = pl.xu_off;
   a.vec_floats = pl.vec_floats;
   a.sf_floats = pl.sf_floats;
+  a.ys_stride = pl.ys_stride;
+  a.nst_c = pl.nst_c;
+  a.c_stage_bytes = pl.c_stage_bytes;
+  a.lg_floats = pl.lg_floats;
   a.timeout_ns = kTimeoutNs;
+  set_offsets(a, info->sms);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   for (int t = 0; t < T; ++t) {
     a.x = x + (long long)t * H;
@@ -310,13 +367,34 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
 }
 
 int fmoe_get_status(fmoe_stream_t stream, unsigned* bits_out) {
-  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return FMOE_ECUDA;
+  if (cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream))) return cuda_fail(e);
   unsigned v = 0, zero = 0;
-  if (cudaMemcpyFromSymbol(&v, g_fmoe_status, sizeof(v)) != cudaSuccess) return FMOE_ECUDA;
-  if (v && cudaMemcpyToSymbol(g_fmoe_status, &zero, sizeof(zero)) != cudaSuccess) return FMOE_ECUDA;
+  if (cudaError_t e = cudaMemcpyFromSymbol(&v, g_fmoe_status, sizeof(v))) return cuda_fail(e);
+  if (v) {
+    if (cudaError_t e = cudaMemcpyToSymbol(g_fmoe_status, &zero, sizeof(zero))) return cuda_fail(e);
+  }
   if (bits_out) *bits_out = v;
   return v ? FMOE_EDEVICE : FMOE_OK;
 }
+
+int fmoe_last_cuda_error(void) { return g_last_cuda_error; }
+
+#ifdef FMOE_TRACE_BUILD
+// Trace builds only: copy the phase timestamps of the last layer launch
+// ([1024][12] u64, ns) to host memory and clear them.
+int fmoe_trace_read(unsigned long long* host) {
+  if (cudaError_t e = cudaMemcpyFromSymbol(host, g_fmoe_trace, sizeof(g_fmoe_trace))) return cuda_fail(e);
+  static unsigned long long zero[1024][kTracePoints];
+  if (cudaError_t e = cudaMemcpyToSymbol(g_fmoe_trace, zero, sizeof(zero))) return cuda_fail(e);
+  return FMOE_OK;
+}
+int fmoe_spins_read(unsigned long long* host4) {
+  if (cudaError_t e = cudaMemcpyFromSymbol(host4, g_fmoe_spins, 4 * sizeof(unsigned long long))) return cuda_fail(e);
+  static unsigned long long zero[4];
+  if (cudaError_t e = cudaMemcpyToSymbol(g_fmoe_spins, zero, sizeof(zero))) return cuda_fail(e);
+  return FMOE_OK;
+}
+#endif
 
 const char* fmoe_strerror(int code) {
   switch (code) {

@@ -9,22 +9,29 @@
 // "MoE-Kombination + Rest + Sigmoid-Gate").
 //
 // How it runs on B200.  One CTA per SM, every CTA co-resident (cooperative
-// launch).  Work is three phases of independent units, dealt round-robin over
-// all warps of the grid:
-//   A  router rows (direct 16-byte loads) and the shared expert's gate/up rows;
+// launch).  Three phases:
+//   A  router rows and the shared expert's gate/up rows (need nothing);
 //   B  the routed experts' gate/up rows (need the routing decision);
-//   C  blocks of kRC output rows of the down projections of every expert,
-//      combined with the routing weights, the shared gate and the residual.
-// Two grid-wide hand-offs separate them: "all router logits written" (before
-// any warp picks experts) and "all SwiGLU activations written" (before down).
-// Both are split-phase: a CTA arrives as soon as its own part is done and
-// waits only when it needs the result, and every wait is time-limited (it sets
-// a status bit instead of hanging).  Each warp streams its units through a
-// private ring of shared-memory stages filled by cp.async.bulk copies completed
-// on an mbarrier, so weight bytes keep flowing while the warp computes, and a
-// warp prefetches its down-projection rows while it waits for the second
-// hand-off.  No float atomics: every output is reduced by one warp in a fixed
-// order, so results are bitwise reproducible.
+//   C  the down projections of every expert over each CTA's own contiguous
+//      block of output rows, then the combine (need all SwiGLU activations).
+// Units of phases A and B are dealt round-robin over all warps of the grid.
+//
+// Hand-offs.  Each CTA publishes its router logits and then bumps a grid
+// counter once (after a fence); each CTA's first warp that needs the routing
+// decision polls that counter, reads the logits and runs the top-K, then wakes
+// the CTA's other warps through an mbarrier.  "All activations written" is a
+// second counter that every CTA bumps once and polls once.  Every wait is
+// time-limited: on expiry the kernel sets a status bit and carries on instead
+// of hanging.
+//
+// Data movement.  Each warp streams its gate/up units through a private ring
+// of shared-memory stages filled by cp.async.bulk copies that complete on an
+// mbarrier.  When its gate/up work is done, the warp re-carves its ring into
+// smaller stages and issues all of its down-projection items at once, so they
+// stream during the second hand-off; L2 is asked to prefetch the shared
+// expert's down rows at kernel start and the routed experts' down rows as soon
+// as the routing is known.  No float atomics: every output is reduced in a
+// fixed order, so results are bitwise reproducible.
 #pragma once
 #include "dequant.cuh"
 
@@ -32,10 +39,26 @@ namespace fmoe {
 
 constexpr int kWarps = 16;        // warps per CTA
 constexpr int kThreads = kWarps * 32;
-constexpr int kRC = 4;            // down rows per phase-C unit
+constexpr int kRC = 4;            // down rows per phase-C item
 constexpr int kMaxTopK = 8;
 constexpr int kMaxSlots = kMaxTopK + 1;
 constexpr int kMaxExperts = 1024; // top-K is one warp with 32 logits per lane
+constexpr int kMaxNstC = 8;       // most down-item stages a warp keeps in flight
+
+// Optional phase trace (compile with -DFMOE_TRACE_BUILD): thread 0 of every CTA
+// stores %globaltimer at fixed points of the kernel into g_fmoe_trace.
+#ifdef FMOE_TRACE_BUILD
+constexpr int kTracePoints = 16;
+__device__ unsigned long long g_fmoe_trace[1024][kTracePoints];
+#define FMOE_TRACE(i) \
+  do { if (threadIdx.x == 0 && blockIdx.x < 1024) g_fmoe_trace[blockIdx.x][i] = globaltimer_ns(); } while (0)
+#define FMOE_TRACE_WARP(i) \
+  do { if ((threadIdx.x & 31) == 0 && blockIdx.x < 1024) \
+    atomicMax(&g_fmoe_trace[blockIdx.x][i], (unsigned long long)globaltimer_ns()); } while (0)
+#else
+#define FMOE_TRACE(i) do { } while (0)
+#define FMOE_TRACE_WARP(i) do { } while (0)
+#endif
 
 struct LayerArgs {
   const uint16_t* w_router;  // [E][H] bf16 bits, or null (single-expert mode)
@@ -48,17 +71,22 @@ struct LayerArgs {
   float* out;                // [H]
   float* logits;             // workspace [E + 1]
   float* act;                // workspace [n_slots][I]
-  unsigned* bar;             // workspace [4]: logits ready, activations ready, done
+  unsigned* bar;             // workspace: [0] logits hand-off, [1] activation hand-off, [2] done ticket
   int* idx_out;              // optional [K]
   float* w_out;              // optional [K]
   float* sg_out;             // optional [1]
   int H, I, E, K, bits_r, bits_s;
   int n_router;              // router rows: E (+1 with w_sgate), 0 in single-expert mode
   int n_slots;               // K routed slots then the shared slot
-  int nst;                   // ring stages per warp
+  int off_a, off_b;          // round-robin slot offsets of phases A and B (in [0, G*kWarps))
+  int nst;                   // ring stages per warp (gate/up phases)
   int stage_bytes;
+  int nst_c;                 // ring stages per warp once re-carved for down items
+  int c_stage_bytes;
   int xs4_off, xs2_off, xu_off;  // float offsets inside the vector region (-1 = absent)
   int vec_floats, sf_floats;
+  int ys_stride;             // rows per CTA (max) in the phase-C result array
+  int lg_floats;             // shared-memory logits (n_router rounded up to 4)
   unsigned long long timeout_ns;
 };
 
@@ -66,6 +94,8 @@ struct Smem {
   char* ring;
   float* vec;
   float2* sf;
+  float* ys;   // [n_slots][ys_stride] per-expert down-projection rows of this CTA
+  float* lg;   // [lg_floats] router logits
   uint64_t* bars;
 };
 
@@ -77,21 +107,28 @@ __device__ __forceinline__ Smem carve_smem(const LayerArgs& a, char* base) {
   off += (size_t)a.vec_floats * 4;
   s.sf = reinterpret_cast<float2*>(base + off);
   off += (size_t)a.sf_floats * 8;
-  s.bars = reinterpret_cast<uint64_t*>(base + off);
+  s.ys = reinterpret_cast<float*>(base + off);
+  off += (size_t)a.n_slots * a.ys_stride * 4;
+  off = (off + 15) & ~(size_t)15;
+  s.lg = reinterpret_cast<float*>(base + off);
+  off += (size_t)a.lg_floats * 4;
+  s.bars = reinterpret_cast<uint64_t*>(base + off);  // [kWarps][nst + kMaxNstC]
   return s;
 }
 
 // ---------------------------------------------------------------------------
-// Unit bookkeeping: unit u of a phase whose numbering starts at slot offset
-// `off` goes to grid-warp slot (u + off) mod GW; slot s is warp s / G of CTA
-// s mod G, so consecutive units land on consecutive CTAs.
+// Work assignment.  Phases A and B: unit u of a phase whose numbering starts at
+// offset `off` goes to grid-warp slot (u + off) mod GW; slot s is warp s / G of
+// CTA s mod G, so consecutive units land on consecutive CTAs.  Phase C: CTA c
+// owns output-row quads [c*nq/G, (c+1)*nq/G) and its warps take the items
+// (slot, quad) of that block round-robin.
 // ---------------------------------------------------------------------------
 struct PhaseList {
   int first, count;
 };
 __device__ __forceinline__ PhaseList phase_list(int n_units, int off, int gslot, int GW) {
   PhaseList p;
-  int f = (gslot - off) % GW;
+  int f = gslot - off;
   if (f < 0) f += GW;
   p.first = f;
   p.count = (n_units > f) ? (n_units - f - 1) / GW + 1 : 0;
@@ -99,38 +136,45 @@ __device__ __forceinline__ PhaseList phase_list(int n_units, int off, int gslot,
 }
 
 struct WarpPlan {
-  PhaseList router, a, b, c;
-  int n_loads;  // ring loads: a.count + b.count + c.count * n_slots
+  PhaseList router, a, b;
+  int q0, nq;      // this CTA's quad block
+  int c_count;     // phase-C items of this warp
+  int n_loads;     // ring loads: a.count + b.count + c_count
 };
 
 __device__ __forceinline__ WarpPlan make_plan(const LayerArgs& a, int cta, int warp, int G) {
   const int GW = G * kWarps;
   const int gslot = warp * G + cta;
-  const int n_static = (a.shared != nullptr) ? a.I : 0;
-  const int n_routed = a.K * a.I;
-  const int n_c = a.H / kRC;
   WarpPlan p;
-  int off = 0;
-  p.router = phase_list(a.n_router, off, gslot, GW);
-  off = (off + a.n_router) % GW;
-  p.a = phase_list(n_static, off, gslot, GW);
-  off = (off + n_static) % GW;
-  p.b = phase_list(n_routed, off, gslot, GW);
-  off = (off + n_routed) % GW;
-  p.c = phase_list(n_c, off, gslot, GW);
-  p.n_loads = p.a.count + p.b.count + p.c.count * a.n_slots;
+  p.router = phase_list(a.n_router, 0, gslot, GW);
+  p.a = phase_list(a.shared != nullptr ? a.I : 0, a.off_a, gslot, GW);
+  p.b = phase_list(a.K * a.I, a.off_b, gslot, GW);
+  const int nq_all = a.H / kRC;  // <= 2048, so cta * nq_all fits in 32 bits
+  p.q0 = cta * nq_all / G;
+  p.nq = (cta + 1) * nq_all / G - p.q0;
+  const int n_items = a.n_slots * p.nq;
+  p.c_count = (n_items > warp) ? (n_items - warp - 1) / kWarps + 1 : 0;
+  p.n_loads = p.a.count + p.b.count + p.c_count;
   return p;
 }
 
 // Per-CTA shared state (static shared memory).
 struct CtaShared {
-  int route_state;     // 0 = not started, 1 = being computed, 2 = ready
+  uint64_t route_bar;   // completes once the routing decision is in this struct
+  uint64_t x_bar;       // completes once x is in shared memory
+  uint64_t staged_bar;  // completes once x is staged in the decode layouts
+  uint64_t lg_bar;      // completes once the router logits are in shared memory
+  float* lg;            // shared-memory copy of the router logits
+  unsigned lg_bytes;
+  int route_state;      // 0 = not started, 1 = being computed, 2 = ready
+  unsigned router_done;    // this CTA's router rows published so far
+  unsigned router_target;  // this CTA's router rows
   int idx[kMaxTopK];
   float w[kMaxTopK];
   float sg;
-  unsigned router_done;
-  unsigned router_target;
 };
+
+__device__ __forceinline__ float* cs_logits(const LayerArgs&, CtaShared& cs) { return cs.lg; }
 
 struct SlotInfo {
   const char* blob;
@@ -154,41 +198,51 @@ __device__ __forceinline__ int codes_row_bytes(int n_in, int bits) { return n_in
 __device__ __forceinline__ int sb_row_bytes(int n_in) { return n_in / 16; }
 __device__ __forceinline__ int sb_superset_cap(int n_in) { return ((n_in / 16 + 15) & ~15) + 16; }
 
-// Issue the bulk copies of ring load `i` (lane 0 only).  Returns false if the
-// load needs the routing decision and it is not known yet.
-__device__ __forceinline__ void issue_load(const LayerArgs& a, const WarpPlan& p, const CtaShared& cs,
-                                           int i, char* stage, uint64_t* bar, int GW) {
+// (slot, row) of gate/up load i < a.count + b.count.
+__device__ __forceinline__ void gu_unit(const LayerArgs& a, const WarpPlan& p, int i, int GW, int& slot,
+                                        int& row) {
+  if (i < p.a.count) {
+    slot = a.K;
+    row = p.a.first + i * GW;
+  } else {
+    const int u = p.b.first + (i - p.a.count) * GW;
+    slot = u / a.I;
+    row = u - slot * a.I;
+  }
+}
+
+// (slot, first row) of phase-C load i >= a.count + b.count.
+__device__ __forceinline__ void c_item(const WarpPlan& p, int i, int warp, int& slot, int& r0) {
+  const int j = warp + (i - p.a.count - p.b.count) * kWarps;
+  slot = j / p.nq;
+  r0 = (p.q0 + (j - slot * p.nq)) * kRC;
+}
+
+// Issue the bulk copies of ring load `i` (lane 0 only).
+//   gate/up stage: gate codes | up codes | gate sb superset | up sb superset
+//   down stage:    kRC code rows | kRC sb rows
+__device__ __noinline__ void issue_load(const LayerArgs& a, const WarpPlan& p, const CtaShared& cs, int i,
+                                           int warp, char* stage, uint64_t* bar, int GW) {
   if (i < p.a.count + p.b.count) {
     int slot, row;
-    if (i < p.a.count) {
-      slot = a.K;
-      row = p.a.first + i * GW;
-    } else {
-      const int u = p.b.first + (i - p.a.count) * GW;
-      slot = u / a.I;
-      row = u % a.I;
-    }
+    gu_unit(a, p, i, GW, slot, row);
     const SlotInfo si = slot_info(a, cs, slot);
     const BlobOff o = blob_offsets(a.H, a.I, si.bits);
     const int cb = codes_row_bytes(a.H, si.bits);
     const int sbr = sb_row_bytes(a.H);
     const int cap = sb_superset_cap(a.H);
-    const char* g_codes = si.blob + o.gc + (long long)row * cb;
-    const char* u_codes = si.blob + o.uc + (long long)row * cb;
     const long long gs0 = o.gsb + (long long)row * sbr, us0 = o.usb + (long long)row * sbr;
     const long long ga = gs0 & ~15LL, ua = us0 & ~15LL;
     const int glen = (int)(((gs0 + sbr + 15) & ~15LL) - ga);
     const int ulen = (int)(((us0 + sbr + 15) & ~15LL) - ua);
     mbar_arrive_expect_tx(bar, 2 * cb + glen + ulen);
-    bulk_g2s(stage, g_codes, cb, bar);
-    bulk_g2s(stage + cb, u_codes, cb, bar);
+    bulk_g2s(stage, si.blob + o.gc + (long long)row * cb, cb, bar);
+    bulk_g2s(stage + cb, si.blob + o.uc + (long long)row * cb, cb, bar);
     bulk_g2s(stage + 2 * cb, si.blob + ga, glen, bar);
     bulk_g2s(stage + 2 * cb + cap, si.blob + ua, ulen, bar);
   } else {
-    const int j = i - p.a.count - p.b.count;
-    const int unit = p.c.first + (j / a.n_slots) * GW;
-    const int slot = j % a.n_slots;
-    const int r0 = unit * kRC;
+    int slot, r0;
+    c_item(p, i, warp, slot, r0);
     const SlotInfo si = slot_info(a, cs, slot);
     const BlobOff o = blob_offsets(a.H, a.I, si.bits);
     const int cb = codes_row_bytes(a.I, si.bits);
@@ -203,20 +257,22 @@ __device__ __forceinline__ void issue_load(const LayerArgs& a, const WarpPlan& p
 // Compute pieces
 // ---------------------------------------------------------------------------
 
-// One router row (bf16) against the unscaled input x (shared memory).
+// One router row (bf16) against the unscaled input x (shared memory), in
+// chunks of 8 16-byte vectors per lane (all loads of a chunk in flight).
+constexpr int kRouterChunk = 8;
 __device__ __forceinline__ float router_dot(const uint16_t* row, const float* xu, int H, int lane) {
   const uint4* rv = reinterpret_cast<const uint4*>(row);
   const int nv = H / 8;
   float acc = 0.f;
-  for (int base = 0; base < nv; base += 32 * 16) {
-    uint4 w[16];
+  for (int base = 0; base < nv; base += 32 * kRouterChunk) {
+    uint4 w[kRouterChunk];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
+    for (int i = 0; i < kRouterChunk; ++i) {
       const int v = base + lane + 32 * i;
       if (v < nv) w[i] = ld_stream_u4(rv + v);
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
+    for (int i = 0; i < kRouterChunk; ++i) {
       const int v = base + lane + 32 * i;
       if (v < nv) {
         const float4 xa = reinterpret_cast<const float4*>(xu)[2 * v];
@@ -281,17 +337,18 @@ __device__ __forceinline__ void pair_dot(const char* st, int H, int sbo_g, int s
 }
 
 // kRC down rows of one expert (stage layout: kRC code rows | kRC sb rows)
-// against that expert's staged activation; adds coef * row dot to acc[r].
+// against that expert's staged activation, which is column block
+// [col0, col0 + I/CPV) of a staged [F4][NVS] array (several same-width experts
+// staged together); sfa points at column col0.  Returns the full row dots.
 template <int BITS>
-__device__ __forceinline__ void down_rows(const char* st, int I, const float4* as, const float2* sfa,
-                                          int lane, float coef, float (&acc)[kRC]) {
+__device__ __forceinline__ void down_rows(const char* st, int I, const float4* as, int NVS, int col0,
+                                          const float2* sfa, int lane, float (&y)[kRC]) {
   constexpr int CPV = 128 / BITS;
   const int NV = I / CPV;
   const int cb = I * BITS / 8;
   const int ng = I / 64;
   const uint32_t* sb = reinterpret_cast<const uint32_t*>(st + kRC * cb);
-  const ulonglong2* xv = reinterpret_cast<const ulonglong2*>(as);
-  float y[kRC];
+  const ulonglong2* xv = reinterpret_cast<const ulonglong2*>(as + col0);
 #pragma unroll
   for (int r = 0; r < kRC; ++r) y[r] = 0.f;
   for (int v = lane; v < NV; v += 32) {
@@ -306,12 +363,12 @@ __device__ __forceinline__ void down_rows(const char* st, int I, const float4* a
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       if (BITS == 4) {
-        const ulonglong2 xa = xv[(2 * t) * NV + v], xb = xv[(2 * t + 1) * NV + v];
+        const ulonglong2 xa = xv[(2 * t) * NVS + v], xb = xv[(2 * t + 1) * NVS + v];
 #pragma unroll
         for (int r = 0; r < kRC; ++r) dot_word4(ac[r], (&w[r].x)[t], xa, xb);
       } else {
-        const ulonglong2 x0 = xv[(4 * t) * NV + v], x1 = xv[(4 * t + 1) * NV + v];
-        const ulonglong2 x2 = xv[(4 * t + 2) * NV + v], x3 = xv[(4 * t + 3) * NV + v];
+        const ulonglong2 x0 = xv[(4 * t) * NVS + v], x1 = xv[(4 * t + 1) * NVS + v];
+        const ulonglong2 x2 = xv[(4 * t + 2) * NVS + v], x3 = xv[(4 * t + 3) * NVS + v];
 #pragma unroll
         for (int r = 0; r < kRC; ++r) dot_word2(ac[r], (&w[r].x)[t], x0, x1, x2, x3);
       }
@@ -325,61 +382,91 @@ __device__ __forceinline__ void down_rows(const char* st, int I, const float4* a
     }
   }
 #pragma unroll
-  for (int r = 0; r < kRC; ++r) acc[r] = fmaf(coef, y[r], acc[r]);
+  for (int r = 0; r < kRC; ++r) y[r] = warp_sum(y[r]);
 }
 
-// Top-K over n logits by one warp: descending logit, lower index first on
-// exact ties; renormalised softmax weights over the selected logits.
-__device__ __forceinline__ void warp_topk(const float* logits, int n, int k, int lane, int* idx_out,
-                                          float* w_out) {
-  float v[kMaxExperts / 32];
+// Top-K by one warp: descending logit, lower index first on exact ties; then
+// renormalised softmax weights over the selected logits.  Each (logit, index)
+// pair is one 64-bit key whose unsigned order is that order: order-preserving
+// float bits above, the complemented index below.  Each lane holds 32 keys in
+// registers and its current maximum; a round is one warp-wide hardware max
+// (__reduce_max_sync) of the maxima's upper halves, one of the lower halves
+// among the lanes that hold that upper half, and a rescan by the single lane
+// that owned the winner.
+__device__ __forceinline__ uint32_t order_bits(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float from_order_bits(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+__device__ __forceinline__ unsigned long long umax64(unsigned long long p, unsigned long long q) {
+  return p > q ? p : q;
+}
+template <int NK>
+__device__ __forceinline__ unsigned long long max_tree(const unsigned long long (&key)[NK]) {
+  unsigned long long m[NK / 2];
 #pragma unroll
-  for (int i = 0; i < kMaxExperts / 32; ++i) {
+  for (int i = 0; i < NK / 2; ++i) m[i] = umax64(key[2 * i], key[2 * i + 1]);
+#pragma unroll
+  for (int w = NK / 4; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) m[i] = umax64(m[2 * i], m[2 * i + 1]);
+  return m[0];
+}
+
+// NK keys per lane (16 covers 512 experts, 32 covers 1024).  kShared: the
+// logits are in this CTA's shared memory, else in global memory.
+template <bool kShared, int NK>
+__device__ __noinline__ void warp_topk_n(const float* lg, int n, int k, int lane, int* idx_out, float* w_out) {
+  unsigned long long key[NK];
+#pragma unroll
+  for (int i = 0; i < NK; ++i) {
     const int e = i * 32 + lane;
-    v[i] = (e < n) ? __ldcg(logits + e) : -INFINITY;
+    key[i] = 0ull;
+    if (e < n)
+      key[i] = ((unsigned long long)order_bits(kShared ? lg[e] : __ldcg(lg + e)) << 32) | (uint32_t)(~(uint32_t)e);
   }
-  float top[kMaxTopK];
-  int topi[kMaxTopK];
+  unsigned long long mine = max_tree<NK>(key);
+  float my_val = 0.f;
+  int my_idx = 0;
+#pragma unroll 1
   for (int kk = 0; kk < k; ++kk) {
-    float best = -INFINITY;
-    int bi = 0x7fffffff;
+    const uint32_t mh = (uint32_t)(mine >> 32);
+    const uint32_t h = __reduce_max_sync(0xffffffffu, mh);
+    const unsigned tie = __ballot_sync(0xffffffffu, mh == h);
+    // usually one lane holds the largest logit; an exact tie needs the index max
+    const uint32_t l = (tie & (tie - 1)) ? __reduce_max_sync(0xffffffffu, mh == h ? (uint32_t)mine : 0u)
+                                         : __shfl_sync(0xffffffffu, (uint32_t)mine, __ffs(tie) - 1);
+    const unsigned long long best = ((unsigned long long)h << 32) | l;
+    if (mine == best) {  // keys are unique: exactly one lane owned the winner
 #pragma unroll
-    for (int i = 0; i < kMaxExperts / 32; ++i) {
-      const int e = i * 32 + lane;
-      if (e < n && (v[i] > best || (v[i] == best && e < bi))) {
-        best = v[i];
-        bi = e;
-      }
+      for (int i = 0; i < NK; ++i)
+        if (key[i] == best) key[i] = 0ull;
+      mine = max_tree<NK>(key);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ob = __shfl_xor_sync(0xffffffffu, best, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ob > best || (ob == best && oi < bi)) {
-        best = ob;
-        bi = oi;
-      }
+    if (lane == kk) {
+      my_val = from_order_bits(h);
+      my_idx = (int)~l;
     }
-    top[kk] = best;
-    topi[kk] = bi;
-#pragma unroll
-    for (int i = 0; i < kMaxExperts / 32; ++i)
-      if (i * 32 + lane == bi) v[i] = -INFINITY;
   }
+  FMOE_TRACE_WARP(14);
   // w_k = exp(l_k - l_0) / sum_j exp(l_j - l_0): softmax restricted to the
   // selected experts, equal to softmax-then-renormalise.
-  float e[kMaxTopK];
-  float s = 0.f;
-  for (int kk = 0; kk < k; ++kk) {
-    e[kk] = expf(top[kk] - top[0]);
-    s += e[kk];
+  const float l0 = __shfl_sync(0xffffffffu, my_val, 0);
+  const float ex = (lane < k) ? expf(my_val - l0) : 0.f;
+  const float s = warp_sum(ex);
+  if (lane < k) {
+    idx_out[lane] = my_idx;
+    w_out[lane] = ex / s;
   }
-  if (lane == 0) {
-    for (int kk = 0; kk < k; ++kk) {
-      idx_out[kk] = topi[kk];
-      w_out[kk] = e[kk] / s;
-    }
-  }
+}
+template <bool kShared>
+__device__ __forceinline__ void warp_topk(const float* lg, int n, int k, int lane, int* idx_out, float* w_out) {
+  if (n <= 512)
+    warp_topk_n<kShared, 16>(lg, n, k, lane, idx_out, w_out);
+  else
+    warp_topk_n<kShared, kMaxExperts / 32>(lg, n, k, lane, idx_out, w_out);
 }
 
 // Wait until *ctr >= target (one thread), for at most limit_ns.
@@ -387,6 +474,7 @@ __device__ __forceinline__ bool grid_wait(const unsigned* ctr, unsigned target, 
   if (ld_acquire_gpu(ctr) >= target) return true;
   const uint64_t t0 = globaltimer_ns();
   while (ld_acquire_gpu(ctr) < target) {
+    FMOE_SPIN(1);
     __nanosleep(64);
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
@@ -394,9 +482,11 @@ __device__ __forceinline__ bool grid_wait(const unsigned* ctr, unsigned target, 
 }
 
 // Make the routing decision available in this CTA's shared state.  The first
-// warp to ask waits for all router logits and runs the top-K; the others wait
-// for it.  Called by whole warps.
-__device__ __noinline__ void ensure_routing(const LayerArgs& a, CtaShared& cs, int lane) {
+// warp to ask waits until every CTA has published its router logits, reads
+// them, runs the top-K and completes the CTA's routing mbarrier, then asks L2
+// to prefetch the routed experts' down rows of this CTA; the other warps sleep
+// on the mbarrier.  Called by whole warps.
+__device__ __noinline__ void ensure_routing(const LayerArgs& a, CtaShared& cs, const WarpPlan& plan, int lane) {
   if (*((volatile int*)&cs.route_state) == 2) return;
   int old = 0;
   if (lane == 0) old = atomicCAS(&cs.route_state, 0, 1);
@@ -405,13 +495,28 @@ __device__ __noinline__ void ensure_routing(const LayerArgs& a, CtaShared& cs, i
     bool ok = true;
     if (lane == 0) ok = grid_wait(&a.bar[0], gridDim.x, a.timeout_ns);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    __syncwarp();
     if (!ok && lane == 0) set_status(kStatusGridBarrierTimeout);
-    warp_topk(a.logits, a.E, a.K, lane, cs.idx, cs.w);
+    FMOE_TRACE_WARP(9);
+    // One bulk copy brings every logit into shared memory (the async proxy
+    // reads what this thread acquired, hence the proxy fence).
+    float* lg = cs_logits(a, cs);
+    if (lane == 0) {
+      fence_proxy_async_global();
+      mbar_arrive_expect_tx(&cs.lg_bar, cs.lg_bytes);
+      bulk_g2s(lg, a.logits, cs.lg_bytes, &cs.lg_bar);
+    }
+    if (!mbar_wait_bounded(&cs.lg_bar, 0, a.timeout_ns) && lane == 0) set_status(kStatusCopyTimeout);
+    const float lsg = a.w_sgate ? lg[a.E] : 0.f;
+    FMOE_TRACE_WARP(12);
+    warp_topk<true>(lg, a.E, a.K, lane, cs.idx, cs.w);
+    __syncwarp();
+    FMOE_TRACE_WARP(10);
     if (lane == 0) {
       // Guard the expert index even on a timed-out (garbage) path.
       for (int k = 0; k < a.K; ++k)
         if (cs.idx[k] < 0 || cs.idx[k] >= a.E) cs.idx[k] = 0;
-      cs.sg = a.w_sgate ? sigmoidf_(__ldcg(a.logits + a.E)) : 1.0f;
+      cs.sg = a.w_sgate ? sigmoidf_(lsg) : 1.0f;
       if (blockIdx.x == 0) {
         for (int k = 0; k < a.K; ++k) {
           if (a.idx_out) a.idx_out[k] = cs.idx[k];
@@ -419,28 +524,39 @@ __device__ __noinline__ void ensure_routing(const LayerArgs& a, CtaShared& cs, i
         }
         if (a.sg_out) *a.sg_out = cs.sg;
       }
-      __threadfence_block();
-      atomicExch(&cs.route_state, 2);
+      *((volatile int*)&cs.route_state) = 2;
+      mbar_arrive(&cs.route_bar);  // release: publishes idx, w, sg to the CTA
+    }
+    FMOE_TRACE_WARP(3);
+    __syncwarp();
+    // L2 prefetch of this CTA's routed down rows, one lane per routed slot.
+    if (lane < a.K && plan.nq > 0) {
+      const SlotInfo si = slot_info(a, cs, lane);
+      const BlobOff o = blob_offsets(a.H, a.I, si.bits);
+      const int cb = codes_row_bytes(a.I, si.bits), sbr = sb_row_bytes(a.I);
+      const long long r0 = (long long)plan.q0 * kRC, nr = (long long)plan.nq * kRC;
+      bulk_prefetch_l2(si.blob + o.dc + r0 * cb, (uint32_t)(nr * cb));
+      bulk_prefetch_l2(si.blob + o.dsb + r0 * sbr, (uint32_t)(nr * sbr));
     }
     __syncwarp();
   } else {
-    bool ok = true;
-    if (lane == 0) {
-      const uint64_t t0 = globaltimer_ns();
-      while (*((volatile int*)&cs.route_state) != 2) {
-        __nanosleep(32);
-        if (globaltimer_ns() - t0 > a.timeout_ns) {
-          ok = false;
-          break;
-        }
-      }
-      if (!ok) set_status(kStatusCtaWaitTimeout);
-      __threadfence_block();
-    }
+    if (!mbar_wait_bounded(&cs.route_bar, 0, a.timeout_ns) && lane == 0) set_status(kStatusCtaWaitTimeout);
     __syncwarp();
   }
 }
 
+// Issue phase-C load i (>= a.count + b.count) into the re-carved ring (lane 0).
+__device__ __forceinline__ void issue_c(const LayerArgs& a, const WarpPlan& p, const CtaShared& cs, int i,
+                                        int warp, char* ring, uint64_t* bars_c, int GW) {
+  const int j = i - p.a.count - p.b.count;
+  fence_proxy_async_smem();
+  issue_load(a, p, cs, i, warp, ring + (size_t)(j % a.nst_c) * a.c_stage_bytes, &bars_c[j % a.nst_c], GW);
+}
+
+// BR, BS: code width of the routed experts and of the shared (or single)
+// expert; each combination is its own instantiation so a launch carries only
+// the dequantisation code it runs.
+template <int BR, int BS>
 __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constant__ LayerArgs a) {
   extern __shared__ __align__(128) char smem_raw[];
   __shared__ CtaShared cs;
@@ -449,60 +565,85 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   const int G = gridDim.x, GW = G * kWarps;
   const WarpPlan plan = make_plan(a, blockIdx.x, warp, G);
   char* my_ring = sm.ring + (size_t)warp * a.nst * a.stage_bytes;
-  uint64_t* my_bars = sm.bars + warp * a.nst;
+  uint64_t* my_bars = sm.bars + warp * (a.nst + kMaxNstC);
+  uint64_t* my_bars_c = my_bars + a.nst;
   const bool layer_mode = a.n_router > 0;
+  const bool router_warp = plan.router.count > 0;
+  // Router rows go to warps w with w*G + cta < n_router, i.e. the first ones.
+  const int n_router_warps = min(kWarps, max(0, (a.n_router - (int)blockIdx.x + G - 1) / G));
+  FMOE_TRACE(0);
 
+  // ---- Set-up: x to shared memory by one bulk copy; prefetches to L2 --------
+  auto router_row_ptr = [&](int e) { return (e < a.E) ? a.w_router + (long long)e * a.H : a.w_sgate; };
   if (tid == 0) {
+    mbar_init(&cs.route_bar, 1);
+    mbar_init(&cs.x_bar, 1);
+    mbar_init(&cs.staged_bar, kWarps - n_router_warps);
+    mbar_init(&cs.lg_bar, 1);
+    cs.lg = sm.lg;
+    cs.lg_bytes = (unsigned)a.lg_floats * 4u;
     cs.route_state = layer_mode ? 0 : 2;
     cs.sg = 1.0f;
     cs.router_done = 0;
-    // router rows owned by this CTA
-    unsigned tgt = 0;
-    for (int w = 0; w < kWarps; ++w) tgt += phase_list(a.n_router, 0, w * G + blockIdx.x, GW).count;
-    cs.router_target = tgt;
+    cs.router_target = n_router_warps;  // n_router < G * kWarps: one row per router warp
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(&cs.x_bar, a.H * 4);
+    bulk_g2s(sm.vec + a.xu_off, a.x, a.H * 4, &cs.x_bar);
   }
   if (lane == 0) {
-    for (int s = 0; s < a.nst; ++s) mbar_init(&my_bars[s], 1);
+    for (int j = 0; j < plan.router.count; ++j) bulk_prefetch_l2(router_row_ptr(plan.router.first + j * GW), a.H * 2);
+    for (int s = 0; s < a.nst + kMaxNstC; ++s) mbar_init(&my_bars[s], 1);
     fence_proxy_async_smem();
   }
+  if (warp == kWarps - 1 && lane == 0 && a.shared && plan.nq > 0) {
+    // the shared expert's down rows of this CTA are known from the start
+    const BlobOff o = blob_offsets(a.H, a.I, a.bits_s);
+    const int cb = codes_row_bytes(a.I, a.bits_s), sbr = sb_row_bytes(a.I);
+    const long long r0 = (long long)plan.q0 * kRC, nr = (long long)plan.nq * kRC;
+    bulk_prefetch_l2(a.shared + o.dc + r0 * cb, (uint32_t)(nr * cb));
+    bulk_prefetch_l2(a.shared + o.dsb + r0 * sbr, (uint32_t)(nr * sbr));
+  }
   __syncthreads();
+  FMOE_TRACE(11);
   if (tid == 0 && layer_mode && cs.router_target == 0) red_release_gpu_add(&a.bar[0], 1);
 
   // Prologue: start the first ring loads that need no routing decision.
   int issued = 0;
   if (lane == 0) {
-    while (issued < plan.n_loads && issued < a.nst && issued < plan.a.count) {
-      issue_load(a, plan, cs, issued, my_ring + (size_t)issued * a.stage_bytes, &my_bars[issued], GW);
+    while (issued < plan.a.count && issued < a.nst) {
+      issue_load(a, plan, cs, issued, warp, my_ring + (size_t)issued * a.stage_bytes, &my_bars[issued], GW);
       ++issued;
     }
   }
   issued = __shfl_sync(0xffffffffu, issued, 0);
 
-  // Stage x: unscaled copy for the router, decode layouts for the experts.
-  if (layer_mode) {
-    float4* xu4 = reinterpret_cast<float4*>(sm.vec + a.xu_off);
-    const float4* x4 = reinterpret_cast<const float4*>(a.x);
-    for (int i = tid; i < a.H / 4; i += kThreads) xu4[i] = __ldcg(x4 + i);
-  }
-  if (a.xs4_off >= 0)
-    stage_vector(a.x, a.H, 4, reinterpret_cast<float4*>(sm.vec + a.xs4_off), sm.sf, tid, kThreads);
-  if (a.xs2_off >= 0)
-    stage_vector(a.x, a.H, 2, reinterpret_cast<float4*>(sm.vec + a.xs2_off),
-                 sm.sf + (a.xs4_off >= 0 ? a.H / 32 : 0), tid, kThreads);
-  __syncthreads();
-
-  // ---- Phase A: router rows --------------------------------------------------
-  for (int j = 0; j < plan.router.count; ++j) {
-    const int e = plan.router.first + j * GW;
-    const uint16_t* row = (e < a.E) ? a.w_router + (long long)e * a.H : a.w_sgate;
-    const float l = router_dot(row, sm.vec + a.xu_off, a.H, lane);
-    if (lane == 0) {
-      a.logits[e] = l;
-      __threadfence();
-      const unsigned d = atomicAdd(&cs.router_done, 1u);
-      if (d + 1 == cs.router_target) red_release_gpu_add(&a.bar[0], 1);
+  if (!mbar_wait_bounded(&cs.x_bar, 0, a.timeout_ns) && lane == 0) set_status(kStatusCopyTimeout);
+  const float* xu = sm.vec + a.xu_off;
+  if (router_warp) {
+    // ---- Phase A, router rows: published, then counted once per CTA ---------
+    for (int j = 0; j < plan.router.count; ++j) {
+      const int e = plan.router.first + j * GW;
+      const float l = router_dot(router_row_ptr(e), xu, a.H, lane);
+      if (lane == 0) {
+        a.logits[e] = l;
+        __threadfence();
+        if (atomicAdd(&cs.router_done, 1u) + 1 == cs.router_target) red_release_gpu_add(&a.bar[0], 1);
+      }
     }
+    FMOE_TRACE_WARP(2);
+  } else {
+    // ---- Stage x into the decode layouts (the non-router warps) --------------
+    const int t0 = tid - n_router_warps * 32, nt = kThreads - n_router_warps * 32;
+    if (BR == 4 || BS == 4)
+      stage_inputs<4, false>(xu, a.H, reinterpret_cast<float4*>(sm.vec + a.xs4_off), sm.sf, t0, nt);
+    if (BR == 2 || BS == 2)
+      stage_inputs<2, false>(xu, a.H, reinterpret_cast<float4*>(sm.vec + a.xs2_off),
+                             sm.sf + (a.xs4_off >= 0 ? a.H / 32 : 0), t0, nt);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&cs.staged_bar);
   }
+  if (!mbar_wait_bounded(&cs.staged_bar, 0, a.timeout_ns) && lane == 0) set_status(kStatusCtaWaitTimeout);
+  FMOE_TRACE(1);
 
   // ---- Ring loop over phases A (static gate/up) and B (routed gate/up) ------
   const int n_gu = plan.a.count + plan.b.count;
@@ -520,16 +661,16 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
       int ready = 0;
       if (lane == 0) ready = *((volatile int*)&cs.route_state) == 2;
       ready = __shfl_sync(0xffffffffu, ready, 0);
-      const bool could = issued >= plan.a.count && issued < i + a.nst && issued < plan.n_loads;
+      const bool could = issued >= plan.a.count && issued < i + a.nst && issued < n_gu;
       if (i >= plan.a.count || (could && ready)) {
-        ensure_routing(a, cs, lane);
+        ensure_routing(a, cs, plan, lane);
         have_routing = true;
       }
     }
     if (lane == 0) {
-      while (issued < plan.n_loads && issued < i + a.nst && (have_routing || issued < plan.a.count)) {
+      while (issued < n_gu && issued < i + a.nst && (have_routing || issued < plan.a.count)) {
         fence_proxy_async_smem();
-        issue_load(a, plan, cs, issued, my_ring + (size_t)(issued % a.nst) * a.stage_bytes,
+        issue_load(a, plan, cs, issued, warp, my_ring + (size_t)(issued % a.nst) * a.stage_bytes,
                    &my_bars[issued % a.nst], GW);
         ++issued;
       }
@@ -539,119 +680,112 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     const char* stage = my_ring + (size_t)st_i * a.stage_bytes;
     if (!mbar_wait_bounded(&my_bars[st_i], (i / a.nst) & 1, a.timeout_ns) && lane == 0)
       set_status(kStatusCopyTimeout);
+    if (i == n_gu - 1) FMOE_TRACE_WARP(13);
     int slot, row;
-    if (i < plan.a.count) {
-      slot = a.K;
-      row = plan.a.first + i * GW;
-    } else {
-      const int u = plan.b.first + (i - plan.a.count) * GW;
-      slot = u / a.I;
-      row = u % a.I;
-    }
-    const SlotInfo si = slot_info(a, cs, slot);
-    const BlobOff o = blob_offsets(a.H, a.I, si.bits);
+    gu_unit(a, plan, i, GW, slot, row);
+    const bool routed = slot < a.K;
+    const BlobOff o = blob_offsets(a.H, a.I, routed ? BR : BS);
     const int sbr = sb_row_bytes(a.H);
     const int sbo_g = (int)((o.gsb + (long long)row * sbr) & 15);
     const int sbo_u = (int)((o.usb + (long long)row * sbr) & 15);
     float g, u;
-    if (si.bits == 4)
-      pair_dot<4>(stage, a.H, sbo_g, sbo_u, xs4, sf4, lane, g, u);
+    if (BR == BS || routed)
+      pair_dot<BR>(stage, a.H, sbo_g, sbo_u, BR == 4 ? xs4 : xs2, BR == 4 ? sf4 : sf2, lane, g, u);
     else
-      pair_dot<2>(stage, a.H, sbo_g, sbo_u, xs2, sf2, lane, g, u);
+      pair_dot<BS>(stage, a.H, sbo_g, sbo_u, BS == 4 ? xs4 : xs2, BS == 4 ? sf4 : sf2, lane, g, u);
     if (lane == 0) a.act[(long long)slot * a.I + row] = g * sigmoidf_(g) * u;
     __syncwarp();
   }
 
-  // Gate/up work of this warp is done: put its first down-projection loads in
-  // flight before joining the hand-off, so they stream during the wait.
-  if (plan.n_loads > n_gu) {
-    if (!have_routing) {
-      ensure_routing(a, cs, lane);
-      have_routing = true;
-    }
-    if (lane == 0) {
-      while (issued < plan.n_loads && issued < n_gu + a.nst) {
-        fence_proxy_async_smem();
-        issue_load(a, plan, cs, issued, my_ring + (size_t)(issued % a.nst) * a.stage_bytes,
-                   &my_bars[issued % a.nst], GW);
-        ++issued;
-      }
-    }
-    issued = __shfl_sync(0xffffffffu, issued, 0);
+  // Gate/up work of this warp is done (its ring is free): re-carve the ring
+  // into down-item stages and put this warp's down items in flight before
+  // joining the hand-off, so they stream during the wait.  (The routing
+  // decision is needed for their addresses; CTA 0 also needs it for the
+  // optional routing outputs.)
+  if (layer_mode && !have_routing && (plan.n_loads > n_gu || (blockIdx.x == 0 && warp == 0))) {
+    ensure_routing(a, cs, plan, lane);
+    have_routing = true;
   }
+  int issued_c = n_gu;
+  if (lane == 0)
+    while (issued_c < plan.n_loads && issued_c < n_gu + a.nst_c) {
+      issue_c(a, plan, cs, issued_c, warp, my_ring, my_bars_c, GW);
+      ++issued_c;
+    }
+  issued_c = __shfl_sync(0xffffffffu, issued_c, 0);
 
   // ---- Hand-off: every activation of the grid is written --------------------
+  FMOE_TRACE_WARP(4);
   __syncthreads();
   if (tid == 0) {
     __threadfence();
     red_release_gpu_add(&a.bar[1], 1);
     if (!grid_wait(&a.bar[1], G, a.timeout_ns)) set_status(kStatusGridBarrierTimeout);
   }
-  __syncthreads();
-  if (warp == 0 && layer_mode && *((volatile int*)&cs.route_state) != 2) ensure_routing(a, cs, lane);
+  FMOE_TRACE(5);
   __syncthreads();
 
-  // Stage every slot's activation in its decode layout.
-  {
-    int vec_off = 0, sf_off = 0;
-    for (int s = 0; s < a.n_slots; ++s) {
-      const int bits = (s < a.K) ? a.bits_r : a.bits_s;
-      stage_vector(a.act + (long long)s * a.I, a.I, bits, reinterpret_cast<float4*>(sm.vec + vec_off),
-                   sm.sf + sf_off, tid, kThreads);
-      vec_off += a.I;
-      sf_off += a.I / 32;
-    }
+  // Stage the activations: the K routed experts (same width, back to back in
+  // the workspace) in one pass, then the shared expert.  Slot s's staged
+  // values start at sm.vec + s * I either way.
+  if (plan.nq > 0) {
+    if (a.K > 0) stage_inputs<BR, true>(a.act, a.K * a.I, reinterpret_cast<float4*>(sm.vec), sm.sf, tid, kThreads);
+    if (a.n_slots > a.K)
+      stage_inputs<BS, true>(a.act + (long long)a.K * a.I, a.I, reinterpret_cast<float4*>(sm.vec + a.K * a.I),
+                             sm.sf + a.K * a.I * BR / 128, tid, kThreads);
   }
+  FMOE_TRACE(6);
   __syncthreads();
 
-  // ---- Phase C: down projections + combine ----------------------------------
-  float accr[kRC];
-  for (int r = 0; r < kRC; ++r) accr[r] = 0.f;
+  // ---- Phase C: down projections of this CTA's rows, one (slot, kRC rows)
+  // item per re-carved stage; the row dots go to shared memory -----------------
   for (int i = n_gu; i < plan.n_loads; ++i) {
-    if (lane == 0) {
-      while (issued < plan.n_loads && issued < i + a.nst) {
-        fence_proxy_async_smem();
-        issue_load(a, plan, cs, issued, my_ring + (size_t)(issued % a.nst) * a.stage_bytes,
-                   &my_bars[issued % a.nst], GW);
-        ++issued;
-      }
-    }
-    issued = __shfl_sync(0xffffffffu, issued, 0);
-    const int st_i = i % a.nst;
-    const char* stage = my_ring + (size_t)st_i * a.stage_bytes;
-    if (!mbar_wait_bounded(&my_bars[st_i], (i / a.nst) & 1, a.timeout_ns) && lane == 0)
-      set_status(kStatusCopyTimeout);
     const int j = i - n_gu;
-    const int slot = j % a.n_slots;
-    const int bits = (slot < a.K) ? a.bits_r : a.bits_s;
-    const float coef = (slot < a.K) ? cs.w[slot] : cs.sg;
-    const float4* as = reinterpret_cast<const float4*>(sm.vec + slot * a.I);
-    const float2* sfa = sm.sf + slot * (a.I / 32);
-    if (bits == 4)
-      down_rows<4>(stage, a.I, as, sfa, lane, coef, accr);
+    if (lane == 0)
+      while (issued_c < plan.n_loads && issued_c < i + a.nst_c) {
+        issue_c(a, plan, cs, issued_c, warp, my_ring, my_bars_c, GW);
+        ++issued_c;
+      }
+    issued_c = __shfl_sync(0xffffffffu, issued_c, 0);
+    const char* stage = my_ring + (size_t)(j % a.nst_c) * a.c_stage_bytes;
+    if (!mbar_wait_bounded(&my_bars_c[j % a.nst_c], (j / a.nst_c) & 1, a.timeout_ns) && lane == 0)
+      set_status(kStatusCopyTimeout);
+    int slot, r0;
+    c_item(plan, i, warp, slot, r0);
+    const bool routed = slot < a.K;
+    const int cpv = 128 / (routed ? BR : BS);
+    // Routed slots share one staged [F4][K*I/CPV] array; the shared slot has
+    // its own [F4][I/CPV] array after it.
+    const float4* as = reinterpret_cast<const float4*>(sm.vec + (routed ? 0 : a.K * a.I));
+    const int nvs = routed ? a.K * a.I / cpv : a.I / cpv;
+    const int col0 = routed ? slot * (a.I / cpv) : 0;
+    const float2* sfa = sm.sf + (routed ? 0 : a.K * a.I * BR / 128) + col0;
+    float y[kRC];
+    if (BR == BS || routed)
+      down_rows<BR>(stage, a.I, as, nvs, col0, sfa, lane, y);
     else
-      down_rows<2>(stage, a.I, as, sfa, lane, coef, accr);
-    __syncwarp();
-    if (slot == a.n_slots - 1) {
-      const int unit = plan.c.first + (j / a.n_slots) * GW;
-      const int r0 = unit * kRC;
-      float tot[kRC];
+      down_rows<BS>(stage, a.I, as, nvs, col0, sfa, lane, y);
+    if (lane == 0) {
+      float* ys = sm.ys + slot * a.ys_stride + (r0 - plan.q0 * kRC);
 #pragma unroll
-      for (int r = 0; r < kRC; ++r) {
-        tot[r] = warp_sum(accr[r]);
-        accr[r] = 0.f;
-      }
-      if (lane == 0) {
-        float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (a.residual) res = __ldg(reinterpret_cast<const float4*>(a.residual + r0));
-        *reinterpret_cast<float4*>(a.out + r0) =
-            make_float4(res.x + tot[0], res.y + tot[1], res.z + tot[2], res.w + tot[3]);
-      }
+      for (int r = 0; r < kRC; ++r) ys[r] = y[r];
     }
+    __syncwarp();
+  }
+  FMOE_TRACE_WARP(7);
+  __syncthreads();
+
+  // ---- Combine: out = residual + sum_k w_k y_k + sg * y_shared, fixed order ---
+  for (int t = tid; t < plan.nq * kRC; t += kThreads) {
+    const int r = plan.q0 * kRC + t;
+    float v = a.residual ? __ldg(a.residual + r) : 0.f;
+    for (int s = 0; s < a.n_slots; ++s) v = fmaf(s < a.K ? cs.w[s] : cs.sg, sm.ys[s * a.ys_stride + t], v);
+    a.out[r] = v;
   }
 
   // ---- Done: the last CTA resets the hand-off counters for the next launch --
   __syncthreads();
+  FMOE_TRACE(8);
   if (tid == 0) {
     const unsigned t = atomicAdd(&a.bar[2], 1u);
     if (t + 1 == (unsigned)G) {

@@ -61,7 +61,7 @@ __global__ void topk_kernel(const float* __restrict__ logits, int T, int E, int 
   const int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (t >= T) return;
   const float* lt = logits + (long long)t * (E + 1);
-  warp_topk(lt, E, K, lane, idx + (long long)t * K, w + (long long)t * K);
+  warp_topk<false>(lt, E, K, lane, idx + (long long)t * K, w + (long long)t * K);
   if (lane == 0 && sgate) sgate[t] = has_sgate ? sigmoidf_(__ldcg(lt + E)) : 1.0f;
 }
 

@@ -181,6 +181,10 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
  * problem; bits are in *bits_out if non-NULL) or FMOE_ECUDA. */
 int fmoe_get_status(fmoe_stream_t stream, unsigned* bits_out);
 
+/* The cudaError_t value of the most recent CUDA call that made an entry point
+ * of this library return FMOE_ECUDA on the calling thread (0 if none). */
+int fmoe_last_cuda_error(void);
+
 /* Static, human-readable text for an error code. */
 const char* fmoe_strerror(int code);
 

@@ -25,6 +25,7 @@ EXPORTED = [
     "fmoe_expert_bytes", "fmoe_blob_offsets", "fmoe_quantize_expert", "fmoe_route_workspace_bytes",
     "fmoe_route", "fmoe_expert_workspace_bytes", "fmoe_expert_forward", "fmoe_workspace_bytes",
     "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status", "fmoe_strerror", "fmoe_last_cuda_error",
+    "fmoe_layer_decode_noalloc",
 ]
 
 
@@ -74,13 +75,14 @@ def lib() -> ctypes.CDLL:
     L.fmoe_workspace_bytes.restype = sz
     L.fmoe_workspace_init.argtypes = [vp, sz, vp]
     L.fmoe_layer_decode.argtypes = [ctypes.POINTER(FmoeLayerC), vp, vp, vp, i, vp, sz, vp, vp, vp]
+    L.fmoe_layer_decode_noalloc.argtypes = [ctypes.POINTER(FmoeLayerC), vp, vp, vp, i, vp, vp, vp]
     L.fmoe_get_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
     L.fmoe_last_cuda_error.argtypes = []
     L.fmoe_last_cuda_error.restype = i
     L.fmoe_strerror.argtypes = [i]
     L.fmoe_strerror.restype = ctypes.c_char_p
     for name in ("fmoe_blob_offsets", "fmoe_quantize_expert", "fmoe_route", "fmoe_expert_forward",
-                 "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status"):
+                 "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status", "fmoe_layer_decode_noalloc"):
         getattr(L, name).restype = i
     _lib = L
     return L
@@ -252,6 +254,21 @@ class Layer:
                                        ws.data_ptr(), ws.numel(), _ptr(idx_out), _ptr(w_out), _stream(stream)),
                "fmoe_layer_decode")
         return out
+
+
+def layer_decode_noalloc(layer: "Layer", x: torch.Tensor, residual: torch.Tensor | None = None,
+                         out: torch.Tensor | None = None, idx_out: torch.Tensor | None = None,
+                         w_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Layer.decode without a workspace argument: the library's fixed device
+    scratch is used instead (see fmoe_layer_decode_noalloc in include/fmoe.h)."""
+    _dev_tensor(x, torch.float32, "x")
+    x2 = x.view(-1, layer.hidden)
+    if out is None:
+        out = torch.empty_like(x2)
+    _check(lib().fmoe_layer_decode_noalloc(ctypes.byref(layer.c), x2.data_ptr(), _ptr(residual), out.data_ptr(),
+                                           x2.shape[0], _ptr(idx_out), _ptr(w_out), _stream(stream)),
+           "fmoe_layer_decode_noalloc")
+    return out
 
 
 def get_status(stream=None) -> int:

@@ -160,6 +160,28 @@ int launch_layer(const LayerArgs& args, const Plan& pl, DevInfo* info, cudaStrea
   return e == cudaSuccess ? FMOE_OK : cuda_fail(e);
 }
 
+// Fixed scratch for fmoe_layer_decode_noalloc: callers that cannot allocate
+// device memory themselves get the decode's workspace from this file-scope
+// array, which every GPU that loads the library keeps until the process exits.
+constexpr size_t kNoallocScratchBytes = 32 << 10;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+// Device address of g_noalloc_scratch per device, looked up once per device
+// (host code only sees a stand-in for the symbol, never its device address).
+void* g_noalloc_ptr[64];
+std::mutex g_noalloc_mu;
+
+int noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch)) return cuda_fail(e);
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FMOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -364,6 +386,24 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
     if (int rc = launch_layer(a, pl, info, s)) return rc;
   }
   return FMOE_OK;
+}
+
+int fmoe_layer_decode_noalloc(const fmoe_layer* L, const float* x, const float* residual, float* out, int T,
+                              int32_t* idx_out_opt, float* w_out_opt, fmoe_stream_t stream) {
+  if (!L) return FMOE_EINVAL;
+  const size_t need = fmoe_workspace_bytes(L, T);
+  if (need == 0) return FMOE_EINVAL;
+  if (need > kNoallocScratchBytes) return FMOE_ENOMEM;  // layer too large for the fixed scratch
+  int dev = 0;
+  if (cudaError_t e = cudaGetDevice(&dev)) return cuda_fail(e);
+  if (dev < 0 || dev >= 64) return FMOE_EINVAL;
+  void* ws = nullptr;
+  if (int rc = noalloc_scratch(dev, &ws)) return rc;
+  // The scratch keeps whatever the previous call left; the hand-off counters
+  // must start at zero, so clear them (the rest is written before it is read).
+  if (cudaError_t e = cudaMemsetAsync(ws, 0, kCounterBytes, reinterpret_cast<cudaStream_t>(stream)))
+    return cuda_fail(e);
+  return fmoe_layer_decode(L, x, residual, out, T, ws, kNoallocScratchBytes, idx_out_opt, w_out_opt, stream);
 }
 
 int fmoe_get_status(fmoe_stream_t stream, unsigned* bits_out) {

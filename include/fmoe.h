@@ -176,6 +176,28 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
                       void* ws, size_t ws_bytes, int32_t* idx_out_opt, float* w_out_opt,
                       fmoe_stream_t stream);
 
+/* fmoe_layer_decode without a caller-provided workspace, for callers that
+ * cannot allocate device memory: code that runs where an allocator must not be
+ * called (inside another library's fixed memory budget, or a host runtime that
+ * hands over only the input and output buffers), or plain C callers with no
+ * device allocator of their own.  The Flash-MoE pages have no counterpart:
+ * this is an interface convenience of this library.
+ *   Arguments, outputs and errors are those of fmoe_layer_decode, minus the
+ *   workspace.  The workspace comes from one fixed 32 KiB array in device
+ *   memory that every GPU which loads the library keeps until the process
+ *   exits; a layer whose fmoe_workspace_bytes() exceeds 32 KiB is rejected
+ *   with FMOE_ENOMEM (the full-size layer of the pages, 512 experts, top-4,
+ *   intermediate 1024, needs about 23 KiB).
+ *   The first call on a device looks the array's device address up (a
+ *   synchronous runtime query); make that first call before capturing a
+ *   stream into a graph.  Every call clears the array's hand-off counters on
+ *   `stream` before the layer kernel runs.
+ *   All calls on a device share the one array: calls that may overlap on the
+ *   GPU (different streams without ordering between them) race and give wrong
+ *   results.  Nothing is allocated or freed by this call. */
+int fmoe_layer_decode_noalloc(const fmoe_layer* L, const float* x, const float* residual, float* out, int T,
+                              int32_t* idx_out_opt, float* w_out_opt, fmoe_stream_t stream);
+
 /* Synchronise `stream`, then read and clear the device status word of the
  * current device.  Returns FMOE_OK, FMOE_EDEVICE (a kernel reported a
  * problem; bits are in *bits_out if non-NULL) or FMOE_ECUDA. */

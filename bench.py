@@ -8,19 +8,21 @@ combine) with the weights resident in HBM.  The default workload is the
 full-size 4-bit layer: hidden 4096, expert intermediate 1024, 512 experts,
 group 64 (3.6 GB of experts per layer, 39.6 MB read per decode).
 
-Timing: W untimed warm-up steps; then K steps, each a replay of the decode call
-captured once in a CUDA graph (so host launch latency is not timed; the
-end-to-end figure keeps it), bracketed by CUDA events on the launching stream,
-with L2 flushed before every step (a 256 MiB write
-outside the event pair) so that the router and shared expert are re-read from
-HBM each time; tokens rotate through a pool of 64 pre-drawn inputs so the
-routed experts change every step.  A barrier and a device synchronise bracket
-the timed region; the value is the total over all ranks divided by the
-slowest rank's time.  With --gpus N > 1 (torchrun) every rank decodes its own
-replica of the layer: the path has no data-path exchange.
+Timing: W untimed warm-up steps; then K steps timed with CUDA events on the
+launching stream, bracketed by a barrier and a device synchronise.  Step j
+decodes token j mod 64 of a pre-drawn pool through layer instance j mod L
+(L = 16 distinct full-size layers, 58 GB of experts): the weights a step reads
+are never L2-resident (inputs larger than L2, no flush between steps).  The
+steps are the library's decode call captured in CUDA graphs of 64 steps, so
+the timed region is device time plus the gaps between back-to-back kernels,
+not Python launch latency (the end-to-end figure keeps that).  The value is
+the total over all ranks divided by the slowest rank's time.  With --gpus
+N > 1 (torchrun) every rank decodes its own replicas: the path has no
+data-path exchange.
 
-The JSON line also carries: the roofline of the layer kernel (algorithmic bytes
-per launch / measured launch time vs the measured HBM copy bandwidth), an
+The JSON line also carries: the latency of one isolated step after a 256 MiB
+L2 flush; the roofline of the layer kernel (algorithmic bytes per launch /
+measured time per launch vs the measured HBM copy bandwidth); an
 end-to-end figure through the same C-ABI call with host buffers (pinned host
 -> device copy of x and residual, decode, device -> host copy of out inside
 the event pair), the SM clocks sampled during the timed region, and the CPU
@@ -235,83 +237,114 @@ def run_fmoe(args, cfg, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     h, i, e, k = cfg["hidden"], cfg["inter"], cfg["experts"], cfg["top_k"]
-    t = SG.make_layer(SEED + rank, 0, h, i, e, cfg["bits"], cfg["shared_bits"], F.blob_offsets, F.expert_bytes,
-                      dev)
-    L = F.Layer(t["w_router"], t["w_sgate"], t["experts"], t["shared"], h, i, k, cfg["bits"],
-                cfg["shared_bits"])
+    NL = args.layers
+    # NL distinct layer instances of the workload, decoded in turn: the weights
+    # a step reads were last touched NL - 1 steps earlier, so they come from
+    # HBM (NL * 40 MB >> 126 MB of L2) without any flush between steps.
+    layers = []
+    for l in range(NL):
+        t = SG.make_layer(SEED + 1000 * rank, l, h, i, e, cfg["bits"], cfg["shared_bits"], F.blob_offsets,
+                          F.expert_bytes, dev)
+        layers.append(F.Layer(t["w_router"], t["w_sgate"], t["experts"], t["shared"], h, i, k, cfg["bits"],
+                              cfg["shared_bits"]))
     xs = torch.from_numpy(S.token_x(SEED + rank, 0, 0, POOL, h)).to(dev)
     rs = torch.from_numpy(S.token_residual(SEED + rank, 0, 0, POOL, h)).to(dev)
     out = torch.empty(POOL, h, dtype=torch.float32, device=dev)
-    ws = L.workspace(1)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ws = [L.workspace(1) for L in layers]
     stream = torch.cuda.current_stream()
 
-    # Each pool entry's decode is one library call captured once into a CUDA
-    # graph, so that a timed step is the device work of the call and not the
-    # Python/ctypes launch latency (the end-to-end figure below keeps that).
+    def decode(j):
+        l = j % NL
+        layers[l].decode(xs[j % POOL], rs[j % POOL], out=out[j % POOL], ws=ws[l])
+
     for j in range(args.warmup):
-        flush.fill_(j & 0xFF)
-        L.decode(xs[j % POOL], rs[j % POOL], out=out[j % POOL], ws=ws)
+        decode(j)
     torch.cuda.synchronize()
     if F.get_status():
         raise RuntimeError("device status word set during warm-up")
-    graphs = []
-    for j in range(POOL):
+
+    # Each captured step is the library's decode call; a graph holds GSTEPS
+    # consecutive steps so that the timed region is device time, without the
+    # Python/ctypes launch latency (the end-to-end figure below keeps that).
+    GSTEPS = 64
+    K = args.steps
+
+    def capture(first, n):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            L.decode(xs[j], rs[j], out=out[j], ws=ws)
-        graphs.append(g)
-    torch.cuda.synchronize()
-    for j in range(min(args.warmup, POOL)):
-        flush.fill_(j & 0xFF)
-        graphs[j].replay()
+            for j in range(first, first + n):
+                decode(j)
+        return g
+
+    g_full = capture(0, GSTEPS)
+    rem = K % GSTEPS
+    g_rem = capture(0, rem) if rem else None
+    g_full.replay()
     torch.cuda.synchronize()
 
-    def step(j):
-        graphs[j % POOL].replay()
-
-    K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     clocks = ClockSampler(local_rank)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.1)
-    for j in range(K):
-        flush.fill_((j + 1) & 0xFF)
-        ev[j][0].record(stream)
-        step(j)
-        ev[j][1].record(stream)
+    ev0.record(stream)
+    for _ in range(K // GSTEPS):
+        g_full.replay()
+    if g_rem is not None:
+        g_rem.replay()
+    ev1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    times_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = float(sum(times_ms))
+    total_ms = ev0.elapsed_time(ev1)
     status = F.get_status()
 
-    # end to end through the same call with host buffers
+    # Latency of one isolated step with L2 flushed before it (single launch,
+    # so it also carries the launch and event overheads of a lone kernel).
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    g_one = [capture(j, 1) for j in range(min(NL, 8))]
+    lat = []
+    for j in range(min(K, 400)):
+        flush.fill_(j & 0xFF)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        g_one[j % len(g_one)].replay()
+        a1.record(stream)
+        lat.append((a0, a1))
+    torch.cuda.synchronize()
+    lat_us = [1000.0 * a.elapsed_time(b) for a, b in lat]
+    del flush
+
+    # End to end through the same call with host buffers: pinned host -> device
+    # copy of x and residual, decode, device -> host copy of out, every step.
     xh = torch.from_numpy(S.token_x(SEED + rank, 0, 1, POOL, h)).pin_memory()
     rh = torch.from_numpy(S.token_residual(SEED + rank, 0, 1, POOL, h)).pin_memory()
     oh = torch.empty(POOL, h, dtype=torch.float32).pin_memory()
     xd = torch.empty(h, dtype=torch.float32, device=dev)
     rd = torch.empty(h, dtype=torch.float32, device=dev)
     od = torch.empty(h, dtype=torch.float32, device=dev)
-    K2 = min(K, 1000)
-    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K2)]
-    for j in range(K2 + 3):
-        flush.fill_(j & 0xFF)
-        if j >= 3:
-            ev2[j - 3][0].record(stream)
+    K2 = min(K, 2000)
+
+    def e2e_step(j):
+        l = j % NL
         xd.copy_(xh[j % POOL], non_blocking=True)
         rd.copy_(rh[j % POOL], non_blocking=True)
-        L.decode(xd, rd, out=od, ws=ws)
+        layers[l].decode(xd, rd, out=od, ws=ws[l])
         oh[j % POOL].copy_(od, non_blocking=True)
-        if j >= 3:
-            ev2[j - 3][1].record(stream)
+
+    for j in range(3):
+        e2e_step(j)
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in ev2)
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0.record(stream)
+    for j in range(K2):
+        e2e_step(j)
+    b1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = b0.elapsed_time(b1)
 
     # max over ranks
     tt = torch.tensor([total_ms, e2e_ms / K2 * K], dtype=torch.float64, device=dev)
@@ -329,15 +362,20 @@ def run_fmoe(args, cfg, rank, world, local_rank):
             "impl": "fmoe", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": total_ms_max / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u4/bf16 weights, f32 compute", "data": "synthetic",
-            "config": {**cfg, "batch": 1, "group": 64, "l2": "flushed before every timed step (256 MiB write)",
-                       "input_pool": POOL, "parallelism": f"replicas x{world}"},
+            "config": {**cfg, "batch": 1, "group": 64,
+                       "l2": f"inputs larger than L2: {NL} distinct layer instances decoded in turn "
+                             f"({NL * e * expert_bytes(h, i, cfg['bits']) / 1e9:.0f} GB of experts), no flush",
+                       "layers_in_rotation": NL, "input_pool": POOL, "parallelism": f"replicas x{world}"},
             "us_per_decode": 1000.0 * total_ms_max / K,
-            "p50_us": 1000.0 * statistics.median(times_ms), "p99_us": 1000.0 * float(np.percentile(times_ms, 99)),
+            "latency_us_l2_flushed": {"p50": statistics.median(lat_us), "p99": float(np.percentile(lat_us, 99)),
+                                      "steps": len(lat_us),
+                                      "note": "one isolated graph launch after a 256 MiB L2 flush"},
             "expert_gbs": ab["experts"] / avg_launch_s / 1e9,
             "expert_frac_of_hbm": ab["experts"] / avg_launch_s / 1e9 / peak,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": profiled_traffic(args.config),
-                         "kernel": "layer_kernel", "algorithmic_bytes_per_launch": ab["total"]},
+                         "kernel": f"layer_kernel<{cfg['bits']},{cfg['shared_bits']}>",
+                         "algorithmic_bytes_per_launch": ab["total"]},
             "e2e": {"value": world * K / (e2e_ms_max / 1000.0), "unit": UNIT, "h2d_bytes_per_step": 2 * h * 4,
                     "d2h_bytes_per_step": h * 4},
             "gpu_launches": K,
@@ -354,7 +392,8 @@ def run_fmoe(args, cfg, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--layers", type=int, default=16, help="distinct layer instances decoded in turn")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["fmoe", "reference"], default="fmoe")
     ap.add_argument("--config", choices=sorted(CONFIGS), default="full4")

@@ -167,6 +167,7 @@ struct CtaShared {
   float* lg;            // shared-memory copy of the router logits
   unsigned lg_bytes;
   int route_state;      // 0 = not started, 1 = being computed, 2 = ready
+  int c_prefetch;          // warps past their gate/up work (the first prefetches down rows)
   unsigned router_done;    // this CTA's router rows published so far
   unsigned router_target;  // this CTA's router rows
   int idx[kMaxTopK];
@@ -529,16 +530,6 @@ __device__ __noinline__ void ensure_routing(const LayerArgs& a, CtaShared& cs, c
     }
     FMOE_TRACE_WARP(3);
     __syncwarp();
-    // L2 prefetch of this CTA's routed down rows, one lane per routed slot.
-    if (lane < a.K && plan.nq > 0) {
-      const SlotInfo si = slot_info(a, cs, lane);
-      const BlobOff o = blob_offsets(a.H, a.I, si.bits);
-      const int cb = codes_row_bytes(a.I, si.bits), sbr = sb_row_bytes(a.I);
-      const long long r0 = (long long)plan.q0 * kRC, nr = (long long)plan.nq * kRC;
-      bulk_prefetch_l2(si.blob + o.dc + r0 * cb, (uint32_t)(nr * cb));
-      bulk_prefetch_l2(si.blob + o.dsb + r0 * sbr, (uint32_t)(nr * sbr));
-    }
-    __syncwarp();
   } else {
     if (!mbar_wait_bounded(&cs.route_bar, 0, a.timeout_ns) && lane == 0) set_status(kStatusCtaWaitTimeout);
     __syncwarp();
@@ -585,6 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     cs.route_state = layer_mode ? 0 : 2;
     cs.sg = 1.0f;
     cs.router_done = 0;
+    cs.c_prefetch = 0;
     cs.router_target = n_router_warps;  // n_router < G * kWarps: one row per router warp
     fence_proxy_async_smem();
     mbar_arrive_expect_tx(&cs.x_bar, a.H * 4);
@@ -595,28 +587,14 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     for (int s = 0; s < a.nst + kMaxNstC; ++s) mbar_init(&my_bars[s], 1);
     fence_proxy_async_smem();
   }
-  if (warp == kWarps - 1 && lane == 0 && a.shared && plan.nq > 0) {
-    // the shared expert's down rows of this CTA are known from the start
-    const BlobOff o = blob_offsets(a.H, a.I, a.bits_s);
-    const int cb = codes_row_bytes(a.I, a.bits_s), sbr = sb_row_bytes(a.I);
-    const long long r0 = (long long)plan.q0 * kRC, nr = (long long)plan.nq * kRC;
-    bulk_prefetch_l2(a.shared + o.dc + r0 * cb, (uint32_t)(nr * cb));
-    bulk_prefetch_l2(a.shared + o.dsb + r0 * sbr, (uint32_t)(nr * sbr));
-  }
   __syncthreads();
   FMOE_TRACE(11);
   if (tid == 0 && layer_mode && cs.router_target == 0) red_release_gpu_add(&a.bar[0], 1);
 
-  // Prologue: start the first ring loads that need no routing decision.
+  // x and the router rows are the critical path to the routing decision, so
+  // they are the only traffic of the first microseconds; the shared expert's
+  // gate/up rows follow once x is staged.
   int issued = 0;
-  if (lane == 0) {
-    while (issued < plan.a.count && issued < a.nst) {
-      issue_load(a, plan, cs, issued, warp, my_ring + (size_t)issued * a.stage_bytes, &my_bars[issued], GW);
-      ++issued;
-    }
-  }
-  issued = __shfl_sync(0xffffffffu, issued, 0);
-
   if (!mbar_wait_bounded(&cs.x_bar, 0, a.timeout_ns) && lane == 0) set_status(kStatusCopyTimeout);
   const float* xu = sm.vec + a.xu_off;
   if (router_warp) {
@@ -641,7 +619,23 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
                              sm.sf + (a.xs4_off >= 0 ? a.H / 32 : 0), t0, nt);
     __syncwarp();
     if (lane == 0) mbar_arrive(&cs.staged_bar);
+    if (warp == kWarps - 1 && lane == 0 && a.shared && plan.nq > 0) {
+      // the shared expert's down rows of this CTA are known from the start
+      const BlobOff o = blob_offsets(a.H, a.I, BS);
+      const int cb = codes_row_bytes(a.I, BS), sbr = sb_row_bytes(a.I);
+      const long long r0 = (long long)plan.q0 * kRC, nr = (long long)plan.nq * kRC;
+      bulk_prefetch_l2(a.shared + o.dc + r0 * cb, (uint32_t)(nr * cb));
+      bulk_prefetch_l2(a.shared + o.dsb + r0 * sbr, (uint32_t)(nr * sbr));
+    }
   }
+  // The shared expert's gate/up loads (no routing decision needed).
+  if (lane == 0) {
+    while (issued < plan.a.count && issued < a.nst) {
+      issue_load(a, plan, cs, issued, warp, my_ring + (size_t)issued * a.stage_bytes, &my_bars[issued], GW);
+      ++issued;
+    }
+  }
+  issued = __shfl_sync(0xffffffffu, issued, 0);
   if (!mbar_wait_bounded(&cs.staged_bar, 0, a.timeout_ns) && lane == 0) set_status(kStatusCtaWaitTimeout);
   FMOE_TRACE(1);
 
@@ -705,6 +699,21 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   if (layer_mode && !have_routing && (plan.n_loads > n_gu || (blockIdx.x == 0 && warp == 0))) {
     ensure_routing(a, cs, plan, lane);
     have_routing = true;
+  }
+  // The CTA's first warp through its gate/up work asks L2 for the routed
+  // experts' down rows of this CTA (one lane per routed slot): late enough not
+  // to compete with the gate/up stream, early enough to land before phase C.
+  if (layer_mode && plan.nq > 0) {
+    int first = 0;
+    if (lane == 0) first = atomicAdd(&cs.c_prefetch, 1) == 0;
+    if (__shfl_sync(0xffffffffu, first, 0) && lane < a.K) {
+      const SlotInfo si = slot_info(a, cs, lane);
+      const BlobOff o = blob_offsets(a.H, a.I, BR);
+      const int cb = codes_row_bytes(a.I, BR), sbr = sb_row_bytes(a.I);
+      const long long r0 = (long long)plan.q0 * kRC, nr = (long long)plan.nq * kRC;
+      bulk_prefetch_l2(si.blob + o.dc + r0 * cb, (uint32_t)(nr * cb));
+      bulk_prefetch_l2(si.blob + o.dsb + r0 * sbr, (uint32_t)(nr * sbr));
+    }
   }
   int issued_c = n_gu;
   if (lane == 0)

@@ -105,47 +105,59 @@ template <int BITS, bool kGlobal>
 __device__ inline void stage_inputs(const float* __restrict__ src, int n, float4* xs, float2* sf, int tid,
                                     int nthreads) {
   constexpr int CPV = 128 / BITS, CPW = 32 / BITS, F4 = CPV / 4;
+  constexpr int kBatch = 4;  // passes whose loads are all issued before any is used
   const int NV = n / CPV, total = NV * F4;
   const int lane = tid & 31;
-  for (int base = tid - lane; base < total; base += nthreads) {
-    const int q = base + lane;
-    const bool on = q < total;
-    const int v = q / F4, j = q % F4;
-    float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (on) val = kGlobal ? __ldcg(reinterpret_cast<const float4*>(src) + q) : reinterpret_cast<const float4*>(src)[q];
-    float mx = fmaxf(fmaxf(fabsf(val.x), fabsf(val.y)), fmaxf(fabsf(val.z), fabsf(val.w)));
-    float sum = (val.x + val.y) + (val.z + val.w);
+  for (int base0 = tid - lane; base0 < total; base0 += kBatch * nthreads) {
+    float4 val[kBatch];
 #pragma unroll
-    for (int o = 1; o < F4; o <<= 1) {
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    for (int b = 0; b < kBatch; ++b) {
+      const int q = base0 + b * nthreads + lane;
+      val[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (q < total)
+        val[b] = kGlobal ? __ldcg(reinterpret_cast<const float4*>(src) + q) : reinterpret_cast<const float4*>(src)[q];
     }
-    // max|x| * 2^S < 2^125; S in [22, 249] keeps 2^(149 - S) and 2^(S - p) finite.
-    int S = 109;
-    if (mx > 0.f) {
-      int e;
-      frexpf(mx, &e);  // mx < 2^e
-      S = 125 - e;
-      S = S < 22 ? 22 : (S > 249 ? 249 : S);
-    }
-    const float* in = &val.x;
-    float4 o;
-    float* out = &o.x;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      int e = S - code_bitpos_t<BITS>((4 * j + c) % CPW);  // in [0, 249]
-      float t = in[c];
-      if (e > 126) {
-        t *= pow2f(126);
-        e -= 126;
+    for (int b = 0; b < kBatch; ++b) {
+      const int base = base0 + b * nthreads;
+      if (base >= total) break;  // warp-uniform
+      const int q = base + lane;
+      const bool on = q < total;
+      const int v = q / F4, j = q % F4;
+      float mx = fmaxf(fmaxf(fabsf(val[b].x), fabsf(val[b].y)), fmaxf(fabsf(val[b].z), fabsf(val[b].w)));
+      float sum = (val[b].x + val[b].y) + (val[b].z + val[b].w);
+#pragma unroll
+      for (int o = 1; o < F4; o <<= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        sum += __shfl_xor_sync(0xffffffffu, sum, o);
       }
-      out[c] = t * pow2f(e);
-    }
-    if (on) {
-      xs[j * NV + v] = o;
-      if (j == 0) {
-        const int fe = 149 - S;  // in [-100, 127]
-        sf[v] = make_float2(sum, pow2f(fe));
+      // max|x| * 2^S < 2^125; S in [22, 249] keeps 2^(149 - S) and 2^(S - p) finite.
+      int S = 109;
+      if (mx > 0.f) {
+        int e;
+        frexpf(mx, &e);  // mx < 2^e
+        S = 125 - e;
+        S = S < 22 ? 22 : (S > 249 ? 249 : S);
+      }
+      const float* in = &val[b].x;
+      float4 o;
+      float* out = &o.x;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        int e = S - code_bitpos_t<BITS>((4 * j + c) % CPW);  // in [0, 249]
+        float t = in[c];
+        if (e > 126) {
+          t *= pow2f(126);
+          e -= 126;
+        }
+        out[c] = t * pow2f(e);
+      }
+      if (on) {
+        xs[j * NV + v] = o;
+        if (j == 0) {
+          const int fe = 149 - S;  // in [-100, 127]
+          sf[v] = make_float2(sum, pow2f(fe));
+        }
       }
     }
   }

@@ -138,12 +138,22 @@ size_t layer_ws_bytes(int E, int I, int K) {
   return kCounterBytes + round_up((size_t)(E + 1) * 4, 256) + round_up((size_t)(K + 1) * I * 4, 256);
 }
 
-// Fill the grid-shape-dependent fields of the kernel arguments.
+// Fill the grid-shape-dependent fields and the blob section offsets.
 void set_offsets(LayerArgs& a, int G) {
   const int GW = G * kWarps;
   const int n_static = a.shared ? a.I : 0;
   a.off_a = a.n_router % GW;
   a.off_b = (int)(((long long)a.n_router + n_static) % GW);
+  for (int r = 0; r < 2; ++r) {
+    const BlobOff o = blob_offsets(a.H, a.I, r == 0 ? a.bits_r : a.bits_s);
+    long long* d = r == 0 ? a.off_r : a.off_s;
+    d[0] = o.gc;
+    d[1] = o.gsb;
+    d[2] = o.uc;
+    d[3] = o.usb;
+    d[4] = o.dc;
+    d[5] = o.dsb;
+  }
 }
 
 int launch_layer(const LayerArgs& args, const Plan& pl, DevInfo* info, cudaStream_t s) {

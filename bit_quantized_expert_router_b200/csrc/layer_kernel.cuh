@@ -87,6 +87,7 @@ struct LayerArgs {
   int vec_floats, sf_floats;
   int ys_stride;             // rows per CTA (max) in the phase-C result array
   int lg_floats;             // shared-memory logits (n_router rounded up to 4)
+  long long off_r[6], off_s[6];  // blob section offsets for the routed / shared code width
   unsigned long long timeout_ns;
 };
 
@@ -173,6 +174,7 @@ struct CtaShared {
   int idx[kMaxTopK];
   float w[kMaxTopK];
   float sg;
+  const char* blob[kMaxSlots];  // blob of each slot (routed ones once the routing is known)
 };
 
 __device__ __forceinline__ float* cs_logits(const LayerArgs&, CtaShared& cs) { return cs.lg; }
@@ -184,13 +186,8 @@ struct SlotInfo {
 
 __device__ __forceinline__ SlotInfo slot_info(const LayerArgs& a, const CtaShared& cs, int slot) {
   SlotInfo si;
-  if (slot < a.K) {
-    si.blob = a.experts + (long long)cs.idx[slot] * a.expert_stride;
-    si.bits = a.bits_r;
-  } else {
-    si.blob = a.shared;
-    si.bits = a.bits_s;
-  }
+  si.blob = cs.blob[slot];
+  si.bits = slot < a.K ? a.bits_r : a.bits_s;
   return si;
 }
 
@@ -222,35 +219,35 @@ __device__ __forceinline__ void c_item(const WarpPlan& p, int i, int warp, int& 
 // Issue the bulk copies of ring load `i` (lane 0 only).
 //   gate/up stage: gate codes | up codes | gate sb superset | up sb superset
 //   down stage:    kRC code rows | kRC sb rows
-__device__ __noinline__ void issue_load(const LayerArgs& a, const WarpPlan& p, const CtaShared& cs, int i,
+__device__ __forceinline__ void issue_load(const LayerArgs& a, const WarpPlan& p, const CtaShared& cs, int i,
                                            int warp, char* stage, uint64_t* bar, int GW) {
   if (i < p.a.count + p.b.count) {
     int slot, row;
     gu_unit(a, p, i, GW, slot, row);
-    const SlotInfo si = slot_info(a, cs, slot);
-    const BlobOff o = blob_offsets(a.H, a.I, si.bits);
-    const int cb = codes_row_bytes(a.H, si.bits);
+    const char* blob = cs.blob[slot];
+    const long long* o = slot < a.K ? a.off_r : a.off_s;
+    const int cb = codes_row_bytes(a.H, slot < a.K ? a.bits_r : a.bits_s);
     const int sbr = sb_row_bytes(a.H);
     const int cap = sb_superset_cap(a.H);
-    const long long gs0 = o.gsb + (long long)row * sbr, us0 = o.usb + (long long)row * sbr;
+    const long long gs0 = o[1] + (long long)row * sbr, us0 = o[3] + (long long)row * sbr;
     const long long ga = gs0 & ~15LL, ua = us0 & ~15LL;
     const int glen = (int)(((gs0 + sbr + 15) & ~15LL) - ga);
     const int ulen = (int)(((us0 + sbr + 15) & ~15LL) - ua);
     mbar_arrive_expect_tx(bar, 2 * cb + glen + ulen);
-    bulk_g2s(stage, si.blob + o.gc + (long long)row * cb, cb, bar);
-    bulk_g2s(stage + cb, si.blob + o.uc + (long long)row * cb, cb, bar);
-    bulk_g2s(stage + 2 * cb, si.blob + ga, glen, bar);
-    bulk_g2s(stage + 2 * cb + cap, si.blob + ua, ulen, bar);
+    bulk_g2s(stage, blob + o[0] + (long long)row * cb, cb, bar);
+    bulk_g2s(stage + cb, blob + o[2] + (long long)row * cb, cb, bar);
+    bulk_g2s(stage + 2 * cb, blob + ga, glen, bar);
+    bulk_g2s(stage + 2 * cb + cap, blob + ua, ulen, bar);
   } else {
     int slot, r0;
     c_item(p, i, warp, slot, r0);
-    const SlotInfo si = slot_info(a, cs, slot);
-    const BlobOff o = blob_offsets(a.H, a.I, si.bits);
-    const int cb = codes_row_bytes(a.I, si.bits);
+    const char* blob = cs.blob[slot];
+    const long long* o = slot < a.K ? a.off_r : a.off_s;
+    const int cb = codes_row_bytes(a.I, slot < a.K ? a.bits_r : a.bits_s);
     const int sbr = sb_row_bytes(a.I);
     mbar_arrive_expect_tx(bar, kRC * (cb + sbr));
-    bulk_g2s(stage, si.blob + o.dc + (long long)r0 * cb, kRC * cb, bar);
-    bulk_g2s(stage + kRC * cb, si.blob + o.dsb + (long long)r0 * sbr, kRC * sbr, bar);
+    bulk_g2s(stage, blob + o[4] + (long long)r0 * cb, kRC * cb, bar);
+    bulk_g2s(stage + kRC * cb, blob + o[5] + (long long)r0 * sbr, kRC * sbr, bar);
   }
 }
 
@@ -515,8 +512,10 @@ __device__ __noinline__ void ensure_routing(const LayerArgs& a, CtaShared& cs, c
     FMOE_TRACE_WARP(10);
     if (lane == 0) {
       // Guard the expert index even on a timed-out (garbage) path.
-      for (int k = 0; k < a.K; ++k)
+      for (int k = 0; k < a.K; ++k) {
         if (cs.idx[k] < 0 || cs.idx[k] >= a.E) cs.idx[k] = 0;
+        cs.blob[k] = a.experts + (long long)cs.idx[k] * a.expert_stride;
+      }
       cs.sg = a.w_sgate ? sigmoidf_(lsg) : 1.0f;
       if (blockIdx.x == 0) {
         for (int k = 0; k < a.K; ++k) {
@@ -577,6 +576,10 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     cs.sg = 1.0f;
     cs.router_done = 0;
     cs.c_prefetch = 0;
+    // The shared (or single) expert; the routed slots point at expert 0 until
+    // the routing decision replaces them (never read before that).
+    for (int k = 0; k < a.K; ++k) cs.blob[k] = a.experts;
+    cs.blob[a.K] = a.shared;
     cs.router_target = n_router_warps;  // n_router < G * kWarps: one row per router warp
     fence_proxy_async_smem();
     mbar_arrive_expect_tx(&cs.x_bar, a.H * 4);
@@ -703,7 +706,9 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   // The CTA's first warp through its gate/up work asks L2 for the routed
   // experts' down rows of this CTA (one lane per routed slot): late enough not
   // to compete with the gate/up stream, early enough to land before phase C.
-  if (layer_mode && plan.nq > 0) {
+  // Only warps that hold the routing decision take part: the routed slots'
+  // blob pointers are set by it.
+  if (layer_mode && have_routing && plan.nq > 0) {
     int first = 0;
     if (lane == 0) first = atomicAdd(&cs.c_prefetch, 1) == 0;
     if (__shfl_sync(0xffffffffu, first, 0) && lane < a.K) {
@@ -759,6 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     const char* stage = my_ring + (size_t)(j % a.nst_c) * a.c_stage_bytes;
     if (!mbar_wait_bounded(&my_bars_c[j % a.nst_c], (j / a.nst_c) & 1, a.timeout_ns) && lane == 0)
       set_status(kStatusCopyTimeout);
+    if (j == 0) FMOE_TRACE_WARP(15);
     int slot, r0;
     c_item(plan, i, warp, slot, r0);
     const bool routed = slot < a.K;
@@ -774,6 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
       down_rows<BR>(stage, a.I, as, nvs, col0, sfa, lane, y);
     else
       down_rows<BS>(stage, a.I, as, nvs, col0, sfa, lane, y);
+    if (j == 0) FMOE_TRACE_WARP(12);
     if (lane == 0) {
       float* ys = sm.ys + slot * a.ys_stride + (r0 - plan.q0 * kRC);
 #pragma unroll

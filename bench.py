@@ -53,6 +53,13 @@ CONFIGS = {
                   experts=512, top_k=4, bits=2, shared_bits=4),
     "tiny": dict(workload="tiny_h512_i128_e16_k4_shared_4bit", hidden=512, inter=128, experts=16, top_k=4,
                  bits=4, shared_bits=4),
+    # 40 independent full-size 4-bit layers (145.6 GB of experts); a step is one
+    # token decoded through all 40 layers.
+    "stacked": dict(workload="stacked_40x_full_h4096_i1024_e512_k4_shared_4bit", hidden=4096, inter=1024,
+                    experts=512, top_k=4, bits=4, shared_bits=4, layers_per_step=40),
+    # 16 tokens per step through the full-size 4-bit layer, grouped by expert.
+    "batch16": dict(workload="batch16_full_h4096_i1024_e512_k4_shared_4bit", hidden=4096, inter=1024,
+                    experts=512, top_k=4, bits=4, shared_bits=4, tokens=16),
 }
 METRIC = "MoE layer decodes/s (batch 1)"
 UNIT = "decodes/s"
@@ -65,12 +72,18 @@ def expert_bytes(h, i, b):
     return 3 * h * i * b // 8 + 3 * h * i // 64 * 4
 
 
-def algorithmic_bytes(cfg) -> dict:
-    """Bytes one decode must read or write at least (each weight once)."""
+def algorithmic_bytes(cfg, distinct_routed: float | None = None) -> dict:
+    """Bytes one decode step must read or write at least (each weight once).
+
+    With several tokens per step, the routed experts are counted once per
+    distinct expert the step selects (`distinct_routed`, measured).
+    """
     h, i, e, k = cfg["hidden"], cfg["inter"], cfg["experts"], cfg["top_k"]
-    experts = k * expert_bytes(h, i, cfg["bits"]) + expert_bytes(h, i, cfg["shared_bits"])
+    tt = cfg.get("tokens", 1)
+    n_routed = k if distinct_routed is None else distinct_routed
+    experts = n_routed * expert_bytes(h, i, cfg["bits"]) + expert_bytes(h, i, cfg["shared_bits"])
     router = e * h * 2 + h * 2
-    vectors = 3 * h * 4  # x, residual in; out
+    vectors = 3 * tt * h * 4  # x, residual in; out
     return dict(experts=experts, router=router, vectors=vectors, total=experts + router + vectors)
 
 
@@ -204,15 +217,23 @@ def run_reference(args, cfg, rank, world):
         t_total += r["seconds"]
         n_total += r["tokens"]
         last = r
-    value = n_total / t_total
+    lps = cfg.get("layers_per_step", 1)
+    tt = cfg.get("tokens", 1)
+    metric, unit = METRIC, UNIT
+    if lps > 1:
+        metric, unit = f"decode steps/s through {lps} MoE layers (batch 1)", "steps/s"
+    elif tt > 1:
+        metric, unit = f"token decodes/s through one MoE layer ({tt}-token batches)", "tokens/s"
+    value = n_total / t_total / lps
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
-        "warmup": warm, "ms_per_step": 1000.0 * t_total / n_total, "higher_is_better": True, "scaling": "weak",
+        "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": steps,
+        "warmup": warm, "ms_per_step": 1000.0 * t_total / n_total * lps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {**{k: v for k, v in cfg.items()}, "batch": 1, "parallelism": "host cores"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": last["cores"], "kind": "oracle",
-                         "sample": f"{n_total} decodes over {steps} steps"},
-        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": last["cores"], "kind": "oracle",
+                         "sample": f"{n_total} single-layer decodes over {steps} steps"
+                                   + (f"; steps/s = decodes/s / {lps}" if lps > 1 else "")},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
@@ -237,7 +258,8 @@ def run_fmoe(args, cfg, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     h, i, e, k = cfg["hidden"], cfg["inter"], cfg["experts"], cfg["top_k"]
-    NL = args.layers
+    LPS = cfg.get("layers_per_step", 1)  # layer decodes per timed step
+    NL = LPS if LPS > 1 else args.layers
     # NL distinct layer instances of the workload, decoded in turn: the weights
     # a step reads were last touched NL - 1 steps earlier, so they come from
     # HBM (NL * 40 MB >> 126 MB of L2) without any flush between steps.
@@ -247,27 +269,46 @@ def run_fmoe(args, cfg, rank, world, local_rank):
                           F.expert_bytes, dev)
         layers.append(F.Layer(t["w_router"], t["w_sgate"], t["experts"], t["shared"], h, i, k, cfg["bits"],
                               cfg["shared_bits"]))
-    xs = torch.from_numpy(S.token_x(SEED + rank, 0, 0, POOL, h)).to(dev)
-    rs = torch.from_numpy(S.token_residual(SEED + rank, 0, 0, POOL, h)).to(dev)
-    out = torch.empty(POOL, h, dtype=torch.float32, device=dev)
-    ws = [L.workspace(1) for L in layers]
+    TT = cfg.get("tokens", 1)  # tokens per decode call
+    shape = (POOL, h) if TT == 1 else (POOL, TT, h)
+    xs = torch.from_numpy(S.token_x(SEED + rank, 0, 0, POOL * TT, h).reshape(shape)).to(dev)
+    rs = torch.from_numpy(S.token_residual(SEED + rank, 0, 0, POOL * TT, h).reshape(shape)).to(dev)
+    out = torch.empty(shape, dtype=torch.float32, device=dev)
+    ws = [L.workspace(TT) for L in layers]
     stream = torch.cuda.current_stream()
+
+    hbuf = torch.empty(2, h, dtype=torch.float32, device=dev)
 
     def decode(j):
         l = j % NL
-        layers[l].decode(xs[j % POOL], rs[j % POOL], out=out[j % POOL], ws=ws[l])
+        if LPS == 1:
+            layers[l].decode(xs[j % POOL], rs[j % POOL], out=out[j % POOL], ws=ws[l])
+        else:
+            # Stacked layers: layer l reads the hidden state layer l - 1 wrote,
+            # as both its input and its residual; layer 0 starts from a pool token.
+            src = xs[(j // NL) % POOL] if l == 0 else hbuf[(l - 1) % 2]
+            layers[l].decode(src, src, out=hbuf[l % 2], ws=ws[l])
 
     for j in range(args.warmup):
         decode(j)
     torch.cuda.synchronize()
     if F.get_status():
         raise RuntimeError("device status word set during warm-up")
+    distinct = None
+    if TT > 1:
+        # distinct routed experts per step, over one period of the rotation
+        idx = torch.empty(TT, k, dtype=torch.int32, device=dev)
+        counts = []
+        for j in range(64):
+            layers[j % NL].decode(xs[j % POOL], rs[j % POOL], out=out[j % POOL], idx_out=idx, ws=ws[j % NL])
+            counts.append(len(set(idx.flatten().tolist())))
+        distinct = float(np.mean(counts))
 
     # Each captured step is the library's decode call; a graph holds GSTEPS
     # consecutive steps so that the timed region is device time, without the
     # Python/ctypes launch latency (the end-to-end figure below keeps that).
-    GSTEPS = 64
-    K = args.steps
+    GSTEPS = 64 if LPS == 1 else LPS
+    K = args.steps * LPS  # layer decodes in the timed region
 
     def capture(first, n):
         g = torch.cuda.CUDAGraph()
@@ -320,49 +361,67 @@ def run_fmoe(args, cfg, rank, world, local_rank):
 
     # End to end through the same call with host buffers: pinned host -> device
     # copy of x and residual, decode, device -> host copy of out, every step.
-    xh = torch.from_numpy(S.token_x(SEED + rank, 0, 1, POOL, h)).pin_memory()
-    rh = torch.from_numpy(S.token_residual(SEED + rank, 0, 1, POOL, h)).pin_memory()
-    oh = torch.empty(POOL, h, dtype=torch.float32).pin_memory()
-    xd = torch.empty(h, dtype=torch.float32, device=dev)
-    rd = torch.empty(h, dtype=torch.float32, device=dev)
-    od = torch.empty(h, dtype=torch.float32, device=dev)
+    xh = torch.from_numpy(S.token_x(SEED + rank, 0, 1, POOL * TT, h).reshape(shape)).pin_memory()
+    rh = torch.from_numpy(S.token_residual(SEED + rank, 0, 1, POOL * TT, h).reshape(shape)).pin_memory()
+    oh = torch.empty(shape, dtype=torch.float32).pin_memory()
+    xd = torch.empty(shape[1:], dtype=torch.float32, device=dev)
+    rd = torch.empty(shape[1:], dtype=torch.float32, device=dev)
+    od = torch.empty(shape[1:], dtype=torch.float32, device=dev)
     K2 = min(K, 2000)
 
     def e2e_step(j):
-        l = j % NL
-        xd.copy_(xh[j % POOL], non_blocking=True)
-        rd.copy_(rh[j % POOL], non_blocking=True)
-        layers[l].decode(xd, rd, out=od, ws=ws[l])
-        oh[j % POOL].copy_(od, non_blocking=True)
+        if LPS == 1:
+            l = j % NL
+            xd.copy_(xh[j % POOL], non_blocking=True)
+            rd.copy_(rh[j % POOL], non_blocking=True)
+            layers[l].decode(xd, rd, out=od, ws=ws[l])
+            oh[j % POOL].copy_(od, non_blocking=True)
+        else:
+            # One token through every layer: its input goes up once and the last
+            # layer's output comes back once.
+            xd.copy_(xh[j % POOL], non_blocking=True)
+            src = xd
+            for l in range(NL):
+                dst = hbuf[l % 2] if l + 1 < NL else od
+                layers[l].decode(src, src, out=dst, ws=ws[l])
+                src = dst
+            oh[j % POOL].copy_(od, non_blocking=True)
 
+    n_e2e = K2 if LPS == 1 else max(1, K2 // LPS)  # e2e steps
     for j in range(3):
         e2e_step(j)
     torch.cuda.synchronize()
     b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     b0.record(stream)
-    for j in range(K2):
+    for j in range(n_e2e):
         e2e_step(j)
     b1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = b0.elapsed_time(b1)
+    e2e_ms_per_decode = b0.elapsed_time(b1) / (n_e2e * LPS)
 
     # max over ranks
-    tt = torch.tensor([total_ms, e2e_ms / K2 * K], dtype=torch.float64, device=dev)
+    tt = torch.tensor([total_ms, e2e_ms_per_decode * K], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
     total_ms_max, e2e_ms_max = float(tt[0]), float(tt[1])
 
     if rank == 0:
-        ab = algorithmic_bytes(cfg)
+        ab = algorithmic_bytes(cfg, distinct)
         peak, peak_kind = peaks()
         avg_launch_s = total_ms / 1000.0 / K
         achieved = ab["total"] / avg_launch_s / 1e9
-        value = world * K / (total_ms_max / 1000.0)
+        steps = K // LPS
+        value = world * steps * TT / (total_ms_max / 1000.0)
+        metric, unit = METRIC, UNIT
+        if LPS > 1:
+            metric, unit = f"decode steps/s through {LPS} MoE layers (batch 1)", "steps/s"
+        elif TT > 1:
+            metric, unit = f"token decodes/s through one MoE layer ({TT}-token batches)", "tokens/s"
         line = {
-            "impl": "fmoe", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
-            "warmup": args.warmup, "ms_per_step": total_ms_max / K, "higher_is_better": True,
+            "impl": "fmoe", "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": total_ms_max / steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u4/bf16 weights, f32 compute", "data": "synthetic",
-            "config": {**cfg, "batch": 1, "group": 64,
+            "config": {**cfg, "batch": TT, "group": 64,
                        "l2": f"inputs larger than L2: {NL} distinct layer instances decoded in turn "
                              f"({NL * e * expert_bytes(h, i, cfg['bits']) / 1e9:.0f} GB of experts), no flush",
                        "layers_in_rotation": NL, "input_pool": POOL, "parallelism": f"replicas x{world}"},
@@ -374,18 +433,27 @@ def run_fmoe(args, cfg, rank, world, local_rank):
             "expert_frac_of_hbm": ab["experts"] / avg_launch_s / 1e9 / peak,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": profiled_traffic(args.config),
-                         "kernel": f"layer_kernel<{cfg['bits']},{cfg['shared_bits']}>",
+                         "kernel": (f"layer_kernel<{cfg['bits']},{cfg['shared_bits']}>" if TT == 1 else
+                                    "grouped decode step (router, prep, gate/up, stage, down launches)"),
                          "algorithmic_bytes_per_launch": ab["total"]},
-            "e2e": {"value": world * K / (e2e_ms_max / 1000.0), "unit": UNIT, "h2d_bytes_per_step": 2 * h * 4,
-                    "d2h_bytes_per_step": h * 4},
-            "gpu_launches": K,
+            "layer_decodes_per_s": world * K / (total_ms_max / 1000.0),
+            "sustained_gbs": world * K * ab["total"] / (total_ms_max / 1000.0) / 1e9,
+            "e2e": {"value": world * K * TT / LPS / (e2e_ms_max / 1000.0), "unit": unit,
+                    "h2d_bytes_per_step": (2 if LPS == 1 else 1) * TT * h * 4, "d2h_bytes_per_step": TT * h * 4},
+            "gpu_launches": K * (1 if TT == 1 else 5),
+            **({"distinct_routed_experts_per_step": distinct} if distinct is not None else {}),
             "clocks": clk,
             "device_status": status,
         }
         if not args.no_cpu_baseline:
-            line["cpu_baseline"] = oracle_sample(cfg, args.cpu_seconds)
-            line["cpu_baseline"].pop("seconds", None)
-            line["cpu_baseline"].pop("tokens", None)
+            cb = oracle_sample(cfg, args.cpu_seconds)
+            cb.pop("seconds", None)
+            cb.pop("tokens", None)
+            if LPS > 1:  # a step is LPS layer decodes
+                cb["value"] /= LPS
+                cb["sample"] += f"; steps/s = decodes/s / {LPS}"
+            cb["unit"] = unit  # one oracle decode is one token through one layer
+            line["cpu_baseline"] = cb
         print(json.dumps(line), flush=True)
 
 

@@ -25,7 +25,7 @@ EXPORTED = [
     "fmoe_expert_bytes", "fmoe_blob_offsets", "fmoe_quantize_expert", "fmoe_route_workspace_bytes",
     "fmoe_route", "fmoe_expert_workspace_bytes", "fmoe_expert_forward", "fmoe_workspace_bytes",
     "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status", "fmoe_strerror", "fmoe_last_cuda_error",
-    "fmoe_layer_decode_noalloc",
+    "fmoe_layer_decode_noalloc", "fmoe_set_wait_limit_ns",
 ]
 
 
@@ -77,6 +77,7 @@ def lib() -> ctypes.CDLL:
     L.fmoe_layer_decode.argtypes = [ctypes.POINTER(FmoeLayerC), vp, vp, vp, i, vp, sz, vp, vp, vp]
     L.fmoe_layer_decode_noalloc.argtypes = [ctypes.POINTER(FmoeLayerC), vp, vp, vp, i, vp, vp, vp]
     L.fmoe_get_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
+    L.fmoe_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong)]
     L.fmoe_last_cuda_error.argtypes = []
     L.fmoe_last_cuda_error.restype = i
     L.fmoe_strerror.argtypes = [i]
@@ -269,6 +270,15 @@ def layer_decode_noalloc(layer: "Layer", x: torch.Tensor, residual: torch.Tensor
                                            x2.shape[0], _ptr(idx_out), _ptr(w_out), _stream(stream)),
            "fmoe_layer_decode_noalloc")
     return out
+
+
+def set_wait_limit_ns(limit_ns: int) -> int:
+    """Set the time limit of the kernels' device-side waits; returns the previous limit."""
+    prev = ctypes.c_ulonglong(0)
+    rc = lib().fmoe_set_wait_limit_ns(ctypes.c_ulonglong(int(limit_ns)), ctypes.byref(prev))
+    if rc != FMOE_OK:
+        raise FmoeError(rc, "fmoe_set_wait_limit_ns")
+    return int(prev.value)
 
 
 def get_status(stream=None) -> int:

@@ -123,6 +123,14 @@ __device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
   return r;
 }
 
+// Read-only input either in shared memory (plain load) or in global memory
+// written by an earlier kernel (non-coherent cached load).
+template <bool kGlobal, typename T>
+__device__ __forceinline__ T ld_in(const T* p) {
+  if constexpr (kGlobal) return __ldg(p);
+  else return *p;
+}
+
 // ---- packed fp32 pairs (sm_100 f32x2) -------------------------------------------
 __device__ __forceinline__ uint64_t pk_u32(uint32_t lo, uint32_t hi) {
   uint64_t r;

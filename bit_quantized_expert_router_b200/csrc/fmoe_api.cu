@@ -1,23 +1,30 @@
 // Host side of libfmoe.so: argument validation, shared-memory planning and
 // launches.  The C ABI is declared (and documented) in include/fmoe.h.
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
 #include "../../include/fmoe.h"
-#include "route_quant_kernels.cuh"
+#include "grouped_kernels.cuh"
 
 using namespace fmoe;
 
 namespace {
 
-constexpr unsigned long long kTimeoutNs = 2000000000ull;  // 2 s bound on every device-side wait
+constexpr unsigned long long kTimeoutNs = 2000000000ull;  // default bound on every device-side wait: 2 s
+constexpr unsigned long long kMinWaitNs = 1000000ull;      // 1 ms
+constexpr unsigned long long kMaxWaitNs = 60000000000ull;  // 60 s
+std::atomic<unsigned long long> g_wait_limit_ns{kTimeoutNs};
 constexpr size_t kCounterBytes = 256;
 constexpr int kMaxNst = 4;
 
 struct DevInfo {
   int sms = 0;
   int max_smem = 0;     // opt-in dynamic shared memory available to the layer kernel
+  int optin = 0;        // opt-in shared memory per block
   bool layer_attr_set[4] = {false, false, false, false};
+  bool grouped_attr_set[4] = {false, false, false, false};
+  int grouped_max_smem = 0;  // dynamic shared memory left by the grouped kernels' static arrays
 };
 
 using LayerFn = void (*)(LayerArgs);
@@ -57,6 +64,14 @@ int dev_info(int* dev_out, DevInfo** info) {
         static_smem = std::max(static_smem, (int)fa.sharedSizeBytes);
       }
     d.max_smem = optin - static_smem;
+    d.optin = optin;
+    int gstatic = 0;
+    for (const void* f : {(const void*)grouped_gateup_kernel<4, 4>, (const void*)grouped_down_kernel<4, 4>}) {
+      cudaFuncAttributes fa;
+      if ((e = cudaFuncGetAttributes(&fa, f)) != cudaSuccess) return cuda_fail(e);
+      gstatic = std::max(gstatic, (int)fa.sharedSizeBytes);
+    }
+    d.grouped_max_smem = optin - gstatic;
   }
   *dev_out = dev;
   *info = &d;
@@ -136,6 +151,144 @@ bool plan_layer(int H, int I, int K, bool has_shared, int bits_r, int bits_s, in
 
 size_t layer_ws_bytes(int E, int I, int K) {
   return kCounterBytes + round_up((size_t)(E + 1) * 4, 256) + round_up((size_t)(K + 1) * I * 4, 256);
+}
+
+// Workspace of the grouped (T >= 2) decode, byte offsets (every section 256-B aligned).
+struct GroupedLayout {
+  size_t logits, meta, slot_expert, slot_pair0, pair_token, tok_pair, tok_w, tok_sg;
+  size_t xs_r, sf_r, xs_s, sf_s, act, as, sfa, total;
+};
+
+GroupedLayout grouped_layout(int E, int H, int I, int K, int T) {
+  GroupedLayout g;
+  size_t off = kCounterBytes;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += round_up(bytes, 256);
+    return o;
+  };
+  const size_t P = (size_t)T * K + T;
+  g.logits = take((size_t)T * (E + 1) * 4);
+  g.meta = take(16);
+  g.slot_expert = take((size_t)kMaxPairs * 4);
+  g.slot_pair0 = take((size_t)(kMaxPairs + 2) * 4);
+  g.pair_token = take((size_t)kMaxPairs * 4);
+  g.tok_pair = take((size_t)T * (K + 1) * 4);
+  g.tok_w = take((size_t)T * K * 4);
+  g.tok_sg = take((size_t)T * 4);
+  g.xs_r = take((size_t)T * H * 4);
+  g.sf_r = take((size_t)T * (H / 32) * 8);
+  g.xs_s = take((size_t)T * H * 4);
+  g.sf_s = take((size_t)T * (H / 32) * 8);
+  g.act = take(P * I * 4);
+  g.as = take(P * I * 4);
+  g.sfa = take(P * (I / 32) * 8);
+  g.total = off;
+  return g;
+}
+
+using GroupedFn = void (*)(GroupArgs);
+struct GroupedFns {
+  GroupedFn prep, gateup, stage, down;
+};
+template <int BR, int BS>
+GroupedFns grouped_fns_t() {
+  return {grouped_prep_kernel<BR, BS>, grouped_gateup_kernel<BR, BS>, grouped_stage_act_kernel<BR, BS>,
+          grouped_down_kernel<BR, BS>};
+}
+GroupedFns grouped_fns(int br, int bs) {
+  if (br == 4) return bs == 4 ? grouped_fns_t<4, 4>() : grouped_fns_t<4, 2>();
+  return bs == 4 ? grouped_fns_t<2, 4>() : grouped_fns_t<2, 2>();
+}
+
+// Launch the grouped decode (router, prep, gate/up, activation staging, down).
+int launch_grouped(const fmoe_layer* L, const float* x, const float* residual, float* out, int T, void* ws,
+                   int32_t* idx_out, float* w_out, DevInfo* info, cudaStream_t s) {
+  const int H = L->hidden, I = L->inter, E = L->n_experts, K = L->top_k, G = info->sms;
+  const bool has_shared = L->shared != nullptr;
+  const int br = L->bits, bs = has_shared ? L->shared_bits : L->bits;
+  const GroupedLayout gl = grouped_layout(E, H, I, K, T);
+  char* w8 = static_cast<char*>(ws);
+  GroupArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.experts = static_cast<const char*>(L->experts);
+  a.expert_stride = L->expert_stride;
+  a.shared = static_cast<const char*>(L->shared);
+  a.x = x;
+  a.residual = residual;
+  a.out = out;
+  a.logits = reinterpret_cast<float*>(w8 + gl.logits);
+  a.tb.meta = reinterpret_cast<int*>(w8 + gl.meta);
+  a.tb.slot_expert = reinterpret_cast<int*>(w8 + gl.slot_expert);
+  a.tb.slot_pair0 = reinterpret_cast<int*>(w8 + gl.slot_pair0);
+  a.tb.pair_token = reinterpret_cast<int*>(w8 + gl.pair_token);
+  a.tb.tok_pair = reinterpret_cast<int*>(w8 + gl.tok_pair);
+  a.tb.tok_w = reinterpret_cast<float*>(w8 + gl.tok_w);
+  a.tb.tok_sg = reinterpret_cast<float*>(w8 + gl.tok_sg);
+  a.xs_r = reinterpret_cast<float4*>(w8 + gl.xs_r);
+  a.sf_r = reinterpret_cast<float2*>(w8 + gl.sf_r);
+  const bool separate = has_shared && bs != br;
+  a.xs_s = reinterpret_cast<float4*>(w8 + (separate ? gl.xs_s : gl.xs_r));
+  a.sf_s = reinterpret_cast<float2*>(w8 + (separate ? gl.sf_s : gl.sf_r));
+  a.act = reinterpret_cast<float*>(w8 + gl.act);
+  a.as = reinterpret_cast<float4*>(w8 + gl.as);
+  a.sfa = reinterpret_cast<float2*>(w8 + gl.sfa);
+  a.idx_out = idx_out;
+  a.w_out = w_out;
+  a.H = H;
+  a.I = I;
+  a.E = E;
+  a.K = K;
+  a.T = T;
+  a.bits_r = br;
+  a.bits_s = bs;
+  a.has_sgate = L->w_sgate != nullptr;
+  a.timeout_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  for (int r = 0; r < 2; ++r) {
+    const BlobOff o = blob_offsets(H, I, r == 0 ? br : bs);
+    long long* d = r == 0 ? a.off_r : a.off_s;
+    d[0] = o.gc;
+    d[1] = o.gsb;
+    d[2] = o.uc;
+    d[3] = o.usb;
+    d[4] = o.dc;
+    d[5] = o.dsb;
+  }
+  // Shared-memory plans: gate/up ring, down ring + per-pair results.
+  int stage = 0, cstage = 0;
+  for (int b : {br, bs}) {
+    const int cap = ((H / 16 + 15) & ~15) + 16;
+    stage = std::max(stage, 2 * (H * b / 8) + 2 * cap);
+    cstage = std::max(cstage, kRC * (I * b / 8 + I / 16));
+  }
+  a.stage_bytes = (int)round_up(stage, 128);
+  a.c_stage_bytes = (int)round_up(cstage, 128);
+  const int budget = info->grouped_max_smem;
+  a.nst = std::min(kMaxNst, (budget - kWarps * kMaxNst * 8) / (kWarps * a.stage_bytes));
+  a.ys_stride = kRC * ((H / kRC + G - 1) / G);
+  const size_t ys_bytes = round_up((size_t)kMaxPairs * a.ys_stride * 4, 16);
+  a.nst_c = std::min(kMaxNstC, (int)((budget - (long long)ys_bytes - kWarps * kMaxNstC * 8) /
+                                     ((long long)kWarps * a.c_stage_bytes)));
+  if (a.nst < 1 || a.nst_c < 1) return FMOE_EINVAL;
+  const size_t smem_gu = (size_t)kWarps * a.nst * a.stage_bytes + (size_t)kWarps * a.nst * 8;
+  const size_t smem_d = (size_t)kWarps * a.nst_c * a.c_stage_bytes + ys_bytes + (size_t)kWarps * a.nst_c * 8;
+  const GroupedFns fns = grouped_fns(br, bs);
+  const int fi = layer_fn_index(br, bs);
+  if (!info->grouped_attr_set[fi]) {
+    for (GroupedFn f : {fns.gateup, fns.down})
+      if (cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, budget))
+        return cuda_fail(e);
+    info->grouped_attr_set[fi] = true;
+  }
+  const int rows = E + (L->w_sgate ? 1 : 0);
+  router_logits_kernel<<<(rows + 7) / 8, 256, 0, s>>>(L->w_router, L->w_sgate, x, T, H, E,
+                                                      const_cast<float*>(a.logits));
+  fns.prep<<<1 + T, kThreads, 0, s>>>(a);
+  fns.gateup<<<G, kThreads, smem_gu, s>>>(a);
+  fns.stage<<<T * K + T, 256, 0, s>>>(a);
+  fns.down<<<G, kThreads, smem_d, s>>>(a);
+  if (cudaError_t e = cudaGetLastError()) return cuda_fail(e);
+  return FMOE_OK;
 }
 
 // Fill the grid-shape-dependent fields and the blob section offsets.
@@ -311,14 +464,16 @@ int fmoe_expert_forward(const void* blob, int hidden, int inter, int bits, const
   a.nst_c = pl.nst_c;
   a.c_stage_bytes = pl.c_stage_bytes;
   a.lg_floats = pl.lg_floats;
-  a.timeout_ns = kTimeoutNs;
+  a.timeout_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   set_offsets(a, info->sms);
   return launch_layer(a, pl, info, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t fmoe_workspace_bytes(const fmoe_layer* L, int T) {
   if (!L || T < 1 || T > FMOE_MAX_TOKENS) return 0;
-  return layer_ws_bytes(L->n_experts, L->inter, L->top_k);
+  const size_t single = layer_ws_bytes(L->n_experts, L->inter, L->top_k);
+  if (T == 1) return single;
+  return std::max(single, grouped_layout(L->n_experts, L->hidden, L->inter, L->top_k, T).total);
 }
 
 int fmoe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream_t stream) {
@@ -383,9 +538,10 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
   a.nst_c = pl.nst_c;
   a.c_stage_bytes = pl.c_stage_bytes;
   a.lg_floats = pl.lg_floats;
-  a.timeout_ns = kTimeoutNs;
+  a.timeout_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   set_offsets(a, info->sms);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (T > 1) return launch_grouped(L, x, residual, out, T, ws, idx_out_opt, w_out_opt, info, s);
   for (int t = 0; t < T; ++t) {
     a.x = x + (long long)t * H;
     a.residual = residual ? residual + (long long)t * H : nullptr;
@@ -428,6 +584,13 @@ int fmoe_get_status(fmoe_stream_t stream, unsigned* bits_out) {
 }
 
 int fmoe_last_cuda_error(void) { return g_last_cuda_error; }
+
+int fmoe_set_wait_limit_ns(unsigned long long limit_ns, unsigned long long* previous_opt) {
+  if (limit_ns < kMinWaitNs || limit_ns > kMaxWaitNs) return FMOE_EINVAL;
+  const unsigned long long old = g_wait_limit_ns.exchange(limit_ns);
+  if (previous_opt) *previous_opt = old;
+  return FMOE_OK;
+}
 
 #ifdef FMOE_TRACE_BUILD
 // Trace builds only: copy the phase timestamps of the last layer launch

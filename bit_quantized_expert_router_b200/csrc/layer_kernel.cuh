@@ -291,8 +291,8 @@ __device__ __forceinline__ float router_dot(const uint16_t* row, const float* xu
 
 // Gate and up rows of one expert (stage layout: gate codes | up codes | gate sb
 // superset | up sb superset) against the staged input.
-template <int BITS>
-__device__ __forceinline__ void pair_dot(const char* st, int H, int sbo_g, int sbo_u, const float4* xs,
+template <int BITS, bool kG>
+__device__ __forceinline__ void pair_dot_src(const char* st, int H, int sbo_g, int sbo_u, const float4* xs,
                                          const float2* sf, int lane, float& g_out, float& u_out) {
   constexpr int CPV = 128 / BITS;
   const int NV = H / CPV;
@@ -308,18 +308,18 @@ __device__ __forceinline__ void pair_dot(const char* st, int H, int sbo_g, int s
     const uint4 wg = cg[v], wu = cu[v];
     const int grp = (BITS == 4) ? (v >> 1) : v;
     const uint32_t sbgw = sbg[grp], sbuw = sbu[grp];
-    const float2 f = sf[v];
+    const float2 f = ld_in<kG>(sf + v);
     uint64_t ag = 0, au = 0;
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       const uint32_t a_ = (&wg.x)[t], b_ = (&wu.x)[t];
       if (BITS == 4) {
-        const ulonglong2 xa = xv[(2 * t) * NV + v], xb = xv[(2 * t + 1) * NV + v];
+        const ulonglong2 xa = ld_in<kG>(xv + (2 * t) * NV + v), xb = ld_in<kG>(xv + (2 * t + 1) * NV + v);
         dot_word4(ag, a_, xa, xb);
         dot_word4(au, b_, xa, xb);
       } else {
-        const ulonglong2 x0 = xv[(4 * t) * NV + v], x1 = xv[(4 * t + 1) * NV + v];
-        const ulonglong2 x2 = xv[(4 * t + 2) * NV + v], x3 = xv[(4 * t + 3) * NV + v];
+        const ulonglong2 x0 = ld_in<kG>(xv + (4 * t) * NV + v), x1 = ld_in<kG>(xv + (4 * t + 1) * NV + v);
+        const ulonglong2 x2 = ld_in<kG>(xv + (4 * t + 2) * NV + v), x3 = ld_in<kG>(xv + (4 * t + 3) * NV + v);
         dot_word2(ag, a_, x0, x1, x2, x3);
         dot_word2(au, b_, x0, x1, x2, x3);
       }
@@ -334,12 +334,18 @@ __device__ __forceinline__ void pair_dot(const char* st, int H, int sbo_g, int s
   u_out = warp_sum(u);
 }
 
+template <int BITS>
+__device__ __forceinline__ void pair_dot(const char* st, int H, int sbo_g, int sbo_u, const float4* xs,
+                                         const float2* sf, int lane, float& g_out, float& u_out) {
+  pair_dot_src<BITS, false>(st, H, sbo_g, sbo_u, xs, sf, lane, g_out, u_out);
+}
+
 // kRC down rows of one expert (stage layout: kRC code rows | kRC sb rows)
 // against that expert's staged activation, which is column block
 // [col0, col0 + I/CPV) of a staged [F4][NVS] array (several same-width experts
 // staged together); sfa points at column col0.  Returns the full row dots.
-template <int BITS>
-__device__ __forceinline__ void down_rows(const char* st, int I, const float4* as, int NVS, int col0,
+template <int BITS, bool kG>
+__device__ __forceinline__ void down_rows_src(const char* st, int I, const float4* as, int NVS, int col0,
                                           const float2* sfa, int lane, float (&y)[kRC]) {
   constexpr int CPV = 128 / BITS;
   const int NV = I / CPV;
@@ -353,7 +359,7 @@ __device__ __forceinline__ void down_rows(const char* st, int I, const float4* a
     uint4 w[kRC];
 #pragma unroll
     for (int r = 0; r < kRC; ++r) w[r] = reinterpret_cast<const uint4*>(st + r * cb)[v];
-    const float2 f = sfa[v];
+    const float2 f = ld_in<kG>(sfa + v);
     const int grp = (BITS == 4) ? (v >> 1) : v;
     uint64_t ac[kRC];
 #pragma unroll
@@ -361,12 +367,12 @@ __device__ __forceinline__ void down_rows(const char* st, int I, const float4* a
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       if (BITS == 4) {
-        const ulonglong2 xa = xv[(2 * t) * NVS + v], xb = xv[(2 * t + 1) * NVS + v];
+        const ulonglong2 xa = ld_in<kG>(xv + (2 * t) * NVS + v), xb = ld_in<kG>(xv + (2 * t + 1) * NVS + v);
 #pragma unroll
         for (int r = 0; r < kRC; ++r) dot_word4(ac[r], (&w[r].x)[t], xa, xb);
       } else {
-        const ulonglong2 x0 = xv[(4 * t) * NVS + v], x1 = xv[(4 * t + 1) * NVS + v];
-        const ulonglong2 x2 = xv[(4 * t + 2) * NVS + v], x3 = xv[(4 * t + 3) * NVS + v];
+        const ulonglong2 x0 = ld_in<kG>(xv + (4 * t) * NVS + v), x1 = ld_in<kG>(xv + (4 * t + 1) * NVS + v);
+        const ulonglong2 x2 = ld_in<kG>(xv + (4 * t + 2) * NVS + v), x3 = ld_in<kG>(xv + (4 * t + 3) * NVS + v);
 #pragma unroll
         for (int r = 0; r < kRC; ++r) dot_word2(ac[r], (&w[r].x)[t], x0, x1, x2, x3);
       }
@@ -381,6 +387,12 @@ __device__ __forceinline__ void down_rows(const char* st, int I, const float4* a
   }
 #pragma unroll
   for (int r = 0; r < kRC; ++r) y[r] = warp_sum(y[r]);
+}
+
+template <int BITS>
+__device__ __forceinline__ void down_rows(const char* st, int I, const float4* as, int NVS, int col0,
+                                          const float2* sfa, int lane, float (&y)[kRC]) {
+  down_rows_src<BITS, false>(st, I, as, NVS, col0, sfa, lane, y);
 }
 
 // Top-K by one warp: descending logit, lower index first on exact ties; then
@@ -468,10 +480,17 @@ __device__ __forceinline__ void warp_topk(const float* lg, int n, int k, int lan
 }
 
 // Wait until *ctr >= target (one thread), for at most limit_ns.
+__device__ __forceinline__ bool counter_reached(unsigned v, unsigned target) {
+  // Counts never exceed the grid size; a value with the top bit set is a
+  // workspace that was not zeroed (or was overwritten), never "reached", so
+  // the wait runs out and reports instead of passing on garbage.
+  return v >= target && v < 0x80000000u;
+}
+
 __device__ __forceinline__ bool grid_wait(const unsigned* ctr, unsigned target, uint64_t limit_ns) {
-  if (ld_acquire_gpu(ctr) >= target) return true;
+  if (counter_reached(ld_acquire_gpu(ctr), target)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (ld_acquire_gpu(ctr) < target) {
+  while (!counter_reached(ld_acquire_gpu(ctr), target)) {
     FMOE_SPIN(1);
     __nanosleep(64);
     if (globaltimer_ns() - t0 > limit_ns) return false;

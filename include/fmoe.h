@@ -207,6 +207,17 @@ int fmoe_get_status(fmoe_stream_t stream, unsigned* bits_out);
  * of this library return FMOE_ECUDA on the calling thread (0 if none). */
 int fmoe_last_cuda_error(void);
 
+/* Set the time limit of every device-side wait of the kernels launched after
+ * this call (process-wide, all devices; default 2 s).  A wait that runs out
+ * sets a bit of the device status word (see fmoe_get_status) and the kernel
+ * carries on to its end without leaving its buffers, so the context stays
+ * usable; the call's outputs are then undefined.  limit_ns must lie in
+ * [1e6, 6e10] (1 ms .. 60 s), else FMOE_EINVAL and nothing changes.  The
+ * previous limit is stored in *previous_opt when non-NULL.  The pages have no
+ * counterpart: this is this library's watchdog.  Not synchronised with
+ * launches in flight on other threads. */
+int fmoe_set_wait_limit_ns(unsigned long long limit_ns, unsigned long long* previous_opt);
+
 /* Static, human-readable text for an error code. */
 const char* fmoe_strerror(int code);
 

@@ -229,3 +229,146 @@ def test_layer_deterministic(F, SG):
     b = L.decode(x, res).clone()
     assert torch.equal(a, b)
     assert F.get_status() == 0
+
+
+def test_stacked_layers_graph(F, SG):
+    """Layers chained as in a stacked decode (each layer's output is the next
+    layer's input and residual), replayed from one CUDA graph; every layer is
+    checked against the oracle on the input the engine actually gave it."""
+    shape = C.FULL4
+    seed, n_layers, n_steps = 11, 3, 2
+    layers = [make_gpu_layer(F, SG, seed, l, shape)[0] for l in range(n_layers)]
+    H, K = shape.hidden, shape.top_k
+    x0 = torch.empty(H, dtype=torch.float32, device=dev())
+    hs = torch.empty(n_layers, H, dtype=torch.float32, device=dev())
+    idx = torch.empty(n_layers, K, dtype=torch.int32, device=dev())
+    ws = [L.workspace(1) for L in layers]
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for L, w in zip(layers, ws):  # resolve the stream's device before capture
+            L.decode(x0, x0, out=hs[0], ws=w)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            src = x0
+            for l, L in enumerate(layers):
+                L.decode(src, src, out=hs[l], idx_out=idx[l], ws=ws[l])
+                src = hs[l]
+    wr = [S.router_bf16(seed, l, shape.n_experts, H) for l in range(n_layers)]
+    for step in range(n_steps):
+        x0.copy_(torch.from_numpy(C.parity_x(seed, 0, step, wr[0], K, H)[0]))
+        g.replay()
+        torch.cuda.synchronize()
+        assert F.get_status() == 0
+        ins = [x0.cpu().numpy().astype(np.float64)] + [hs[l].cpu().numpy().astype(np.float64)
+                                                         for l in range(n_layers - 1)]
+        for l in range(n_layers):
+            x = ins[l].astype(np.float32)
+            r = C.oracle_layer(seed, l, shape, x, x)
+            got = idx[l].cpu().numpy().tolist()
+            lg = O.router_logits(wr[l], x)
+            if O.top5_min_gap(lg, K) >= C.NEAR_TIE:
+                assert got == r["idx"].tolist(), f"layer {l} step {step}"
+            else:  # a near-tie: the selection must still be a valid top-K
+                assert min(lg[got]) >= np.sort(lg)[-K] - C.NEAR_TIE
+                continue
+            out = hs[l].cpu().numpy()
+            C.assert_close(out, r["out"], f"stacked layer {l} step {step}")
+            ma, _ = C.errors(out.astype(np.float64) - x, r["out"] - x)
+            assert ma <= C.MAX_ABS, f"layer {l} step {step}: MoE part max-abs {ma:.3e}"
+    del g
+
+
+# ---------------------------------------------------------------------------
+# Grouped decode (T >= 2 tokens in one call)
+# ---------------------------------------------------------------------------
+
+def run_grouped_case(F, SG, shape, T, seed=31, layer=0, with_shared=True, with_sgate=True, identical=False,
+                     residual=True):
+    L, t = make_gpu_layer(F, SG, seed, layer, shape, with_shared, with_sgate)
+    wr = S.router_bf16(seed, layer, shape.n_experts, shape.hidden)
+    x = C.parity_x(seed, layer, 0, wr, shape.top_k, shape.hidden, 1 if identical else T)
+    if identical:
+        x = np.repeat(x, T, axis=0)
+    res = S.token_residual(seed, layer, 0, T, shape.hidden) if residual else np.zeros((T, shape.hidden), np.float32)
+    if identical:
+        res = np.repeat(res[:1], T, axis=0)
+    idx = torch.empty(T, shape.top_k, dtype=torch.int32, device=dev())
+    w = torch.empty(T, shape.top_k, dtype=torch.float32, device=dev())
+    out = L.decode(torch.from_numpy(x).to(dev()), torch.from_numpy(res).to(dev()) if residual else None,
+                   idx_out=idx, w_out=w)
+    assert F.get_status() == 0
+    got = out.cpu().numpy()
+    gi, gw = idx.cpu().numpy(), w.cpu().numpy()
+    for k in range(T):
+        if identical and k > 0:
+            assert np.array_equal(got[k], got[0]) and np.array_equal(gi[k], gi[0])
+            continue
+        r = C.oracle_layer(seed, layer, shape, x[k], res[k], with_shared, with_sgate)
+        assert gi[k].tolist() == r["idx"].tolist(), f"token {k}"
+        C.assert_close(gw[k], r["w"], f"token {k} w", max_abs=1e-6, rel_l2=1e-6)
+        C.assert_close(got[k], r["out"], f"{shape.name} T={T} token {k}")
+    return L, x, res, got
+
+
+def test_grouped_full_4bit_16_tokens(F, SG):
+    run_grouped_case(F, SG, C.FULL4, 16)
+
+
+def test_grouped_full_2bit_16_tokens(F, SG):
+    run_grouped_case(F, SG, C.FULL2, 16, seed=32, residual=False)
+
+
+def test_grouped_two_tokens_full(F, SG):
+    run_grouped_case(F, SG, C.FULL4, 2, seed=33)
+
+
+@pytest.mark.parametrize("shape,T,with_shared,with_sgate", [
+    (C.Shape("shared_heavy_h512_i128_e8_k4", 512, 128, 8, 4, 4), 16, True, True),
+    (C.Shape("ragged_h320_i192_e24_k3", 320, 192, 24, 3, 4), 7, True, True),
+    (C.Shape("no_shared_h512_i128_e16_k4", 512, 128, 16, 4, 4), 16, False, True),
+    (C.Shape("ungated_h512_i128_e16_k2_2bit", 512, 128, 16, 2, 2, 2), 9, True, False),
+    (C.Shape("mixed_h1024_i256_e64_k8_r4_s2", 1024, 256, 64, 8, 4, 2), 16, True, True),
+    (C.Shape("mixed_h1024_i256_e64_k1_r2_s4", 1024, 256, 64, 1, 2, 4), 3, True, True),
+    (C.Shape("e1024_h2048_i256_k4", 2048, 256, 1024, 4, 4), 16, True, True),
+])
+def test_grouped_edge_shapes(F, SG, shape, T, with_shared, with_sgate):
+    run_grouped_case(F, SG, shape, T, with_shared=with_shared, with_sgate=with_sgate)
+
+
+def test_grouped_identical_tokens_share_every_expert(F, SG):
+    """All tokens equal: one slot per expert holding every token."""
+    run_grouped_case(F, SG, C.Shape("identical_h1024_i256_e64_k4", 1024, 256, 64, 4, 4), 16, identical=True)
+
+
+def test_grouped_matches_single_token_calls(F, SG):
+    """A batch gives each token the routing and (within the fp tolerance) the
+    output of decoding that token alone."""
+    L, x, res, got = run_grouped_case(F, SG, C.TINY, 12, seed=34)
+    for k in range(12):
+        idx = torch.empty(1, C.TINY.top_k, dtype=torch.int32, device=dev())
+        one = L.decode(torch.from_numpy(x[k]).to(dev()), torch.from_numpy(res[k]).to(dev()), idx_out=idx)
+        C.assert_close(got[k], one.cpu().numpy()[0], f"token {k} batch vs alone", max_abs=1e-5, rel_l2=1e-6)
+
+
+def test_grouped_deterministic_and_graph_replay(F, SG):
+    shape, T = C.FULL4, 16
+    L, t = make_gpu_layer(F, SG, 35, 0, shape)
+    x = torch.from_numpy(S.token_x(35, 0, 0, T, shape.hidden)).to(dev())
+    res = torch.from_numpy(S.token_residual(35, 0, 0, T, shape.hidden)).to(dev())
+    out = torch.empty(T, shape.hidden, dtype=torch.float32, device=dev())
+    ws = L.workspace(T)
+    a = L.decode(x, res, ws=ws).clone()
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        L.decode(x, res, out=out, ws=ws)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            L.decode(x, res, out=out, ws=ws)
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(a, out)
+    assert F.get_status() == 0
+    del g

@@ -14,6 +14,7 @@ enum : unsigned {
   kStatusGridBarrierTimeout = 1u,  // a grid-wide wait ran past its time limit
   kStatusCopyTimeout = 2u,         // a bulk copy did not complete in time
   kStatusCtaWaitTimeout = 4u,      // an intra-CTA hand-off ran past its time limit
+  kStatusMmaTimeout = 8u,          // tensor-core work did not complete in time
 };
 
 __device__ __forceinline__ void set_status(unsigned bits) { atomicOr(&g_fmoe_status, bits); }

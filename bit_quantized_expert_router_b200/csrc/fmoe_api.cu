@@ -5,7 +5,7 @@
 #include <mutex>
 
 #include "../../include/fmoe.h"
-#include "grouped_kernels.cuh"
+#include "shared_tc.cuh"
 
 using namespace fmoe;
 
@@ -155,8 +155,8 @@ size_t layer_ws_bytes(int E, int I, int K) {
 
 // Workspace of the grouped (T >= 2) decode, byte offsets (every section 256-B aligned).
 struct GroupedLayout {
-  size_t logits, meta, slot_expert, slot_pair0, pair_token, tok_pair, tok_w, tok_sg;
-  size_t xs_r, sf_r, xs_s, sf_s, act, as, sfa, total;
+  size_t logits, meta, slot_expert, slot_pair0, pair_token, pair_slot, tok_pair, tok_w, tok_sg;
+  size_t xs_r, sf_r, xs_s, sf_s, gu_part, as, sfa, y_part, sh_gu, sh_y, total;
 };
 
 GroupedLayout grouped_layout(int E, int H, int I, int K, int T) {
@@ -173,6 +173,7 @@ GroupedLayout grouped_layout(int E, int H, int I, int K, int T) {
   g.slot_expert = take((size_t)kMaxPairs * 4);
   g.slot_pair0 = take((size_t)(kMaxPairs + 2) * 4);
   g.pair_token = take((size_t)kMaxPairs * 4);
+  g.pair_slot = take((size_t)kMaxPairs * 4);
   g.tok_pair = take((size_t)T * (K + 1) * 4);
   g.tok_w = take((size_t)T * K * 4);
   g.tok_sg = take((size_t)T * 4);
@@ -180,9 +181,13 @@ GroupedLayout grouped_layout(int E, int H, int I, int K, int T) {
   g.sf_r = take((size_t)T * (H / 32) * 8);
   g.xs_s = take((size_t)T * H * 4);
   g.sf_s = take((size_t)T * (H / 32) * 8);
-  g.act = take(P * I * 4);
+  g.gu_part = take(P * kMaxChunks * I * 8);
   g.as = take(P * I * 4);
   g.sfa = take(P * (I / 32) * 8);
+  g.y_part = take(P * kMaxChunks * H * 4);
+  // tensor-core shared expert partials (used when H and I are multiples of 512)
+  g.sh_gu = take((size_t)2 * (H / kTcK) * kMaxTokens * I * 4);
+  g.sh_y = take((size_t)(I / kTcK) * kMaxTokens * H * 4);
   g.total = off;
   return g;
 }
@@ -196,6 +201,7 @@ GroupedFns grouped_fns_t() {
   return {grouped_prep_kernel<BR, BS>, grouped_gateup_kernel<BR, BS>, grouped_stage_act_kernel<BR, BS>,
           grouped_down_kernel<BR, BS>};
 }
+// (the combine and the router are independent of the code widths)
 GroupedFns grouped_fns(int br, int bs) {
   if (br == 4) return bs == 4 ? grouped_fns_t<4, 4>() : grouped_fns_t<4, 2>();
   return bs == 4 ? grouped_fns_t<2, 4>() : grouped_fns_t<2, 2>();
@@ -222,6 +228,7 @@ int launch_grouped(const fmoe_layer* L, const float* x, const float* residual, f
   a.tb.slot_expert = reinterpret_cast<int*>(w8 + gl.slot_expert);
   a.tb.slot_pair0 = reinterpret_cast<int*>(w8 + gl.slot_pair0);
   a.tb.pair_token = reinterpret_cast<int*>(w8 + gl.pair_token);
+  a.tb.pair_slot = reinterpret_cast<int*>(w8 + gl.pair_slot);
   a.tb.tok_pair = reinterpret_cast<int*>(w8 + gl.tok_pair);
   a.tb.tok_w = reinterpret_cast<float*>(w8 + gl.tok_w);
   a.tb.tok_sg = reinterpret_cast<float*>(w8 + gl.tok_sg);
@@ -230,9 +237,18 @@ int launch_grouped(const fmoe_layer* L, const float* x, const float* residual, f
   const bool separate = has_shared && bs != br;
   a.xs_s = reinterpret_cast<float4*>(w8 + (separate ? gl.xs_s : gl.xs_r));
   a.sf_s = reinterpret_cast<float2*>(w8 + (separate ? gl.sf_s : gl.sf_r));
-  a.act = reinterpret_cast<float*>(w8 + gl.act);
+  a.gu_part = reinterpret_cast<float2*>(w8 + gl.gu_part);
   a.as = reinterpret_cast<float4*>(w8 + gl.as);
   a.sfa = reinterpret_cast<float2*>(w8 + gl.sfa);
+  a.y_part = reinterpret_cast<float*>(w8 + gl.y_part);
+  a.sh_gu = reinterpret_cast<float*>(w8 + gl.sh_gu);
+  a.sh_y = reinterpret_cast<float*>(w8 + gl.sh_y);
+  a.w_router = L->w_router;
+  a.w_sgate = L->w_sgate;
+  // The shared expert runs on the tensor cores when its matrices tile into
+  // 128-row x 512-input tiles; otherwise it is one more slot of the CUDA-core
+  // kernels.
+  a.shared_tc = has_shared && H % kTcK == 0 && I % kTcK == 0;
   a.idx_out = idx_out;
   a.w_out = w_out;
   a.H = H;
@@ -254,39 +270,52 @@ int launch_grouped(const fmoe_layer* L, const float* x, const float* residual, f
     d[4] = o.dc;
     d[5] = o.dsb;
   }
-  // Shared-memory plans: gate/up ring, down ring + per-pair results.
+  // Shared-memory plans: per-warp rings of gate/up stages (full-row sized:
+  // gate and up codes, each row's scale/bias superset) and of down stages
+  // (kRC code rows and one scale/bias copy spanning them).
   int stage = 0, cstage = 0;
   for (int b : {br, bs}) {
     const int cap = ((H / 16 + 15) & ~15) + 16;
     stage = std::max(stage, 2 * (H * b / 8) + 2 * cap);
-    cstage = std::max(cstage, kRC * (I * b / 8 + I / 16));
+    cstage = std::max(cstage, kRC * (I * b / 8) + (int)round_up((size_t)kRC * (I / 16), 16) + 32);
   }
   a.stage_bytes = (int)round_up(stage, 128);
   a.c_stage_bytes = (int)round_up(cstage, 128);
   const int budget = info->grouped_max_smem;
   a.nst = std::min(kMaxNst, (budget - kWarps * kMaxNst * 8) / (kWarps * a.stage_bytes));
-  a.ys_stride = kRC * ((H / kRC + G - 1) / G);
-  const size_t ys_bytes = round_up((size_t)kMaxPairs * a.ys_stride * 4, 16);
-  a.nst_c = std::min(kMaxNstC, (int)((budget - (long long)ys_bytes - kWarps * kMaxNstC * 8) /
-                                     ((long long)kWarps * a.c_stage_bytes)));
+  a.nst_c = std::min(kMaxNstC, (budget - kWarps * kMaxNstC * 8) / (kWarps * a.c_stage_bytes));
   if (a.nst < 1 || a.nst_c < 1) return FMOE_EINVAL;
   const size_t smem_gu = (size_t)kWarps * a.nst * a.stage_bytes + (size_t)kWarps * a.nst * 8;
-  const size_t smem_d = (size_t)kWarps * a.nst_c * a.c_stage_bytes + ys_bytes + (size_t)kWarps * a.nst_c * 8;
+  const size_t smem_d = (size_t)kWarps * a.nst_c * a.c_stage_bytes + (size_t)kWarps * a.nst_c * 8;
   const GroupedFns fns = grouped_fns(br, bs);
   const int fi = layer_fn_index(br, bs);
+  const GroupedFn tc1 = bs == 4 ? router_shared_gu_kernel<4> : router_shared_gu_kernel<2>;
+  const GroupedFn tc2 = br == 4 ? (bs == 4 ? prep_shared_down_kernel<4, 4> : prep_shared_down_kernel<4, 2>)
+                                : (bs == 4 ? prep_shared_down_kernel<2, 4> : prep_shared_down_kernel<2, 2>);
   if (!info->grouped_attr_set[fi]) {
     for (GroupedFn f : {fns.gateup, fns.down})
       if (cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, budget))
         return cuda_fail(e);
+    for (GroupedFn f : {tc1, tc2})
+      if (cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes))
+        return cuda_fail(e);
     info->grouped_attr_set[fi] = true;
   }
   const int rows = E + (L->w_sgate ? 1 : 0);
-  router_logits_kernel<<<(rows + 7) / 8, 256, 0, s>>>(L->w_router, L->w_sgate, x, T, H, E,
-                                                      const_cast<float*>(a.logits));
-  fns.prep<<<1 + T, kThreads, 0, s>>>(a);
+  const int router_ctas = (rows + kRouterRows - 1) / kRouterRows;
+  if (a.shared_tc) {
+    const int n_gu = 2 * (I / kTcRows) * (H / kTcK), n_down = (H / kTcRows) * (I / kTcK);
+    tc1<<<std::max(router_ctas, n_gu), kThreads, kTcSmemBytes, s>>>(a);
+    tc2<<<1 + T + n_down, kThreads, kTcSmemBytes, s>>>(a);
+  } else {
+    router_tokens_kernel<<<router_ctas, kThreads, 0, s>>>(L->w_router, L->w_sgate, x, T, H, E,
+                                                         const_cast<float*>(a.logits));
+    fns.prep<<<1 + T, kThreads, 0, s>>>(a);
+  }
   fns.gateup<<<G, kThreads, smem_gu, s>>>(a);
-  fns.stage<<<T * K + T, 256, 0, s>>>(a);
+  fns.stage<<<T * K + T, kStageThreads, (size_t)I * 4, s>>>(a);
   fns.down<<<G, kThreads, smem_d, s>>>(a);
+  grouped_combine_kernel<<<(unsigned)(((long long)T * H + 255) / 256), 256, 0, s>>>(a);
   if (cudaError_t e = cudaGetLastError()) return cuda_fail(e);
   return FMOE_OK;
 }

@@ -9,21 +9,29 @@
 // expert chosen by n tokens are read once and applied to all n.
 //
 // Steps (one launch each, all on the caller's stream):
-//   router   logits[t][e] for every token, each router row read once
-//            (router_logits_kernel);
+//   router   logits[t][e] for every token; each CTA owns a few router rows and
+//            reads every token's input once;
 //   prep     CTA 0: top-K per token (one warp each), then the grouping: the
 //            (token, k) pairs sorted by (expert, token), one slot per distinct
 //            expert in ascending expert order, the shared expert last with all
 //            T tokens; CTAs 1..T: each token's input staged in the decode
 //            layouts (stage_inputs) into the workspace;
-//   gate/up  every (slot, row) unit reads the gate and up rows once and
-//            produces silu(g) * u for each token of the slot;
-//   stage    each pair's activation vector staged for the down projection;
-//   down     each CTA owns a block of output rows; for every slot it reads the
-//            down rows of its block once and applies them to each token of the
-//            slot; then the combine, per token in fixed k order.
-// No float atomics anywhere: results are bitwise reproducible and equal for a
-// token whatever else is in the batch, up to the order of the combine.
+//   gate/up  units (slot, input chunk, row); every unit reads its gate and up
+//            row chunk once and applies it to each token of the slot, giving
+//            partial dot products per chunk;
+//   stage    per pair: the chunk partials summed in order, silu(g) * u, and the
+//            activation staged for the down projection;
+//   down     units (slot, input chunk, 4 output rows), as gate/up;
+//   combine  per token and output row: residual + sum_k w_k y_k + sg * y_shared
+//            with each y summed over its chunks in order.
+// Scheduling of gate/up and down: the units are ordered (slot, chunk, row)
+// and cut into one contiguous range per CTA of equal estimated cost (bytes
+// plus per-token work); inside a CTA consecutive units go to consecutive
+// warps, so the warps of a CTA work on the same slot and chunk at the same
+// time and share its staged inputs through L1.  A slot with many tokens has
+// its inputs split into chunks so that one chunk of all its tokens' inputs
+// stays within a fixed budget.  No float atomics: every sum has a fixed
+// order, so results are bitwise reproducible.
 #pragma once
 #include "route_quant_kernels.cuh"
 
@@ -31,7 +39,24 @@ namespace fmoe {
 
 constexpr int kMaxTokens = 16;
 constexpr int kMaxPairs = kMaxTokens * kMaxTopK + kMaxTokens;
-constexpr int kUnitCostBase = 2;  // gate/up unit cost = kUnitCostBase + tokens of its slot
+constexpr int kMaxChunks = 8;              // input chunks per slot, at most
+constexpr int kChunkBudget = 32 << 10;     // bytes of staged inputs of one (slot, chunk)
+constexpr int kUnitCostBase = 2;           // unit cost = chunk length * (kUnitCostBase + tokens)
+constexpr int kRouterRows = 4;             // router rows per CTA
+
+// Chunks the n_in inputs of a slot with n_tok tokens are split into: the
+// fewest (a divisor of n_in / 64, at most kMaxChunks) that keep n_tok chunks of
+// staged fp32 inputs within kChunkBudget, else the most allowed.
+__host__ __device__ inline int input_chunks(int n_tok, int n_in) {
+  const int ng = n_in / 64;
+  int best = 1;
+  for (int d = 1; d <= kMaxChunks && d <= ng; ++d) {
+    if (ng % d) continue;
+    best = d;
+    if ((long long)n_tok * (n_in / d) * 4 <= kChunkBudget) return d;
+  }
+  return best;
+}
 
 // Grouping tables (workspace).
 struct GroupTables {
@@ -39,6 +64,7 @@ struct GroupTables {
   int* slot_expert;  // [slots] expert id, -1 = the shared expert
   int* slot_pair0;   // [slots + 1] first pair of each slot
   int* pair_token;   // [pairs]
+  int* pair_slot;    // [pairs]
   int* tok_pair;     // [T][K + 1] pair of (t, k); column K: the shared pair (-1 if none)
   float* tok_w;      // [T][K]
   float* tok_sg;     // [T]
@@ -53,45 +79,126 @@ struct GroupArgs {
   float* out;             // [T][H]
   const float* logits;    // [T][E + 1]
   GroupTables tb;
-  float4* xs_r;  // [T][H/4] staged inputs for the routed code width
-  float2* sf_r;  // [T][H*BR/128]
-  float4* xs_s;  // same for the shared expert's width (aliases xs_r when equal)
+  float4* xs_r;     // [T][H/4] staged inputs for the routed code width
+  float2* sf_r;     // [T][H*BR/128]
+  float4* xs_s;     // same for the shared expert's width (aliases xs_r when equal)
   float2* sf_s;
-  float* act;    // [pairs][I] silu(g) * u
-  float4* as;    // [pairs][I/4] staged activations
-  float2* sfa;   // [pairs][I/32]
-  int* idx_out;  // optional [T][K]
-  float* w_out;  // optional [T][K]
+  float2* gu_part;  // [pairs][kMaxChunks][I] {gate, up} partial dot products
+  float4* as;       // [pairs][I/4] staged activations
+  float2* sfa;      // [pairs][I/32]
+  float* y_part;    // [pairs][kMaxChunks][H] partial down projections
+  int* idx_out;     // optional [T][K]
+  float* w_out;     // optional [T][K]
+  const uint16_t* w_router;  // [E][H] bf16
+  const uint16_t* w_sgate;   // [H] bf16 or null
+  float* sh_gu;     // tensor-core shared expert: [2][H/512][16][I] gate/up partials
+  float* sh_y;      // [I/512][16][H] down partials
   int H, I, E, K, T, bits_r, bits_s;
   int has_sgate;
+  int shared_tc;    // the shared expert runs on the tensor cores (not as a slot)
   int nst, stage_bytes;      // gate/up ring
   int nst_c, c_stage_bytes;  // down ring
-  int ys_stride;             // rows per CTA (max) of the down results
   long long off_r[6], off_s[6];
   unsigned long long timeout_ns;
 };
 
 // ---------------------------------------------------------------------------
+// router: logits[t][r] = W_r[r] . x[t] (row E: the shared gate vector)
+// ---------------------------------------------------------------------------
+// Router rows r0 .. r0 + kRouterRows - 1 for all T tokens; all threads of the
+// CTA call it.  Each thread takes 16-byte weight vectors of the rows and the
+// matching inputs of every token; per-warp sums are combined in fixed order.
+__device__ __noinline__ void router_rows_tokens(const uint16_t* __restrict__ w_router,
+                                                const uint16_t* __restrict__ w_sgate, const float* __restrict__ x,
+                                                int T, int H, int E, int r0, float* __restrict__ logits) {
+  __shared__ float part[kWarps][kRouterRows * kMaxTokens];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int rows = E + (w_sgate ? 1 : 0);
+  float acc[kRouterRows][kMaxTokens];
+#pragma unroll
+  for (int r = 0; r < kRouterRows; ++r)
+#pragma unroll
+    for (int t = 0; t < kMaxTokens; ++t) acc[r][t] = 0.f;
+  const int nv = H / 8;  // 16-byte vectors of 8 bf16 weights
+  for (int v = tid; v < nv; v += kThreads) {
+    uint4 w[kRouterRows];
+#pragma unroll
+    for (int r = 0; r < kRouterRows; ++r) {
+      const int row = r0 + r;
+      w[r] = make_uint4(0u, 0u, 0u, 0u);
+      if (row < rows) w[r] = ld_stream_u4((row < E ? w_router + (long long)row * H : w_sgate) + 8 * v);
+    }
+#pragma unroll
+    for (int t = 0; t < kMaxTokens; ++t) {
+      if (t < T) {
+        const float4* xt = reinterpret_cast<const float4*>(x + (long long)t * H) + 2 * v;
+        const float4 xa = __ldg(xt), xb = __ldg(xt + 1);
+#pragma unroll
+        for (int r = 0; r < kRouterRows; ++r) {
+          float s = acc[r][t];
+          s = fmaf(bf16_lo(w[r].x), xa.x, s);
+          s = fmaf(bf16_hi(w[r].x), xa.y, s);
+          s = fmaf(bf16_lo(w[r].y), xa.z, s);
+          s = fmaf(bf16_hi(w[r].y), xa.w, s);
+          s = fmaf(bf16_lo(w[r].z), xb.x, s);
+          s = fmaf(bf16_hi(w[r].z), xb.y, s);
+          s = fmaf(bf16_lo(w[r].w), xb.z, s);
+          s = fmaf(bf16_hi(w[r].w), xb.w, s);
+          acc[r][t] = s;
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < kRouterRows; ++r)
+#pragma unroll
+    for (int t = 0; t < kMaxTokens; ++t) {
+      if (t < T) {
+        const float s = warp_sum(acc[r][t]);
+        if (lane == 0) part[warp][r * kMaxTokens + t] = s;
+      }
+    }
+  __syncthreads();
+  if (tid < kRouterRows * T) {
+    const int r = tid / T, t = tid - r * T, row = r0 + r;
+    float s = 0.f;
+    for (int w = 0; w < kWarps; ++w) s += part[w][r * kMaxTokens + t];
+    if (row < rows) logits[(long long)t * (E + 1) + row] = s;
+  }
+  __syncthreads();  // `part` is reused by the next call
+}
+
+__global__ void __launch_bounds__(kThreads) router_tokens_kernel(const uint16_t* __restrict__ w_router,
+                                                                 const uint16_t* __restrict__ w_sgate,
+                                                                 const float* __restrict__ x, int T, int H, int E,
+                                                                 float* __restrict__ logits) {
+  router_rows_tokens(w_router, w_sgate, x, T, H, E, blockIdx.x * kRouterRows, logits);
+}
+
+// ---------------------------------------------------------------------------
 // prep: top-K per token, grouping, input staging
 // ---------------------------------------------------------------------------
+// CTA `b` of the prep step (0 <= b <= T): b = 0 routes and groups, b > 0
+// stages token b - 1's input.
 template <int BR, int BS>
-__global__ void __launch_bounds__(kThreads) grouped_prep_kernel(const __grid_constant__ GroupArgs a) {
+__device__ __noinline__ void prep_cta(const GroupArgs& a, int b) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (blockIdx.x > 0) {
-    const int t = blockIdx.x - 1;
+  const bool shared_slot = a.shared != nullptr && !a.shared_tc;  // the shared expert runs as a slot
+  if (b > 0) {
+    const int t = b - 1;
     const float* x = a.x + (long long)t * a.H;
     stage_inputs<BR, true>(x, a.H, a.xs_r + (long long)t * (a.H / 4), a.sf_r + (long long)t * (a.H * BR / 128), tid,
                            kThreads);
-    if (a.shared != nullptr && a.xs_s != a.xs_r)
+    if (shared_slot && a.xs_s != a.xs_r)
       stage_inputs<BS, true>(x, a.H, a.xs_s + (long long)t * (a.H / 4), a.sf_s + (long long)t * (a.H * BS / 128),
                              tid, kThreads);
     return;
   }
   __shared__ int s_idx[kMaxTokens * kMaxTopK];
   __shared__ float s_w[kMaxTokens * kMaxTopK];
-  __shared__ int s_rank[kMaxTokens * kMaxTopK];
   __shared__ int s_se[kMaxTokens * kMaxTopK];  // expert of sorted pair p
   __shared__ int s_start[kMaxTokens * kMaxTopK];
+  __shared__ int s_slot[kMaxTokens * kMaxTopK];
   const int T = a.T, K = a.K, NP = T * K;
   if (warp < T) {
     const float* lt = a.logits + (long long)warp * (a.E + 1);
@@ -99,15 +206,15 @@ __global__ void __launch_bounds__(kThreads) grouped_prep_kernel(const __grid_con
     if (lane == 0) a.tb.tok_sg[warp] = a.has_sgate ? sigmoidf_(__ldcg(lt + a.E)) : 1.0f;
   }
   __syncthreads();
-  // Rank of pair j = t*K + k in (expert, j) order, i.e. (expert, token) order
-  // since a token's top-K experts are distinct; ties on j keep the ranks a
-  // permutation whatever the indices are.
   if (tid < NP) {
     int e = s_idx[tid];
     if (e < 0 || e >= a.E) e = 0;  // (cannot happen: top-K indices lie in [0, E))
     s_idx[tid] = e;
   }
   __syncthreads();
+  // Rank of pair j = t*K + k in (expert, j) order, i.e. (expert, token) order
+  // since a token's top-K experts are distinct; ties on j keep the ranks a
+  // permutation whatever the indices are.
   if (tid < NP) {
     const int e = s_idx[tid], t = tid / K;
     int rank = 0;
@@ -115,7 +222,6 @@ __global__ void __launch_bounds__(kThreads) grouped_prep_kernel(const __grid_con
       const int e2 = s_idx[j];
       rank += (e2 < e) || (e2 == e && j < tid);
     }
-    s_rank[tid] = rank;
     s_se[rank] = e;
     a.tb.pair_token[rank] = t;
     a.tb.tok_pair[t * (K + 1) + tid % K] = rank;
@@ -126,21 +232,28 @@ __global__ void __launch_bounds__(kThreads) grouped_prep_kernel(const __grid_con
   __syncthreads();
   if (tid < NP) s_start[tid] = (tid == 0) || s_se[tid] != s_se[tid - 1];
   __syncthreads();
-  if (tid < NP && s_start[tid]) {
+  if (tid < NP) {
     int slot = -1;
     for (int j = 0; j <= tid; ++j) slot += s_start[j];
-    a.tb.slot_expert[slot] = s_se[tid];
-    a.tb.slot_pair0[slot] = tid;
+    s_slot[tid] = slot;
+    a.tb.pair_slot[tid] = slot;
+    if (s_start[tid]) {
+      a.tb.slot_expert[slot] = s_se[tid];
+      a.tb.slot_pair0[slot] = tid;
+    }
   }
+  __syncthreads();
+  const int nr = NP > 0 ? s_slot[NP - 1] + 1 : 0;
   if (tid < T) {
-    a.tb.tok_pair[tid * (K + 1) + K] = a.shared != nullptr ? NP + tid : -1;
-    if (a.shared != nullptr) a.tb.pair_token[NP + tid] = tid;
+    a.tb.tok_pair[tid * (K + 1) + K] = shared_slot ? NP + tid : -1;
+    if (shared_slot) {
+      a.tb.pair_token[NP + tid] = tid;
+      a.tb.pair_slot[NP + tid] = nr;
+    }
   }
   if (tid == 0) {
-    int nr = 0;
-    for (int j = 0; j < NP; ++j) nr += s_start[j];
     int ns = nr, np = NP;
-    if (a.shared != nullptr) {
+    if (shared_slot) {
       a.tb.slot_expert[nr] = -1;
       a.tb.slot_pair0[nr] = NP;
       ns = nr + 1;
@@ -152,91 +265,242 @@ __global__ void __launch_bounds__(kThreads) grouped_prep_kernel(const __grid_con
   }
 }
 
-// ---------------------------------------------------------------------------
-// gate/up
-// ---------------------------------------------------------------------------
-
-// First unit (flattened slot * I + row) whose cost interval starts at or after
-// `target`; slot s's units each cost kUnitCostBase + n_s.
-__device__ __forceinline__ int first_unit(long long target, const int* pair0, int ns, int I) {
-  long long cc = 0;
-  for (int s = 0; s < ns; ++s) {
-    const long long c = kUnitCostBase + (pair0[s + 1] - pair0[s]);
-    const long long span = c * I;
-    if (target < cc + span) return s * I + (int)((target - cc + c - 1) / c);
-    cc += span;
-  }
-  return ns * I;
+template <int BR, int BS>
+__global__ void __launch_bounds__(kThreads) grouped_prep_kernel(const __grid_constant__ GroupArgs a) {
+  prep_cta<BR, BS>(a, blockIdx.x);
 }
 
-template <int BR, int BS>
-__global__ void __launch_bounds__(kThreads, 1) grouped_gateup_kernel(const __grid_constant__ GroupArgs a) {
-  extern __shared__ __align__(128) char smem_raw[];
-  __shared__ int s_pair0[kMaxPairs + 2];
-  __shared__ int s_expert[kMaxPairs + 1];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// ---------------------------------------------------------------------------
+// Unit scheduling shared by gate/up and down
+// ---------------------------------------------------------------------------
+// Units of slot s: input_chunks(n_s, kin) chunks x ru row units, chunk-major.
+struct CtaSched {
+  int ns;
+  int* pair0;   // [ns + 1]
+  int* expert;  // [ns]
+  int* nk;      // [ns]
+  int* ubase;   // [ns + 1] units before slot s
+  int u0, u1;   // this CTA's units
+};
+
+// Load the slot tables and cut this CTA's range; all threads call it.
+__device__ inline void cta_sched(const GroupArgs& a, int kin, int ru, CtaSched& cs, int* s_pair0, int* s_expert,
+                                 int* s_nk, int* s_ubase, int* s_range) {
+  const int tid = threadIdx.x;
   const int ns = a.tb.meta[0];
-  for (int s = tid; s <= ns; s += kThreads) {
+  for (int s = tid; s <= ns; s += blockDim.x) {
     s_pair0[s] = a.tb.slot_pair0[s];
     if (s < ns) s_expert[s] = a.tb.slot_expert[s];
   }
+  __syncthreads();
+  if (tid == 0) {
+    long long total = 0;
+    int ub = 0;
+    for (int s = 0; s < ns; ++s) {
+      const int n = s_pair0[s + 1] - s_pair0[s];
+      s_nk[s] = input_chunks(n, kin);
+      s_ubase[s] = ub;
+      ub += s_nk[s] * ru;
+      total += (long long)ru * kin * (kUnitCostBase + n);
+    }
+    s_ubase[ns] = ub;
+    // first unit whose cost interval starts at or after `target`
+    auto first_unit = [&](long long target) {
+      long long cc = 0;
+      for (int s = 0; s < ns; ++s) {
+        const int n = s_pair0[s + 1] - s_pair0[s];
+        const long long uc = (long long)(kin / s_nk[s]) * (kUnitCostBase + n);
+        const long long span = uc * s_nk[s] * ru;
+        if (target < cc + span) return s_ubase[s] + (int)((target - cc + uc - 1) / uc);
+        cc += span;
+      }
+      return s_ubase[ns];
+    };
+    const long long G = gridDim.x, b = blockIdx.x;
+    s_range[0] = first_unit(total * b / G);
+    s_range[1] = first_unit(total * (b + 1) / G);
+  }
+  __syncthreads();
+  cs.ns = ns;
+  cs.pair0 = s_pair0;
+  cs.expert = s_expert;
+  cs.nk = s_nk;
+  cs.ubase = s_ubase;
+  cs.u0 = s_range[0];
+  cs.u1 = s_range[1];
+}
+
+// (slot, chunk, row unit) of unit u; `s` is a cursor that only moves forward.
+__device__ __forceinline__ void locate(const CtaSched& cs, int ru, int u, int& s, int& c, int& r) {
+  while (cs.ubase[s + 1] <= u) ++s;
+  const int w = u - cs.ubase[s];
+  c = w / ru;
+  r = w - c * ru;
+}
+
+// ---------------------------------------------------------------------------
+// Dot products over one input chunk
+// ---------------------------------------------------------------------------
+// Gate and up row chunks (nvc vectors each) against one token's staged input:
+// vectors v0 .. v0+nvc-1 of a [F4][NV] staged array.
+template <int BITS>
+__device__ __forceinline__ void gu_dot_chunk(const char* st, int nvc, int cb, int cap, int sbo_g, int sbo_u,
+                                             const float4* xs, int NV, int v0, const float2* sf, int lane,
+                                             float& g_out, float& u_out) {
+  const uint4* cg = reinterpret_cast<const uint4*>(st);
+  const uint4* cu = reinterpret_cast<const uint4*>(st + cb);
+  const uint32_t* sbg = reinterpret_cast<const uint32_t*>(st + 2 * cb + sbo_g);
+  const uint32_t* sbu = reinterpret_cast<const uint32_t*>(st + 2 * cb + cap + sbo_u);
+  const ulonglong2* xv = reinterpret_cast<const ulonglong2*>(xs) + v0;
+  float g = 0.f, u = 0.f;
+  for (int v = lane; v < nvc; v += 32) {
+    const uint4 wg = cg[v], wu = cu[v];
+    const int grp = (BITS == 4) ? (v >> 1) : v;
+    const uint32_t sbgw = sbg[grp], sbuw = sbu[grp];
+    const float2 f = __ldg(sf + v0 + v);
+    uint64_t ag = 0, au = 0;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const uint32_t a_ = (&wg.x)[t], b_ = (&wu.x)[t];
+      if (BITS == 4) {
+        const ulonglong2 xa = __ldg(xv + (2 * t) * NV + v), xb = __ldg(xv + (2 * t + 1) * NV + v);
+        dot_word4(ag, a_, xa, xb);
+        dot_word4(au, b_, xa, xb);
+      } else {
+        const ulonglong2 x0 = __ldg(xv + (4 * t) * NV + v), x1 = __ldg(xv + (4 * t + 1) * NV + v);
+        const ulonglong2 x2 = __ldg(xv + (4 * t + 2) * NV + v), x3 = __ldg(xv + (4 * t + 3) * NV + v);
+        dot_word2(ag, a_, x0, x1, x2, x3);
+        dot_word2(au, b_, x0, x1, x2, x3);
+      }
+    }
+    const float2 dg = unpk_f32(ag), du = unpk_f32(au);
+    g = fmaf(bf16_lo(sbgw) * f.y, dg.x + dg.y, g);
+    g = fmaf(bf16_hi(sbgw), f.x, g);
+    u = fmaf(bf16_lo(sbuw) * f.y, du.x + du.y, u);
+    u = fmaf(bf16_hi(sbuw), f.x, u);
+  }
+  g_out = warp_sum(g);
+  u_out = warp_sum(u);
+}
+
+// kRC down-row chunks (nvc vectors each, rows cb bytes apart in the stage;
+// scale/bias words of row j at sbw + j * sb_stride) against one staged
+// activation (vectors v0 .. v0+nvc-1 of a [F4][NV] array).
+template <int BITS>
+__device__ __forceinline__ void down_dot_chunk(const char* st, int nvc, int cb, const uint32_t* sbw, int sb_stride,
+                                               const float4* as, int NV, int v0, const float2* sfa, int lane,
+                                               float (&y)[kRC]) {
+  const ulonglong2* xv = reinterpret_cast<const ulonglong2*>(as) + v0;
+#pragma unroll
+  for (int r = 0; r < kRC; ++r) y[r] = 0.f;
+  for (int v = lane; v < nvc; v += 32) {
+    uint4 w[kRC];
+#pragma unroll
+    for (int r = 0; r < kRC; ++r) w[r] = reinterpret_cast<const uint4*>(st + r * cb)[v];
+    const float2 f = __ldg(sfa + v0 + v);
+    const int grp = (BITS == 4) ? (v >> 1) : v;
+    uint64_t ac[kRC];
+#pragma unroll
+    for (int r = 0; r < kRC; ++r) ac[r] = 0;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      if (BITS == 4) {
+        const ulonglong2 xa = __ldg(xv + (2 * t) * NV + v), xb = __ldg(xv + (2 * t + 1) * NV + v);
+#pragma unroll
+        for (int r = 0; r < kRC; ++r) dot_word4(ac[r], (&w[r].x)[t], xa, xb);
+      } else {
+        const ulonglong2 x0 = __ldg(xv + (4 * t) * NV + v), x1 = __ldg(xv + (4 * t + 1) * NV + v);
+        const ulonglong2 x2 = __ldg(xv + (4 * t + 2) * NV + v), x3 = __ldg(xv + (4 * t + 3) * NV + v);
+#pragma unroll
+        for (int r = 0; r < kRC; ++r) dot_word2(ac[r], (&w[r].x)[t], x0, x1, x2, x3);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kRC; ++r) {
+      const uint32_t sbv = sbw[r * sb_stride + grp];
+      const float2 d = unpk_f32(ac[r]);
+      y[r] = fmaf(bf16_lo(sbv) * f.y, d.x + d.y, y[r]);
+      y[r] = fmaf(bf16_hi(sbv), f.x, y[r]);
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < kRC; ++r) y[r] = warp_sum(y[r]);
+}
+
+// ---------------------------------------------------------------------------
+// gate/up
+// ---------------------------------------------------------------------------
+template <int BR, int BS>
+__global__ void __launch_bounds__(kThreads, 1) grouped_gateup_kernel(const __grid_constant__ GroupArgs a) {
+  extern __shared__ __align__(128) char smem_raw[];
+  __shared__ int s_pair0[kMaxPairs + 2], s_expert[kMaxPairs + 1], s_nk[kMaxPairs + 1], s_ubase[kMaxPairs + 2];
+  __shared__ int s_range[2];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   char* my_ring = smem_raw + (size_t)warp * a.nst * a.stage_bytes;
   uint64_t* my_bars = reinterpret_cast<uint64_t*>(smem_raw + (size_t)kWarps * a.nst * a.stage_bytes) + warp * a.nst;
   if (lane == 0) {
     for (int s = 0; s < a.nst; ++s) mbar_init(&my_bars[s], 1);
     fence_proxy_async_smem();
   }
-  __syncthreads();
-
-  // This warp's units: an equal share of the total cost, contiguous.
-  long long total = 0;
-  for (int s = 0; s < ns; ++s) total += (long long)(kUnitCostBase + s_pair0[s + 1] - s_pair0[s]) * a.I;
-  const long long GW = (long long)gridDim.x * kWarps, gw = (long long)blockIdx.x * kWarps + warp;
-  const int u0 = first_unit(total * gw / GW, s_pair0, ns, a.I);
-  const int u1 = first_unit(total * (gw + 1) / GW, s_pair0, ns, a.I);
-  const int n = u1 - u0;
-
+  CtaSched cs;
+  cta_sched(a, a.H, a.I, cs, s_pair0, s_expert, s_nk, s_ubase, s_range);  // includes __syncthreads
+  // this warp's units: cs.u0 + warp + i * kWarps
+  const int n = cs.u1 - cs.u0 > warp ? (cs.u1 - cs.u0 - warp - 1) / kWarps + 1 : 0;
   const int sbr = sb_row_bytes(a.H), cap = sb_superset_cap(a.H);
+
+  int s_issue = 0;
   auto issue = [&](int i) {  // lane 0
-    const int u = u0 + i, s = u / a.I, row = u - s * a.I;
-    const int e = s_expert[s];
+    int s, c, row;
+    locate(cs, a.I, cs.u0 + warp + i * kWarps, s_issue, c, row);
+    s = s_issue;
+    const int e = cs.expert[s];
+    const int bits = e >= 0 ? BR : BS;
     const char* blob = e >= 0 ? a.experts + (long long)e * a.expert_stride : a.shared;
     const long long* o = e >= 0 ? a.off_r : a.off_s;
-    const int cb = codes_row_bytes(a.H, e >= 0 ? BR : BS);
-    const long long gs0 = o[1] + (long long)row * sbr, us0 = o[3] + (long long)row * sbr;
+    const int cl = a.H / cs.nk[s];  // inputs per chunk
+    const int cb = cl * bits / 8;
+    const long long code0 = (long long)row * (a.H * bits / 8) + (long long)c * cb;
+    const long long gs0 = o[1] + (long long)row * sbr + c * (cl / 16), us0 = o[3] + (long long)row * sbr + c * (cl / 16);
     const long long ga = gs0 & ~15LL, ua = us0 & ~15LL;
-    const int glen = (int)(((gs0 + sbr + 15) & ~15LL) - ga);
-    const int ulen = (int)(((us0 + sbr + 15) & ~15LL) - ua);
+    const int glen = (int)(((gs0 + cl / 16 + 15) & ~15LL) - ga);
+    const int ulen = (int)(((us0 + cl / 16 + 15) & ~15LL) - ua);
     char* stage = my_ring + (size_t)(i % a.nst) * a.stage_bytes;
     uint64_t* bar = &my_bars[i % a.nst];
     mbar_arrive_expect_tx(bar, 2 * cb + glen + ulen);
-    bulk_g2s(stage, blob + o[0] + (long long)row * cb, cb, bar);
-    bulk_g2s(stage + cb, blob + o[2] + (long long)row * cb, cb, bar);
+    bulk_g2s(stage, blob + o[0] + code0, cb, bar);
+    bulk_g2s(stage + cb, blob + o[2] + code0, cb, bar);
     bulk_g2s(stage + 2 * cb, blob + ga, glen, bar);
     bulk_g2s(stage + 2 * cb + cap, blob + ua, ulen, bar);
   };
   if (lane == 0)
     for (int i = 0; i < n && i < a.nst; ++i) issue(i);
 
+  int s_cur = 0;
   for (int i = 0; i < n; ++i) {
     const char* stage = my_ring + (size_t)(i % a.nst) * a.stage_bytes;
     if (!mbar_wait_bounded(&my_bars[i % a.nst], (i / a.nst) & 1, a.timeout_ns) && lane == 0)
       set_status(kStatusCopyTimeout);
-    const int u = u0 + i, s = u / a.I, row = u - s * a.I;
-    const bool routed = s_expert[s] >= 0;
+    int c, row;
+    locate(cs, a.I, cs.u0 + warp + i * kWarps, s_cur, c, row);
+    const int s = s_cur;
+    const bool routed = cs.expert[s] >= 0;
+    const int cl = a.H / cs.nk[s];
     const BlobOff o = blob_offsets(a.H, a.I, routed ? BR : BS);
-    const int sbo_g = (int)((o.gsb + (long long)row * sbr) & 15);
-    const int sbo_u = (int)((o.usb + (long long)row * sbr) & 15);
-    for (int p = s_pair0[s]; p < s_pair0[s + 1]; ++p) {
+    const int sbo_g = (int)((o.gsb + (long long)row * sbr + c * (cl / 16)) & 15);
+    const int sbo_u = (int)((o.usb + (long long)row * sbr + c * (cl / 16)) & 15);
+    for (int p = cs.pair0[s]; p < cs.pair0[s + 1]; ++p) {
       const int t = a.tb.pair_token[p];
       float g, up;
-      if (routed || BR == BS)
-        pair_dot_src<BR, true>(stage, a.H, sbo_g, sbo_u, a.xs_r + (long long)t * (a.H / 4),
-                               a.sf_r + (long long)t * (a.H * BR / 128), lane, g, up);
-      else
-        pair_dot_src<BS, true>(stage, a.H, sbo_g, sbo_u, a.xs_s + (long long)t * (a.H / 4),
-                               a.sf_s + (long long)t * (a.H * BS / 128), lane, g, up);
-      if (lane == 0) a.act[(long long)p * a.I + row] = g * sigmoidf_(g) * up;
+      if (routed || BR == BS) {
+        constexpr int CPV = 128 / BR;
+        gu_dot_chunk<BR>(stage, cl / CPV, cl * BR / 8, cap, sbo_g, sbo_u, a.xs_r + (long long)t * (a.H / 4),
+                         a.H / CPV, c * (cl / CPV), a.sf_r + (long long)t * (a.H / CPV), lane, g, up);
+      } else {
+        constexpr int CPV = 128 / BS;
+        gu_dot_chunk<BS>(stage, cl / CPV, cl * BS / 8, cap, sbo_g, sbo_u, a.xs_s + (long long)t * (a.H / 4),
+                         a.H / CPV, c * (cl / CPV), a.sf_s + (long long)t * (a.H / CPV), lane, g, up);
+      }
+      if (lane == 0) a.gu_part[((long long)p * kMaxChunks + c) * a.I + row] = make_float2(g, up);
     }
     __syncwarp();
     if (lane == 0 && i + a.nst < n) {
@@ -247,87 +511,119 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gateup_kernel(const __gri
 }
 
 // ---------------------------------------------------------------------------
-// stage the activations (one CTA per pair)
+// stage: act = silu(g) * u from the chunk partials, staged for the down
+// projection (one CTA per pair)
 // ---------------------------------------------------------------------------
+constexpr int kStageThreads = 256;
+
 template <int BR, int BS>
-__global__ void __launch_bounds__(256) grouped_stage_act_kernel(const __grid_constant__ GroupArgs a) {
+__global__ void __launch_bounds__(kStageThreads) grouped_stage_act_kernel(const __grid_constant__ GroupArgs a) {
+  extern __shared__ __align__(16) float act[];  // [I]
   const int p = blockIdx.x;
   if (p >= a.tb.meta[1]) return;
-  const bool routed = p < a.T * a.K;
-  const float* src = a.act + (long long)p * a.I;
+  const int s = a.tb.pair_slot[p];
+  const int n = a.tb.slot_pair0[s + 1] - a.tb.slot_pair0[s];
+  const int nk = input_chunks(n, a.H);
+  const float2* part = a.gu_part + (long long)p * kMaxChunks * a.I;
+  for (int r = threadIdx.x; r < a.I; r += kStageThreads) {
+    float g = 0.f, u = 0.f;
+    for (int c = 0; c < nk; ++c) {
+      const float2 v = __ldcg(part + (long long)c * a.I + r);
+      g += v.x;
+      u += v.y;
+    }
+    act[r] = g * sigmoidf_(g) * u;
+  }
+  __syncthreads();
   float4* as = a.as + (long long)p * (a.I / 4);
   float2* sf = a.sfa + (long long)p * (a.I / 32);
-  if (routed || BR == BS)
-    stage_inputs<BR, true>(src, a.I, as, sf, threadIdx.x, blockDim.x);
+  if (a.tb.slot_expert[s] >= 0 || BR == BS)
+    stage_inputs<BR, false>(act, a.I, as, sf, threadIdx.x, kStageThreads);
   else
-    stage_inputs<BS, true>(src, a.I, as, sf, threadIdx.x, blockDim.x);
+    stage_inputs<BS, false>(act, a.I, as, sf, threadIdx.x, kStageThreads);
 }
 
 // ---------------------------------------------------------------------------
-// down + combine
+// down
 // ---------------------------------------------------------------------------
 template <int BR, int BS>
 __global__ void __launch_bounds__(kThreads, 1) grouped_down_kernel(const __grid_constant__ GroupArgs a) {
   extern __shared__ __align__(128) char smem_raw[];
-  __shared__ int s_pair0[kMaxPairs + 2];
-  __shared__ int s_expert[kMaxPairs + 1];
+  __shared__ int s_pair0[kMaxPairs + 2], s_expert[kMaxPairs + 1], s_nk[kMaxPairs + 1], s_ubase[kMaxPairs + 2];
+  __shared__ int s_range[2];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int G = gridDim.x;
-  const int ns = a.tb.meta[0];
-  for (int s = tid; s <= ns; s += kThreads) {
-    s_pair0[s] = a.tb.slot_pair0[s];
-    if (s < ns) s_expert[s] = a.tb.slot_expert[s];
-  }
   char* my_ring = smem_raw + (size_t)warp * a.nst_c * a.c_stage_bytes;
-  size_t off = (size_t)kWarps * a.nst_c * a.c_stage_bytes;
-  float* ys = reinterpret_cast<float*>(smem_raw + off);  // [pairs][ys_stride]
-  off += (size_t)kMaxPairs * a.ys_stride * 4;
-  uint64_t* my_bars = reinterpret_cast<uint64_t*>(smem_raw + off) + warp * a.nst_c;
+  uint64_t* my_bars =
+      reinterpret_cast<uint64_t*>(smem_raw + (size_t)kWarps * a.nst_c * a.c_stage_bytes) + warp * a.nst_c;
   if (lane == 0) {
     for (int s = 0; s < a.nst_c; ++s) mbar_init(&my_bars[s], 1);
     fence_proxy_async_smem();
   }
-  __syncthreads();
+  const int nq = a.H / kRC;
+  CtaSched cs;
+  cta_sched(a, a.I, nq, cs, s_pair0, s_expert, s_nk, s_ubase, s_range);
+  const int n = cs.u1 - cs.u0 > warp ? (cs.u1 - cs.u0 - warp - 1) / kWarps + 1 : 0;
+  const int sbr = sb_row_bytes(a.I);  // bytes of one row's scale/bias words
 
-  const int nq_all = a.H / kRC;
-  const int q0 = (int)((long long)blockIdx.x * nq_all / G);
-  const int nq = (int)((long long)(blockIdx.x + 1) * nq_all / G) - q0;
-  const int n_items = ns * nq;
-  const int n = n_items > warp ? (n_items - warp - 1) / kWarps + 1 : 0;  // items j = warp + i * kWarps
-  const int sbr = sb_row_bytes(a.I);
-
+  int s_issue = 0;
   auto issue = [&](int i) {  // lane 0
-    const int j = warp + i * kWarps, s = j / nq, r0 = (q0 + j - s * nq) * kRC;
-    const int e = s_expert[s];
+    int c, q;
+    locate(cs, nq, cs.u0 + warp + i * kWarps, s_issue, c, q);
+    const int s = s_issue;
+    const int e = cs.expert[s];
+    const int bits = e >= 0 ? BR : BS;
     const char* blob = e >= 0 ? a.experts + (long long)e * a.expert_stride : a.shared;
     const long long* o = e >= 0 ? a.off_r : a.off_s;
-    const int cb = codes_row_bytes(a.I, e >= 0 ? BR : BS);
+    const int cl = a.I / cs.nk[s];
+    const int cb = cl * bits / 8, rowb = a.I * bits / 8;
+    const long long r0 = (long long)q * kRC;
     char* stage = my_ring + (size_t)(i % a.nst_c) * a.c_stage_bytes;
     uint64_t* bar = &my_bars[i % a.nst_c];
-    mbar_arrive_expect_tx(bar, kRC * (cb + sbr));
-    bulk_g2s(stage, blob + o[4] + (long long)r0 * cb, kRC * cb, bar);
-    bulk_g2s(stage + kRC * cb, blob + o[5] + (long long)r0 * sbr, kRC * sbr, bar);
+    // kRC code row chunks, then one copy covering the rows' scale/bias chunks
+    const long long sb0 = o[5] + r0 * sbr + c * (cl / 16);
+    const long long sba = sb0 & ~15LL;
+    const int sblen = (int)(((sb0 + (kRC - 1) * sbr + cl / 16 + 15) & ~15LL) - sba);
+    mbar_arrive_expect_tx(bar, kRC * cb + sblen);
+    if (cs.nk[s] == 1) {
+      bulk_g2s(stage, blob + o[4] + r0 * rowb, kRC * cb, bar);
+    } else {
+#pragma unroll
+      for (int j = 0; j < kRC; ++j) bulk_g2s(stage + j * cb, blob + o[4] + (r0 + j) * rowb + (long long)c * cb, cb, bar);
+    }
+    bulk_g2s(stage + kRC * cb, blob + sba, sblen, bar);
   };
   if (lane == 0)
     for (int i = 0; i < n && i < a.nst_c; ++i) issue(i);
 
+  int s_cur = 0;
   for (int i = 0; i < n; ++i) {
     const char* stage = my_ring + (size_t)(i % a.nst_c) * a.c_stage_bytes;
     if (!mbar_wait_bounded(&my_bars[i % a.nst_c], (i / a.nst_c) & 1, a.timeout_ns) && lane == 0)
       set_status(kStatusCopyTimeout);
-    const int j = warp + i * kWarps, s = j / nq, rl = (j - s * nq) * kRC;
-    const bool routed = s_expert[s] >= 0;
-    for (int p = s_pair0[s]; p < s_pair0[s + 1]; ++p) {
+    int c, q;
+    locate(cs, nq, cs.u0 + warp + i * kWarps, s_cur, c, q);
+    const int s = s_cur;
+    const bool routed = cs.expert[s] >= 0;
+    const int cl = a.I / cs.nk[s];
+    const BlobOff o = blob_offsets(a.H, a.I, routed ? BR : BS);
+    const long long sb0 = o.dsb + (long long)q * kRC * sbr + c * (cl / 16);
+    const int bits = routed ? BR : BS;
+    const int cb = cl * bits / 8;
+    const uint32_t* sbw = reinterpret_cast<const uint32_t*>(stage + kRC * cb + (sb0 & 15));
+    for (int p = cs.pair0[s]; p < cs.pair0[s + 1]; ++p) {
       float y[kRC];
       const float4* as = a.as + (long long)p * (a.I / 4);
       const float2* sf = a.sfa + (long long)p * (a.I / 32);
-      if (routed || BR == BS)
-        down_rows_src<BR, true>(stage, a.I, as, a.I * BR / 128, 0, sf, lane, y);
-      else
-        down_rows_src<BS, true>(stage, a.I, as, a.I * BS / 128, 0, sf, lane, y);
+      if (routed || BR == BS) {
+        constexpr int CPV = 128 / BR;
+        down_dot_chunk<BR>(stage, cl / CPV, cb, sbw, sbr / 4, as, a.I / CPV, c * (cl / CPV), sf, lane, y);
+      } else {
+        constexpr int CPV = 128 / BS;
+        down_dot_chunk<BS>(stage, cl / CPV, cb, sbw, sbr / 4, as, a.I / CPV, c * (cl / CPV), sf, lane, y);
+      }
       if (lane == 0) {
-#pragma unroll
-        for (int r = 0; r < kRC; ++r) ys[p * a.ys_stride + rl + r] = y[r];
+        float* dst = a.y_part + ((long long)p * kMaxChunks + c) * a.H + (long long)q * kRC;
+        *reinterpret_cast<float4*>(dst) = make_float4(y[0], y[1], y[2], y[3]);
       }
     }
     __syncwarp();
@@ -336,18 +632,34 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_down_kernel(const __grid_
       issue(i + a.nst_c);
     }
   }
-  __syncthreads();
+}
 
-  // out[t] = residual[t] + sum_k w[t][k] y[pair(t,k)] + sg[t] y[shared pair of t], fixed order
-  const int rows = nq * kRC, K = a.K;
-  for (int q = tid; q < a.T * rows; q += kThreads) {
-    const int t = q / rows, rl = q - t * rows, h = q0 * kRC + rl;
-    float v = a.residual ? __ldg(a.residual + (long long)t * a.H + h) : 0.f;
-    const int* tp = a.tb.tok_pair + t * (K + 1);
-    for (int k = 0; k < K; ++k) v = fmaf(a.tb.tok_w[t * K + k], ys[tp[k] * a.ys_stride + rl], v);
-    if (tp[K] >= 0) v = fmaf(a.tb.tok_sg[t], ys[tp[K] * a.ys_stride + rl], v);
-    a.out[(long long)t * a.H + h] = v;
+// ---------------------------------------------------------------------------
+// combine: out[t] = residual[t] + sum_k w[t][k] y[pair(t,k)] + sg[t] y[shared pair of t]
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float pair_output(const GroupArgs& a, int p, int h) {
+  const int s = a.tb.pair_slot[p];
+  const int nk = input_chunks(a.tb.slot_pair0[s + 1] - a.tb.slot_pair0[s], a.I);
+  const float* y = a.y_part + (long long)p * kMaxChunks * a.H + h;
+  float v = 0.f;
+  for (int c = 0; c < nk; ++c) v += __ldcg(y + (long long)c * a.H);
+  return v;
+}
+
+__global__ void __launch_bounds__(256) grouped_combine_kernel(const __grid_constant__ GroupArgs a) {
+  const long long q = blockIdx.x * 256LL + threadIdx.x;
+  if (q >= (long long)a.T * a.H) return;
+  const int t = (int)(q / a.H), h = (int)(q - (long long)t * a.H);
+  float v = a.residual ? __ldg(a.residual + q) : 0.f;
+  const int* tp = a.tb.tok_pair + t * (a.K + 1);
+  for (int k = 0; k < a.K; ++k) v = fmaf(a.tb.tok_w[t * a.K + k], pair_output(a, tp[k], h), v);
+  if (tp[a.K] >= 0) v = fmaf(a.tb.tok_sg[t], pair_output(a, tp[a.K], h), v);
+  if (a.shared_tc) {
+    float y = 0.f;
+    for (int ks = 0; ks < a.I / 512; ++ks) y += __ldcg(a.sh_y + ((long long)ks * kMaxTokens + t) * a.H + h);
+    v = fmaf(a.tb.tok_sg[t], y, v);
   }
+  a.out[q] = v;
 }
 
 }  // namespace fmoe

@@ -331,14 +331,22 @@ def test_grouped_two_tokens_full(F, SG):
     (C.Shape("mixed_h1024_i256_e64_k8_r4_s2", 1024, 256, 64, 8, 4, 2), 16, True, True),
     (C.Shape("mixed_h1024_i256_e64_k1_r2_s4", 1024, 256, 64, 1, 2, 4), 3, True, True),
     (C.Shape("e1024_h2048_i256_k4", 2048, 256, 1024, 4, 4), 16, True, True),
-])
+    # H and I multiples of 512: the shared expert runs on the tensor cores
+    (C.Shape("tc_h1024_i512_e64_k4", 1024, 512, 64, 4, 4), 16, True, True),
+    (C.Shape("tc_h1024_i512_e32_k8_r2_s4", 1024, 512, 32, 8, 2, 4), 16, True, True),
+    (C.Shape("tc_h2048_i512_e64_k2_r4_s2", 2048, 512, 64, 2, 4, 2), 5, True, True),
+    (C.Shape("tc_ungated_h1024_i1024_e16_k4", 1024, 1024, 16, 4, 4), 3, True, False),
+], ids=lambda v: v.name if isinstance(v, C.Shape) else str(v))
 def test_grouped_edge_shapes(F, SG, shape, T, with_shared, with_sgate):
     run_grouped_case(F, SG, shape, T, with_shared=with_shared, with_sgate=with_sgate)
 
 
-def test_grouped_identical_tokens_share_every_expert(F, SG):
+@pytest.mark.parametrize("shape", [C.Shape("identical_h1024_i256_e64_k4", 1024, 256, 64, 4, 4),
+                                   C.Shape("identical_tc_h1024_i512_e64_k4", 1024, 512, 64, 4, 4)],
+                         ids=lambda v: v.name)
+def test_grouped_identical_tokens_share_every_expert(F, SG, shape):
     """All tokens equal: one slot per expert holding every token."""
-    run_grouped_case(F, SG, C.Shape("identical_h1024_i256_e64_k4", 1024, 256, 64, 4, 4), 16, identical=True)
+    run_grouped_case(F, SG, shape, 16, identical=True)
 
 
 def test_grouped_matches_single_token_calls(F, SG):

@@ -1,5 +1,5 @@
 /*
- * fmoe — single-token quantised Mixture-of-Experts layer decode on NVIDIA B200
+ * fmoe — quantised Mixture-of-Experts layer decode (one token or a few) on NVIDIA B200
  * (sm_100a).  C ABI of libfmoe.so.
  *
  * What the library computes is the MoE step of the Flash-MoE engine, as its
@@ -168,7 +168,12 @@ int fmoe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream_t stream);
  *   ws: workspace of ws_bytes >= fmoe_workspace_bytes(L, T), zero-filled
  *   before its first use; calls sharing a workspace must be stream-ordered.
  * The whole layer runs on the GPU; the routing decision never returns to the
- * host.  Limits: as fmoe_route and fmoe_expert_forward, plus
+ * host.  T = 1 runs one persistent kernel.  T >= 2 groups the tokens by
+ * expert: every distinct selected expert's weights are read once per call and
+ * applied to each token that chose it, and the shared expert (every token)
+ * runs on the tensor cores when hidden and inter are multiples of 512; each
+ * token's result is the single-token result (same routing, outputs within
+ * fp32 rounding).  Limits: as fmoe_route and fmoe_expert_forward, plus
  * (top_k + 1) * inter <= 10240.  Errors: FMOE_EINVAL, FMOE_ENOMEM, FMOE_ECUDA.
  * Kernel-side problems (a time-limited wait that ran out) are reported by
  * fmoe_get_status(). */

@@ -568,6 +568,8 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
   a.c_stage_bytes = pl.c_stage_bytes;
   a.lg_floats = pl.lg_floats;
   a.timeout_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  // A router warp's row (2H bytes) fits in its ring: copy it there at entry.
+  a.router_smem = (long long)pl.nst * pl.stage_bytes >= 2LL * H ? 1 : 0;
   set_offsets(a, info->sms);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (T > 1) return launch_grouped(L, x, residual, out, T, ws, idx_out_opt, w_out_opt, info, s);

@@ -16,10 +16,10 @@
 //      block of output rows, then the combine (need all SwiGLU activations).
 // Units of phases A and B are dealt round-robin over all warps of the grid.
 //
-// Hand-offs.  Each CTA publishes its router logits and then bumps a grid
-// counter once (after a fence); each CTA's first warp that needs the routing
-// decision polls that counter, reads the logits and runs the top-K, then wakes
-// the CTA's other warps through an mbarrier.  "All activations written" is a
+// Hand-offs.  Each router warp stores its logit and counts it with one
+// release add on a grid counter; each CTA's first warp that needs the routing
+// decision polls until every router row is counted, reads the logits and runs
+// the top-K, then wakes the CTA's other warps through an mbarrier.  "All activations written" is a
 // second counter that every CTA bumps once and polls once.  Every wait is
 // time-limited: on expiry the kernel sets a status bit and carries on instead
 // of hanging.
@@ -48,7 +48,7 @@ constexpr int kMaxNstC = 8;       // most down-item stages a warp keeps in fligh
 // Optional phase trace (compile with -DFMOE_TRACE_BUILD): thread 0 of every CTA
 // stores %globaltimer at fixed points of the kernel into g_fmoe_trace.
 #ifdef FMOE_TRACE_BUILD
-constexpr int kTracePoints = 16;
+constexpr int kTracePoints = 24;
 __device__ unsigned long long g_fmoe_trace[1024][kTracePoints];
 #define FMOE_TRACE(i) \
   do { if (threadIdx.x == 0 && blockIdx.x < 1024) g_fmoe_trace[blockIdx.x][i] = globaltimer_ns(); } while (0)
@@ -71,7 +71,7 @@ struct LayerArgs {
   float* out;                // [H]
   float* logits;             // workspace [E + 1]
   float* act;                // workspace [n_slots][I]
-  unsigned* bar;             // workspace: [0] logits hand-off, [1] activation hand-off, [2] done ticket
+  unsigned* bar;             // workspace: [0] router rows published, [1] CTAs past gate/up, [2] done ticket
   int* idx_out;              // optional [K]
   float* w_out;              // optional [K]
   float* sg_out;             // optional [1]
@@ -89,6 +89,7 @@ struct LayerArgs {
   int lg_floats;             // shared-memory logits (n_router rounded up to 4)
   long long off_r[6], off_s[6];  // blob section offsets for the routed / shared code width
   unsigned long long timeout_ns;
+  int router_smem;           // 1: each router warp's row is bulk-copied into its ring at entry
 };
 
 struct Smem {
@@ -165,12 +166,12 @@ struct CtaShared {
   uint64_t x_bar;       // completes once x is in shared memory
   uint64_t staged_bar;  // completes once x is staged in the decode layouts
   uint64_t lg_bar;      // completes once the router logits are in shared memory
+  uint64_t rbar[kWarps];  // router warp w's row is in its ring (router_smem)
+  unsigned long long param_touch;  // see the kernel's set-up
   float* lg;            // shared-memory copy of the router logits
   unsigned lg_bytes;
   int route_state;      // 0 = not started, 1 = being computed, 2 = ready
   int c_prefetch;          // warps past their gate/up work (the first prefetches down rows)
-  unsigned router_done;    // this CTA's router rows published so far
-  unsigned router_target;  // this CTA's router rows
   int idx[kMaxTopK];
   float w[kMaxTopK];
   float sg;
@@ -289,6 +290,26 @@ __device__ __forceinline__ float router_dot(const uint16_t* row, const float* xu
   return warp_sum(acc);
 }
 
+// The same dot product with the row in shared memory.
+__device__ __forceinline__ float router_dot_smem(const uint16_t* row, const float* xu, int H, int lane) {
+  const uint4* rv = reinterpret_cast<const uint4*>(row);
+  const float4* xv = reinterpret_cast<const float4*>(xu);
+  float acc0 = 0.f, acc1 = 0.f;
+  for (int v = lane; v < H / 8; v += 32) {
+    const uint4 w = rv[v];
+    const float4 xa = xv[2 * v], xb = xv[2 * v + 1];
+    acc0 = fmaf(bf16_lo(w.x), xa.x, acc0);
+    acc1 = fmaf(bf16_hi(w.x), xa.y, acc1);
+    acc0 = fmaf(bf16_lo(w.y), xa.z, acc0);
+    acc1 = fmaf(bf16_hi(w.y), xa.w, acc1);
+    acc0 = fmaf(bf16_lo(w.z), xb.x, acc0);
+    acc1 = fmaf(bf16_hi(w.z), xb.y, acc1);
+    acc0 = fmaf(bf16_lo(w.w), xb.z, acc0);
+    acc1 = fmaf(bf16_hi(w.w), xb.w, acc1);
+  }
+  return warp_sum(acc0 + acc1);
+}
+
 // Gate and up rows of one expert (stage layout: gate codes | up codes | gate sb
 // superset | up sb superset) against the staged input.
 template <int BITS, bool kG>
@@ -396,13 +417,11 @@ __device__ __forceinline__ void down_rows(const char* st, int I, const float4* a
 }
 
 // Top-K by one warp: descending logit, lower index first on exact ties; then
-// renormalised softmax weights over the selected logits.  Each (logit, index)
-// pair is one 64-bit key whose unsigned order is that order: order-preserving
-// float bits above, the complemented index below.  Each lane holds 32 keys in
-// registers and its current maximum; a round is one warp-wide hardware max
-// (__reduce_max_sync) of the maxima's upper halves, one of the lower halves
-// among the lanes that hold that upper half, and a rescan by the single lane
-// that owned the winner.
+// renormalised softmax weights over the selected logits.  Logits become
+// 32-bit keys whose unsigned order is the float order; each lane holds its
+// keys in registers with the position of its largest; a round is one
+// warp-wide hardware max of the lanes' largest keys, one hardware min of the
+// expert indices that hold it (the tie rule), and a rescan by the winner lane.
 __device__ __forceinline__ uint32_t order_bits(float v) {
   const uint32_t u = __float_as_uint(v);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
@@ -410,54 +429,44 @@ __device__ __forceinline__ uint32_t order_bits(float v) {
 __device__ __forceinline__ float from_order_bits(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
-__device__ __forceinline__ unsigned long long umax64(unsigned long long p, unsigned long long q) {
-  return p > q ? p : q;
-}
-template <int NK>
-__device__ __forceinline__ unsigned long long max_tree(const unsigned long long (&key)[NK]) {
-  unsigned long long m[NK / 2];
-#pragma unroll
-  for (int i = 0; i < NK / 2; ++i) m[i] = umax64(key[2 * i], key[2 * i + 1]);
-#pragma unroll
-  for (int w = NK / 4; w >= 1; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) m[i] = umax64(m[2 * i], m[2 * i + 1]);
-  return m[0];
-}
-
 // NK keys per lane (16 covers 512 experts, 32 covers 1024).  kShared: the
 // logits are in this CTA's shared memory, else in global memory.
 template <bool kShared, int NK>
 __device__ __noinline__ void warp_topk_n(const float* lg, int n, int k, int lane, int* idx_out, float* w_out) {
-  unsigned long long key[NK];
+  // Keys: order-preserving 32-bit images of the logits (0 = empty).  Each
+  // lane keeps the position of its largest key (lowest position on ties);
+  // per round the warp takes the largest key, and among equal keys the lowest
+  // expert index, and only the winner lane rescans its keys.
+  uint32_t key[NK];
 #pragma unroll
   for (int i = 0; i < NK; ++i) {
     const int e = i * 32 + lane;
-    key[i] = 0ull;
-    if (e < n)
-      key[i] = ((unsigned long long)order_bits(kShared ? lg[e] : __ldcg(lg + e)) << 32) | (uint32_t)(~(uint32_t)e);
+    key[i] = e < n ? order_bits(kShared ? lg[e] : __ldcg(lg + e)) : 0u;
   }
-  unsigned long long mine = max_tree<NK>(key);
+  uint32_t mine = key[0];
+  int mi = 0;
+#pragma unroll
+  for (int i = 1; i < NK; ++i)
+    if (key[i] > mine) { mine = key[i]; mi = i; }
   float my_val = 0.f;
   int my_idx = 0;
 #pragma unroll 1
   for (int kk = 0; kk < k; ++kk) {
-    const uint32_t mh = (uint32_t)(mine >> 32);
-    const uint32_t h = __reduce_max_sync(0xffffffffu, mh);
-    const unsigned tie = __ballot_sync(0xffffffffu, mh == h);
-    // usually one lane holds the largest logit; an exact tie needs the index max
-    const uint32_t l = (tie & (tie - 1)) ? __reduce_max_sync(0xffffffffu, mh == h ? (uint32_t)mine : 0u)
-                                         : __shfl_sync(0xffffffffu, (uint32_t)mine, __ffs(tie) - 1);
-    const unsigned long long best = ((unsigned long long)h << 32) | l;
-    if (mine == best) {  // keys are unique: exactly one lane owned the winner
+    const uint32_t h = __reduce_max_sync(0xffffffffu, mine);
+    const uint32_t e = __reduce_min_sync(0xffffffffu, mine == h ? (uint32_t)(mi * 32 + lane) : 0xffffffffu);
+    if ((int)(e & 31u) == lane) {  // the winner lane drops the key and rescans
 #pragma unroll
       for (int i = 0; i < NK; ++i)
-        if (key[i] == best) key[i] = 0ull;
-      mine = max_tree<NK>(key);
+        if (i == mi) key[i] = 0u;
+      mine = key[0];
+      mi = 0;
+#pragma unroll
+      for (int i = 1; i < NK; ++i)
+        if (key[i] > mine) { mine = key[i]; mi = i; }
     }
     if (lane == kk) {
       my_val = from_order_bits(h);
-      my_idx = (int)~l;
+      my_idx = (int)e;
     }
   }
   FMOE_TRACE_WARP(14);
@@ -510,7 +519,7 @@ __device__ __noinline__ void ensure_routing(const LayerArgs& a, CtaShared& cs, c
   old = __shfl_sync(0xffffffffu, old, 0);
   if (old == 0) {
     bool ok = true;
-    if (lane == 0) ok = grid_wait(&a.bar[0], gridDim.x, a.timeout_ns);
+    if (lane == 0) ok = grid_wait(&a.bar[0], (unsigned)a.n_router, a.timeout_ns);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     __syncwarp();
     if (!ok && lane == 0) set_status(kStatusGridBarrierTimeout);
@@ -525,7 +534,7 @@ __device__ __noinline__ void ensure_routing(const LayerArgs& a, CtaShared& cs, c
     }
     if (!mbar_wait_bounded(&cs.lg_bar, 0, a.timeout_ns) && lane == 0) set_status(kStatusCopyTimeout);
     const float lsg = a.w_sgate ? lg[a.E] : 0.f;
-    FMOE_TRACE_WARP(12);
+    FMOE_TRACE_WARP(17);
     warp_topk<true>(lg, a.E, a.K, lane, cs.idx, cs.w);
     __syncwarp();
     FMOE_TRACE_WARP(10);
@@ -536,6 +545,7 @@ __device__ __noinline__ void ensure_routing(const LayerArgs& a, CtaShared& cs, c
         cs.blob[k] = a.experts + (long long)cs.idx[k] * a.expert_stride;
       }
       cs.sg = a.w_sgate ? sigmoidf_(lsg) : 1.0f;
+      FMOE_TRACE_WARP(23);
       if (blockIdx.x == 0) {
         for (int k = 0; k < a.K; ++k) {
           if (a.idx_out) a.idx_out[k] = cs.idx[k];
@@ -593,41 +603,72 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     cs.lg_bytes = (unsigned)a.lg_floats * 4u;
     cs.route_state = layer_mode ? 0 : 2;
     cs.sg = 1.0f;
-    cs.router_done = 0;
     cs.c_prefetch = 0;
+    // Read every kernel parameter once now, while x is in flight, so that the
+    // later first uses (routing, publishing, outputs) hit the constant cache.
+    {
+      unsigned long long t = (uintptr_t)a.w_router ^ (uintptr_t)a.w_sgate ^ (uintptr_t)a.experts ^
+                             (unsigned long long)a.expert_stride ^ (uintptr_t)a.shared ^ (uintptr_t)a.x ^
+                             (uintptr_t)a.residual ^ (uintptr_t)a.out ^ (uintptr_t)a.logits ^ (uintptr_t)a.act ^
+                             (uintptr_t)a.bar ^ (uintptr_t)a.idx_out ^ (uintptr_t)a.w_out ^ (uintptr_t)a.sg_out ^
+                             a.timeout_ns;
+      t += (unsigned)(a.H ^ a.I ^ a.E ^ a.K ^ a.bits_r ^ a.bits_s ^ a.n_router ^ a.n_slots ^ a.off_a ^ a.off_b ^
+                      a.nst ^ a.stage_bytes ^ a.nst_c ^ a.c_stage_bytes ^ a.xs4_off ^ a.xs2_off ^ a.xu_off ^
+                      a.vec_floats ^ a.sf_floats ^ a.ys_stride ^ a.lg_floats ^ a.router_smem);
+      for (int i = 0; i < 6; ++i) t += (unsigned long long)(a.off_r[i] ^ a.off_s[i]);
+      *(volatile unsigned long long*)&cs.param_touch = t;
+    }
     // The shared (or single) expert; the routed slots point at expert 0 until
     // the routing decision replaces them (never read before that).
     for (int k = 0; k < a.K; ++k) cs.blob[k] = a.experts;
     cs.blob[a.K] = a.shared;
-    cs.router_target = n_router_warps;  // n_router < G * kWarps: one row per router warp
     fence_proxy_async_smem();
     mbar_arrive_expect_tx(&cs.x_bar, a.H * 4);
     bulk_g2s(sm.vec + a.xu_off, a.x, a.H * 4, &cs.x_bar);
   }
   if (lane == 0) {
-    for (int j = 0; j < plan.router.count; ++j) bulk_prefetch_l2(router_row_ptr(plan.router.first + j * GW), a.H * 2);
+    if (a.router_smem && plan.router.count == 1) {
+      // The router row is the first thing this warp needs after x: bring it
+      // into the warp's (still unused) ring now, alongside x.
+      mbar_init(&cs.rbar[warp], 1);
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&cs.rbar[warp], a.H * 2);
+      bulk_g2s(my_ring, router_row_ptr(plan.router.first), a.H * 2, &cs.rbar[warp]);
+    } else {
+      for (int j = 0; j < plan.router.count; ++j)
+        bulk_prefetch_l2(router_row_ptr(plan.router.first + j * GW), a.H * 2);
+    }
     for (int s = 0; s < a.nst + kMaxNstC; ++s) mbar_init(&my_bars[s], 1);
     fence_proxy_async_smem();
   }
   __syncthreads();
   FMOE_TRACE(11);
-  if (tid == 0 && layer_mode && cs.router_target == 0) red_release_gpu_add(&a.bar[0], 1);
 
   // x and the router rows are the critical path to the routing decision, so
   // they are the only traffic of the first microseconds; the shared expert's
   // gate/up rows follow once x is staged.
   int issued = 0;
   if (!mbar_wait_bounded(&cs.x_bar, 0, a.timeout_ns) && lane == 0) set_status(kStatusCopyTimeout);
+  FMOE_TRACE_WARP(16);
   const float* xu = sm.vec + a.xu_off;
   if (router_warp) {
     // ---- Phase A, router rows: published, then counted once per CTA ---------
     for (int j = 0; j < plan.router.count; ++j) {
       const int e = plan.router.first + j * GW;
-      const float l = router_dot(router_row_ptr(e), xu, a.H, lane);
+      float l;
+      if (a.router_smem && plan.router.count == 1) {
+        if (!mbar_wait_bounded(&cs.rbar[warp], 0, a.timeout_ns) && lane == 0) set_status(kStatusCopyTimeout);
+        FMOE_TRACE_WARP(20);
+        l = router_dot_smem(reinterpret_cast<const uint16_t*>(my_ring), xu, a.H, lane);
+        FMOE_TRACE_WARP(21);
+      } else {
+        l = router_dot(router_row_ptr(e), xu, a.H, lane);
+      }
       if (lane == 0) {
+        // The release orders this thread's logit store before its count.
         a.logits[e] = l;
-        __threadfence();
-        if (atomicAdd(&cs.router_done, 1u) + 1 == cs.router_target) red_release_gpu_add(&a.bar[0], 1);
+        red_release_gpu_add(&a.bar[0], 1);
+        FMOE_TRACE_WARP(22);
       }
     }
     FMOE_TRACE_WARP(2);
@@ -640,6 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
       stage_inputs<2, false>(xu, a.H, reinterpret_cast<float4*>(sm.vec + a.xs2_off),
                              sm.sf + (a.xs4_off >= 0 ? a.H / 32 : 0), t0, nt);
     __syncwarp();
+    FMOE_TRACE_WARP(18);
     if (lane == 0) mbar_arrive(&cs.staged_bar);
     if (warp == kWarps - 1 && lane == 0 && a.shared && plan.nq > 0) {
       // the shared expert's down rows of this CTA are known from the start
@@ -650,8 +692,11 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
       bulk_prefetch_l2(a.shared + o.dsb + r0 * sbr, (uint32_t)(nr * sbr));
     }
   }
-  // The shared expert's gate/up loads (no routing decision needed).
+  // The shared expert's gate/up loads (no routing decision needed).  A
+  // router warp's ring held its router row: its reads come before the copies.
+  __syncwarp();
   if (lane == 0) {
+    if (router_warp && a.router_smem) fence_proxy_async_smem();
     while (issued < plan.a.count && issued < a.nst) {
       issue_load(a, plan, cs, issued, warp, my_ring + (size_t)issued * a.stage_bytes, &my_bars[issued], GW);
       ++issued;
@@ -697,6 +742,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     if (!mbar_wait_bounded(&my_bars[st_i], (i / a.nst) & 1, a.timeout_ns) && lane == 0)
       set_status(kStatusCopyTimeout);
     if (i == n_gu - 1) FMOE_TRACE_WARP(13);
+    if (i == 0 && plan.a.count > 0) FMOE_TRACE_WARP(19);
     int slot, row;
     gu_unit(a, plan, i, GW, slot, row);
     const bool routed = slot < a.K;

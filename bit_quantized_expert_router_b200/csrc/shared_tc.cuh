@@ -210,7 +210,7 @@ __device__ __forceinline__ char* align1024(char* p) {
 // tokens, then (CTAs below 2 * (I/128) * (H/512)) one gate or up tile.
 template <int BS>
 __global__ void __launch_bounds__(kThreads, 1) router_shared_gu_kernel(const __grid_constant__ GroupArgs a) {
-  extern __shared__ __align__(1024) char smem_raw[];
+  extern __shared__ __align__(128) char smem_raw[];  // (aligned to 1024 below)
   char* sbase = align1024(smem_raw);
   const int b = blockIdx.x;
   const int rows = a.E + (a.w_sgate ? 1 : 0);
@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1) router_shared_gu_kernel(const __g
 // partials (summed over the input tiles in order).
 template <int BR, int BS>
 __global__ void __launch_bounds__(kThreads, 1) prep_shared_down_kernel(const __grid_constant__ GroupArgs a) {
-  extern __shared__ __align__(1024) char smem_raw[];
+  extern __shared__ __align__(128) char smem_raw[];  // (aligned to 1024 below)
   const int b = blockIdx.x;
   if (b <= a.T) {
     prep_cta<BR, BS>(a, b);

@@ -154,6 +154,29 @@ __device__ __forceinline__ float warp_sum(float v) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
+// Two warp sums at once: returns the sum of `a` over the warp on lanes 0..15
+// and the sum of `b` on lanes 16..31 (5 shuffles instead of 10).
+__device__ __forceinline__ float warp_sum2_split(float a, float b, int lane) {
+  const bool hi = (lane & 16) != 0;
+  float keep = hi ? b : a;
+  keep += __shfl_xor_sync(0xffffffffu, hi ? a : b, 16);
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) keep += __shfl_xor_sync(0xffffffffu, keep, o);
+  return keep;
+}
+// Four warp sums at once: lane l returns the sum of y[(l >> 3) & 3] over the
+// warp (so lanes 0, 8, 16, 24 hold rows 0..3; 6 shuffles instead of 20).
+__device__ __forceinline__ float warp_sum4_split(const float (&y)[4], int lane) {
+  const bool b4 = (lane & 16) != 0, b3 = (lane & 8) != 0;
+  float k0 = b4 ? y[2] : y[0], k1 = b4 ? y[3] : y[1];
+  k0 += __shfl_xor_sync(0xffffffffu, b4 ? y[0] : y[2], 16);
+  k1 += __shfl_xor_sync(0xffffffffu, b4 ? y[1] : y[3], 16);
+  float keep = b3 ? k1 : k0;
+  keep += __shfl_xor_sync(0xffffffffu, b3 ? k0 : k1, 8);
+#pragma unroll
+  for (int o = 4; o > 0; o >>= 1) keep += __shfl_xor_sync(0xffffffffu, keep, o);
+  return keep;
+}
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

@@ -338,6 +338,29 @@ __device__ __forceinline__ void locate(const CtaSched& cs, int ru, int u, int& s
   r = w - c * ru;
 }
 
+// A warp's units are u0 + warp + i * kWarps: one division to find the first,
+// then each step moves kWarps units on, which crosses at most one chunk and
+// one slot boundary because every chunk has ru >= kWarps units.
+struct UnitCursor {
+  int s, c, r;
+};
+__device__ __forceinline__ UnitCursor cursor_at(const CtaSched& cs, int ru, int u) {
+  UnitCursor k;
+  k.s = 0;
+  locate(cs, ru, u, k.s, k.c, k.r);
+  return k;
+}
+__device__ __forceinline__ void cursor_step(const CtaSched& cs, int ru, UnitCursor& k) {
+  k.r += kWarps;
+  if (k.r >= ru) {
+    k.r -= ru;
+    if (++k.c >= cs.nk[k.s]) {
+      k.c = 0;
+      ++k.s;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Dot products over one input chunk
 // ---------------------------------------------------------------------------
@@ -379,8 +402,10 @@ __device__ __forceinline__ void gu_dot_chunk(const char* st, int nvc, int cb, in
     u = fmaf(bf16_lo(sbuw) * f.y, du.x + du.y, u);
     u = fmaf(bf16_hi(sbuw), f.x, u);
   }
-  g_out = warp_sum(g);
-  u_out = warp_sum(u);
+  // g on lanes 0..15 (lane 0 is the one that uses it), u broadcast
+  const float v = warp_sum2_split(g, u, lane);
+  g_out = v;
+  u_out = __shfl_sync(0xffffffffu, v, 16);
 }
 
 // kRC down-row chunks (nvc vectors each, rows cb bytes apart in the stage;
@@ -423,8 +448,118 @@ __device__ __forceinline__ void down_dot_chunk(const char* st, int nvc, int cb, 
       y[r] = fmaf(bf16_hi(sbv), f.x, y[r]);
     }
   }
+  // row (lane >> 3) & 3 on each lane: lanes 0, 8, 16, 24 hold rows 0..3
+  y[0] = warp_sum4_split(y, lane);
+}
+
+// Two gate/up units (stages stA, stB: rows of the same slot and input chunk)
+// against one token's staged input, each input load serving four rows.
+// Results: unit A's g, u on lane 0, unit B's g, u on lane 16.
+template <int BITS>
+__device__ __forceinline__ void gu_dot_chunk2(const char* stA, const char* stB, int nvc, int cb, int cap, int sbo_gA,
+                                              int sbo_uA, int sbo_gB, int sbo_uB, const float4* xs, int NV, int v0,
+                                              const float2* sf, int lane, float& g_out, float& u_out) {
+  const uint4* cgA = reinterpret_cast<const uint4*>(stA);
+  const uint4* cuA = reinterpret_cast<const uint4*>(stA + cb);
+  const uint4* cgB = reinterpret_cast<const uint4*>(stB);
+  const uint4* cuB = reinterpret_cast<const uint4*>(stB + cb);
+  const uint32_t* sgA = reinterpret_cast<const uint32_t*>(stA + 2 * cb + sbo_gA);
+  const uint32_t* suA = reinterpret_cast<const uint32_t*>(stA + 2 * cb + cap + sbo_uA);
+  const uint32_t* sgB = reinterpret_cast<const uint32_t*>(stB + 2 * cb + sbo_gB);
+  const uint32_t* suB = reinterpret_cast<const uint32_t*>(stB + 2 * cb + cap + sbo_uB);
+  const ulonglong2* xv = reinterpret_cast<const ulonglong2*>(xs) + v0;
+  float y[4] = {0.f, 0.f, 0.f, 0.f};  // gA, uA, gB, uB
+  for (int v = lane; v < nvc; v += 32) {
+    const uint4 w0 = cgA[v], w1 = cuA[v], w2 = cgB[v], w3 = cuB[v];
+    const int grp = (BITS == 4) ? (v >> 1) : v;
+    const uint32_t sb[4] = {sgA[grp], suA[grp], sgB[grp], suB[grp]};
+    const float2 f = __ldg(sf + v0 + v);
+    uint64_t ac[4] = {0, 0, 0, 0};
 #pragma unroll
-  for (int r = 0; r < kRC; ++r) y[r] = warp_sum(y[r]);
+    for (int t = 0; t < 4; ++t) {
+      const uint32_t c0 = (&w0.x)[t], c1 = (&w1.x)[t], c2 = (&w2.x)[t], c3 = (&w3.x)[t];
+      if (BITS == 4) {
+        const ulonglong2 xa = __ldg(xv + (2 * t) * NV + v), xb = __ldg(xv + (2 * t + 1) * NV + v);
+        dot_word4(ac[0], c0, xa, xb);
+        dot_word4(ac[1], c1, xa, xb);
+        dot_word4(ac[2], c2, xa, xb);
+        dot_word4(ac[3], c3, xa, xb);
+      } else {
+        const ulonglong2 x0 = __ldg(xv + (4 * t) * NV + v), x1 = __ldg(xv + (4 * t + 1) * NV + v);
+        const ulonglong2 x2 = __ldg(xv + (4 * t + 2) * NV + v), x3 = __ldg(xv + (4 * t + 3) * NV + v);
+        dot_word2(ac[0], c0, x0, x1, x2, x3);
+        dot_word2(ac[1], c1, x0, x1, x2, x3);
+        dot_word2(ac[2], c2, x0, x1, x2, x3);
+        dot_word2(ac[3], c3, x0, x1, x2, x3);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float2 d = unpk_f32(ac[r]);
+      y[r] = fmaf(bf16_lo(sb[r]) * f.y, d.x + d.y, y[r]);
+      y[r] = fmaf(bf16_hi(sb[r]), f.x, y[r]);
+    }
+  }
+  const float v = warp_sum4_split(y, lane);  // lanes 0, 8, 16, 24: gA, uA, gB, uB
+  g_out = v;
+  u_out = __shfl_down_sync(0xffffffffu, v, 8);
+}
+
+// Two down units (stA, stB: kRC rows each, same slot and input chunk) against
+// one staged activation, each activation load serving 2 * kRC rows.  Results:
+// lane 8r holds row r of A in yA and row r of B in yB.
+template <int BITS>
+__device__ __forceinline__ void down_dot_chunk2(const char* stA, const char* stB, int nvc, int cb,
+                                                const uint32_t* sbwA, const uint32_t* sbwB, int sb_stride,
+                                                const float4* as, int NV, int v0, const float2* sfa, int lane,
+                                                float& yA, float& yB) {
+  const ulonglong2* xv = reinterpret_cast<const ulonglong2*>(as) + v0;
+  float ya[kRC], yb[kRC];
+#pragma unroll
+  for (int r = 0; r < kRC; ++r) ya[r] = yb[r] = 0.f;
+  for (int v = lane; v < nvc; v += 32) {
+    uint4 wa[kRC], wb[kRC];
+#pragma unroll
+    for (int r = 0; r < kRC; ++r) {
+      wa[r] = reinterpret_cast<const uint4*>(stA + r * cb)[v];
+      wb[r] = reinterpret_cast<const uint4*>(stB + r * cb)[v];
+    }
+    const float2 f = __ldg(sfa + v0 + v);
+    const int grp = (BITS == 4) ? (v >> 1) : v;
+    uint64_t aa[kRC], ab[kRC];
+#pragma unroll
+    for (int r = 0; r < kRC; ++r) aa[r] = ab[r] = 0;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      if (BITS == 4) {
+        const ulonglong2 xa = __ldg(xv + (2 * t) * NV + v), xb = __ldg(xv + (2 * t + 1) * NV + v);
+#pragma unroll
+        for (int r = 0; r < kRC; ++r) {
+          dot_word4(aa[r], (&wa[r].x)[t], xa, xb);
+          dot_word4(ab[r], (&wb[r].x)[t], xa, xb);
+        }
+      } else {
+        const ulonglong2 x0 = __ldg(xv + (4 * t) * NV + v), x1 = __ldg(xv + (4 * t + 1) * NV + v);
+        const ulonglong2 x2 = __ldg(xv + (4 * t + 2) * NV + v), x3 = __ldg(xv + (4 * t + 3) * NV + v);
+#pragma unroll
+        for (int r = 0; r < kRC; ++r) {
+          dot_word2(aa[r], (&wa[r].x)[t], x0, x1, x2, x3);
+          dot_word2(ab[r], (&wb[r].x)[t], x0, x1, x2, x3);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kRC; ++r) {
+      const uint32_t sa = sbwA[r * sb_stride + grp], sbv = sbwB[r * sb_stride + grp];
+      const float2 da = unpk_f32(aa[r]), db = unpk_f32(ab[r]);
+      ya[r] = fmaf(bf16_lo(sa) * f.y, da.x + da.y, ya[r]);
+      ya[r] = fmaf(bf16_hi(sa), f.x, ya[r]);
+      yb[r] = fmaf(bf16_lo(sbv) * f.y, db.x + db.y, yb[r]);
+      yb[r] = fmaf(bf16_hi(sbv), f.x, yb[r]);
+    }
+  }
+  yA = warp_sum4_split(ya, lane);
+  yB = warp_sum4_split(yb, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -448,11 +583,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gateup_kernel(const __gri
   const int n = cs.u1 - cs.u0 > warp ? (cs.u1 - cs.u0 - warp - 1) / kWarps + 1 : 0;
   const int sbr = sb_row_bytes(a.H), cap = sb_superset_cap(a.H);
 
-  int s_issue = 0;
-  auto issue = [&](int i) {  // lane 0
-    int s, c, row;
-    locate(cs, a.I, cs.u0 + warp + i * kWarps, s_issue, c, row);
-    s = s_issue;
+  UnitCursor ki = cursor_at(cs, a.I, cs.u0 + warp);  // next unit to issue
+  auto issue = [&](int i) {  // lane 0; units are issued in order
+    const int s = ki.s, c = ki.c, row = ki.r;
+    cursor_step(cs, a.I, ki);
     const int e = cs.expert[s];
     const int bits = e >= 0 ? BR : BS;
     const char* blob = e >= 0 ? a.experts + (long long)e * a.expert_stride : a.shared;
@@ -475,38 +609,64 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gateup_kernel(const __gri
   if (lane == 0)
     for (int i = 0; i < n && i < a.nst; ++i) issue(i);
 
-  int s_cur = 0;
-  for (int i = 0; i < n; ++i) {
+  UnitCursor kc = cursor_at(cs, a.I, cs.u0 + warp);  // unit being computed
+  for (int i = 0; i < n;) {
+    // Two consecutive units of the same slot and input chunk are computed in
+    // one pass (each input load then serves four rows).
+    UnitCursor kn = kc;
+    cursor_step(cs, a.I, kn);
+    const bool two = a.nst >= 2 && i + 1 < n && kn.s == kc.s && kn.c == kc.c;
     const char* stage = my_ring + (size_t)(i % a.nst) * a.stage_bytes;
+    const char* stage2 = my_ring + (size_t)((i + 1) % a.nst) * a.stage_bytes;
     if (!mbar_wait_bounded(&my_bars[i % a.nst], (i / a.nst) & 1, a.timeout_ns) && lane == 0)
       set_status(kStatusCopyTimeout);
-    int c, row;
-    locate(cs, a.I, cs.u0 + warp + i * kWarps, s_cur, c, row);
-    const int s = s_cur;
+    if (two && !mbar_wait_bounded(&my_bars[(i + 1) % a.nst], ((i + 1) / a.nst) & 1, a.timeout_ns) && lane == 0)
+      set_status(kStatusCopyTimeout);
+    const int s = kc.s, c = kc.c, row = kc.r, row2 = kn.r;
     const bool routed = cs.expert[s] >= 0;
     const int cl = a.H / cs.nk[s];
-    const BlobOff o = blob_offsets(a.H, a.I, routed ? BR : BS);
-    const int sbo_g = (int)((o.gsb + (long long)row * sbr + c * (cl / 16)) & 15);
-    const int sbo_u = (int)((o.usb + (long long)row * sbr + c * (cl / 16)) & 15);
+    const long long* o = routed ? a.off_r : a.off_s;
+    const int sbo_g = (int)((o[1] + (long long)row * sbr + c * (cl / 16)) & 15);
+    const int sbo_u = (int)((o[3] + (long long)row * sbr + c * (cl / 16)) & 15);
+    const int sbo_g2 = (int)((o[1] + (long long)row2 * sbr + c * (cl / 16)) & 15);
+    const int sbo_u2 = (int)((o[3] + (long long)row2 * sbr + c * (cl / 16)) & 15);
     for (int p = cs.pair0[s]; p < cs.pair0[s + 1]; ++p) {
       const int t = a.tb.pair_token[p];
       float g, up;
+      float2* dst = a.gu_part + ((long long)p * kMaxChunks + c) * a.I;
       if (routed || BR == BS) {
         constexpr int CPV = 128 / BR;
-        gu_dot_chunk<BR>(stage, cl / CPV, cl * BR / 8, cap, sbo_g, sbo_u, a.xs_r + (long long)t * (a.H / 4),
-                         a.H / CPV, c * (cl / CPV), a.sf_r + (long long)t * (a.H / CPV), lane, g, up);
+        const float4* xs = a.xs_r + (long long)t * (a.H / 4);
+        const float2* sf = a.sf_r + (long long)t * (a.H / CPV);
+        if (two)
+          gu_dot_chunk2<BR>(stage, stage2, cl / CPV, cl * BR / 8, cap, sbo_g, sbo_u, sbo_g2, sbo_u2, xs, a.H / CPV,
+                            c * (cl / CPV), sf, lane, g, up);
+        else
+          gu_dot_chunk<BR>(stage, cl / CPV, cl * BR / 8, cap, sbo_g, sbo_u, xs, a.H / CPV, c * (cl / CPV), sf, lane,
+                           g, up);
       } else {
         constexpr int CPV = 128 / BS;
-        gu_dot_chunk<BS>(stage, cl / CPV, cl * BS / 8, cap, sbo_g, sbo_u, a.xs_s + (long long)t * (a.H / 4),
-                         a.H / CPV, c * (cl / CPV), a.sf_s + (long long)t * (a.H / CPV), lane, g, up);
+        const float4* xs = a.xs_s + (long long)t * (a.H / 4);
+        const float2* sf = a.sf_s + (long long)t * (a.H / CPV);
+        if (two)
+          gu_dot_chunk2<BS>(stage, stage2, cl / CPV, cl * BS / 8, cap, sbo_g, sbo_u, sbo_g2, sbo_u2, xs, a.H / CPV,
+                            c * (cl / CPV), sf, lane, g, up);
+        else
+          gu_dot_chunk<BS>(stage, cl / CPV, cl * BS / 8, cap, sbo_g, sbo_u, xs, a.H / CPV, c * (cl / CPV), sf, lane,
+                           g, up);
       }
-      if (lane == 0) a.gu_part[((long long)p * kMaxChunks + c) * a.I + row] = make_float2(g, up);
+      if (lane == 0) dst[row] = make_float2(g, up);
+      if (two && lane == 16) dst[row2] = make_float2(g, up);
     }
     __syncwarp();
-    if (lane == 0 && i + a.nst < n) {
+    if (lane == 0) {
       fence_proxy_async_smem();
-      issue(i + a.nst);
+      if (i + a.nst < n) issue(i + a.nst);
+      if (two && i + 1 + a.nst < n) issue(i + 1 + a.nst);
     }
+    i += two ? 2 : 1;
+    kc = kn;
+    if (two) cursor_step(cs, a.I, kc);
   }
 }
 
@@ -565,11 +725,10 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_down_kernel(const __grid_
   const int n = cs.u1 - cs.u0 > warp ? (cs.u1 - cs.u0 - warp - 1) / kWarps + 1 : 0;
   const int sbr = sb_row_bytes(a.I);  // bytes of one row's scale/bias words
 
-  int s_issue = 0;
-  auto issue = [&](int i) {  // lane 0
-    int c, q;
-    locate(cs, nq, cs.u0 + warp + i * kWarps, s_issue, c, q);
-    const int s = s_issue;
+  UnitCursor ki = cursor_at(cs, nq, cs.u0 + warp);  // next unit to issue
+  auto issue = [&](int i) {  // lane 0; units are issued in order
+    const int s = ki.s, c = ki.c, q = ki.r;
+    cursor_step(cs, nq, ki);
     const int e = cs.expert[s];
     const int bits = e >= 0 ? BR : BS;
     const char* blob = e >= 0 ? a.experts + (long long)e * a.expert_stride : a.shared;
@@ -595,42 +754,62 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_down_kernel(const __grid_
   if (lane == 0)
     for (int i = 0; i < n && i < a.nst_c; ++i) issue(i);
 
-  int s_cur = 0;
-  for (int i = 0; i < n; ++i) {
+  UnitCursor kc = cursor_at(cs, nq, cs.u0 + warp);  // unit being computed
+  for (int i = 0; i < n;) {
+    // Two consecutive units of the same slot and input chunk are computed in
+    // one pass (each activation load then serves 2 * kRC rows).
+    UnitCursor kn = kc;
+    cursor_step(cs, nq, kn);
+    const bool two = a.nst_c >= 2 && i + 1 < n && kn.s == kc.s && kn.c == kc.c;
     const char* stage = my_ring + (size_t)(i % a.nst_c) * a.c_stage_bytes;
+    const char* stage2 = my_ring + (size_t)((i + 1) % a.nst_c) * a.c_stage_bytes;
     if (!mbar_wait_bounded(&my_bars[i % a.nst_c], (i / a.nst_c) & 1, a.timeout_ns) && lane == 0)
       set_status(kStatusCopyTimeout);
-    int c, q;
-    locate(cs, nq, cs.u0 + warp + i * kWarps, s_cur, c, q);
-    const int s = s_cur;
+    if (two && !mbar_wait_bounded(&my_bars[(i + 1) % a.nst_c], ((i + 1) / a.nst_c) & 1, a.timeout_ns) && lane == 0)
+      set_status(kStatusCopyTimeout);
+    const int s = kc.s, c = kc.c, q = kc.r, q2 = kn.r;
     const bool routed = cs.expert[s] >= 0;
     const int cl = a.I / cs.nk[s];
-    const BlobOff o = blob_offsets(a.H, a.I, routed ? BR : BS);
-    const long long sb0 = o.dsb + (long long)q * kRC * sbr + c * (cl / 16);
+    const long long sbbase = (routed ? a.off_r : a.off_s)[5] + c * (cl / 16);
+    const long long sb0 = sbbase + (long long)q * kRC * sbr, sb2 = sbbase + (long long)q2 * kRC * sbr;
     const int bits = routed ? BR : BS;
     const int cb = cl * bits / 8;
     const uint32_t* sbw = reinterpret_cast<const uint32_t*>(stage + kRC * cb + (sb0 & 15));
+    const uint32_t* sbw2 = reinterpret_cast<const uint32_t*>(stage2 + kRC * cb + (sb2 & 15));
     for (int p = cs.pair0[s]; p < cs.pair0[s + 1]; ++p) {
-      float y[kRC];
+      float y[kRC], y2 = 0.f;
       const float4* as = a.as + (long long)p * (a.I / 4);
       const float2* sf = a.sfa + (long long)p * (a.I / 32);
       if (routed || BR == BS) {
         constexpr int CPV = 128 / BR;
-        down_dot_chunk<BR>(stage, cl / CPV, cb, sbw, sbr / 4, as, a.I / CPV, c * (cl / CPV), sf, lane, y);
+        if (two)
+          down_dot_chunk2<BR>(stage, stage2, cl / CPV, cb, sbw, sbw2, sbr / 4, as, a.I / CPV, c * (cl / CPV), sf, lane,
+                              y[0], y2);
+        else
+          down_dot_chunk<BR>(stage, cl / CPV, cb, sbw, sbr / 4, as, a.I / CPV, c * (cl / CPV), sf, lane, y);
       } else {
         constexpr int CPV = 128 / BS;
-        down_dot_chunk<BS>(stage, cl / CPV, cb, sbw, sbr / 4, as, a.I / CPV, c * (cl / CPV), sf, lane, y);
+        if (two)
+          down_dot_chunk2<BS>(stage, stage2, cl / CPV, cb, sbw, sbw2, sbr / 4, as, a.I / CPV, c * (cl / CPV), sf, lane,
+                              y[0], y2);
+        else
+          down_dot_chunk<BS>(stage, cl / CPV, cb, sbw, sbr / 4, as, a.I / CPV, c * (cl / CPV), sf, lane, y);
       }
-      if (lane == 0) {
-        float* dst = a.y_part + ((long long)p * kMaxChunks + c) * a.H + (long long)q * kRC;
-        *reinterpret_cast<float4*>(dst) = make_float4(y[0], y[1], y[2], y[3]);
+      float* dst = a.y_part + ((long long)p * kMaxChunks + c) * a.H + (lane >> 3);
+      if ((lane & 7) == 0) {
+        dst[(long long)q * kRC] = y[0];
+        if (two) dst[(long long)q2 * kRC] = y2;
       }
     }
     __syncwarp();
-    if (lane == 0 && i + a.nst_c < n) {
+    if (lane == 0) {
       fence_proxy_async_smem();
-      issue(i + a.nst_c);
+      if (i + a.nst_c < n) issue(i + a.nst_c);
+      if (two && i + 1 + a.nst_c < n) issue(i + 1 + a.nst_c);
     }
+    i += two ? 2 : 1;
+    kc = kn;
+    if (two) cursor_step(cs, nq, kc);
   }
 }
 

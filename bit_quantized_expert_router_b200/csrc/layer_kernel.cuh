@@ -39,7 +39,7 @@ namespace fmoe {
 
 constexpr int kWarps = 16;        // warps per CTA
 constexpr int kThreads = kWarps * 32;
-constexpr int kRC = 4;            // down rows per phase-C item
+constexpr int kRC = 4;            // down rows per phase-C item (the split row reduction assumes 4)
 constexpr int kMaxTopK = 8;
 constexpr int kMaxSlots = kMaxTopK + 1;
 constexpr int kMaxExperts = 1024; // top-K is one warp with 32 logits per lane
@@ -351,8 +351,10 @@ __device__ __forceinline__ void pair_dot_src(const char* st, int H, int sbo_g, i
     u = fmaf(bf16_lo(sbuw) * f.y, du.x + du.y, u);
     u = fmaf(bf16_hi(sbuw), f.x, u);
   }
-  g_out = warp_sum(g);
-  u_out = warp_sum(u);
+  // g on lanes 0..15 (lane 0 is the one that uses it), u broadcast
+  const float v = warp_sum2_split(g, u, lane);
+  g_out = v;
+  u_out = __shfl_sync(0xffffffffu, v, 16);
 }
 
 template <int BITS>
@@ -406,8 +408,8 @@ __device__ __forceinline__ void down_rows_src(const char* st, int I, const float
       y[r] = fmaf(bf16_hi(sbw), f.x, y[r]);
     }
   }
-#pragma unroll
-  for (int r = 0; r < kRC; ++r) y[r] = warp_sum(y[r]);
+  // row (lane >> 3) & 3 on each lane: lanes 0, 8, 16, 24 hold rows 0..3
+  y[0] = warp_sum4_split(y, lane);
 }
 
 template <int BITS>
@@ -846,11 +848,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     else
       down_rows<BS>(stage, a.I, as, nvs, col0, sfa, lane, y);
     if (j == 0) FMOE_TRACE_WARP(12);
-    if (lane == 0) {
-      float* ys = sm.ys + slot * a.ys_stride + (r0 - plan.q0 * kRC);
-#pragma unroll
-      for (int r = 0; r < kRC; ++r) ys[r] = y[r];
-    }
+    if ((lane & 7) == 0) sm.ys[slot * a.ys_stride + (r0 - plan.q0 * kRC) + (lane >> 3)] = y[0];
     __syncwarp();
   }
   FMOE_TRACE_WARP(7);

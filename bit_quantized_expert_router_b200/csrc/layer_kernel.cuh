@@ -17,12 +17,13 @@
 // Units of phases A and B are dealt round-robin over all warps of the grid.
 //
 // Hand-offs.  Each router warp stores its logit and counts it with one
-// release add on a grid counter; each CTA's first warp that needs the routing
-// decision polls until every router row is counted, reads the logits and runs
-// the top-K, then wakes the CTA's other warps through an mbarrier.  "All activations written" is a
-// second counter that every CTA bumps once and polls once.  Every wait is
-// time-limited: on expiry the kernel sets a status bit and carries on instead
-// of hanging.
+// release add on a grid counter.  Every CTA then takes the routing decision
+// with all of its warps: one warp polls until every router row is counted and
+// copies the logits into shared memory, each warp selects the top K of its
+// slice, and one warp merges the candidates (two CTA barriers).  "All
+// activations written" is a second counter that every CTA bumps once and
+// polls once.  Every wait is time-limited: on expiry the kernel sets a status
+// bit and carries on instead of hanging.
 //
 // Data movement.  Each warp streams its gate/up units through a private ring
 // of shared-memory stages filled by cp.async.bulk copies that complete on an
@@ -162,23 +163,24 @@ __device__ __forceinline__ WarpPlan make_plan(const LayerArgs& a, int cta, int w
 
 // Per-CTA shared state (static shared memory).
 struct CtaShared {
-  uint64_t route_bar;   // completes once the routing decision is in this struct
   uint64_t x_bar;       // completes once x is in shared memory
   uint64_t staged_bar;  // completes once x is staged in the decode layouts
+  uint64_t rdot_bar;    // completes once this CTA's router dot products are done
   uint64_t lg_bar;      // completes once the router logits are in shared memory
   uint64_t rbar[kWarps];  // router warp w's row is in its ring (router_smem)
   unsigned long long param_touch;  // see the kernel's set-up
   float* lg;            // shared-memory copy of the router logits
   unsigned lg_bytes;
-  int route_state;      // 0 = not started, 1 = being computed, 2 = ready
   int c_prefetch;          // warps past their gate/up work (the first prefetches down rows)
   int idx[kMaxTopK];
   float w[kMaxTopK];
   float sg;
   const char* blob[kMaxSlots];  // blob of each slot (routed ones once the routing is known)
+  uint32_t cand_key[kWarps * kMaxTopK];  // per-warp top-K candidates (order-preserving keys)
+  uint32_t cand_idx[kWarps * kMaxTopK];  // and their expert indices
+  uint32_t sel_key[kMaxTopK];            // the selected keys, in rank order
 };
 
-__device__ __forceinline__ float* cs_logits(const LayerArgs&, CtaShared& cs) { return cs.lg; }
 
 struct SlotInfo {
   const char* blob;
@@ -363,6 +365,7 @@ __device__ __forceinline__ void pair_dot(const char* st, int H, int sbo_g, int s
   pair_dot_src<BITS, false>(st, H, sbo_g, sbo_u, xs, sf, lane, g_out, u_out);
 }
 
+
 // kRC down rows of one expert (stage layout: kRC code rows | kRC sb rows)
 // against that expert's staged activation, which is column block
 // [col0, col0 + I/CPV) of a staged [F4][NVS] array (several same-width experts
@@ -417,6 +420,7 @@ __device__ __forceinline__ void down_rows(const char* st, int I, const float4* a
                                           const float2* sfa, int lane, float (&y)[kRC]) {
   down_rows_src<BITS, false>(st, I, as, NVS, col0, sfa, lane, y);
 }
+
 
 // Top-K by one warp: descending logit, lower index first on exact ties; then
 // renormalised softmax weights over the selected logits.  Logits become
@@ -509,61 +513,142 @@ __device__ __forceinline__ bool grid_wait(const unsigned* ctr, unsigned target, 
   return true;
 }
 
-// Make the routing decision available in this CTA's shared state.  The first
-// warp to ask waits until every CTA has published its router logits, reads
-// them, runs the top-K and completes the CTA's routing mbarrier, then asks L2
-// to prefetch the routed experts' down rows of this CTA; the other warps sleep
-// on the mbarrier.  Called by whole warps.
-__device__ __noinline__ void ensure_routing(const LayerArgs& a, CtaShared& cs, const WarpPlan& plan, int lane) {
-  if (*((volatile int*)&cs.route_state) == 2) return;
-  int old = 0;
-  if (lane == 0) old = atomicCAS(&cs.route_state, 0, 1);
-  old = __shfl_sync(0xffffffffu, old, 0);
-  if (old == 0) {
+// Top-K rounds over keys held by a warp, NK per lane, each with its expert
+// index (empty slots: key 0): per round the largest key wins and, among equal
+// keys, the lowest expert index; only the winner lane rescans.  Lane kk < k
+// ends with the kk-th winner's key and index.
+template <int NK>
+__device__ __forceinline__ void warp_select(uint32_t (&key)[NK], const uint32_t (&eix)[NK], int k, int lane,
+                                            uint32_t& out_key, uint32_t& out_idx) {
+  uint32_t mk = key[0], mx = eix[0];
+  int mp = 0;
+#pragma unroll
+  for (int i = 1; i < NK; ++i)
+    if (key[i] > mk || (key[i] == mk && eix[i] < mx)) { mk = key[i]; mx = eix[i]; mp = i; }
+  out_key = 0u;
+  out_idx = 0u;
+#pragma unroll 1
+  for (int kk = 0; kk < k; ++kk) {
+    const uint32_t h = __reduce_max_sync(0xffffffffu, mk);
+    const uint32_t e = __reduce_min_sync(0xffffffffu, mk == h ? mx : 0xffffffffu);
+    if (mk == h && mx == e) {  // the winner drops its key and rescans
+#pragma unroll
+      for (int i = 0; i < NK; ++i)
+        if (i == mp) key[i] = 0u;
+      mk = key[0];
+      mx = eix[0];
+      mp = 0;
+#pragma unroll
+      for (int i = 1; i < NK; ++i)
+        if (key[i] > mk || (key[i] == mk && eix[i] < mx)) { mk = key[i]; mx = eix[i]; mp = i; }
+    }
+    if (lane == kk) {
+      out_key = h;
+      out_idx = e;
+    }
+  }
+}
+
+// Stage 1 of the CTA's top-K: warp w selects the top k of its slice of the
+// logits (NKW * 32 consecutive experts from w * NKW * 32) into the candidates.
+template <int NKW>
+__device__ __forceinline__ void slice_topk(const float* lg, int n, int k, int warp, int lane, CtaShared& cs) {
+  uint32_t key[NKW], eix[NKW];
+#pragma unroll
+  for (int i = 0; i < NKW; ++i) {
+    const int e = (warp * NKW + i) * 32 + lane;
+    key[i] = e < n ? order_bits(lg[e]) : 0u;
+    eix[i] = e < n ? (uint32_t)e : 0xffffffffu;
+  }
+  uint32_t hk, hi;
+  warp_select<NKW>(key, eix, k, lane, hk, hi);
+  if (lane < k) {
+    cs.cand_key[warp * k + lane] = hk;
+    cs.cand_idx[warp * k + lane] = hi;
+  }
+}
+
+// The routing decision of this CTA, computed by all of its warps together;
+// every warp calls this once, before it computes any unit (layer mode).
+//   Warp 0 waits until every router row is counted and bulk-copies the logits
+//   into shared memory; each warp selects the top K of its slice of the
+//   logits; after a CTA barrier the candidates are ranked in parallel (the
+//   global top K is among them, ties included); after a second barrier warp 0
+//   computes the weights, and a third publishes the decision to the CTA.
+__device__ __noinline__ void cta_routing(const LayerArgs& a, CtaShared& cs, int warp, int lane) {
+  float* lg = cs.lg;
+  if (warp == 0) {
     bool ok = true;
     if (lane == 0) ok = grid_wait(&a.bar[0], (unsigned)a.n_router, a.timeout_ns);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    __syncwarp();
     if (!ok && lane == 0) set_status(kStatusGridBarrierTimeout);
     FMOE_TRACE_WARP(9);
-    // One bulk copy brings every logit into shared memory (the async proxy
-    // reads what this thread acquired, hence the proxy fence).
-    float* lg = cs_logits(a, cs);
+    // (the async proxy reads what this thread acquired, hence the proxy fence)
     if (lane == 0) {
       fence_proxy_async_global();
       mbar_arrive_expect_tx(&cs.lg_bar, cs.lg_bytes);
       bulk_g2s(lg, a.logits, cs.lg_bytes, &cs.lg_bar);
     }
-    if (!mbar_wait_bounded(&cs.lg_bar, 0, a.timeout_ns) && lane == 0) set_status(kStatusCopyTimeout);
-    const float lsg = a.w_sgate ? lg[a.E] : 0.f;
-    FMOE_TRACE_WARP(17);
-    warp_topk<true>(lg, a.E, a.K, lane, cs.idx, cs.w);
-    __syncwarp();
-    FMOE_TRACE_WARP(10);
-    if (lane == 0) {
-      // Guard the expert index even on a timed-out (garbage) path.
-      for (int k = 0; k < a.K; ++k) {
-        if (cs.idx[k] < 0 || cs.idx[k] >= a.E) cs.idx[k] = 0;
-        cs.blob[k] = a.experts + (long long)cs.idx[k] * a.expert_stride;
-      }
-      cs.sg = a.w_sgate ? sigmoidf_(lsg) : 1.0f;
-      FMOE_TRACE_WARP(23);
-      if (blockIdx.x == 0) {
-        for (int k = 0; k < a.K; ++k) {
-          if (a.idx_out) a.idx_out[k] = cs.idx[k];
-          if (a.w_out) a.w_out[k] = cs.w[k];
-        }
-        if (a.sg_out) *a.sg_out = cs.sg;
-      }
-      *((volatile int*)&cs.route_state) = 2;
-      mbar_arrive(&cs.route_bar);  // release: publishes idx, w, sg to the CTA
-    }
-    FMOE_TRACE_WARP(3);
-    __syncwarp();
-  } else {
-    if (!mbar_wait_bounded(&cs.route_bar, 0, a.timeout_ns) && lane == 0) set_status(kStatusCtaWaitTimeout);
-    __syncwarp();
   }
+  if (!mbar_wait_bounded(&cs.lg_bar, 0, a.timeout_ns) && lane == 0) set_status(kStatusCopyTimeout);
+  FMOE_TRACE_WARP(17);
+  if (a.E <= kWarps * 32)
+    slice_topk<1>(lg, a.E, a.K, warp, lane, cs);
+  else
+    slice_topk<kMaxExperts / (kWarps * 32)>(lg, a.E, a.K, warp, lane, cs);
+  FMOE_TRACE_WARP(14);
+  __syncthreads();
+  // Stage 2: each candidate's rank among the nc candidates (larger key first,
+  // then lower expert index) is counted by P threads over nc_pad / P
+  // candidates each and summed over those P lanes; the K candidates of rank
+  // < K are the decision, written in rank order.
+  {
+    const int nc = kWarps * a.K;
+    int nc_pad = kWarps;
+    while (nc_pad < nc) nc_pad <<= 1;  // 16 .. 128
+    // P threads per candidate (consecutive lanes, a power of two dividing 32),
+    // each comparing against nc_pad / P >= 1 candidates
+    const int P = min(kThreads / nc_pad, nc_pad);
+    const int tid = warp * 32 + lane;
+    const int c = tid / P, part = tid - c * P, per = nc_pad / P;
+    const uint32_t ck = c < nc ? cs.cand_key[c] : 0u, ci = c < nc ? cs.cand_idx[c] : 0xffffffffu;
+    int rank = 0;
+    for (int j = part * per; j < part * per + per && j < nc; ++j) {
+      const uint32_t k2 = cs.cand_key[j], i2 = cs.cand_idx[j];
+      rank += (k2 > ck) || (k2 == ck && i2 < ci);
+    }
+    for (int o = P >> 1; o > 0; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+    if (part == 0 && c < nc && rank < a.K) {
+      cs.sel_key[rank] = ck;
+      cs.idx[rank] = ci < (uint32_t)a.E ? (int)ci : 0;  // (always in range)
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // w_k = exp(l_k - l_0) / sum_j exp(l_j - l_0): softmax restricted to the
+    // selected experts, equal to softmax-then-renormalise.
+    const float val = lane < a.K ? from_order_bits(cs.sel_key[lane]) : 0.f;
+    const float l0 = __shfl_sync(0xffffffffu, val, 0);
+    const float ex = (lane < a.K) ? expf(val - l0) : 0.f;
+    const float ssum = warp_sum(ex);
+    if (lane < a.K) {
+      const int idx = cs.idx[lane];
+      const float w = ex / ssum;
+      cs.w[lane] = w;
+      cs.blob[lane] = a.experts + (long long)idx * a.expert_stride;
+      if (blockIdx.x == 0) {
+        if (a.idx_out) a.idx_out[lane] = idx;
+        if (a.w_out) a.w_out[lane] = w;
+      }
+    }
+    if (lane == 0) {
+      cs.sg = a.w_sgate ? sigmoidf_(lg[a.E]) : 1.0f;
+      if (blockIdx.x == 0 && a.sg_out) *a.sg_out = cs.sg;
+    }
+    FMOE_TRACE_WARP(10);
+  }
+  __syncthreads();
+  FMOE_TRACE_WARP(3);
 }
 
 // Issue phase-C load i (>= a.count + b.count) into the re-carved ring (lane 0).
@@ -597,13 +682,12 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   // ---- Set-up: x to shared memory by one bulk copy; prefetches to L2 --------
   auto router_row_ptr = [&](int e) { return (e < a.E) ? a.w_router + (long long)e * a.H : a.w_sgate; };
   if (tid == 0) {
-    mbar_init(&cs.route_bar, 1);
     mbar_init(&cs.x_bar, 1);
     mbar_init(&cs.staged_bar, kWarps - n_router_warps);
+    mbar_init(&cs.rdot_bar, n_router_warps > 0 ? n_router_warps : 1);
     mbar_init(&cs.lg_bar, 1);
     cs.lg = sm.lg;
     cs.lg_bytes = (unsigned)a.lg_floats * 4u;
-    cs.route_state = layer_mode ? 0 : 2;
     cs.sg = 1.0f;
     cs.c_prefetch = 0;
     // Read every kernel parameter once now, while x is in flight, so that the
@@ -666,6 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
       } else {
         l = router_dot(router_row_ptr(e), xu, a.H, lane);
       }
+      if (lane == 0 && j == 0) mbar_arrive(&cs.rdot_bar);  // staging may start
       if (lane == 0) {
         // The release orders this thread's logit store before its count.
         a.logits[e] = l;
@@ -676,6 +761,10 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     FMOE_TRACE_WARP(2);
   } else {
     // ---- Stage x into the decode layouts (the non-router warps) --------------
+    // The router dot products are on the critical path: staging waits for them
+    // so that they run without competition for the CTA's issue slots.
+    if (n_router_warps > 0 && !mbar_wait_bounded(&cs.rdot_bar, 0, a.timeout_ns) && lane == 0)
+      set_status(kStatusCtaWaitTimeout);
     const int t0 = tid - n_router_warps * 32, nt = kThreads - n_router_warps * 32;
     if (BR == 4 || BS == 4)
       stage_inputs<4, false>(xu, a.H, reinterpret_cast<float4*>(sm.vec + a.xs4_off), sm.sf, t0, nt);
@@ -705,6 +794,8 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     }
   }
   issued = __shfl_sync(0xffffffffu, issued, 0);
+  // Every warp of the CTA takes part in the routing decision (layer mode).
+  if (layer_mode) cta_routing(a, cs, warp, lane);
   if (!mbar_wait_bounded(&cs.staged_bar, 0, a.timeout_ns) && lane == 0) set_status(kStatusCtaWaitTimeout);
   FMOE_TRACE(1);
 
@@ -714,24 +805,11 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   const float4* xs2 = reinterpret_cast<const float4*>(sm.vec + (a.xs2_off >= 0 ? a.xs2_off : 0));
   const float2* sf4 = sm.sf;
   const float2* sf2 = sm.sf + (a.xs4_off >= 0 ? a.H / 32 : 0);
-  bool have_routing = !layer_mode;
 
+  // The routing decision is known from here on: issue freely.
   for (int i = 0; i < n_gu; ++i) {
-    // Loads from index plan.a.count on need the routing decision: block for it
-    // when the warp is about to consume such a load, otherwise take it only if
-    // it is already there.
-    if (!have_routing) {
-      int ready = 0;
-      if (lane == 0) ready = *((volatile int*)&cs.route_state) == 2;
-      ready = __shfl_sync(0xffffffffu, ready, 0);
-      const bool could = issued >= plan.a.count && issued < i + a.nst && issued < n_gu;
-      if (i >= plan.a.count || (could && ready)) {
-        ensure_routing(a, cs, plan, lane);
-        have_routing = true;
-      }
-    }
     if (lane == 0) {
-      while (issued < n_gu && issued < i + a.nst && (have_routing || issued < plan.a.count)) {
+      while (issued < n_gu && issued < i + a.nst) {
         fence_proxy_async_smem();
         issue_load(a, plan, cs, issued, warp, my_ring + (size_t)(issued % a.nst) * a.stage_bytes,
                    &my_bars[issued % a.nst], GW);
@@ -748,10 +826,10 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     int slot, row;
     gu_unit(a, plan, i, GW, slot, row);
     const bool routed = slot < a.K;
-    const BlobOff o = blob_offsets(a.H, a.I, routed ? BR : BS);
+    const long long* o = routed ? a.off_r : a.off_s;
     const int sbr = sb_row_bytes(a.H);
-    const int sbo_g = (int)((o.gsb + (long long)row * sbr) & 15);
-    const int sbo_u = (int)((o.usb + (long long)row * sbr) & 15);
+    const int sbo_g = (int)((o[1] + (long long)row * sbr) & 15);
+    const int sbo_u = (int)((o[3] + (long long)row * sbr) & 15);
     float g, u;
     if (BR == BS || routed)
       pair_dot<BR>(stage, a.H, sbo_g, sbo_u, BR == 4 ? xs4 : xs2, BR == 4 ? sf4 : sf2, lane, g, u);
@@ -763,19 +841,11 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
 
   // Gate/up work of this warp is done (its ring is free): re-carve the ring
   // into down-item stages and put this warp's down items in flight before
-  // joining the hand-off, so they stream during the wait.  (The routing
-  // decision is needed for their addresses; CTA 0 also needs it for the
-  // optional routing outputs.)
-  if (layer_mode && !have_routing && (plan.n_loads > n_gu || (blockIdx.x == 0 && warp == 0))) {
-    ensure_routing(a, cs, plan, lane);
-    have_routing = true;
-  }
+  // joining the hand-off, so they stream during the wait.
   // The CTA's first warp through its gate/up work asks L2 for the routed
   // experts' down rows of this CTA (one lane per routed slot): late enough not
   // to compete with the gate/up stream, early enough to land before phase C.
-  // Only warps that hold the routing decision take part: the routed slots'
-  // blob pointers are set by it.
-  if (layer_mode && have_routing && plan.nq > 0) {
+  if (layer_mode && plan.nq > 0) {
     int first = 0;
     if (lane == 0) first = atomicAdd(&cs.c_prefetch, 1) == 0;
     if (__shfl_sync(0xffffffffu, first, 0) && lane < a.K) {

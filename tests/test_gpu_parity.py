@@ -380,3 +380,34 @@ def test_grouped_deterministic_and_graph_replay(F, SG):
     assert torch.equal(a, out)
     assert F.get_status() == 0
     del g
+
+
+@pytest.mark.parametrize("T", [1, 6])
+def test_layer_exact_ties_pick_lowest_indices(F, SG, T):
+    """Every router row equal: all logits tie exactly, and the decision is the
+    K lowest expert indices with equal weights (single token and grouped)."""
+    shape = C.Shape("ties_h512_i128_e40_k4", 512, 128, 40, 4, 4)
+    seed, layer = 41, 0
+    t = SG.make_layer(seed, layer, shape.hidden, shape.inter, shape.n_experts, shape.bits, shape.shared_bits,
+                      F.blob_offsets, F.expert_bytes, dev())
+    wr_host = S.router_bf16(seed, layer, shape.n_experts, shape.hidden)
+    wr_tied = np.repeat(wr_host[7:8], shape.n_experts, axis=0)
+    w_router = t["w_router"].clone()
+    w_router.copy_(torch.from_numpy(wr_tied.view(np.int16)).to(dev()))
+    L = F.Layer(w_router, t["w_sgate"], t["experts"], t["shared"], shape.hidden, shape.inter, shape.top_k,
+                shape.bits, shape.shared_bits)
+    x = S.token_x(seed, layer, 0, T, shape.hidden)
+    res = S.token_residual(seed, layer, 0, T, shape.hidden)
+    idx = torch.empty(T, shape.top_k, dtype=torch.int32, device=dev())
+    w = torch.empty(T, shape.top_k, dtype=torch.float32, device=dev())
+    out = L.decode(torch.from_numpy(x).to(dev()), torch.from_numpy(res).to(dev()), idx_out=idx, w_out=w)
+    assert F.get_status() == 0
+    w_sg = S.sgate_bf16(seed, layer, shape.hidden)
+    shared = C.cpu_blob(seed, layer, S.SHARED_EXPERT_ID, shape.hidden, shape.inter, shape.shared_bits)
+    for k in range(T):
+        assert idx.cpu().numpy()[k].tolist() == [0, 1, 2, 3]
+        C.assert_close(w.cpu().numpy()[k], np.full(4, 0.25), "tied weights", max_abs=1e-7, rel_l2=1e-7)
+        r = O.layer_decode(wr_tied, w_sg, lambda e: C.cpu_blob(seed, layer, e, shape.hidden, shape.inter, shape.bits),
+                           shared, x[k], res[k], shape.top_k, shape.hidden, shape.inter, shape.bits, shape.shared_bits)
+        assert r["idx"].tolist() == [0, 1, 2, 3]
+        C.assert_close(out.cpu().numpy()[k], r["out"], f"tied token {k}")

@@ -114,6 +114,21 @@ def profiled_traffic(cfg_name: str):
     return d.get("dram_bytes_per_launch")
 
 
+def max_over_ranks(values, world: int, device) -> list:
+    """Element-wise maximum of per-rank values; every rank gets the result."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def whole_job_rate(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Units all ranks processed divided by the slowest rank's time (per second)."""
+    return world * units_per_rank / (max_ms / 1000.0)
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -400,10 +415,7 @@ def run_fmoe(args, cfg, rank, world, local_rank):
     e2e_ms_per_decode = b0.elapsed_time(b1) / (n_e2e * LPS)
 
     # max over ranks
-    tt = torch.tensor([total_ms, e2e_ms_per_decode * K], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-    total_ms_max, e2e_ms_max = float(tt[0]), float(tt[1])
+    total_ms_max, e2e_ms_max = max_over_ranks([total_ms, e2e_ms_per_decode * K], world, dev)
 
     if rank == 0:
         ab = algorithmic_bytes(cfg, distinct)
@@ -411,7 +423,7 @@ def run_fmoe(args, cfg, rank, world, local_rank):
         avg_launch_s = total_ms / 1000.0 / K
         achieved = ab["total"] / avg_launch_s / 1e9
         steps = K // LPS
-        value = world * steps * TT / (total_ms_max / 1000.0)
+        value = whole_job_rate(steps * TT, world, total_ms_max)
         metric, unit = METRIC, UNIT
         if LPS > 1:
             metric, unit = f"decode steps/s through {LPS} MoE layers (batch 1)", "steps/s"
@@ -436,9 +448,9 @@ def run_fmoe(args, cfg, rank, world, local_rank):
                          "kernel": (f"layer_kernel<{cfg['bits']},{cfg['shared_bits']}>" if TT == 1 else
                                     "grouped decode step (router, prep, gate/up, stage, down launches)"),
                          "algorithmic_bytes_per_launch": ab["total"]},
-            "layer_decodes_per_s": world * K / (total_ms_max / 1000.0),
+            "layer_decodes_per_s": whole_job_rate(K, world, total_ms_max),
             "sustained_gbs": world * K * ab["total"] / (total_ms_max / 1000.0) / 1e9,
-            "e2e": {"value": world * K * TT / LPS / (e2e_ms_max / 1000.0), "unit": unit,
+            "e2e": {"value": whole_job_rate(K * TT / LPS, world, e2e_ms_max), "unit": unit,
                     "h2d_bytes_per_step": (2 if LPS == 1 else 1) * TT * h * 4, "d2h_bytes_per_step": TT * h * 4},
             "gpu_launches": K * (1 if TT == 1 else 5),
             **({"distinct_routed_experts_per_step": distinct} if distinct is not None else {}),

@@ -432,8 +432,10 @@ def run_fmoe(args, cfg, rank, world, local_rank):
         line = {
             "impl": "fmoe", "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": steps,
             "warmup": args.warmup, "ms_per_step": total_ms_max / steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "u4/bf16 weights, f32 compute", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {**cfg, "batch": TT, "group": 64,
+                       "weights": f"{cfg['bits']}-bit routed / {cfg['shared_bits']}-bit shared codes, bf16 scale+bias "
+                                  "per group of 64, bf16 router",
                        "l2": f"inputs larger than L2: {NL} distinct layer instances decoded in turn "
                              f"({NL * e * expert_bytes(h, i, cfg['bits']) / 1e9:.0f} GB of experts), no flush",
                        "layers_in_rotation": NL, "input_pool": POOL, "parallelism": f"replicas x{world}"},

@@ -155,7 +155,7 @@ size_t layer_ws_bytes(int E, int I, int K) {
 
 // Workspace of the grouped (T >= 2) decode, byte offsets (every section 256-B aligned).
 struct GroupedLayout {
-  size_t logits, meta, slot_expert, slot_pair0, pair_token, pair_slot, tok_pair, tok_w, tok_sg;
+  size_t logits, meta, slot_expert, slot_pair0, pair_token, pair_slot, pair_nk, tok_pair, tok_w, tok_sg;
   size_t xs_r, sf_r, xs_s, sf_s, gu_part, as, sfa, y_part, sh_gu, sh_y, total;
 };
 
@@ -174,6 +174,7 @@ GroupedLayout grouped_layout(int E, int H, int I, int K, int T) {
   g.slot_pair0 = take((size_t)(kMaxPairs + 2) * 4);
   g.pair_token = take((size_t)kMaxPairs * 4);
   g.pair_slot = take((size_t)kMaxPairs * 4);
+  g.pair_nk = take((size_t)kMaxPairs * 4);
   g.tok_pair = take((size_t)T * (K + 1) * 4);
   g.tok_w = take((size_t)T * K * 4);
   g.tok_sg = take((size_t)T * 4);
@@ -229,6 +230,7 @@ int launch_grouped(const fmoe_layer* L, const float* x, const float* residual, f
   a.tb.slot_pair0 = reinterpret_cast<int*>(w8 + gl.slot_pair0);
   a.tb.pair_token = reinterpret_cast<int*>(w8 + gl.pair_token);
   a.tb.pair_slot = reinterpret_cast<int*>(w8 + gl.pair_slot);
+  a.tb.pair_nk = reinterpret_cast<int*>(w8 + gl.pair_nk);
   a.tb.tok_pair = reinterpret_cast<int*>(w8 + gl.tok_pair);
   a.tb.tok_w = reinterpret_cast<float*>(w8 + gl.tok_w);
   a.tb.tok_sg = reinterpret_cast<float*>(w8 + gl.tok_sg);
@@ -315,7 +317,7 @@ int launch_grouped(const fmoe_layer* L, const float* x, const float* residual, f
   fns.gateup<<<G, kThreads, smem_gu, s>>>(a);
   fns.stage<<<T * K + T, kStageThreads, (size_t)I * 4, s>>>(a);
   fns.down<<<G, kThreads, smem_d, s>>>(a);
-  grouped_combine_kernel<<<(unsigned)(((long long)T * H + 255) / 256), 256, 0, s>>>(a);
+  grouped_combine_kernel<<<dim3((H / 4 + kCombineThreads - 1) / kCombineThreads, T), kCombineThreads, 0, s>>>(a);
   if (cudaError_t e = cudaGetLastError()) return cuda_fail(e);
   return FMOE_OK;
 }

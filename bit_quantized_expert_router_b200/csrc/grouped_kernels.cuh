@@ -65,6 +65,7 @@ struct GroupTables {
   int* slot_pair0;   // [slots + 1] first pair of each slot
   int* pair_token;   // [pairs]
   int* pair_slot;    // [pairs]
+  int* pair_nk;      // [pairs] input chunks of the pair's slot: gate/up (bits 0-7), down (bits 8-15)
   int* tok_pair;     // [T][K + 1] pair of (t, k); column K: the shared pair (-1 if none)
   float* tok_w;      // [T][K]
   float* tok_sg;     // [T]
@@ -149,15 +150,26 @@ __device__ __noinline__ void router_rows_tokens(const uint16_t* __restrict__ w_r
       }
     }
   }
+  // Transposed warp reduction of the 64 sums: each of 5 halving steps keeps
+  // the half of the values selected by one lane bit and adds the partner's
+  // copy of it (62 shuffles in all); lane l ends with sums 2l and 2l + 1
+  // (index r * 16 + t).
+  {
+    float* v = &acc[0][0];
 #pragma unroll
-  for (int r = 0; r < kRouterRows; ++r)
+    for (int o = 16, n = kRouterRows * kMaxTokens; o >= 1; o >>= 1, n >>= 1) {
+      const bool hi = (lane & o) != 0;
 #pragma unroll
-    for (int t = 0; t < kMaxTokens; ++t) {
-      if (t < T) {
-        const float s = warp_sum(acc[r][t]);
-        if (lane == 0) part[warp][r * kMaxTokens + t] = s;
+      for (int j = 0; j < n / 2; ++j) {
+        const float keep = hi ? v[j + n / 2] : v[j];
+        const float send = hi ? v[j] : v[j + n / 2];
+        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
       }
     }
+    part[warp][2 * lane] = v[0];
+    part[warp][2 * lane + 1] = v[1];
+  }
+  static_assert(kRouterRows * kMaxTokens == 64, "the transposed reduction assumes 64 sums per lane");
   __syncthreads();
   if (tid < kRouterRows * T) {
     const int r = tid / T, t = tid - r * T, row = r0 + r;
@@ -243,12 +255,18 @@ __device__ __noinline__ void prep_cta(const GroupArgs& a, int b) {
     }
   }
   __syncthreads();
+  if (tid < NP) {  // tokens of this pair's slot -> its chunk counts
+    int n = 0;
+    for (int j = 0; j < NP; ++j) n += s_slot[j] == s_slot[tid];
+    a.tb.pair_nk[tid] = input_chunks(n, a.H) | (input_chunks(n, a.I) << 8);
+  }
   const int nr = NP > 0 ? s_slot[NP - 1] + 1 : 0;
   if (tid < T) {
     a.tb.tok_pair[tid * (K + 1) + K] = shared_slot ? NP + tid : -1;
     if (shared_slot) {
       a.tb.pair_token[NP + tid] = tid;
       a.tb.pair_slot[NP + tid] = nr;
+      a.tb.pair_nk[NP + tid] = input_chunks(T, a.H) | (input_chunks(T, a.I) << 8);
     }
   }
   if (tid == 0) {
@@ -681,9 +699,8 @@ __global__ void __launch_bounds__(kStageThreads) grouped_stage_act_kernel(const 
   extern __shared__ __align__(16) float act[];  // [I]
   const int p = blockIdx.x;
   if (p >= a.tb.meta[1]) return;
-  const int s = a.tb.pair_slot[p];
-  const int n = a.tb.slot_pair0[s + 1] - a.tb.slot_pair0[s];
-  const int nk = input_chunks(n, a.H);
+  const int nk = a.tb.pair_nk[p] & 0xFF;
+  const bool routed = p < a.T * a.K;  // routed pairs come first
   const float2* part = a.gu_part + (long long)p * kMaxChunks * a.I;
   for (int r = threadIdx.x; r < a.I; r += kStageThreads) {
     float g = 0.f, u = 0.f;
@@ -697,7 +714,7 @@ __global__ void __launch_bounds__(kStageThreads) grouped_stage_act_kernel(const 
   __syncthreads();
   float4* as = a.as + (long long)p * (a.I / 4);
   float2* sf = a.sfa + (long long)p * (a.I / 32);
-  if (a.tb.slot_expert[s] >= 0 || BR == BS)
+  if (routed || BR == BS)
     stage_inputs<BR, false>(act, a.I, as, sf, threadIdx.x, kStageThreads);
   else
     stage_inputs<BS, false>(act, a.I, as, sf, threadIdx.x, kStageThreads);
@@ -815,30 +832,56 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_down_kernel(const __grid_
 
 // ---------------------------------------------------------------------------
 // combine: out[t] = residual[t] + sum_k w[t][k] y[pair(t,k)] + sg[t] y[shared pair of t]
+// One CTA per (token, 1024 outputs); each thread takes 4 consecutive outputs.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float pair_output(const GroupArgs& a, int p, int h) {
-  const int s = a.tb.pair_slot[p];
-  const int nk = input_chunks(a.tb.slot_pair0[s + 1] - a.tb.slot_pair0[s], a.I);
-  const float* y = a.y_part + (long long)p * kMaxChunks * a.H + h;
-  float v = 0.f;
-  for (int c = 0; c < nk; ++c) v += __ldcg(y + (long long)c * a.H);
-  return v;
-}
+constexpr int kCombineThreads = 256;
 
-__global__ void __launch_bounds__(256) grouped_combine_kernel(const __grid_constant__ GroupArgs a) {
-  const long long q = blockIdx.x * 256LL + threadIdx.x;
-  if (q >= (long long)a.T * a.H) return;
-  const int t = (int)(q / a.H), h = (int)(q - (long long)t * a.H);
-  float v = a.residual ? __ldg(a.residual + q) : 0.f;
-  const int* tp = a.tb.tok_pair + t * (a.K + 1);
-  for (int k = 0; k < a.K; ++k) v = fmaf(a.tb.tok_w[t * a.K + k], pair_output(a, tp[k], h), v);
-  if (tp[a.K] >= 0) v = fmaf(a.tb.tok_sg[t], pair_output(a, tp[a.K], h), v);
-  if (a.shared_tc) {
-    float y = 0.f;
-    for (int ks = 0; ks < a.I / 512; ++ks) y += __ldcg(a.sh_y + ((long long)ks * kMaxTokens + t) * a.H + h);
-    v = fmaf(a.tb.tok_sg[t], y, v);
+__global__ void __launch_bounds__(kCombineThreads) grouped_combine_kernel(const __grid_constant__ GroupArgs a) {
+  __shared__ int s_pair[kMaxTopK + 1], s_nk[kMaxTopK + 1];
+  __shared__ float s_w[kMaxTopK + 1];
+  const int t = blockIdx.y, K = a.K;
+  if (threadIdx.x <= K) {
+    const int p = a.tb.tok_pair[t * (K + 1) + threadIdx.x];
+    s_pair[threadIdx.x] = p;
+    s_nk[threadIdx.x] = p >= 0 ? (__ldcg(a.tb.pair_nk + p) >> 8) & 0xFF : 0;
+    s_w[threadIdx.x] = threadIdx.x < K ? a.tb.tok_w[t * K + threadIdx.x] : a.tb.tok_sg[t];
   }
-  a.out[q] = v;
+  __syncthreads();
+  const int h = (blockIdx.x * kCombineThreads + threadIdx.x) * 4;
+  if (h >= a.H) return;
+  const long long q = (long long)t * a.H + h;
+  float4 v = a.residual ? __ldg(reinterpret_cast<const float4*>(a.residual + q)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  auto add = [&](float w, float4 y) {
+    v.x = fmaf(w, y.x, v.x);
+    v.y = fmaf(w, y.y, v.y);
+    v.z = fmaf(w, y.z, v.z);
+    v.w = fmaf(w, y.w, v.w);
+  };
+  for (int k = 0; k <= K; ++k) {  // routed pairs in k order, then the shared pair
+    const int p = s_pair[k];
+    if (p < 0) continue;
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < s_nk[k]; ++c) {
+      const float4 u = __ldcg(reinterpret_cast<const float4*>(a.y_part + ((long long)p * kMaxChunks + c) * a.H + h));
+      y.x += u.x;
+      y.y += u.y;
+      y.z += u.z;
+      y.w += u.w;
+    }
+    add(s_w[k], y);
+  }
+  if (a.shared_tc) {
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int ks = 0; ks < a.I / 512; ++ks) {
+      const float4 u = __ldcg(reinterpret_cast<const float4*>(a.sh_y + ((long long)ks * kMaxTokens + t) * a.H + h));
+      y.x += u.x;
+      y.y += u.y;
+      y.z += u.z;
+      y.w += u.w;
+    }
+    add(s_w[K], y);
+  }
+  *reinterpret_cast<float4*>(a.out + q) = v;
 }
 
 }  // namespace fmoe

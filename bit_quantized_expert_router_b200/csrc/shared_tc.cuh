@@ -76,36 +76,46 @@ __device__ __noinline__ void tc_tile(char* sbase, const char* __restrict__ codes
   }
 
   // A: codes -> bf16, 128-byte-swizzled K-major, one 16 KB tile per group.
-  for (int idx = tid; idx < kTcRows * kTcGroups; idx += kThreads) {
-    const int g = idx % kTcGroups, r = idx / kTcGroups;
-    const char* p = codes + (long long)(r0 + r) * row_bytes + (long long)(k0 + g * 64) * BITS / 8;
-    char* dst = sbase + kTcA + g * (kTcRows * 128);
-    uint32_t w[8];
-    if (BITS == 4) {
-      const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(p)), w1 = __ldg(reinterpret_cast<const uint4*>(p) + 1);
-      w[0] = w0.x; w[1] = w0.y; w[2] = w0.z; w[3] = w0.w;
-      w[4] = w1.x; w[5] = w1.y; w[6] = w1.z; w[7] = w1.w;
+  // Each thread converts kPer (row, group) blocks; all their loads are issued
+  // before the first conversion.
+  {
+    constexpr int kPer = kTcRows * kTcGroups / kThreads;  // 2
+    constexpr int kWords = 64 * BITS / 32;                // code words per block
+    uint32_t w[kPer][kWords];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {  // chunk c = codes 8c .. 8c+7 = word c
-        const uint32_t x = w[c];
-        uint4 o;
-        o.x = ints_to_bf16x2(x & 0xFu, (x >> 4) & 0xFu);
-        o.y = ints_to_bf16x2((x >> 8) & 0xFu, (x >> 12) & 0xFu);
-        o.z = ints_to_bf16x2((x >> 16) & 0xFu, (x >> 20) & 0xFu);
-        o.w = ints_to_bf16x2((x >> 24) & 0xFu, (x >> 28) & 0xFu);
-        *reinterpret_cast<uint4*>(dst + sw128_offset(r, 8 * c)) = o;
+    for (int q = 0; q < kPer; ++q) {
+      const int idx = tid + q * kThreads, g = idx % kTcGroups, r = idx / kTcGroups;
+      const uint4* p = reinterpret_cast<const uint4*>(codes + (long long)(r0 + r) * row_bytes +
+                                                      (long long)(k0 + g * 64) * BITS / 8);
+#pragma unroll
+      for (int u = 0; u < kWords / 4; ++u) {
+        const uint4 v = __ldg(p + u);
+        w[q][4 * u] = v.x;
+        w[q][4 * u + 1] = v.y;
+        w[q][4 * u + 2] = v.z;
+        w[q][4 * u + 3] = v.w;
       }
-    } else {
-      const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(p));
-      w[0] = w0.x; w[1] = w0.y; w[2] = w0.z; w[3] = w0.w;
+    }
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {  // chunk c = codes 8c .. 8c+7 = half c%2 of word c/2
-        const uint32_t x = w[c >> 1] >> (16 * (c & 1));
+    for (int q = 0; q < kPer; ++q) {
+      const int idx = tid + q * kThreads, g = idx % kTcGroups, r = idx / kTcGroups;
+      char* dst = sbase + kTcA + g * (kTcRows * 128);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {  // chunk c = codes 8c .. 8c+7
         uint4 o;
-        o.x = ints_to_bf16x2(x & 3u, (x >> 2) & 3u);
-        o.y = ints_to_bf16x2((x >> 4) & 3u, (x >> 6) & 3u);
-        o.z = ints_to_bf16x2((x >> 8) & 3u, (x >> 10) & 3u);
-        o.w = ints_to_bf16x2((x >> 12) & 3u, (x >> 14) & 3u);
+        if (BITS == 4) {
+          const uint32_t x = w[q][c];
+          o.x = ints_to_bf16x2(x & 0xFu, (x >> 4) & 0xFu);
+          o.y = ints_to_bf16x2((x >> 8) & 0xFu, (x >> 12) & 0xFu);
+          o.z = ints_to_bf16x2((x >> 16) & 0xFu, (x >> 20) & 0xFu);
+          o.w = ints_to_bf16x2((x >> 24) & 0xFu, (x >> 28) & 0xFu);
+        } else {  // half c % 2 of word c / 2
+          const uint32_t x = w[q][c >> 1] >> (16 * (c & 1));
+          o.x = ints_to_bf16x2(x & 3u, (x >> 2) & 3u);
+          o.y = ints_to_bf16x2((x >> 4) & 3u, (x >> 6) & 3u);
+          o.z = ints_to_bf16x2((x >> 8) & 3u, (x >> 10) & 3u);
+          o.w = ints_to_bf16x2((x >> 12) & 3u, (x >> 14) & 3u);
+        }
         *reinterpret_cast<uint4*>(dst + sw128_offset(r, 8 * c)) = o;
       }
     }
@@ -254,22 +264,25 @@ __global__ void __launch_bounds__(kThreads, 1) prep_shared_down_kernel(const __g
   const float* gp = a.sh_gu;
   const float* up = a.sh_gu + (long long)KSg * kMaxTokens * a.I;
   const int I = a.I;
+  // (per float4 of inputs, the partials of all input tiles are loaded together
+  // and then summed in tile order)
   auto src = [gp, up, I, KSg](int t, int k, float (&v)[16]) {
-    float g[16], u[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) g[i] = u[i] = 0.f;
-    for (int s = 0; s < KSg; ++s) {
-      const float4* pg = reinterpret_cast<const float4*>(gp + ((long long)s * kMaxTokens + t) * I + k);
-      const float4* pu = reinterpret_cast<const float4*>(up + ((long long)s * kMaxTokens + t) * I + k);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 a4 = __ldcg(pg + i), b4 = __ldcg(pu + i);
-        g[4 * i] += a4.x; g[4 * i + 1] += a4.y; g[4 * i + 2] += a4.z; g[4 * i + 3] += a4.w;
-        u[4 * i] += b4.x; u[4 * i + 1] += b4.y; u[4 * i + 2] += b4.z; u[4 * i + 3] += b4.w;
+    for (int i = 0; i < 4; ++i) {
+      float4 g = make_float4(0.f, 0.f, 0.f, 0.f), u = g;
+#pragma unroll 8
+      for (int s = 0; s < KSg; ++s) {
+        const long long off = ((long long)s * kMaxTokens + t) * I + k;
+        const float4 a4 = __ldcg(reinterpret_cast<const float4*>(gp + off) + i);
+        const float4 b4 = __ldcg(reinterpret_cast<const float4*>(up + off) + i);
+        g.x += a4.x; g.y += a4.y; g.z += a4.z; g.w += a4.w;
+        u.x += b4.x; u.y += b4.y; u.z += b4.z; u.w += b4.w;
       }
+      v[4 * i] = g.x * sigmoidf_(g.x) * u.x;
+      v[4 * i + 1] = g.y * sigmoidf_(g.y) * u.y;
+      v[4 * i + 2] = g.z * sigmoidf_(g.z) * u.z;
+      v[4 * i + 3] = g.w * sigmoidf_(g.w) * u.w;
     }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = g[i] * sigmoidf_(g[i]) * u[i];
   };
   const char* codes = a.shared + a.off_s[4];
   const uint32_t* sbw = reinterpret_cast<const uint32_t*>(a.shared + a.off_s[5]);

@@ -284,15 +284,30 @@ def top5_min_gap(logits: np.ndarray, k: int = 4) -> float:
 # The layer
 # ---------------------------------------------------------------------------
 
+def rms_norm(x, w_bf16, eps: float) -> np.ndarray:
+    """x / sqrt(mean(x^2) + eps) * w, in fp64 with the bf16 weight widened exactly.
+
+    The pages name the step only ("combine + norm" feeding the next layer,
+    [P2 "Verzögerte GPU-Experten-Berechnung"]); this is the plain RMS
+    normalisation with a per-element weight.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt(np.mean(x * x) + eps) * bf16_to_f64(w_bf16)
+
+
 def layer_decode(w_router_bf16, w_sgate_bf16, get_expert_blob, shared_blob,
                  x, residual, top_k: int, hidden: int, inter: int, bits: int,
-                 shared_bits: int = 4) -> dict:
+                 shared_bits: int = 4, norm_w_bf16=None, norm_eps: float = 1e-6) -> dict:
     """One MoE layer for one token.
 
     out = residual + sum_k w_k * y_{idx_k} + sg * y_shared
     ([P2 "Metal-Compute-Shader"]: "MoE-Kombination + Rest + Sigmoid-Gate").
     ``get_expert_blob(e)`` returns expert e's blob; ``shared_blob`` may be None.
+    With ``norm_w_bf16`` the layer's input is first ``rms_norm(x, norm_w, eps)``
+    (the residual is not normalised).
     """
+    if norm_w_bf16 is not None:
+        x = rms_norm(x, norm_w_bf16, norm_eps)
     r = route(w_router_bf16, w_sgate_bf16, x, top_k)
     out = np.asarray(residual, dtype=np.float64).copy()
     ys = []

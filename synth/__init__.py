@@ -41,6 +41,7 @@ TAG_X = 0x7E5
 TAG_RES = 0x2E5
 TAG_SGATE = 0x5647E
 TAG_DENSE = 0xDE45E
+TAG_NORM = 0x40235
 
 GROUP = 64  # quantisation group length along the input dimension
 
@@ -164,6 +165,13 @@ def sgate_bf16(seed: int, layer: int, hidden: int) -> np.ndarray:
     """uint16 [H] bf16 bit patterns of the shared-expert gate vector, ~N(0, 0.02)."""
     g = _rng(seed, TAG_SGATE, layer)
     w = g.normal(0.0, 0.02, size=hidden).astype(np.float32)
+    return bf16_bits_rne(w)
+
+
+def norm_bf16(seed: int, layer: int, hidden: int) -> np.ndarray:
+    """uint16 [H] bf16 bit patterns of an RMS-norm weight, ~N(1, 0.1)."""
+    g = _rng(seed, TAG_NORM, layer)
+    w = g.normal(1.0, 0.1, size=hidden).astype(np.float32)
     return bf16_bits_rne(w)
 
 

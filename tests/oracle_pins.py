@@ -375,6 +375,22 @@ def pin_layer(O):
     r = O.layer_decode(wr, None, lambda e: b2, shared, x, res, 1, hidden, inter, 2, shared_bits=4)
     np.testing.assert_allclose(r["out"], res + O.expert_forward(b2, hidden, inter, 2, x) + ysh,
                                rtol=1e-12, atol=1e-12)
+    # (e) input RMS norm (unit weight, eps 0): the layer sees x / rms(x), so scaling
+    # x by a power of two leaves the decision and the MoE output unchanged,
+    # and the result equals the un-normalised layer on x / rms(x)
+    ones = np.full(hidden, 0x3F80, dtype=np.uint16)
+    zero = np.zeros(hidden)
+    rn = O.layer_decode(wr, None, lambda e: blobs[e], shared, x, zero, 2, hidden, inter, bits,
+                        norm_w_bf16=ones, norm_eps=0.0)
+    rs = O.layer_decode(wr, None, lambda e: blobs[e], shared, x * 8.0, zero, 2, hidden, inter, bits,
+                        norm_w_bf16=ones, norm_eps=0.0)
+    assert rn["idx"].tolist() == rs["idx"].tolist()
+    np.testing.assert_allclose(rs["out"], rn["out"], rtol=1e-12, atol=1e-12)
+    xn = x / math.sqrt(float(np.mean(x * x)))
+    r0 = O.layer_decode(wr, None, lambda e: blobs[e], shared, xn, zero, 2, hidden, inter, bits)
+    np.testing.assert_allclose(rn["out"], r0["out"], rtol=1e-12, atol=1e-12)
+    assert np.max(np.abs(rn["out"] - O.layer_decode(wr, None, lambda e: blobs[e], shared, x, zero, 2, hidden,
+                                                    inter, bits)["out"])) > 1e-6  # the norm matters here
 
 
 def pin_quantizer(O):
@@ -423,6 +439,30 @@ def pin_quantizer(O):
         assert np.max(np.abs(m - ref)) < 0.02 * 8 / 15
 
 
+def pin_rms_norm(O):
+    """RMS normalisation against closed forms (eps = 0 unless stated)."""
+    one = np.full(8, 0x3F80, dtype=np.uint16)  # bf16 1.0
+    # a constant vector normalises to +-1 exactly
+    assert np.array_equal(O.rms_norm(np.full(8, -3.0), one, 0.0), np.full(8, -1.0))
+    # (3, 4): mean of squares 12.5, so the result is (3, 4) / sqrt(12.5) = (3, 4) * sqrt(2) / 5
+    got = O.rms_norm(np.array([3.0, 4.0]), one[:2], 0.0)
+    np.testing.assert_allclose(got, np.array([3.0, 4.0]) * np.sqrt(2.0) / 5.0, rtol=1e-15, atol=0)
+    # scale invariance by powers of two (exact), and mean of squares 1 with unit weight
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal(256)
+    y = O.rms_norm(x, np.full(256, 0x3F80, dtype=np.uint16), 0.0)
+    assert np.array_equal(O.rms_norm(x * 2.0**-7, np.full(256, 0x3F80, dtype=np.uint16), 0.0), y)
+    assert abs(np.mean(y * y) - 1.0) < 1e-14
+    # the weight multiplies element by element (bf16 2.0 = 0x4000, 0.5 = 0x3F00)
+    w = np.where(np.arange(256) % 2 == 0, 0x4000, 0x3F00).astype(np.uint16)
+    yw = O.rms_norm(x, w, 0.0)
+    assert np.array_equal(yw[0::2], 2.0 * y[0::2]) and np.array_equal(yw[1::2], 0.5 * y[1::2])
+    # eps keeps a zero input finite (zero)
+    assert np.array_equal(O.rms_norm(np.zeros(4), one[:4], 1e-6), np.zeros(4))
+    # eps enters under the root: x = (1, 1), eps = 3 -> 1 / sqrt(4) = 0.5
+    assert np.array_equal(O.rms_norm(np.ones(2), one[:2], 3.0), np.full(2, 0.5))
+
+
 ALL_PINS = [pin_expert_size, pin_packing_golden, pin_fma_identity_exact, pin_constant_codes,
             pin_one_hot, pin_permutation_expert, pin_dense_bruteforce, pin_activations,
-            pin_routing, pin_layer, pin_quantizer]
+            pin_routing, pin_layer, pin_quantizer, pin_rms_norm]

@@ -120,6 +120,27 @@ def _quantize_floor(w, bits):
     return O.pack_codes(q.reshape(n, kdim), bits), sbits.astype(np.uint32) | (bbits.astype(np.uint32) << 16)
 
 
+def _rms_norm_mean_abs(x, w_bf16, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return x / (np.mean(np.abs(x)) + eps) * O.bf16_to_f64(w_bf16)
+
+
+def _rms_norm_no_sqrt(x, w_bf16, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return x / (np.mean(x * x) + eps) * O.bf16_to_f64(w_bf16)
+
+
+def _rms_norm_no_weight(x, w_bf16, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt(np.mean(x * x) + eps)
+
+
+def _layer_ignores_norm(*a, **kw):
+    kw.pop("norm_w_bf16", None)
+    kw.pop("norm_eps", None)
+    return ORIG_LAYER(*a, **kw)
+
+
 ORIG_ROUTE = O.route
 ORIG_LAYER = O.layer_decode
 ORIG_QUANT = O.quantize_matrix
@@ -141,6 +162,10 @@ MUTANTS = {
     "expert_bytes_wrong": ("expert_bytes", _expert_bytes_bf16_once),
     "quantizer_bias_is_max": ("quantize_matrix", _quantize_bias_max),
     "quantizer_floor": ("quantize_matrix", _quantize_floor),
+    "rms_norm_mean_abs": ("rms_norm", _rms_norm_mean_abs),
+    "rms_norm_no_sqrt": ("rms_norm", _rms_norm_no_sqrt),
+    "rms_norm_no_weight": ("rms_norm", _rms_norm_no_weight),
+    "layer_ignores_norm": ("layer_decode", _layer_ignores_norm),
 }
 
 

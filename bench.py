@@ -54,7 +54,7 @@ CONFIGS = {
     "tiny": dict(workload="tiny_h512_i128_e16_k4_shared_4bit", hidden=512, inter=128, experts=16, top_k=4,
                  bits=4, shared_bits=4),
     # 40 independent full-size 4-bit layers (145.6 GB of experts); a step is one
-    # token decoded through all 40 layers.
+    # token decoded through all 40 layers, each normalising its input.
     "stacked": dict(workload="stacked_40x_full_h4096_i1024_e512_k4_shared_4bit", hidden=4096, inter=1024,
                     experts=512, top_k=4, bits=4, shared_bits=4, layers_per_step=40),
     # 16 tokens per step through the full-size 4-bit layer, grouped by expert.
@@ -287,8 +287,10 @@ def run_fmoe(args, cfg, rank, world, local_rank):
     for l in range(NL):
         t = SG.make_layer(SEED + 1000 * rank, l, h, i, e, cfg["bits"], cfg["shared_bits"], F.blob_offsets,
                           F.expert_bytes, dev)
+        # stacked layers normalise their input (the decoder stack's RMS norm)
+        nw = SG.bf16_tensor(S.norm_bf16(SEED + 1000 * rank, l, h), dev) if LPS > 1 else None
         layers.append(F.Layer(t["w_router"], t["w_sgate"], t["experts"], t["shared"], h, i, k, cfg["bits"],
-                              cfg["shared_bits"]))
+                              cfg["shared_bits"], norm_weight=nw))
     TT = cfg.get("tokens", 1)  # tokens per decode call
     shape = (POOL, h) if TT == 1 else (POOL, TT, h)
     xs = torch.from_numpy(S.token_x(SEED + rank, 0, 0, POOL * TT, h).reshape(shape)).to(dev)
@@ -305,7 +307,8 @@ def run_fmoe(args, cfg, rank, world, local_rank):
             layers[l].decode(xs[j % POOL], rs[j % POOL], out=out[j % POOL], ws=ws[l])
         else:
             # Stacked layers: layer l reads the hidden state layer l - 1 wrote,
-            # as both its input and its residual; layer 0 starts from a pool token.
+            # as its input (normalised inside) and its residual; layer 0 starts
+            # from a pool token.
             src = xs[(j // NL) % POOL] if l == 0 else hbuf[(l - 1) % 2]
             layers[l].decode(src, src, out=hbuf[l % 2], ws=ws[l])
 

@@ -45,6 +45,7 @@ class FmoeLayerC(ctypes.Structure):
         ("expert_stride", ctypes.c_int64), ("shared", ctypes.c_void_p), ("hidden", ctypes.c_int),
         ("inter", ctypes.c_int), ("n_experts", ctypes.c_int), ("top_k", ctypes.c_int),
         ("bits", ctypes.c_int), ("shared_bits", ctypes.c_int), ("group", ctypes.c_int),
+        ("norm_weight", ctypes.c_void_p), ("norm_eps", ctypes.c_float),
     ]
 
 
@@ -202,7 +203,8 @@ class Layer:
     """Device-resident weights of one MoE layer (all tensors on one GPU).
 
     experts: uint8 [E][stride] packed routed experts; shared: uint8 blob or None;
-    w_router: int16 [E][H] bf16 bits; w_sgate: int16 [H] bf16 bits or None.
+    w_router: int16 [E][H] bf16 bits; w_sgate: int16 [H] bf16 bits or None;
+    norm_weight: int16 [H] bf16 bits or None (input RMS norm with norm_eps).
     """
     w_router: torch.Tensor
     w_sgate: torch.Tensor | None
@@ -213,9 +215,13 @@ class Layer:
     top_k: int
     bits: int = 4
     shared_bits: int = 4
+    norm_weight: torch.Tensor | None = None
+    norm_eps: float = 1e-6
 
     def __post_init__(self):
         _dev_tensor(self.w_router, torch.int16, "w_router")
+        if self.norm_weight is not None:
+            _dev_tensor(self.norm_weight, torch.int16, "norm_weight")
         if self.w_sgate is not None:
             _dev_tensor(self.w_sgate, torch.int16, "w_sgate")
         _dev_tensor(self.experts, torch.uint8, "experts")
@@ -227,7 +233,8 @@ class Layer:
             expert_stride=self.experts.stride(0) if self.experts.dim() == 2 else expert_bytes(
                 self.hidden, self.inter, self.bits),
             shared=_ptr(self.shared), hidden=self.hidden, inter=self.inter, n_experts=self.n_experts,
-            top_k=self.top_k, bits=self.bits, shared_bits=self.shared_bits, group=GROUP)
+            top_k=self.top_k, bits=self.bits, shared_bits=self.shared_bits, group=GROUP,
+            norm_weight=_ptr(self.norm_weight), norm_eps=float(self.norm_eps))
         self._ws = None
 
     def workspace_bytes(self, T: int = 1) -> int:

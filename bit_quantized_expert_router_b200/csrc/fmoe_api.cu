@@ -156,7 +156,7 @@ size_t layer_ws_bytes(int E, int I, int K) {
 // Workspace of the grouped (T >= 2) decode, byte offsets (every section 256-B aligned).
 struct GroupedLayout {
   size_t logits, meta, slot_expert, slot_pair0, pair_token, pair_slot, pair_nk, tok_pair, tok_w, tok_sg;
-  size_t xs_r, sf_r, xs_s, sf_s, gu_part, as, sfa, y_part, sh_gu, sh_y, total;
+  size_t xs_r, sf_r, xs_s, sf_s, gu_part, as, sfa, y_part, sh_gu, sh_y, xn, total;
 };
 
 GroupedLayout grouped_layout(int E, int H, int I, int K, int T) {
@@ -189,6 +189,7 @@ GroupedLayout grouped_layout(int E, int H, int I, int K, int T) {
   // tensor-core shared expert partials (used when H and I are multiples of 512)
   g.sh_gu = take((size_t)2 * (H / kTcK) * kMaxTokens * I * 4);
   g.sh_y = take((size_t)(I / kTcK) * kMaxTokens * H * 4);
+  g.xn = take((size_t)T * H * 4);  // the normalised inputs (input norm)
   g.total = off;
   return g;
 }
@@ -211,6 +212,7 @@ GroupedFns grouped_fns(int br, int bs) {
 // Launch the grouped decode (router, prep, gate/up, activation staging, down).
 int launch_grouped(const fmoe_layer* L, const float* x, const float* residual, float* out, int T, void* ws,
                    int32_t* idx_out, float* w_out, DevInfo* info, cudaStream_t s) {
+  const float* x_in = x;
   const int H = L->hidden, I = L->inter, E = L->n_experts, K = L->top_k, G = info->sms;
   const bool has_shared = L->shared != nullptr;
   const int br = L->bits, bs = has_shared ? L->shared_bits : L->bits;
@@ -221,6 +223,9 @@ int launch_grouped(const fmoe_layer* L, const float* x, const float* residual, f
   a.experts = static_cast<const char*>(L->experts);
   a.expert_stride = L->expert_stride;
   a.shared = static_cast<const char*>(L->shared);
+  // With an input norm every later step reads the normalised inputs.
+  float* xn = reinterpret_cast<float*>(w8 + gl.xn);
+  if (L->norm_weight) x = xn;
   a.x = x;
   a.residual = residual;
   a.out = out;
@@ -303,6 +308,8 @@ int launch_grouped(const fmoe_layer* L, const float* x, const float* residual, f
         return cuda_fail(e);
     info->grouped_attr_set[fi] = true;
   }
+  if (L->norm_weight)
+    rms_norm_tokens_kernel<<<T, kNormThreads, 0, s>>>(x_in, L->norm_weight, L->norm_eps, H, xn);
   const int rows = E + (L->w_sgate ? 1 : 0);
   const int router_ctas = (rows + kRouterRows - 1) / kRouterRows;
   if (a.shared_tc) {
@@ -528,6 +535,8 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
       (L->w_sgate && !aligned(L->w_sgate, 16)) || !aligned(x, 16) || !aligned(out, 16) ||
       (residual && !aligned(residual, 16)) || !aligned(ws, 256) || x == out)
     return FMOE_EINVAL;
+  if (L->norm_weight && (!aligned(L->norm_weight, 16) || !(L->norm_eps >= 0.f) || !(L->norm_eps < INFINITY)))
+    return FMOE_EINVAL;
   if (ws_bytes < fmoe_workspace_bytes(L, T)) return FMOE_ENOMEM;
   int dev;
   DevInfo* info;
@@ -570,6 +579,8 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
   a.c_stage_bytes = pl.c_stage_bytes;
   a.lg_floats = pl.lg_floats;
   a.timeout_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  a.norm_w = L->norm_weight;
+  a.norm_eps = L->norm_eps;
   // A router warp's row (2H bytes) fits in its ring: copy it there at entry.
   a.router_smem = (long long)pl.nst * pl.stage_bytes >= 2LL * H ? 1 : 0;
   set_offsets(a, info->sms);

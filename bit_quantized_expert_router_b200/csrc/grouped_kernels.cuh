@@ -188,6 +188,30 @@ __global__ void __launch_bounds__(kThreads) router_tokens_kernel(const uint16_t*
 }
 
 // ---------------------------------------------------------------------------
+// input RMS norm: xn[t] = x[t] / sqrt(mean(x[t]^2) + eps) * w (one CTA per token)
+// ---------------------------------------------------------------------------
+constexpr int kNormThreads = 256;
+
+__global__ void __launch_bounds__(kNormThreads) rms_norm_tokens_kernel(const float* __restrict__ x,
+                                                                       const uint16_t* __restrict__ w, float eps,
+                                                                       int H, float* __restrict__ xn) {
+  __shared__ float red[kNormThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const float* xt = x + (long long)blockIdx.x * H;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < H; i += kNormThreads) ss = fmaf(xt[i], xt[i], ss);
+  ss = warp_sum(ss);
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int k = 0; k < kNormThreads / 32; ++k) tot += red[k];
+  const float r = 1.0f / sqrtf(tot / (float)H + eps);
+  for (int i = threadIdx.x; i < H; i += kNormThreads)
+    xn[(long long)blockIdx.x * H + i] = xt[i] * r * __uint_as_float((uint32_t)__ldg(w + i) << 16);
+}
+
+// ---------------------------------------------------------------------------
 // prep: top-K per token, grouping, input staging
 // ---------------------------------------------------------------------------
 // CTA `b` of the prep step (0 <= b <= T): b = 0 routes and groups, b > 0

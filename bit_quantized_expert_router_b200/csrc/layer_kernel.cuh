@@ -91,6 +91,8 @@ struct LayerArgs {
   long long off_r[6], off_s[6];  // blob section offsets for the routed / shared code width
   unsigned long long timeout_ns;
   int router_smem;           // 1: each router warp's row is bulk-copied into its ring at entry
+  const uint16_t* norm_w;    // [H] bf16 RMS-norm weight of the input, or null
+  float norm_eps;
 };
 
 struct Smem {
@@ -169,6 +171,7 @@ struct CtaShared {
   uint64_t lg_bar;      // completes once the router logits are in shared memory
   uint64_t rbar[kWarps];  // router warp w's row is in its ring (router_smem)
   unsigned long long param_touch;  // see the kernel's set-up
+  float red[kWarps];               // per-warp partial sums (input norm)
   float* lg;            // shared-memory copy of the router logits
   unsigned lg_bytes;
   int c_prefetch;          // warps past their gate/up work (the first prefetches down rows)
@@ -702,6 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
                       a.nst ^ a.stage_bytes ^ a.nst_c ^ a.c_stage_bytes ^ a.xs4_off ^ a.xs2_off ^ a.xu_off ^
                       a.vec_floats ^ a.sf_floats ^ a.ys_stride ^ a.lg_floats ^ a.router_smem);
       for (int i = 0; i < 6; ++i) t += (unsigned long long)(a.off_r[i] ^ a.off_s[i]);
+      t ^= (uintptr_t)a.norm_w ^ (unsigned long long)__float_as_uint(a.norm_eps);
       *(volatile unsigned long long*)&cs.param_touch = t;
     }
     // The shared (or single) expert; the routed slots point at expert 0 until
@@ -709,8 +713,11 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     for (int k = 0; k < a.K; ++k) cs.blob[k] = a.experts;
     cs.blob[a.K] = a.shared;
     fence_proxy_async_smem();
-    mbar_arrive_expect_tx(&cs.x_bar, a.H * 4);
+    // x, and the input-norm weight (into the staging area, free until the
+    // staging that follows the norm)
+    mbar_arrive_expect_tx(&cs.x_bar, a.H * 4 + (a.norm_w ? a.H * 2 : 0));
     bulk_g2s(sm.vec + a.xu_off, a.x, a.H * 4, &cs.x_bar);
+    if (a.norm_w) bulk_g2s(sm.vec + (a.xs4_off >= 0 ? a.xs4_off : a.xs2_off), a.norm_w, a.H * 2, &cs.x_bar);
   }
   if (lane == 0) {
     if (a.router_smem && plan.router.count == 1) {
@@ -736,6 +743,24 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   int issued = 0;
   if (!mbar_wait_bounded(&cs.x_bar, 0, a.timeout_ns) && lane == 0) set_status(kStatusCopyTimeout);
   FMOE_TRACE_WARP(16);
+  if (a.norm_w) {
+    // Input RMS norm, in place: x <- x / sqrt(mean(x^2) + eps) * w.  Every
+    // thread sums the per-warp partials in the same order, so all use the
+    // same factor.
+    float* xw = sm.vec + a.xu_off;
+    const uint16_t* wn = reinterpret_cast<const uint16_t*>(sm.vec + (a.xs4_off >= 0 ? a.xs4_off : a.xs2_off));
+    float ss = 0.f;
+    for (int i = tid; i < a.H; i += kThreads) ss = fmaf(xw[i], xw[i], ss);
+    ss = warp_sum(ss);
+    if (lane == 0) cs.red[warp] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) tot += cs.red[w];
+    const float r = 1.0f / sqrtf(tot / (float)a.H + a.norm_eps);
+    for (int i = tid; i < a.H; i += kThreads) xw[i] = xw[i] * r * __uint_as_float((uint32_t)wn[i] << 16);
+    __syncthreads();
+  }
   const float* xu = sm.vec + a.xu_off;
   if (router_warp) {
     // ---- Phase A, router rows: published, then counted once per CTA ---------

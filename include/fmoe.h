@@ -147,6 +147,14 @@ typedef struct {
   int bits;                 /* routed experts: 4 or 2 */
   int shared_bits;          /* shared expert: 4 or 2 */
   int group;                /* must be 64 */
+  /* Optional input normalisation (the "norm" that ends the previous layer's
+   * step in [P2] "Verzögerte GPU-Experten-Berechnung", here fused into the
+   * start of this layer): when norm_weight is non-NULL the experts and the
+   * router see x / sqrt(mean(x^2) + norm_eps) * norm_weight instead of x; the
+   * residual is used as given.  norm_weight: [hidden] bf16 bits, 16-byte
+   * aligned; norm_eps: finite, >= 0 (1e-6 is usual). */
+  const uint16_t* norm_weight;
+  float norm_eps;
 } fmoe_layer;
 
 /* Workspace bytes needed by fmoe_layer_decode for T tokens. */

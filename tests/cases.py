@@ -40,7 +40,7 @@ def cpu_blob(seed: int, layer: int, expert: int, hidden: int, inter: int, bits: 
 
 
 def parity_x(seed: int, layer: int, step: int, w_router_bf16: np.ndarray, top_k: int, hidden: int,
-             n_tokens: int = 1) -> np.ndarray:
+             n_tokens: int = 1, norm_w=None, norm_eps: float = 1e-6) -> np.ndarray:
     """Token vectors whose router logits have no near-tie among the top K+1.
 
     A token is redrawn from an independent substream until the smallest gap
@@ -51,7 +51,8 @@ def parity_x(seed: int, layer: int, step: int, w_router_bf16: np.ndarray, top_k:
     for t in range(n_tokens):
         for redraw in range(1000):
             x = S.token_x(seed, layer, step * 64 + t, 1, hidden, redraw)[0]
-            lg = O.router_logits(w_router_bf16, x)
+            xr = x if norm_w is None else O.rms_norm(x, norm_w, norm_eps)  # what the router sees
+            lg = O.router_logits(w_router_bf16, xr)
             if O.top5_min_gap(lg, top_k) >= NEAR_TIE:
                 out[t] = x
                 break
@@ -61,7 +62,7 @@ def parity_x(seed: int, layer: int, step: int, w_router_bf16: np.ndarray, top_k:
 
 
 def oracle_layer(seed: int, layer: int, shape: Shape, x: np.ndarray, residual: np.ndarray,
-                 with_shared: bool = True, with_sgate: bool = True) -> dict:
+                 with_shared: bool = True, with_sgate: bool = True, norm_w=None, norm_eps: float = 1e-6) -> dict:
     """Oracle output of one token through a synthetic layer."""
     H, I = shape.hidden, shape.inter
     w_router = S.router_bf16(seed, layer, shape.n_experts, H)
@@ -75,7 +76,7 @@ def oracle_layer(seed: int, layer: int, shape: Shape, x: np.ndarray, residual: n
         return cache[e]
 
     return O.layer_decode(w_router, w_sg, get, shared, x, residual, shape.top_k, H, I, shape.bits,
-                          shape.shared_bits)
+                          shape.shared_bits, norm_w_bf16=norm_w, norm_eps=norm_eps)
 
 
 def errors(got: np.ndarray, want: np.ndarray) -> tuple[float, float]:

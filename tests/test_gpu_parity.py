@@ -411,3 +411,36 @@ def test_layer_exact_ties_pick_lowest_indices(F, SG, T):
                            shared, x[k], res[k], shape.top_k, shape.hidden, shape.inter, shape.bits, shape.shared_bits)
         assert r["idx"].tolist() == [0, 1, 2, 3]
         C.assert_close(out.cpu().numpy()[k], r["out"], f"tied token {k}")
+
+
+# ---------------------------------------------------------------------------
+# Input RMS norm (the next layer's norm fused into the layer start)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("shape,T", [(C.TINY, 1), (C.FULL4, 1), (C.FULL2, 1), (C.TINY, 7), (C.FULL4, 16),
+                                     (C.Shape("norm_h1024_i256_e64_k4", 1024, 256, 64, 4, 4), 5)],
+                         ids=lambda v: v.name if isinstance(v, C.Shape) else str(v))
+def test_layer_input_norm(F, SG, shape, T):
+    seed, layer, eps = 51, 2, 1e-5
+    L0, t = make_gpu_layer(F, SG, seed, layer, shape)
+    nw = S.norm_bf16(seed, layer, shape.hidden)
+    L = F.Layer(t["w_router"], t["w_sgate"], t["experts"], t["shared"], shape.hidden, shape.inter, shape.top_k,
+                shape.bits, shape.shared_bits, norm_weight=SG.bf16_tensor(nw, dev()), norm_eps=eps)
+    wr = S.router_bf16(seed, layer, shape.n_experts, shape.hidden)
+    # un-normalised inputs of different scales (the norm removes most of the
+    # scale); the near-tie screen looks at what the router will see
+    x = np.empty((T, shape.hidden), dtype=np.float32)
+    for k in range(T):
+        for redraw in range(1000):
+            xk = S.token_x(seed, layer, k, 1, shape.hidden, redraw)[0] * np.float32(0.5 + k)
+            if O.top5_min_gap(O.router_logits(wr, O.rms_norm(xk, nw, eps)), shape.top_k) >= C.NEAR_TIE:
+                x[k] = xk
+                break
+    res = S.token_residual(seed, layer, 0, T, shape.hidden)
+    idx = torch.empty(T, shape.top_k, dtype=torch.int32, device=dev())
+    out = L.decode(torch.from_numpy(x).to(dev()), torch.from_numpy(res).to(dev()), idx_out=idx)
+    assert F.get_status() == 0
+    for k in range(T):
+        r = C.oracle_layer(seed, layer, shape, x[k], res[k], norm_w=nw, norm_eps=eps)
+        assert idx.cpu().numpy()[k].tolist() == r["idx"].tolist(), f"token {k}"
+        C.assert_close(out.cpu().numpy()[k], r["out"], f"{shape.name} T={T} token {k} (input norm)")

@@ -1,0 +1,115 @@
+"""Stacked decode at full size: 40 chained layers, 64 steps, replayed from one
+CUDA graph (the bench's stacked workload).
+
+Layer l's input and residual are layer l - 1's output (layer 0 starts from a
+pool token); each layer RMS-normalises its input with its own weight (as a
+decoder stack does), so the hidden state stays bounded over the 40 layers.
+Every layer is checked on the input the engine actually gave it:
+the routing of all 40 x 64 (layer, step) pairs against the fp64 router, and
+the full output against the oracle on every layer of the first and last step
+plus 32 random pairs.  An input whose top-(K+1) router logits have an adjacent
+gap below the near-tie bound only needs a valid top-K (within that bound).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth as S
+from tests import cases as C
+
+pytestmark = pytest.mark.gpu
+
+N_LAYERS, N_STEPS, SEED, EPS = 40, 64, 13, 1e-6
+
+
+@pytest.fixture(scope="module")
+def F():
+    from bit_quantized_expert_router_b200 import build as B
+    B.build_engine()
+    import synth.gpu as SG
+    SG.build()
+    import bit_quantized_expert_router_b200 as F
+    F.lib()
+    return F
+
+
+def test_stacked_40_layers_64_steps(F):
+    import synth.gpu as SG
+    shape = C.FULL4
+    H, K, E = shape.hidden, shape.top_k, shape.n_experts
+    torch.cuda.empty_cache()
+    need = N_LAYERS * E * F.expert_bytes(H, shape.inter, shape.bits) * 1.03
+    if torch.cuda.mem_get_info()[0] < need:
+        pytest.skip(f"needs {need / 1e9:.0f} GB of free device memory")
+    dev = torch.device("cuda:0")
+    layers, norms = [], []
+    for l in range(N_LAYERS):
+        t = SG.make_layer(SEED, l, H, shape.inter, E, shape.bits, shape.shared_bits, F.blob_offsets,
+                          F.expert_bytes, dev)
+        norms.append(S.norm_bf16(SEED, l, H))
+        layers.append(F.Layer(t["w_router"], t["w_sgate"], t["experts"], t["shared"], H, shape.inter, K,
+                              shape.bits, shape.shared_bits, norm_weight=SG.bf16_tensor(norms[l], dev),
+                              norm_eps=EPS))
+    x0 = torch.empty(H, dtype=torch.float32, device=dev)
+    hs = torch.empty(N_LAYERS, H, dtype=torch.float32, device=dev)
+    idx = torch.empty(N_LAYERS, K, dtype=torch.int32, device=dev)
+    ws = [L.workspace(1) for L in layers]
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for L, w in zip(layers, ws):  # resolve the stream's device before capture
+            L.decode(x0, x0, out=hs[0], ws=w)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            src = x0
+            for l, L in enumerate(layers):
+                L.decode(src, src, out=hs[l], idx_out=idx[l], ws=ws[l])
+                src = hs[l]
+    wr0 = S.router_bf16(SEED, 0, E, H)
+    inputs = np.empty((N_STEPS, N_LAYERS, H), dtype=np.float32)  # the input each layer got
+    outs = np.empty((N_STEPS, N_LAYERS, H), dtype=np.float32)
+    got_idx = np.empty((N_STEPS, N_LAYERS, K), dtype=np.int64)
+    for step in range(N_STEPS):
+        x = C.parity_x(SEED, 0, step, wr0, K, H, norm_w=norms[0], norm_eps=EPS)[0]
+        x0.copy_(torch.from_numpy(x))
+        g.replay()
+        torch.cuda.synchronize()
+        assert F.get_status() == 0
+        o = hs.cpu().numpy()
+        inputs[step, 0] = x
+        inputs[step, 1:] = o[:-1]
+        outs[step] = o
+        got_idx[step] = idx.cpu().numpy()
+    del g
+
+    # routing of every (layer, step) pair against the fp64 router
+    near_ties = 0
+    for l in range(N_LAYERS):
+        wr = O.bf16_to_f64(S.router_bf16(SEED, l, E, H))
+        xn = np.stack([O.rms_norm(inputs[step, l], norms[l], EPS) for step in range(N_STEPS)])
+        lg_all = xn @ wr.T  # [steps][E]: what the router of layer l sees
+        for step in range(N_STEPS):
+            lg = lg_all[step]
+            want = O.top_k_order(lg, K)
+            got = got_idx[step, l].tolist()
+            if O.top5_min_gap(lg, K) >= C.NEAR_TIE:
+                assert got == list(want), f"layer {l} step {step}"
+            else:
+                near_ties += 1
+                assert len(set(got)) == K and min(lg[got]) >= np.sort(lg)[-K] - C.NEAR_TIE
+    assert near_ties <= N_LAYERS * N_STEPS // 20  # near-ties are rare
+
+    # full outputs on a sample of pairs
+    rng = np.random.default_rng(SEED)
+    pairs = [(0, l) for l in range(N_LAYERS)] + [(N_STEPS - 1, l) for l in range(N_LAYERS)]
+    pairs += [(int(rng.integers(N_STEPS)), int(rng.integers(N_LAYERS))) for _ in range(32)]
+    for step, l in pairs:
+        x = inputs[step, l]
+        lg = O.router_logits(S.router_bf16(SEED, l, E, H), O.rms_norm(x, norms[l], EPS))
+        if O.top5_min_gap(lg, K) < C.NEAR_TIE:
+            continue  # the selection may legitimately differ from the oracle's
+        r = C.oracle_layer(SEED, l, shape, x, x, norm_w=norms[l], norm_eps=EPS)
+        C.assert_close(outs[step, l], r["out"], f"stacked layer {l} step {step}")
+    del layers, ws
+    torch.cuda.empty_cache()

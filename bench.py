@@ -277,6 +277,7 @@ def run_fmoe(args, cfg, rank, world, local_rank):
         dist.barrier()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    F.set_dependent_launch(args.launch == "dependent")
     h, i, e, k = cfg["hidden"], cfg["inter"], cfg["experts"], cfg["top_k"]
     LPS = cfg.get("layers_per_step", 1)  # layer decodes per timed step
     NL = LPS if LPS > 1 else args.layers
@@ -446,7 +447,8 @@ def run_fmoe(args, cfg, rank, world, local_rank):
                                   "per group of 64, bf16 router",
                        "l2": f"inputs larger than L2: {NL} distinct layer instances decoded in turn "
                              f"({NL * e * expert_bytes(h, i, cfg['bits']) / 1e9:.0f} GB of experts), no flush",
-                       "layers_in_rotation": NL, "input_pool": POOL, "parallelism": f"replicas x{world}"},
+                       "layers_in_rotation": NL, "input_pool": POOL, "parallelism": f"replicas x{world}",
+                       **({"launch": args.launch} if TT == 1 else {})},
             "us_per_decode": 1000.0 * total_ms_max / K,
             "latency_us_l2_flushed": {"p50": statistics.median(lat_us), "p99": float(np.percentile(lat_us, 99)),
                                       "steps": len(lat_us),
@@ -489,6 +491,9 @@ def main():
     ap.add_argument("--config", choices=sorted(CONFIGS), default="full4")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--launch", choices=["dependent", "cooperative"], default="dependent",
+                    help="single-token layer kernel: programmatic dependent launch (overlaps the previous "
+                         "decode's end) or cooperative launch")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -25,7 +25,7 @@ EXPORTED = [
     "fmoe_expert_bytes", "fmoe_blob_offsets", "fmoe_quantize_expert", "fmoe_route_workspace_bytes",
     "fmoe_route", "fmoe_expert_workspace_bytes", "fmoe_expert_forward", "fmoe_workspace_bytes",
     "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status", "fmoe_strerror", "fmoe_last_cuda_error",
-    "fmoe_layer_decode_noalloc", "fmoe_set_wait_limit_ns",
+    "fmoe_layer_decode_noalloc", "fmoe_set_wait_limit_ns", "fmoe_set_dependent_launch",
 ]
 
 
@@ -79,6 +79,7 @@ def lib() -> ctypes.CDLL:
     L.fmoe_layer_decode_noalloc.argtypes = [ctypes.POINTER(FmoeLayerC), vp, vp, vp, i, vp, vp, vp]
     L.fmoe_get_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
     L.fmoe_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong)]
+    L.fmoe_set_dependent_launch.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
     L.fmoe_last_cuda_error.argtypes = []
     L.fmoe_last_cuda_error.restype = i
     L.fmoe_strerror.argtypes = [i]
@@ -286,6 +287,17 @@ def set_wait_limit_ns(limit_ns: int) -> int:
     if rc != FMOE_OK:
         raise FmoeError(rc, "fmoe_set_wait_limit_ns")
     return int(prev.value)
+
+
+def set_dependent_launch(enable: bool) -> bool:
+    """Launch the single-token layer kernel as a programmatic dependent launch
+    (True, the default: it overlaps the previous kernel's end) or as a
+    cooperative launch (False); returns the previous setting."""
+    prev = ctypes.c_int(0)
+    rc = lib().fmoe_set_dependent_launch(1 if enable else 0, ctypes.byref(prev))
+    if rc != FMOE_OK:
+        raise FmoeError(rc, "fmoe_set_dependent_launch")
+    return bool(prev.value)
 
 
 def get_status(stream=None) -> int:

@@ -95,6 +95,15 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 }
 
 // Prefetch `bytes` (multiple of 16, 16-byte aligned) of global memory into L2.
+// Programmatic dependent launch: let the next grid on the stream be
+// scheduled (its CTAs start as this grid's CTAs leave), and wait until the
+// previous grid on the stream has completed with its writes visible (no-op
+// when the launch had no programmatic dependency).
+__device__ __forceinline__ void grid_dep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }

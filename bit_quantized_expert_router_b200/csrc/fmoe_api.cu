@@ -15,6 +15,7 @@ constexpr unsigned long long kTimeoutNs = 2000000000ull;  // default bound on ev
 constexpr unsigned long long kMinWaitNs = 1000000ull;      // 1 ms
 constexpr unsigned long long kMaxWaitNs = 60000000000ull;  // 60 s
 std::atomic<unsigned long long> g_wait_limit_ns{kTimeoutNs};
+std::atomic<int> g_dependent_launch{1};
 constexpr size_t kCounterBytes = 256;
 constexpr int kMaxNst = 4;
 
@@ -23,6 +24,7 @@ struct DevInfo {
   int max_smem = 0;     // opt-in dynamic shared memory available to the layer kernel
   int optin = 0;        // opt-in shared memory per block
   bool layer_attr_set[4] = {false, false, false, false};
+  int layer_occupancy[4] = {-1, -1, -1, -1};  // resident CTAs per SM at pl.smem (-1: not asked yet)
   bool grouped_attr_set[4] = {false, false, false, false};
   int grouped_max_smem = 0;  // dynamic shared memory left by the grouped kernels' static arrays
 };
@@ -356,8 +358,35 @@ int launch_layer(const LayerArgs& args, const Plan& pl, DevInfo* info, cudaStrea
     info->layer_attr_set[fi] = true;
   }
   LayerArgs a = args;
-  void* kargs[] = {&a};
-  cudaError_t e = cudaLaunchCooperativeKernel((const void*)fn, dim3(info->sms), dim3(kThreads), kargs, pl.smem, s);
+  if (!g_dependent_launch.load(std::memory_order_relaxed)) {
+    void* kargs[] = {&a};
+    cudaError_t e = cudaLaunchCooperativeKernel((const void*)fn, dim3(info->sms), dim3(kThreads), kargs, pl.smem, s);
+    return e == cudaSuccess ? FMOE_OK : cuda_fail(e);
+  }
+  // Programmatic dependent launch: this grid's CTAs may start while the
+  // previous kernel on the stream finishes (the kernel waits for it before
+  // its first dependent access).  A plain launch gives no co-residency
+  // guarantee, so it is only made when one CTA fits on every SM; the grid
+  // is then resident once the previous grid has left (the grid barriers are
+  // bounded waits either way).
+  if (info->layer_occupancy[fi] < 0) {
+    int n = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kThreads, pl.smem);
+    if (e != cudaSuccess) return cuda_fail(e);
+    info->layer_occupancy[fi] = n;
+  }
+  if (info->layer_occupancy[fi] < 1) return FMOE_EINVAL;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(info->sms);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, fn, a);
   return e == cudaSuccess ? FMOE_OK : cuda_fail(e);
 }
 
@@ -632,6 +661,13 @@ int fmoe_last_cuda_error(void) { return g_last_cuda_error; }
 int fmoe_set_wait_limit_ns(unsigned long long limit_ns, unsigned long long* previous_opt) {
   if (limit_ns < kMinWaitNs || limit_ns > kMaxWaitNs) return FMOE_EINVAL;
   const unsigned long long old = g_wait_limit_ns.exchange(limit_ns);
+  if (previous_opt) *previous_opt = old;
+  return FMOE_OK;
+}
+
+int fmoe_set_dependent_launch(int enable, int* previous_opt) {
+  if (enable != 0 && enable != 1) return FMOE_EINVAL;
+  const int old = g_dependent_launch.exchange(enable);
   if (previous_opt) *previous_opt = old;
   return FMOE_OK;
 }

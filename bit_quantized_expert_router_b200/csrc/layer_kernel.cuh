@@ -49,7 +49,7 @@ constexpr int kMaxNstC = 8;       // most down-item stages a warp keeps in fligh
 // Optional phase trace (compile with -DFMOE_TRACE_BUILD): thread 0 of every CTA
 // stores %globaltimer at fixed points of the kernel into g_fmoe_trace.
 #ifdef FMOE_TRACE_BUILD
-constexpr int kTracePoints = 24;
+constexpr int kTracePoints = 25;
 __device__ unsigned long long g_fmoe_trace[1024][kTracePoints];
 #define FMOE_TRACE(i) \
   do { if (threadIdx.x == 0 && blockIdx.x < 1024) g_fmoe_trace[blockIdx.x][i] = globaltimer_ns(); } while (0)
@@ -681,8 +681,12 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   // Router rows go to warps w with w*G + cta < n_router, i.e. the first ones.
   const int n_router_warps = min(kWarps, max(0, (a.n_router - (int)blockIdx.x + G - 1) / G));
   FMOE_TRACE(0);
+  // The next layer decode on the stream may be scheduled now: its CTAs take
+  // the SMs this grid's CTAs leave, and do their weight-only set-up while
+  // this grid ends.
+  grid_dep_launch_dependents();
 
-  // ---- Set-up: x to shared memory by one bulk copy; prefetches to L2 --------
+  // ---- Set-up: weights only until the previous grid on the stream is done ---
   auto router_row_ptr = [&](int e) { return (e < a.E) ? a.w_router + (long long)e * a.H : a.w_sgate; };
   if (tid == 0) {
     mbar_init(&cs.x_bar, 1);
@@ -713,10 +717,9 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     for (int k = 0; k < a.K; ++k) cs.blob[k] = a.experts;
     cs.blob[a.K] = a.shared;
     fence_proxy_async_smem();
-    // x, and the input-norm weight (into the staging area, free until the
-    // staging that follows the norm)
+    // x (issued below, after the dependency wait), and the input-norm weight
+    // (into the staging area, free until the staging that follows the norm)
     mbar_arrive_expect_tx(&cs.x_bar, a.H * 4 + (a.norm_w ? a.H * 2 : 0));
-    bulk_g2s(sm.vec + a.xu_off, a.x, a.H * 4, &cs.x_bar);
     if (a.norm_w) bulk_g2s(sm.vec + (a.xs4_off >= 0 ? a.xs4_off : a.xs2_off), a.norm_w, a.H * 2, &cs.x_bar);
   }
   if (lane == 0) {
@@ -736,6 +739,11 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   }
   __syncthreads();
   FMOE_TRACE(11);
+  // x, the residual, the workspace and the outputs may be the previous grid's:
+  // no access to them before it has completed.
+  grid_dep_wait();
+  FMOE_TRACE(24);
+  if (tid == 0) bulk_g2s(sm.vec + a.xu_off, a.x, a.H * 4, &cs.x_bar);
 
   // x and the router rows are the critical path to the routing decision, so
   // they are the only traffic of the first microseconds; the shared expert's

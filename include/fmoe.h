@@ -231,6 +231,28 @@ int fmoe_last_cuda_error(void);
  * launches in flight on other threads. */
 int fmoe_set_wait_limit_ns(unsigned long long limit_ns, unsigned long long* previous_opt);
 
+/* How the single-token layer kernel (fmoe_layer_decode with T = 1,
+ * fmoe_layer_decode_noalloc with T = 1, fmoe_expert_forward) is launched,
+ * process-wide, for the calls made after this one.
+ *   1 (default): programmatic dependent launch.  The grid may start while the
+ *     previous kernel on the stream finishes: each CTA sets up its barriers
+ *     and copies its share of the router weights before it waits for that
+ *     kernel, and reads no input, output or workspace byte before.  Back-to-
+ *     back layer decodes overlap one's start with the other's end.  The
+ *     kernel's grid barriers need all of its CTAs resident at once; a plain
+ *     launch does not promise that, so it is made only when one CTA fits on
+ *     every SM (else FMOE_EINVAL), and a grid that other work keeps from
+ *     becoming resident ends with a bounded-wait status bit (see
+ *     fmoe_set_wait_limit_ns) instead of results.
+ *   0: cooperative launch, all CTAs resident by the driver's guarantee, no
+ *     overlap with the previous kernel.
+ * Outputs are bit-identical either way.  enable must be 0 or 1, else
+ * FMOE_EINVAL and nothing changes; the previous setting is stored in
+ * *previous_opt when non-NULL.  The pages have no counterpart: launch
+ * mechanics of this library.  Not synchronised with launches in flight on
+ * other threads. */
+int fmoe_set_dependent_launch(int enable, int* previous_opt);
+
 /* Static, human-readable text for an error code. */
 const char* fmoe_strerror(int code);
 

@@ -95,5 +95,10 @@ def test_invalid_arguments_rejected_on_host(F):
     assert L.fmoe_workspace_bytes(ctypes.byref(c), 1) >= 256 + 513 * 4 + 5 * 1024 * 4
     assert L.fmoe_workspace_bytes(ctypes.byref(c), 0) == 0
     assert L.fmoe_route_workspace_bytes(17, 512) == 0
+    # launch-mode switch: only 0 and 1, nothing changes otherwise
+    prev = ctypes.c_int(-1)
+    assert L.fmoe_set_dependent_launch(2, ctypes.byref(prev)) == F.FMOE_EINVAL and prev.value == -1
+    assert L.fmoe_set_dependent_launch(0, ctypes.byref(prev)) == F.FMOE_OK and prev.value == 1
+    assert L.fmoe_set_dependent_launch(1, ctypes.byref(prev)) == F.FMOE_OK and prev.value == 0
     for code in range(5):
         assert len(F.strerror(code)) >= 2 and F.strerror(code) != F.strerror(99)

@@ -41,7 +41,16 @@ def test_wait_limit_bounds(F):
     assert F.set_wait_limit_ns(prev) == 2_000_000_000
 
 
-def test_unreachable_counter_times_out_and_recovers(F):
+@pytest.mark.parametrize("dependent", [True, False], ids=["dependent_launch", "cooperative_launch"])
+def test_unreachable_counter_times_out_and_recovers(F, dependent):
+    prev_mode = F.set_dependent_launch(dependent)
+    try:
+        unreachable_counter_case(F)
+    finally:
+        F.set_dependent_launch(prev_mode)
+
+
+def unreachable_counter_case(F):
     import synth.gpu as SG
     shape, seed, layer = C.TINY, 21, 0
     dev = torch.device("cuda:0")

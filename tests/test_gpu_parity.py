@@ -279,6 +279,63 @@ def test_stacked_layers_graph(F, SG):
     del g
 
 
+@pytest.mark.parametrize("shape", [C.FULL4, C.TINY], ids=["full4", "tiny"])
+def test_dependent_launch_matches_cooperative(F, SG, shape):
+    """Back-to-back chained decodes of three layers that share ONE workspace
+    (so each grid's counters are the previous grid's), run as programmatic
+    dependent launches (eagerly and from a graph) and as cooperative launches:
+    all outputs, indices and weights are bit-identical, and layer 0 agrees
+    with the oracle."""
+    seed, n_layers = 17, 3
+    layers = [make_gpu_layer(F, SG, seed, l, shape)[0] for l in range(n_layers)]
+    H, K = shape.hidden, shape.top_k
+    ws = layers[0].workspace(1)
+    x0 = torch.from_numpy(C.parity_x(seed, 0, 0, S.router_bf16(seed, 0, shape.n_experts, H), K, H)[0]).to(dev())
+
+    def chain(hs, idx, w):
+        src = x0
+        for l, L in enumerate(layers):
+            L.decode(src, src, out=hs[l], idx_out=idx[l], w_out=w[l], ws=ws)
+            src = hs[l]
+
+    def bufs():
+        return (torch.full((n_layers, H), float("nan"), device=dev()),
+                torch.full((n_layers, K), -1, dtype=torch.int32, device=dev()),
+                torch.full((n_layers, K), float("nan"), device=dev()))
+
+    runs = {}
+    prev = F.set_dependent_launch(True)
+    try:
+        for mode in (True, False):
+            F.set_dependent_launch(mode)
+            eager = bufs()
+            for _ in range(3):
+                chain(*eager)
+            assert F.get_status() == 0
+            graphed = bufs()
+            stream = torch.cuda.Stream()
+            stream.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(stream):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    chain(*graphed)
+                for _ in range(3):
+                    g.replay()
+            stream.synchronize()
+            assert F.get_status() == 0
+            del g
+            runs[mode] = (eager, graphed)
+    finally:
+        F.set_dependent_launch(prev)
+    ref = runs[False][0]
+    for mode in (True, False):
+        for got in runs[mode]:
+            for a, b in zip(got, ref):
+                assert torch.equal(a, b), f"dependent={mode}"
+    r = C.oracle_layer(seed, 0, shape, x0.cpu().numpy(), x0.cpu().numpy())
+    C.assert_close(ref[0][0].cpu().numpy(), r["out"], "chain layer 0")
+
+
 # ---------------------------------------------------------------------------
 # Grouped decode (T >= 2 tokens in one call)
 # ---------------------------------------------------------------------------

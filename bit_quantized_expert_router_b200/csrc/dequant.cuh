@@ -105,7 +105,10 @@ template <int BITS, bool kGlobal>
 __device__ inline void stage_inputs(const float* __restrict__ src, int n, float4* xs, float2* sf, int tid,
                                     int nthreads) {
   constexpr int CPV = 128 / BITS, CPW = 32 / BITS, F4 = CPV / 4;
-  constexpr int kBatch = 4;  // passes whose loads are all issued before any is used
+  // passes whose loads are all issued before any is used: global sources need
+  // the loads in flight together; from shared memory one pass at a time keeps
+  // this code (run once per launch, from a cold instruction cache) short
+  constexpr int kBatch = kGlobal ? 4 : 1;
   const int NV = n / CPV, total = NV * F4;
   const int lane = tid & 31;
   for (int base0 = tid - lane; base0 < total; base0 += kBatch * nthreads) {

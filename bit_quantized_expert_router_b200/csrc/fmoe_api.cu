@@ -17,6 +17,11 @@ constexpr unsigned long long kMaxWaitNs = 60000000000ull;  // 60 s
 std::atomic<unsigned long long> g_wait_limit_ns{kTimeoutNs};
 std::atomic<int> g_dependent_launch{1};
 constexpr size_t kCounterBytes = 256;
+// Every workspace starts with the counters, then the single-token decode's
+// tagged router logits (sized for the most experts, so that no other use of a
+// workspace, whatever its layer's shape, ever writes these bytes).
+constexpr size_t kTagBytes = (kTagWords * 8 + 255) / 256 * 256;
+constexpr size_t kHeaderBytes = kCounterBytes + kTagBytes;
 constexpr int kMaxNst = 4;
 
 struct DevInfo {
@@ -103,7 +108,7 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Shared-memory plan of the layer kernel (see carve_smem in layer_kernel.cuh).
 struct Plan {
-  int nst, stage_bytes, nst_c, c_stage_bytes, xs4_off, xs2_off, xu_off, vec_floats, sf_floats, ys_stride, lg_floats;
+  int nst, stage_bytes, nst_c, c_stage_bytes, xs4_off, xs2_off, xu_off, vec_floats, sf_floats, ys_stride;
   size_t smem;
 };
 
@@ -135,9 +140,8 @@ bool plan_layer(int H, int I, int K, bool has_shared, int bits_r, int bits_s, in
   const int nq = H / kRC;
   p->ys_stride = kRC * ((nq + G - 1) / G);
   p->stage_bytes = stage;
-  p->lg_floats = (int)round_up((size_t)n_router, 4);
   const size_t fixed = (size_t)p->vec_floats * 4 + (size_t)p->sf_floats * 8 +
-                       round_up((size_t)n_slots * p->ys_stride * 4, 16) + (size_t)p->lg_floats * 4;
+                       round_up((size_t)n_slots * p->ys_stride * 4, 16);
   p->c_stage_bytes = cstage;
   for (int nst = kMaxNst; nst >= 1; --nst) {
     const size_t total = (size_t)kWarps * nst * stage + fixed + (size_t)kWarps * (nst + kMaxNstC) * 8;
@@ -151,8 +155,8 @@ bool plan_layer(int H, int I, int K, bool has_shared, int bits_r, int bits_s, in
   return false;
 }
 
-size_t layer_ws_bytes(int E, int I, int K) {
-  return kCounterBytes + round_up((size_t)(E + 1) * 4, 256) + round_up((size_t)(K + 1) * I * 4, 256);
+size_t layer_ws_bytes(int I, int K) {
+  return kHeaderBytes + round_up((size_t)(K + 1) * I * 4, 256);
 }
 
 // Workspace of the grouped (T >= 2) decode, byte offsets (every section 256-B aligned).
@@ -163,7 +167,7 @@ struct GroupedLayout {
 
 GroupedLayout grouped_layout(int E, int H, int I, int K, int T) {
   GroupedLayout g;
-  size_t off = kCounterBytes;
+  size_t off = kHeaderBytes;
   auto take = [&](size_t bytes) {
     const size_t o = off;
     off += round_up(bytes, 256);
@@ -489,7 +493,7 @@ int fmoe_route(const uint16_t* w_router, const uint16_t* w_sgate, const float* x
 
 size_t fmoe_expert_workspace_bytes(int hidden, int inter) {
   if (!shape_ok(hidden, inter)) return 0;
-  return kCounterBytes + round_up((size_t)inter * 4, 256);
+  return kHeaderBytes + round_up((size_t)inter * 4, 256);
 }
 
 int fmoe_expert_forward(const void* blob, int hidden, int inter, int bits, const float* x, float* y,
@@ -511,7 +515,7 @@ int fmoe_expert_forward(const void* blob, int hidden, int inter, int bits, const
   a.out = y;
   char* w8 = static_cast<char*>(ws);
   a.bar = reinterpret_cast<unsigned*>(w8);
-  a.act = reinterpret_cast<float*>(w8 + kCounterBytes);
+  a.act = reinterpret_cast<float*>(w8 + kHeaderBytes);
   a.H = hidden;
   a.I = inter;
   a.E = 0;
@@ -530,7 +534,6 @@ int fmoe_expert_forward(const void* blob, int hidden, int inter, int bits, const
   a.ys_stride = pl.ys_stride;
   a.nst_c = pl.nst_c;
   a.c_stage_bytes = pl.c_stage_bytes;
-  a.lg_floats = pl.lg_floats;
   a.timeout_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   set_offsets(a, info->sms);
   return launch_layer(a, pl, info, reinterpret_cast<cudaStream_t>(stream));
@@ -538,7 +541,7 @@ int fmoe_expert_forward(const void* blob, int hidden, int inter, int bits, const
 
 size_t fmoe_workspace_bytes(const fmoe_layer* L, int T) {
   if (!L || T < 1 || T > FMOE_MAX_TOKENS) return 0;
-  const size_t single = layer_ws_bytes(L->n_experts, L->inter, L->top_k);
+  const size_t single = layer_ws_bytes(L->inter, L->top_k);
   if (T == 1) return single;
   return std::max(single, grouped_layout(L->n_experts, L->hidden, L->inter, L->top_k, T).total);
 }
@@ -586,8 +589,8 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
   a.shared = static_cast<const char*>(L->shared);
   char* w8 = static_cast<char*>(ws);
   a.bar = reinterpret_cast<unsigned*>(w8);
-  a.logits = reinterpret_cast<float*>(w8 + kCounterBytes);
-  a.act = reinterpret_cast<float*>(w8 + kCounterBytes + round_up((size_t)(E + 1) * 4, 256));
+  a.tlog = reinterpret_cast<unsigned long long*>(w8 + kCounterBytes);
+  a.act = reinterpret_cast<float*>(w8 + kHeaderBytes);
   a.H = H;
   a.I = I;
   a.E = E;
@@ -606,7 +609,6 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
   a.ys_stride = pl.ys_stride;
   a.nst_c = pl.nst_c;
   a.c_stage_bytes = pl.c_stage_bytes;
-  a.lg_floats = pl.lg_floats;
   a.timeout_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   a.norm_w = L->norm_weight;
   a.norm_eps = L->norm_eps;
@@ -638,9 +640,10 @@ int fmoe_layer_decode_noalloc(const fmoe_layer* L, const float* x, const float* 
   if (dev < 0 || dev >= 64) return FMOE_EINVAL;
   void* ws = nullptr;
   if (int rc = noalloc_scratch(dev, &ws)) return rc;
-  // The scratch keeps whatever the previous call left; the hand-off counters
-  // must start at zero, so clear them (the rest is written before it is read).
-  if (cudaError_t e = cudaMemsetAsync(ws, 0, kCounterBytes, reinterpret_cast<cudaStream_t>(stream)))
+  // The scratch keeps whatever the previous call left: clear the counters and
+  // the tagged logits (epoch 0, no word tagged), as a fresh workspace has them;
+  // the rest is written before it is read.
+  if (cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes, reinterpret_cast<cudaStream_t>(stream)))
     return cuda_fail(e);
   return fmoe_layer_decode(L, x, residual, out, T, ws, kNoallocScratchBytes, idx_out_opt, w_out_opt, stream);
 }

@@ -44,6 +44,7 @@ constexpr int kRC = 4;            // down rows per phase-C item (the split row r
 constexpr int kMaxTopK = 8;
 constexpr int kMaxSlots = kMaxTopK + 1;
 constexpr int kMaxExperts = 1024; // top-K is one warp with 32 logits per lane
+constexpr int kTagWords = kMaxExperts + 1;  // tagged-logit words of a workspace (routers and the gate)
 constexpr int kMaxNstC = 8;       // most down-item stages a warp keeps in flight
 
 // Optional phase trace (compile with -DFMOE_TRACE_BUILD): thread 0 of every CTA
@@ -70,9 +71,11 @@ struct LayerArgs {
   const float* x;            // [H]
   const float* residual;     // [H] or null
   float* out;                // [H]
-  float* logits;             // workspace [E + 1]
+  // workspace [n_router] tagged logits: word e = (tag << 32) | bits of logit e,
+  // tag = this launch's epoch + 1 (written by the router warps only)
+  unsigned long long* tlog;
   float* act;                // workspace [n_slots][I]
-  unsigned* bar;             // workspace: [0] router rows published, [1] CTAs past gate/up, [2] done ticket
+  unsigned* bar;             // workspace: [0] launch epoch, [1] CTAs past gate/up, [2] done ticket
   int* idx_out;              // optional [K]
   float* w_out;              // optional [K]
   float* sg_out;             // optional [1]
@@ -87,7 +90,6 @@ struct LayerArgs {
   int xs4_off, xs2_off, xu_off;  // float offsets inside the vector region (-1 = absent)
   int vec_floats, sf_floats;
   int ys_stride;             // rows per CTA (max) in the phase-C result array
-  int lg_floats;             // shared-memory logits (n_router rounded up to 4)
   long long off_r[6], off_s[6];  // blob section offsets for the routed / shared code width
   unsigned long long timeout_ns;
   int router_smem;           // 1: each router warp's row is bulk-copied into its ring at entry
@@ -100,7 +102,6 @@ struct Smem {
   float* vec;
   float2* sf;
   float* ys;   // [n_slots][ys_stride] per-expert down-projection rows of this CTA
-  float* lg;   // [lg_floats] router logits
   uint64_t* bars;
 };
 
@@ -115,8 +116,6 @@ __device__ __forceinline__ Smem carve_smem(const LayerArgs& a, char* base) {
   s.ys = reinterpret_cast<float*>(base + off);
   off += (size_t)a.n_slots * a.ys_stride * 4;
   off = (off + 15) & ~(size_t)15;
-  s.lg = reinterpret_cast<float*>(base + off);
-  off += (size_t)a.lg_floats * 4;
   s.bars = reinterpret_cast<uint64_t*>(base + off);  // [kWarps][nst + kMaxNstC]
   return s;
 }
@@ -167,13 +166,9 @@ __device__ __forceinline__ WarpPlan make_plan(const LayerArgs& a, int cta, int w
 struct CtaShared {
   uint64_t x_bar;       // completes once x is in shared memory
   uint64_t staged_bar;  // completes once x is staged in the decode layouts
-  uint64_t rdot_bar;    // completes once this CTA's router dot products are done
-  uint64_t lg_bar;      // completes once the router logits are in shared memory
   uint64_t rbar[kWarps];  // router warp w's row is in its ring (router_smem)
   unsigned long long param_touch;  // see the kernel's set-up
   float red[kWarps];               // per-warp partial sums (input norm)
-  float* lg;            // shared-memory copy of the router logits
-  unsigned lg_bytes;
   int c_prefetch;          // warps past their gate/up work (the first prefetches down rows)
   int idx[kMaxTopK];
   float w[kMaxTopK];
@@ -552,53 +547,74 @@ __device__ __forceinline__ void warp_select(uint32_t (&key)[NK], const uint32_t 
   }
 }
 
-// Stage 1 of the CTA's top-K: warp w selects the top k of its slice of the
-// logits (NKW * 32 consecutive experts from w * NKW * 32) into the candidates.
+// Stage 1 of the CTA's top-K.  Each lane holds NKW logits of its warp's slice
+// (NKW * 32 consecutive experts from w * NKW * 32) as order-preserving keys,
+// read from the tagged words as soon as they carry this launch's tag (warp 0's
+// lane 0 also reads the shared gate's logit, which it returns); the warp then
+// selects the top k of its slice into the candidates.  The tag check replaces
+// a grid barrier: a word is this launch's logit or it is not read.
 template <int NKW>
-__device__ __forceinline__ void slice_topk(const float* lg, int n, int k, int warp, int lane, CtaShared& cs) {
+__device__ __forceinline__ float slice_topk(const LayerArgs& a, unsigned tag, int warp, int lane, CtaShared& cs) {
   uint32_t key[NKW], eix[NKW];
+  unsigned pend = 0;
 #pragma unroll
   for (int i = 0; i < NKW; ++i) {
     const int e = (warp * NKW + i) * 32 + lane;
-    key[i] = e < n ? order_bits(lg[e]) : 0u;
-    eix[i] = e < n ? (uint32_t)e : 0xffffffffu;
+    key[i] = 0u;
+    eix[i] = e < a.E ? (uint32_t)e : 0xffffffffu;
+    if (e < a.E) pend |= 1u << i;
   }
+  if (warp == 0 && lane == 0 && a.n_router > a.E) pend |= 1u << NKW;
+  float gate_logit = 0.f;
+  uint64_t t0 = 0;
+  while (pend) {
+    unsigned long long v[NKW + 1];
+#pragma unroll
+    for (int i = 0; i <= NKW; ++i) {
+      const int e = i < NKW ? (warp * NKW + i) * 32 + lane : a.E;
+      v[i] = (pend >> i & 1u) ? ld_relaxed_gpu_u64(a.tlog + e) : 0ull;
+    }
+#pragma unroll
+    for (int i = 0; i <= NKW; ++i) {
+      if ((pend >> i & 1u) && (unsigned)(v[i] >> 32) == tag) {
+        const float l = __uint_as_float((unsigned)v[i]);
+        if (i < NKW) key[i] = order_bits(l); else gate_logit = l;
+        pend &= ~(1u << i);
+      }
+    }
+    if (!pend) break;
+    FMOE_SPIN(2);
+    const uint64_t now = globaltimer_ns();
+    if (t0 == 0) {
+      t0 = now;
+    } else if (now - t0 > a.timeout_ns) {
+      set_status(kStatusGridBarrierTimeout);
+      break;
+    }
+  }
+  FMOE_TRACE_WARP(17);
   uint32_t hk, hi;
-  warp_select<NKW>(key, eix, k, lane, hk, hi);
-  if (lane < k) {
-    cs.cand_key[warp * k + lane] = hk;
-    cs.cand_idx[warp * k + lane] = hi;
+  warp_select<NKW>(key, eix, a.K, lane, hk, hi);
+  if (lane < a.K) {
+    cs.cand_key[warp * a.K + lane] = hk;
+    cs.cand_idx[warp * a.K + lane] = hi;
   }
+  return gate_logit;
 }
 
 // The routing decision of this CTA, computed by all of its warps together;
 // every warp calls this once, before it computes any unit (layer mode).
-//   Warp 0 waits until every router row is counted and bulk-copies the logits
-//   into shared memory; each warp selects the top K of its slice of the
-//   logits; after a CTA barrier the candidates are ranked in parallel (the
+//   Each warp takes the top K of its slice of the logits as they are
+//   published; after a CTA barrier the candidates are ranked in parallel (the
 //   global top K is among them, ties included); after a second barrier warp 0
 //   computes the weights, and a third publishes the decision to the CTA.
 __device__ __noinline__ void cta_routing(const LayerArgs& a, CtaShared& cs, int warp, int lane) {
-  float* lg = cs.lg;
-  if (warp == 0) {
-    bool ok = true;
-    if (lane == 0) ok = grid_wait(&a.bar[0], (unsigned)a.n_router, a.timeout_ns);
-    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    if (!ok && lane == 0) set_status(kStatusGridBarrierTimeout);
-    FMOE_TRACE_WARP(9);
-    // (the async proxy reads what this thread acquired, hence the proxy fence)
-    if (lane == 0) {
-      fence_proxy_async_global();
-      mbar_arrive_expect_tx(&cs.lg_bar, cs.lg_bytes);
-      bulk_g2s(lg, a.logits, cs.lg_bytes, &cs.lg_bar);
-    }
-  }
-  if (!mbar_wait_bounded(&cs.lg_bar, 0, a.timeout_ns) && lane == 0) set_status(kStatusCopyTimeout);
-  FMOE_TRACE_WARP(17);
+  const unsigned tag = ld_relaxed_gpu(&a.bar[0]) + 1u;
+  float gate_logit;
   if (a.E <= kWarps * 32)
-    slice_topk<1>(lg, a.E, a.K, warp, lane, cs);
+    gate_logit = slice_topk<1>(a, tag, warp, lane, cs);
   else
-    slice_topk<kMaxExperts / (kWarps * 32)>(lg, a.E, a.K, warp, lane, cs);
+    gate_logit = slice_topk<kMaxExperts / (kWarps * 32)>(a, tag, warp, lane, cs);
   FMOE_TRACE_WARP(14);
   __syncthreads();
   // Stage 2: each candidate's rank among the nc candidates (larger key first,
@@ -645,7 +661,7 @@ __device__ __noinline__ void cta_routing(const LayerArgs& a, CtaShared& cs, int 
       }
     }
     if (lane == 0) {
-      cs.sg = a.w_sgate ? sigmoidf_(lg[a.E]) : 1.0f;
+      cs.sg = a.w_sgate ? sigmoidf_(gate_logit) : 1.0f;
       if (blockIdx.x == 0 && a.sg_out) *a.sg_out = cs.sg;
     }
     FMOE_TRACE_WARP(10);
@@ -691,10 +707,6 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   if (tid == 0) {
     mbar_init(&cs.x_bar, 1);
     mbar_init(&cs.staged_bar, kWarps - n_router_warps);
-    mbar_init(&cs.rdot_bar, n_router_warps > 0 ? n_router_warps : 1);
-    mbar_init(&cs.lg_bar, 1);
-    cs.lg = sm.lg;
-    cs.lg_bytes = (unsigned)a.lg_floats * 4u;
     cs.sg = 1.0f;
     cs.c_prefetch = 0;
     // Read every kernel parameter once now, while x is in flight, so that the
@@ -702,12 +714,12 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     {
       unsigned long long t = (uintptr_t)a.w_router ^ (uintptr_t)a.w_sgate ^ (uintptr_t)a.experts ^
                              (unsigned long long)a.expert_stride ^ (uintptr_t)a.shared ^ (uintptr_t)a.x ^
-                             (uintptr_t)a.residual ^ (uintptr_t)a.out ^ (uintptr_t)a.logits ^ (uintptr_t)a.act ^
+                             (uintptr_t)a.residual ^ (uintptr_t)a.out ^ (uintptr_t)a.tlog ^ (uintptr_t)a.act ^
                              (uintptr_t)a.bar ^ (uintptr_t)a.idx_out ^ (uintptr_t)a.w_out ^ (uintptr_t)a.sg_out ^
                              a.timeout_ns;
       t += (unsigned)(a.H ^ a.I ^ a.E ^ a.K ^ a.bits_r ^ a.bits_s ^ a.n_router ^ a.n_slots ^ a.off_a ^ a.off_b ^
                       a.nst ^ a.stage_bytes ^ a.nst_c ^ a.c_stage_bytes ^ a.xs4_off ^ a.xs2_off ^ a.xu_off ^
-                      a.vec_floats ^ a.sf_floats ^ a.ys_stride ^ a.lg_floats ^ a.router_smem);
+                      a.vec_floats ^ a.sf_floats ^ a.ys_stride ^ a.router_smem);
       for (int i = 0; i < 6; ++i) t += (unsigned long long)(a.off_r[i] ^ a.off_s[i]);
       t ^= (uintptr_t)a.norm_w ^ (unsigned long long)__float_as_uint(a.norm_eps);
       *(volatile unsigned long long*)&cs.param_touch = t;
@@ -744,6 +756,9 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   grid_dep_wait();
   FMOE_TRACE(24);
   if (tid == 0) bulk_g2s(sm.vec + a.xu_off, a.x, a.H * 4, &cs.x_bar);
+  // The tag of this launch's router logits (the epoch the previous launch on
+  // this workspace left, plus one).
+  const unsigned ptag = (router_warp && lane == 0) ? ld_relaxed_gpu(&a.bar[0]) + 1u : 0u;
 
   // x and the router rows are the critical path to the routing decision, so
   // they are the only traffic of the first microseconds; the shared expert's
@@ -783,21 +798,16 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
       } else {
         l = router_dot(router_row_ptr(e), xu, a.H, lane);
       }
-      if (lane == 0 && j == 0) mbar_arrive(&cs.rdot_bar);  // staging may start
       if (lane == 0) {
-        // The release orders this thread's logit store before its count.
-        a.logits[e] = l;
-        red_release_gpu_add(&a.bar[0], 1);
+        st_relaxed_gpu_u64(a.tlog + e, ((unsigned long long)ptag << 32) | __float_as_uint(l));
         FMOE_TRACE_WARP(22);
       }
     }
     FMOE_TRACE_WARP(2);
   } else {
     // ---- Stage x into the decode layouts (the non-router warps) --------------
-    // The router dot products are on the critical path: staging waits for them
-    // so that they run without competition for the CTA's issue slots.
-    if (n_router_warps > 0 && !mbar_wait_bounded(&cs.rdot_bar, 0, a.timeout_ns) && lane == 0)
-      set_status(kStatusCtaWaitTimeout);
+    // At once, alongside the router dot products: the staging is what keeps
+    // these warps from polling for the logits.
     const int t0 = tid - n_router_warps * 32, nt = kThreads - n_router_warps * 32;
     if (BR == 4 || BS == 4)
       stage_inputs<4, false>(xu, a.H, reinterpret_cast<float4*>(sm.vec + a.xs4_off), sm.sf, t0, nt);
@@ -909,14 +919,21 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   FMOE_TRACE(5);
   __syncthreads();
 
-  // Stage the activations: the K routed experts (same width, back to back in
-  // the workspace) in one pass, then the shared expert.  Slot s's staged
-  // values start at sm.vec + s * I either way.
+  // Stage the activations.  With one code width every slot (back to back in
+  // the workspace) is staged in one pass, as one [F4][n_slots*I/CPV] array;
+  // otherwise the K routed experts in one pass and the shared expert in a
+  // second, its own [F4][I/CPV] array at sm.vec + K * I.  Slot s's scale pairs
+  // start at sm.sf + s * I / CPV either way.
   if (plan.nq > 0) {
-    if (a.K > 0) stage_inputs<BR, true>(a.act, a.K * a.I, reinterpret_cast<float4*>(sm.vec), sm.sf, tid, kThreads);
-    if (a.n_slots > a.K)
-      stage_inputs<BS, true>(a.act + (long long)a.K * a.I, a.I, reinterpret_cast<float4*>(sm.vec + a.K * a.I),
-                             sm.sf + a.K * a.I * BR / 128, tid, kThreads);
+    if (BR == BS) {
+      stage_inputs<BR, true>(a.act, a.n_slots * a.I, reinterpret_cast<float4*>(sm.vec), sm.sf, tid, kThreads);
+    } else {
+      if (a.K > 0)
+        stage_inputs<BR, true>(a.act, a.K * a.I, reinterpret_cast<float4*>(sm.vec), sm.sf, tid, kThreads);
+      if (a.n_slots > a.K)
+        stage_inputs<BS, true>(a.act + (long long)a.K * a.I, a.I, reinterpret_cast<float4*>(sm.vec + a.K * a.I),
+                               sm.sf + a.K * a.I * BR / 128, tid, kThreads);
+    }
   }
   FMOE_TRACE(6);
   __syncthreads();
@@ -939,12 +956,14 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     c_item(plan, i, warp, slot, r0);
     const bool routed = slot < a.K;
     const int cpv = 128 / (routed ? BR : BS);
-    // Routed slots share one staged [F4][K*I/CPV] array; the shared slot has
-    // its own [F4][I/CPV] array after it.
-    const float4* as = reinterpret_cast<const float4*>(sm.vec + (routed ? 0 : a.K * a.I));
-    const int nvs = routed ? a.K * a.I / cpv : a.I / cpv;
-    const int col0 = routed ? slot * (a.I / cpv) : 0;
-    const float2* sfa = sm.sf + (routed ? 0 : a.K * a.I * BR / 128) + col0;
+    // One code width: every slot is column block slot of one staged array.
+    // Otherwise the routed slots share one [F4][K*I/CPV] array and the shared
+    // slot has its own [F4][I/CPV] array after it.
+    const bool one = BR == BS || routed;
+    const float4* as = reinterpret_cast<const float4*>(sm.vec + (one ? 0 : a.K * a.I));
+    const int nvs = (BR == BS ? a.n_slots : routed ? a.K : 1) * (a.I / cpv);
+    const int col0 = one ? slot * (a.I / cpv) : 0;
+    const float2* sfa = sm.sf + (one ? 0 : a.K * a.I * BR / 128) + col0;
     float y[kRC];
     if (BR == BS || routed)
       down_rows<BR>(stage, a.I, as, nvs, col0, sfa, lane, y);
@@ -965,13 +984,23 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     a.out[r] = v;
   }
 
-  // ---- Done: the last CTA resets the hand-off counters for the next launch --
+  // ---- Done: the last CTA advances the epoch and resets the counters -------
   __syncthreads();
   FMOE_TRACE(8);
   if (tid == 0) {
     const unsigned t = atomicAdd(&a.bar[2], 1u);
     if (t + 1 == (unsigned)G) {
-      atomicExch(&a.bar[0], 0u);
+      // Every CTA is past its last use of the epoch.  Tags run 1 .. 2^32 - 1
+      // (epoch + 1); before the epoch would reach 2^32 - 1 the tagged words are
+      // cleared (tag 0 never matches) and it restarts at 0, so no word left by
+      // an earlier launch ever carries a later launch's tag.
+      unsigned ep = ld_relaxed_gpu(&a.bar[0]) + 1u;
+      if (ep == 0xFFFFFFFFu) {
+        if (a.tlog)
+          for (int e = 0; e < kTagWords; ++e) st_relaxed_gpu_u64(a.tlog + e, 0ull);
+        ep = 0u;
+      }
+      atomicExch(&a.bar[0], ep);
       atomicExch(&a.bar[1], 0u);
       atomicExch(&a.bar[2], 0u);
       __threadfence();

@@ -200,7 +200,7 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
  *   memory that every GPU which loads the library keeps until the process
  *   exits; a layer whose fmoe_workspace_bytes() exceeds 32 KiB is rejected
  *   with FMOE_ENOMEM (the full-size layer of the pages, 512 experts, top-4,
- *   intermediate 1024, needs about 23 KiB).
+ *   intermediate 1024, needs about 29 KiB).
  *   The first call on a device looks the array's device address up (a
  *   synchronous runtime query); make that first call before capturing a
  *   stream into a graph.  Every call clears the array's hand-off counters on

@@ -1,12 +1,13 @@
 """Failure detection on the GPU without a fault: a time-limited wait that runs out.
 
 The layer kernel's CTAs hand off through counters in the caller's workspace.
-Here the two hand-off counters are left at a value no launch can bring to its
-target (as if the workspace had not been zeroed), with a short wait limit.
-Every wait on them must run out, the kernel must end on its own and report
-through the status word, the context must stay usable, and the next launch
-on the same workspace must be correct again (the kernel's last CTA resets the
-counters on its way out).
+Here the activation hand-off counter is left at a value no launch can bring
+to its target (as if the workspace had not been zeroed), with a short wait
+limit.  Every wait on it must run out, the kernel must end on its own and
+report through the status word, the context must stay usable, and the next
+launch on the same workspace must be correct again (the kernel's last CTA
+resets the counter on its way out).  Both launch modes (programmatic
+dependent and cooperative) are covered.
 """
 import numpy as np
 import pytest
@@ -67,14 +68,16 @@ def unreachable_counter_case(F):
 
     prev = F.set_wait_limit_ns(20_000_000)  # 20 ms
     try:
-        counters = ws[:8].view(torch.int32)
-        counters.fill_(-1024)  # 0xFFFFFC00: above any grid size, never "reached"
+        counters = ws[:12].view(torch.int32)
+        epoch = int(counters[0])
+        counters[1:2].fill_(-1024)  # hand-off counter 0xFFFFFC00: above any grid size, never "reached"
         L.decode(xd, rd, ws=ws)
         bits = F.get_status()  # synchronises: the launch ended on its own
         assert bits & STATUS_GRID_BARRIER_TIMEOUT, f"status bits {bits:#x}"
         assert F.get_status() == 0  # read-and-clear
-        # the last CTA put every hand-off counter back to zero
-        assert ws[:12].view(torch.int32).cpu().tolist() == [0, 0, 0]
+        # the last CTA advanced the launch epoch and put both hand-off
+        # counters back to zero
+        assert counters.cpu().tolist() == [epoch + 1, 0, 0]
     finally:
         F.set_wait_limit_ns(prev)
 

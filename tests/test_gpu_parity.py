@@ -336,6 +336,53 @@ def test_dependent_launch_matches_cooperative(F, SG, shape):
     C.assert_close(ref[0][0].cpu().numpy(), r["out"], "chain layer 0")
 
 
+def test_routing_epoch_wraps(F, SG):
+    """The router logits are published as words tagged with the workspace's
+    launch epoch + 1.  Started two launches before the epoch would reach
+    2^32 - 1, three decodes must all be right: the second clears the tagged
+    words and restarts the epoch at 0, so the third (tag 1) reads no stale
+    word."""
+    shape, seed = C.FULL4, 23
+    L, _ = make_gpu_layer(F, SG, seed, 0, shape)
+    H, K = shape.hidden, shape.top_k
+    wr = S.router_bf16(seed, 0, shape.n_experts, H)
+    xs = C.parity_x(seed, 0, 0, wr, K, H, 3)
+    res = S.token_residual(seed, 0, 0, 3, H)
+    ws = L.workspace(1)
+    epoch = ws[:4].view(torch.int32)
+    epoch.fill_(-3)  # 0xFFFFFFFD
+    expect_epoch = [-2, 0, 1]  # 0xFFFFFFFE, then the wrap to 0
+    for i in range(3):
+        idx = torch.empty(1, K, dtype=torch.int32, device=dev())
+        out = L.decode(torch.from_numpy(xs[i]).to(dev()), torch.from_numpy(res[i]).to(dev()), idx_out=idx, ws=ws)
+        assert F.get_status() == 0
+        assert int(epoch.cpu()[0]) == expect_epoch[i], f"decode {i}"
+        if i == 1:  # the wrap cleared every tagged word
+            tags = ws[256:256 + 1025 * 8].view(torch.int64).cpu().numpy()
+            assert (tags == 0).all()
+        r = C.oracle_layer(seed, 0, shape, xs[i], res[i])
+        assert idx.cpu().numpy()[0].tolist() == r["idx"].tolist(), f"decode {i}"
+        C.assert_close(out.cpu().numpy()[0], r["out"], f"decode {i} across the epoch wrap")
+
+
+def test_workspace_shared_by_grouped_and_single_token(F, SG):
+    """One workspace used in turn by single-token and grouped decodes of the
+    layer: every single-token result equals the one from a fresh workspace
+    (the grouped decode never writes the tagged router words)."""
+    shape, seed, T = C.FULL4, 29, 16
+    L, _ = make_gpu_layer(F, SG, seed, 0, shape)
+    H = shape.hidden
+    xs = torch.from_numpy(S.token_x(seed, 0, 0, T, H)).to(dev())
+    res = torch.from_numpy(S.token_residual(seed, 0, 0, T, H)).to(dev())
+    fresh = torch.zeros(L.workspace_bytes(1), dtype=torch.uint8, device=dev())
+    want = [L.decode(xs[t], res[t], ws=fresh).clone() for t in range(3)]
+    ws = torch.zeros(L.workspace_bytes(T), dtype=torch.uint8, device=dev())
+    for t in range(3):
+        L.decode(xs, res, ws=ws)
+        assert torch.equal(L.decode(xs[t], res[t], ws=ws), want[t]), f"token {t}"
+        assert F.get_status() == 0
+
+
 # ---------------------------------------------------------------------------
 # Grouped decode (T >= 2 tokens in one call)
 # ---------------------------------------------------------------------------

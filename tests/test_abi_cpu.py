@@ -92,7 +92,17 @@ def test_invalid_arguments_rejected_on_host(F):
     assert decode(ws_bytes=16) == F.FMOE_ENOMEM
     assert decode(inter=4096) == F.FMOE_EINVAL  # (K+1)*I above the staging limit
     c = F.FmoeLayerC(**base)
-    assert L.fmoe_workspace_bytes(ctypes.byref(c), 1) >= 256 + 513 * 4 + 5 * 1024 * 4
+    # workspace header: 256 B of counters, then the tagged router logits sized
+    # for the most experts (1025 words of 8 B, rounded to 256): 8448 B; then
+    # the activations [K+1][I] fp32
+    header = 256 + (1025 * 8 + 255) // 256 * 256
+    assert header == 8704
+    assert L.fmoe_workspace_bytes(ctypes.byref(c), 1) == header + 5 * 1024 * 4
+    assert L.fmoe_expert_workspace_bytes(4096, 1024) == header + 1024 * 4
+    # a grouped workspace serves single-token calls of the layer too
+    assert L.fmoe_workspace_bytes(ctypes.byref(c), 16) > L.fmoe_workspace_bytes(ctypes.byref(c), 1)
+    small = F.FmoeLayerC(**{**base, "n_experts": 16, "inter": 128})
+    assert L.fmoe_workspace_bytes(ctypes.byref(small), 1) == header + 5 * 128 * 4  # header independent of E
     assert L.fmoe_workspace_bytes(ctypes.byref(c), 0) == 0
     assert L.fmoe_route_workspace_bytes(17, 512) == 0
     # launch-mode switch: only 0 and 1, nothing changes otherwise

@@ -55,6 +55,9 @@ Readings where the pages are silent (each one is listed in the design notes):
   IEEE fp32: s = bf16(fl(fl(max - min) / (2^b - 1))), bias = bf16(min),
   q = clamp(rint(fl(fl(w - bias) / s)), 0, 2^b - 1), q = 0 when s == 0.
 
+A second, independent step: the gated delta-rule update of the linear-
+attention state (delta_update, at the end of this file).
+
 Parity status: every function here is pinned by the CPU tests against closed
 forms, exact rational arithmetic, brute force and the expert size the pages
 print (6.75 MB per 4-bit expert).  Agreement with the pages' own engine
@@ -364,3 +367,50 @@ def quantize_expert(w_gate: np.ndarray, w_up: np.ndarray, w_down: np.ndarray,
     parts = {name: quantize_matrix(m, bits)
              for name, m in (("gate", w_gate), ("up", w_up), ("down", w_down))}
     return assemble_blob(parts, hidden, inter, bits)
+
+
+# ---------------------------------------------------------------------------
+# The linear-attention state update (a second, independent decode step)
+# ---------------------------------------------------------------------------
+
+def delta_update(state, q, k, v, alpha, beta):
+    """Gated delta-rule recurrence of a multi-head state, T tokens in turn.
+
+    The pages name the routines only: the GatedDeltaNet recurrence updates a
+    64-head x 128x128 state matrix with single-precision scale, matrix-vector
+    and rank-1-update calls ([P2 "Accelerate-BLAS für lineare
+    Aufmerksamkeit"], [P1 "Técnicas innovadoras" §5], [P3 "Uso do
+    Accelerate BLAS"], [P5 "Points clés du projet"]).  Read in that order,
+    per head and token:
+
+      S <- alpha * S                  (scale)
+      u <- S k                        (matrix-vector)
+      S <- S + beta * (v - u) k^T     (rank-1 update)
+      o <- S q                        (matrix-vector: the readout)
+
+    which is the gated delta rule S' = alpha S (I - beta k k^T) + beta v k^T,
+    o = S' q.  Shapes: state [heads][dv][dk] (row i of a head holds the dk
+    key coefficients of value i), q and k [T][heads][dk], v [T][heads][dv],
+    alpha and beta [T][heads].  Each token is computed in fp64 from the fp32
+    state; the state is stored back in fp32 after every token (single
+    precision, as the pages' routines are).  Returns (state' as float32,
+    o [T][heads][dv] as float64); the input state is not modified.
+    """
+    S = np.array(state, dtype=np.float32)
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    alpha = np.asarray(alpha, dtype=np.float64)
+    beta = np.asarray(beta, dtype=np.float64)
+    T, heads = alpha.shape
+    dv = S.shape[1]
+    o = np.empty((T, heads, dv), dtype=np.float64)
+    for t in range(T):
+        for h in range(heads):
+            Sh = S[h].astype(np.float64)
+            Sh = alpha[t, h] * Sh
+            u = Sh @ k[t, h]
+            Sh = Sh + beta[t, h] * np.outer(v[t, h] - u, k[t, h])
+            o[t, h] = Sh @ q[t, h]
+            S[h] = Sh.astype(np.float32)
+    return S, o

@@ -463,6 +463,90 @@ def pin_rms_norm(O):
     assert np.array_equal(O.rms_norm(np.ones(2), one[:2], 3.0), np.full(2, 0.5))
 
 
+def _delta_inputs(rng, T, heads, dk, dv, unit_k=True):
+    S = (0.1 * rng.standard_normal((heads, dv, dk))).astype(np.float32)
+    q = rng.standard_normal((T, heads, dk))
+    k = rng.standard_normal((T, heads, dk))
+    if unit_k:
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((T, heads, dv))
+    alpha = rng.uniform(0.8, 1.0, (T, heads))
+    beta = rng.uniform(0.0, 1.0, (T, heads))
+    return S, q, k, v, alpha, beta
+
+
+def pin_delta_rule(O):
+    """The delta-rule update against its defining properties and an exact
+    brute force (the stepwise oracle is checked against the matrix form
+    alpha S (I - beta k k^T) + beta v k^T, computed differently)."""
+    rng = np.random.default_rng(31)
+    # (a) matrix form, one token, several heads: S' and o = S' q
+    S, q, k, v, alpha, beta = _delta_inputs(rng, 1, 3, 16, 12)
+    got_S, got_o = O.delta_update(S, q, k, v, alpha, beta)
+    for h in range(3):
+        S64 = S[h].astype(np.float64)
+        M = alpha[0, h] * S64 @ (np.eye(16) - beta[0, h] * np.outer(k[0, h], k[0, h])) \
+            + beta[0, h] * np.outer(v[0, h], k[0, h])
+        np.testing.assert_allclose(got_S[h], M.astype(np.float32), rtol=2e-7, atol=1e-7)
+        np.testing.assert_allclose(got_o[0, h], M @ q[0, h], rtol=1e-12, atol=1e-12)
+    # (b) beta = 0 is a pure decay: S' = fl32(alpha S), o = alpha S q
+    S, q, k, v, alpha, _ = _delta_inputs(rng, 1, 2, 8, 8)
+    got_S, got_o = O.delta_update(S, q, k, v, alpha, np.zeros((1, 2)))
+    for h in range(2):
+        assert np.array_equal(got_S[h], (alpha[0, h] * S[h].astype(np.float64)).astype(np.float32))
+        np.testing.assert_allclose(got_o[0, h], alpha[0, h] * S[h].astype(np.float64) @ q[0, h], rtol=1e-13)
+    # (c) alpha = beta = 1 with a unit key writes v at k: S' k = v (the rule's
+    # defining property), and leaves every direction orthogonal to k alone
+    S, q, k, v, _, _ = _delta_inputs(rng, 1, 1, 32, 20)
+    got_S, _ = O.delta_update(S, q, k, v, np.ones((1, 1)), np.ones((1, 1)))
+    np.testing.assert_allclose(got_S[0].astype(np.float64) @ k[0, 0], v[0, 0], rtol=0, atol=2e-6)
+    w = rng.standard_normal(32)
+    w -= (w @ k[0, 0]) * k[0, 0]
+    np.testing.assert_allclose(got_S[0].astype(np.float64) @ w, S[0].astype(np.float64) @ w, rtol=0, atol=2e-6)
+    # (d) exact brute force on small integers and dyadic gates (every value
+    # and intermediate exact in fp64 and the state exact in fp32), two tokens
+    from fractions import Fraction as Fr
+    heads, dk, dv, T = 2, 3, 2, 2
+    Si = rng.integers(-4, 5, (heads, dv, dk))
+    qi = rng.integers(-3, 4, (T, heads, dk))
+    ki = rng.integers(-2, 3, (T, heads, dk))
+    vi = rng.integers(-5, 6, (T, heads, dv))
+    al = np.array([[0.5, 1.0], [0.75, 0.5]])
+    be = np.array([[0.25, 0.5], [1.0, 0.125]])
+    got_S, got_o = O.delta_update(Si.astype(np.float32), qi, ki, vi, al, be)
+    for h in range(heads):
+        M = [[Fr(int(Si[h, i, j])) for j in range(dk)] for i in range(dv)]
+        for t in range(T):
+            a_, b_ = Fr(al[t, h]), Fr(be[t, h])
+            M = [[a_ * M[i][j] for j in range(dk)] for i in range(dv)]
+            u = [sum(M[i][j] * int(ki[t, h, j]) for j in range(dk)) for i in range(dv)]
+            M = [[M[i][j] + b_ * (int(vi[t, h, i]) - u[i]) * int(ki[t, h, j]) for j in range(dk)]
+                 for i in range(dv)]
+            for i in range(dv):
+                assert got_o[t, h, i] == float(sum(M[i][j] * int(qi[t, h, j]) for j in range(dk))), (t, h, i)
+        for i in range(dv):
+            for j in range(dk):
+                assert got_S[h, i, j] == np.float32(float(M[i][j])), (h, i, j)
+    # (e) heads are independent and the state rows are the value dimension:
+    # permuting the heads, or the values (rows of S and entries of v), permutes
+    # the results the same way
+    S, q, k, v, alpha, beta = _delta_inputs(rng, 2, 4, 8, 6)
+    ref_S, ref_o = O.delta_update(S, q, k, v, alpha, beta)
+    ph = np.array([2, 0, 3, 1])
+    pS, po = O.delta_update(S[ph], q[:, ph], k[:, ph], v[:, ph], alpha[:, ph], beta[:, ph])
+    assert np.array_equal(pS, ref_S[ph]) and np.array_equal(po, ref_o[:, ph])
+    pr = np.array([5, 3, 1, 0, 2, 4])
+    pS, po = O.delta_update(S[:, pr], q, k, v[:, :, pr], alpha, beta)
+    # (the library's matrix-vector product may sum a row in another order at
+    # another position: equal to rounding)
+    np.testing.assert_allclose(pS, ref_S[:, pr], rtol=1e-6, atol=1e-9)
+    np.testing.assert_allclose(po, ref_o[:, :, pr], rtol=1e-12, atol=1e-12)
+    # (f) the input state is left as it was
+    S0 = S.copy()
+    O.delta_update(S, q, k, v, alpha, beta)
+    assert np.array_equal(S, S0)
+
+
 ALL_PINS = [pin_expert_size, pin_packing_golden, pin_fma_identity_exact, pin_constant_codes,
             pin_one_hot, pin_permutation_expert, pin_dense_bruteforce, pin_activations,
-            pin_routing, pin_layer, pin_quantizer, pin_rms_norm]
+            pin_routing, pin_layer, pin_quantizer, pin_rms_norm, pin_delta_rule]

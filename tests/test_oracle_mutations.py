@@ -141,6 +141,42 @@ def _layer_ignores_norm(*a, **kw):
     return ORIG_LAYER(*a, **kw)
 
 
+def _delta_variant(order):
+    """A delta-rule oracle with one slip, chosen by `order`."""
+    def step(Sh, a_, b_, kk, vv, qq):
+        if order == "gemv_before_scale":
+            u = Sh @ kk
+            Sn = a_ * Sh + b_ * np.outer(vv - u, kk)
+        elif order == "correction_sign":
+            Sa = a_ * Sh
+            Sn = Sa - b_ * np.outer(vv - Sa @ kk, kk)
+        elif order == "scale_after_update":
+            Sn = a_ * (Sh + b_ * np.outer(vv - Sh @ kk, kk))
+        elif order == "no_beta":
+            Sa = a_ * Sh
+            Sn = Sa + np.outer(vv - Sa @ kk, kk)
+        elif order == "transposed_outer":
+            Sa = a_ * Sh
+            Sn = Sa + b_ * np.outer(kk, vv - Sa @ kk)
+        else:  # readout_before_update
+            Sa = a_ * Sh
+            return Sa + b_ * np.outer(vv - Sa @ kk, kk), Sh @ qq
+        return Sn, Sn @ qq
+
+    def fn(state, q, k, v, alpha, beta):
+        S = np.array(state, dtype=np.float32)
+        q, k, v = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
+        alpha, beta = np.asarray(alpha, dtype=np.float64), np.asarray(beta, dtype=np.float64)
+        T, heads = alpha.shape
+        o = np.empty((T, heads, S.shape[1]))
+        for t in range(T):
+            for h in range(heads):
+                Sn, o[t, h] = step(S[h].astype(np.float64), alpha[t, h], beta[t, h], k[t, h], v[t, h], q[t, h])
+                S[h] = Sn.astype(np.float32)
+        return S, o
+    return fn
+
+
 ORIG_ROUTE = O.route
 ORIG_LAYER = O.layer_decode
 ORIG_QUANT = O.quantize_matrix
@@ -166,6 +202,12 @@ MUTANTS = {
     "rms_norm_no_sqrt": ("rms_norm", _rms_norm_no_sqrt),
     "rms_norm_no_weight": ("rms_norm", _rms_norm_no_weight),
     "layer_ignores_norm": ("layer_decode", _layer_ignores_norm),
+    "delta_gemv_before_scale": ("delta_update", _delta_variant("gemv_before_scale")),
+    "delta_correction_sign": ("delta_update", _delta_variant("correction_sign")),
+    "delta_scale_after_update": ("delta_update", _delta_variant("scale_after_update")),
+    "delta_no_beta": ("delta_update", _delta_variant("no_beta")),
+    "delta_transposed_outer": ("delta_update", _delta_variant("transposed_outer")),
+    "delta_readout_before_update": ("delta_update", _delta_variant("readout_before_update")),
 }
 
 

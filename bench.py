@@ -1,6 +1,6 @@
 """Benchmark: single-token MoE layer decode on B200 through the C-ABI engine.
 
-python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fmoe|reference] [--config full4|full2|tiny]
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fmoe|reference] [--config full4|full2|tiny|stacked|batch16|deltanet]
 
 One step = one token decoded through one full MoE layer (router GEMV over 512
 experts, softmax/top-4/renormalise, 4 routed + 1 shared 4-bit experts, fused
@@ -57,11 +57,16 @@ CONFIGS = {
     # token decoded through all 40 layers, each normalising its input.
     "stacked": dict(workload="stacked_40x_full_h4096_i1024_e512_k4_shared_4bit", hidden=4096, inter=1024,
                     experts=512, top_k=4, bits=4, shared_bits=4, layers_per_step=40),
+    # The linear-attention state update: one token through one layer's
+    # 64-head x 128x128 gated delta-rule state (45 such layers in rotation).
+    "deltanet": dict(workload="gated_delta_h64_dk128_dv128", kind="deltanet", heads=64, dk=128, dv=128,
+                     layers=45),
     # 16 tokens per step through the full-size 4-bit layer, grouped by expert.
     "batch16": dict(workload="batch16_full_h4096_i1024_e512_k4_shared_4bit", hidden=4096, inter=1024,
                     experts=512, top_k=4, bits=4, shared_bits=4, tokens=16),
 }
 METRIC = "MoE layer decodes/s (batch 1)"
+DELTA_METRIC = "GatedDeltaNet state updates/s (64 heads x 128x128, one token, batch 1)"
 UNIT = "decodes/s"
 SEED = 2026
 POOL = 64
@@ -481,6 +486,226 @@ def run_fmoe(args, cfg, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# The linear-attention state update (config "deltanet")
+# ---------------------------------------------------------------------------
+
+DELTA_KERNEL_SOURCES = ("common.cuh", "deltanet.cuh")
+
+
+def delta_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_quantized_expert_router_b200", "csrc")
+    for f in DELTA_KERNEL_SOURCES:
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def delta_bytes(cfg) -> int:
+    """Algorithmic bytes of one token's update: the state read and written,
+    q and k read, v read and o written, the two gates read (all fp32)."""
+    H, dk, dv = cfg["heads"], cfg["dk"], cfg["dv"]
+    return 4 * (2 * H * dv * dk + 2 * H * dk + 2 * H * dv + 2 * H)
+
+
+def delta_oracle_sample(cfg, budget_s: float, max_steps: int = 100000) -> dict:
+    """Time the oracle (as it stands) on state updates of the same shape."""
+    import oracle as O
+    H, dk, dv = cfg["heads"], cfg["dk"], cfg["dv"]
+    st = S.delta_state(SEED, 0, H, dv, dk)
+    toks = [S.delta_tokens(SEED, 0, j, 1, H, dk, dv) for j in range(8)]
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        tk = toks[n % len(toks)]
+        st, _ = O.delta_update(st, tk["q"], tk["k"], tk["v"], tk["alpha"], tk["beta"])
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= max_steps:
+            break
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    return dict(value=n / el, unit="updates/s", cores=cores, kind="oracle", seconds=el, tokens=n,
+                sample=f"{n} one-token updates of the {cfg['workload']} state (fp64 numpy oracle), {el:.1f} s")
+
+
+def run_reference_delta(args, cfg, rank, world):
+    if rank != 0:
+        return
+    steps, warm = args.steps, args.warmup
+    per_step_budget = max(0.05, min(5.0, 60.0 / max(1, steps + warm)))
+    for _ in range(warm):
+        delta_oracle_sample(cfg, per_step_budget * 0.2, max_steps=1)
+    t_total, n_total, last = 0.0, 0, None
+    for _ in range(steps):
+        r = delta_oracle_sample(cfg, per_step_budget, max_steps=4)
+        t_total += r["seconds"]
+        n_total += r["tokens"]
+        last = r
+    value = n_total / t_total
+    line = {
+        "impl": "reference", "metric": DELTA_METRIC, "value": value, "unit": "updates/s", "n_gpus": world,
+        "steps": steps, "warmup": warm, "ms_per_step": 1000.0 * t_total / n_total, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {**cfg, "batch": 1, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "updates/s", "cores": last["cores"], "kind": "oracle",
+                         "sample": f"{n_total} one-token state updates over {steps} steps"},
+        "e2e": {"value": value, "unit": "updates/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_delta(args, cfg, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import bit_quantized_expert_router_b200 as F
+    from bit_quantized_expert_router_b200 import build as B
+
+    if rank == 0 or not os.path.exists(F.LIB_PATH):
+        B.build_engine()
+    if world > 1:
+        dist.barrier()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    H, dk, dv, NL = cfg["heads"], cfg["dk"], cfg["dv"], cfg["layers"]
+    # NL layer states updated in turn: 45 x 4 MiB = 180 MiB, larger than L2,
+    # so a step's state comes from HBM without any flush between steps.
+    states = torch.stack([torch.from_numpy(S.delta_state(SEED + 1000 * rank, l, H, dv, dk)) for l in range(NL)]).to(dev)
+    pool = [S.delta_tokens(SEED + rank, 0, j, 1, H, dk, dv) for j in range(POOL)]
+    tok = {n: torch.from_numpy(np.stack([p[n] for p in pool])).to(dev) for n in pool[0]}
+    o = torch.empty(POOL, 1, H, dv, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(j):
+        t = j % POOL
+        F.delta_update(states[j % NL], tok["q"][t], tok["k"][t], tok["v"][t], tok["alpha"][t], tok["beta"][t],
+                       o=o[t])
+
+    for j in range(args.warmup):
+        step(j)
+    torch.cuda.synchronize()
+    GSTEPS = 64
+    K = args.steps
+
+    def capture(first, n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for j in range(first, first + n):
+                step(j)
+        return g
+
+    g_full = capture(0, GSTEPS)
+    rem = K % GSTEPS
+    g_rem = capture(0, rem) if rem else None
+    g_full.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.1)
+    ev0.record(stream)
+    for _ in range(K // GSTEPS):
+        g_full.replay()
+    if g_rem is not None:
+        g_rem.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = ev0.elapsed_time(ev1)
+
+    # one isolated update after a 256 MiB L2 flush
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    g_one = capture(0, 1)
+    lat = []
+    for j in range(min(K, 400)):
+        flush.fill_(j & 0xFF)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        g_one.replay()
+        a1.record(stream)
+        lat.append((a0, a1))
+    torch.cuda.synchronize()
+    lat_us = [1000.0 * a.elapsed_time(b) for a, b in lat]
+    del flush
+
+    # End to end through the same call with host buffers: the token's q, k, v
+    # and gates go up from pinned memory and its readout comes back, every step.
+    host = {n: torch.from_numpy(np.stack([p[n] for p in pool])).pin_memory() for n in pool[0]}
+    dbuf = {n: torch.empty_like(tok[n][0]) for n in tok}
+    oh = torch.empty(POOL, 1, H, dv, dtype=torch.float32).pin_memory()
+    od = torch.empty(1, H, dv, dtype=torch.float32, device=dev)
+    K2 = min(K, 2000)
+
+    def e2e_step(j):
+        t = j % POOL
+        for n in dbuf:
+            dbuf[n].copy_(host[n][t], non_blocking=True)
+        F.delta_update(states[j % NL], dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], o=od)
+        oh[t].copy_(od, non_blocking=True)
+
+    for j in range(3):
+        e2e_step(j)
+    torch.cuda.synchronize()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0.record(stream)
+    for j in range(K2):
+        e2e_step(j)
+    b1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = b0.elapsed_time(b1) / K2
+    total_ms_max, e2e_ms_max = max_over_ranks([total_ms, e2e_ms * K], world, dev)
+    status = F.get_status()
+
+    if rank == 0:
+        ab = delta_bytes(cfg)
+        peak, peak_kind = peaks()
+        achieved = ab / (total_ms / 1000.0 / K) / 1e9
+        traffic = None
+        pj = os.path.join(ROOT, "profiles", "delta_update_deltanet.json")
+        if os.path.exists(pj):
+            d = json.load(open(pj))
+            if d.get("source_hash") == delta_source_hash():
+                traffic = d.get("dram_bytes_per_launch")
+        h2d = sum(int(dbuf[n].numel()) * 4 for n in dbuf)
+        line = {
+            "impl": "fmoe", "metric": DELTA_METRIC, "value": whole_job_rate(K, world, total_ms_max),
+            "unit": "updates/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": total_ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {**cfg, "batch": 1,
+                       "l2": f"inputs larger than L2: {NL} layer states of {H * dv * dk * 4 / 2**20:.0f} MiB "
+                             f"updated in turn, no flush",
+                       "input_pool": POOL, "parallelism": f"replicas x{world}"},
+            "us_per_update": 1000.0 * total_ms_max / K,
+            "latency_us_l2_flushed": {"p50": statistics.median(lat_us), "p99": float(np.percentile(lat_us, 99)),
+                                      "steps": len(lat_us),
+                                      "note": "one isolated graph launch after a 256 MiB L2 flush"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic, "kernel": f"delta_update_kernel<{dk // 128}>",
+                         "algorithmic_bytes_per_launch": ab},
+            "e2e": {"value": whole_job_rate(K, world, e2e_ms_max), "unit": "updates/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": int(od.numel()) * 4},
+            "gpu_launches": K,
+            "clocks": clk,
+            "device_status": status,
+        }
+        if not args.no_cpu_baseline:
+            cb = delta_oracle_sample(cfg, args.cpu_seconds)
+            cb.pop("seconds", None)
+            cb.pop("tokens", None)
+            line["cpu_baseline"] = cb
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -501,9 +726,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    delta = cfg.get("kind") == "deltanet"
     if args.impl == "reference":
         if rank == 0:
-            run_reference(args, cfg, rank, world)
+            (run_reference_delta if delta else run_reference)(args, cfg, rank, world)
         return
     if world > 1:
         import datetime
@@ -513,7 +739,7 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        run_fmoe(args, cfg, rank, world, local_rank)
+        (run_delta if delta else run_fmoe)(args, cfg, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

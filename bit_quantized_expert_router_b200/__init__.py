@@ -25,7 +25,7 @@ EXPORTED = [
     "fmoe_expert_bytes", "fmoe_blob_offsets", "fmoe_quantize_expert", "fmoe_route_workspace_bytes",
     "fmoe_route", "fmoe_expert_workspace_bytes", "fmoe_expert_forward", "fmoe_workspace_bytes",
     "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status", "fmoe_strerror", "fmoe_last_cuda_error",
-    "fmoe_layer_decode_noalloc", "fmoe_set_wait_limit_ns", "fmoe_set_dependent_launch",
+    "fmoe_layer_decode_noalloc", "fmoe_set_wait_limit_ns", "fmoe_set_dependent_launch", "fmoe_delta_update",
 ]
 
 
@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
     L.fmoe_get_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
     L.fmoe_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong)]
     L.fmoe_set_dependent_launch.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
+    L.fmoe_delta_update.argtypes = [vp] * 7 + [i, i, i, i, vp]
     L.fmoe_last_cuda_error.argtypes = []
     L.fmoe_last_cuda_error.restype = i
     L.fmoe_strerror.argtypes = [i]
@@ -287,6 +288,27 @@ def set_wait_limit_ns(limit_ns: int) -> int:
     if rc != FMOE_OK:
         raise FmoeError(rc, "fmoe_set_wait_limit_ns")
     return int(prev.value)
+
+
+def delta_update(state: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, alpha: torch.Tensor,
+                 beta: torch.Tensor, o: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Gated delta-rule update of `state` [heads][dv][dk] (in place) for the T
+    tokens of q, k [T][heads][dk], v [T][heads][dv], alpha, beta [T][heads];
+    returns the readouts o [T][heads][dv] (all fp32, on one GPU)."""
+    for name, t in (("state", state), ("q", q), ("k", k), ("v", v), ("alpha", alpha), ("beta", beta)):
+        _dev_tensor(t, torch.float32, name)
+    heads, dv, dk = state.shape
+    T = alpha.shape[0]
+    if q.shape != (T, heads, dk) or k.shape != (T, heads, dk) or v.shape != (T, heads, dv) or \
+            alpha.shape != (T, heads) or beta.shape != (T, heads):
+        raise ValueError("delta_update: inconsistent shapes")
+    if o is None:
+        o = torch.empty(T, heads, dv, dtype=torch.float32, device=state.device)
+    _dev_tensor(o, torch.float32, "o")
+    _check(lib().fmoe_delta_update(state.data_ptr(), q.data_ptr(), k.data_ptr(), v.data_ptr(), alpha.data_ptr(),
+                                   beta.data_ptr(), o.data_ptr(), heads, dk, dv, T, _stream(stream)),
+           "fmoe_delta_update")
+    return o
 
 
 def set_dependent_launch(enable: bool) -> bool:

@@ -5,6 +5,7 @@
 #include <mutex>
 
 #include "../../include/fmoe.h"
+#include "deltanet.cuh"
 #include "shared_tc.cuh"
 
 using namespace fmoe;
@@ -665,6 +666,57 @@ int fmoe_set_wait_limit_ns(unsigned long long limit_ns, unsigned long long* prev
   if (limit_ns < kMinWaitNs || limit_ns > kMaxWaitNs) return FMOE_EINVAL;
   const unsigned long long old = g_wait_limit_ns.exchange(limit_ns);
   if (previous_opt) *previous_opt = old;
+  return FMOE_OK;
+}
+
+bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + bn && y < x + an;
+}
+
+int fmoe_delta_update(float* state, const float* q, const float* k, const float* v, const float* alpha,
+                      const float* beta, float* o, int heads, int dk, int dv, int T, fmoe_stream_t stream) {
+  if (!state || !q || !k || !v || !alpha || !beta || !o) return FMOE_EINVAL;
+  if (heads < 1 || heads > FMOE_DELTA_MAX_DIM || dv < 1 || dv > FMOE_DELTA_MAX_DIM || T < 1 ||
+      T > FMOE_DELTA_MAX_DIM || dk < 128 || dk > 512 || dk % 128 != 0)
+    return FMOE_EINVAL;
+  if (!aligned(state, 16) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 4) || !aligned(alpha, 4) ||
+      !aligned(beta, 4) || !aligned(o, 4))
+    return FMOE_EINVAL;
+  // The state and the readout are written: neither may overlap the other or an input.
+  const size_t sb = (size_t)heads * dv * dk * 4, kb = (size_t)T * heads * dk * 4, vb = (size_t)T * heads * dv * 4,
+               gb = (size_t)T * heads * 4;
+  const void* in[5] = {q, k, v, alpha, beta};
+  const size_t inb[5] = {kb, kb, vb, gb, gb};
+  if (overlaps(state, sb, o, vb)) return FMOE_EINVAL;
+  for (int j = 0; j < 5; ++j)
+    if (overlaps(state, sb, in[j], inb[j]) || overlaps(o, vb, in[j], inb[j])) return FMOE_EINVAL;
+  int dev;
+  DevInfo* info;
+  if (int rc = dev_info(&dev, &info)) return rc;
+  if (int rc = check_stream(stream, dev)) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DeltaArgs a;
+  a.state = state;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.alpha = alpha;
+  a.beta = beta;
+  a.o = o;
+  a.heads = heads;
+  a.dk = dk;
+  a.dv = dv;
+  a.T = T;
+  const long long rows = (long long)heads * dv;
+  const unsigned grid = (unsigned)((rows + kDeltaWarps - 1) / kDeltaWarps);
+  switch (dk / 128) {
+    case 1: delta_update_kernel<1><<<grid, kDeltaWarps * 32, 0, s>>>(a); break;
+    case 2: delta_update_kernel<2><<<grid, kDeltaWarps * 32, 0, s>>>(a); break;
+    case 3: delta_update_kernel<3><<<grid, kDeltaWarps * 32, 0, s>>>(a); break;
+    default: delta_update_kernel<4><<<grid, kDeltaWarps * 32, 0, s>>>(a); break;
+  }
+  if (cudaError_t e = cudaGetLastError()) return cuda_fail(e);
   return FMOE_OK;
 }
 

@@ -231,6 +231,34 @@ int fmoe_last_cuda_error(void);
  * launches in flight on other threads. */
 int fmoe_set_wait_limit_ns(unsigned long long limit_ns, unsigned long long* previous_opt);
 
+/* ---- Linear-attention state update (a second, independent decode step) ---- */
+
+#define FMOE_DELTA_MAX_DIM 65536
+
+/* Gated delta-rule update of a multi-head state for T tokens in turn, in
+ * place, with the readout after each token.  Per head h and token t, in the
+ * order of the routines the pages name for the GatedDeltaNet recurrence
+ * (single-precision scale, matrix-vector and rank-1 update on a 64-head x
+ * 128x128 state: [P2] "Accelerate-BLAS für lineare Aufmerksamkeit", [P3]
+ * "Uso do Accelerate BLAS"):
+ *   S_h <- alpha[t][h] * S_h
+ *   u   <- S_h k[t][h]
+ *   S_h <- S_h + beta[t][h] * (v[t][h] - u) k[t][h]^T
+ *   o[t][h] <- S_h q[t][h]
+ * i.e. S' = alpha S (I - beta k k^T) + beta v k^T, o = S' q.  How q, k, v and
+ * the gates are produced from a token is outside this call.
+ *   state: device [heads][dv][dk] fp32 (row i of a head: the dk key
+ *          coefficients of value i), read and written once per call.
+ *   q, k: device [T][heads][dk] fp32; v: [T][heads][dv]; alpha, beta:
+ *          [T][heads]; o: device [T][heads][dv] fp32 out.
+ * Arithmetic in fp32 (the state stays fp32 between tokens).  Limits: dk in
+ * {128, 256, 384, 512}; 1 <= heads, dv, T <= FMOE_DELTA_MAX_DIM; state, q, k
+ * 16-byte aligned, the rest 4-byte aligned; state and o may not overlap each
+ * other or any input.  Errors: FMOE_EINVAL, FMOE_ECUDA.  Nothing is
+ * allocated. */
+int fmoe_delta_update(float* state, const float* q, const float* k, const float* v, const float* alpha,
+                      const float* beta, float* o, int heads, int dk, int dv, int T, fmoe_stream_t stream);
+
 /* How the single-token layer kernel (fmoe_layer_decode with T = 1,
  * fmoe_layer_decode_noalloc with T = 1, fmoe_expert_forward) is launched,
  * process-wide, for the calls made after this one.

@@ -10,7 +10,11 @@ GEMV, no routing, no activation.  It only produces
   distributions (scale ~ U(1e-3, 4e-3), bias = -m * scale * (1 + U(-0.1, 0.1))
   with m = 8 at 4 bits and m = 1.5 at 2 bits),
 * bf16 router rows and the bf16 shared-gate vector ~ N(0, 0.02),
-* fp32 token vectors x and residual ~ N(0, 1).
+* fp32 token vectors x and residual ~ N(0, 1);
+* for the linear-attention state update: an fp32 state ~ N(0, 0.1^2) per
+  element, and per token and head a key of unit length (a standard normal
+  vector divided by its length), a query ~ N(0, 1/dk) per element, a value
+  ~ N(0, 1), a decay gate alpha ~ U(0.9, 1) and a write gate beta ~ U(0, 1).
 
 Code words and (scale, bias) pairs come from a counter-based generator: the
 i-th output of SplitMix64 (Steele, Lea and Flood, "Fast splittable
@@ -42,6 +46,8 @@ TAG_RES = 0x2E5
 TAG_SGATE = 0x5647E
 TAG_DENSE = 0xDE45E
 TAG_NORM = 0x40235
+TAG_DSTATE = 0xD57A7
+TAG_DTOK = 0xD70C5
 
 GROUP = 64  # quantisation group length along the input dimension
 
@@ -192,3 +198,22 @@ def dense_matrix(seed: int, tag: int, n_rows: int, n_in: int, std: float = 0.02)
     """fp32 dense matrix ~ N(0, std) (input for the quantiser)."""
     g = _rng(seed, TAG_DENSE, tag)
     return (g.standard_normal((n_rows, n_in), dtype=np.float32) * np.float32(std)).astype(np.float32)
+
+
+def delta_state(seed: int, layer: int, heads: int, dv: int, dk: int) -> np.ndarray:
+    """fp32 [heads][dv][dk] ~ N(0, 0.1^2)."""
+    g = _rng(seed, TAG_DSTATE, layer)
+    return (g.standard_normal((heads, dv, dk), dtype=np.float32) * np.float32(0.1)).astype(np.float32)
+
+
+def delta_tokens(seed: int, layer: int, step: int, n_tokens: int, heads: int, dk: int, dv: int) -> dict:
+    """fp32 inputs of n_tokens state updates: q, k [T][heads][dk], v [T][heads][dv],
+    alpha, beta [T][heads] (distributions in the module docstring)."""
+    g = _rng(seed, TAG_DTOK, layer, step)
+    k = g.standard_normal((n_tokens, heads, dk))
+    k = (k / np.linalg.norm(k, axis=-1, keepdims=True)).astype(np.float32)
+    q = (g.standard_normal((n_tokens, heads, dk)) / np.sqrt(dk)).astype(np.float32)
+    v = g.standard_normal((n_tokens, heads, dv), dtype=np.float32)
+    alpha = g.uniform(0.9, 1.0, (n_tokens, heads)).astype(np.float32)
+    beta = g.uniform(0.0, 1.0, (n_tokens, heads)).astype(np.float32)
+    return {"q": q, "k": k, "v": v, "alpha": alpha, "beta": beta}

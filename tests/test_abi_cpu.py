@@ -105,6 +105,23 @@ def test_invalid_arguments_rejected_on_host(F):
     assert L.fmoe_workspace_bytes(ctypes.byref(small), 1) == header + 5 * 128 * 4  # header independent of E
     assert L.fmoe_workspace_bytes(ctypes.byref(c), 0) == 0
     assert L.fmoe_route_workspace_bytes(17, 512) == 0
+    # delta-rule update: shapes, alignment and overlap are checked on the host.
+    # The defaults are disjoint stand-ins (the 64 x 128 x 128 state spans 4 MiB
+    # from 1 MiB; every other buffer lies beyond it); only variants with one
+    # fault each are called, so no call gets past validation.
+    MiB = 1 << 20
+
+    def delta(state=MiB, q=8 * MiB, k=9 * MiB, v=10 * MiB, alpha=11 * MiB, beta=12 * MiB, o=13 * MiB,
+              heads=64, dk=128, dv=128, T=1):
+        return L.fmoe_delta_update(state, q, k, v, alpha, beta, o, heads, dk, dv, T, None)
+
+    for kw in (dict(state=None), dict(o=None), dict(alpha=None),
+               dict(dk=64), dict(dk=640), dict(dk=200), dict(heads=0), dict(dv=0), dict(T=0),
+               dict(heads=65537), dict(state=MiB + 8), dict(q=8 * MiB + 4), dict(v=10 * MiB + 2),
+               dict(o=MiB + 4096),           # readout inside the state
+               dict(q=MiB + 1024),           # an input inside the state
+               dict(o=10 * MiB + 256)):      # readout overlapping v
+        assert delta(**kw) == F.FMOE_EINVAL, kw
     # launch-mode switch: only 0 and 1, nothing changes otherwise
     prev = ctypes.c_int(-1)
     assert L.fmoe_set_dependent_launch(2, ctypes.byref(prev)) == F.FMOE_EINVAL and prev.value == -1

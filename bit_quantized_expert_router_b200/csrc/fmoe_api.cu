@@ -709,7 +709,8 @@ int fmoe_delta_update(float* state, const float* q, const float* k, const float*
   a.dv = dv;
   a.T = T;
   const long long rows = (long long)heads * dv;
-  const unsigned grid = (unsigned)((rows + kDeltaWarps - 1) / kDeltaWarps);
+  const long long per_cta = (long long)kDeltaWarps * delta_rows_per_warp(dk / 128);
+  const unsigned grid = (unsigned)((rows + per_cta - 1) / per_cta);
   switch (dk / 128) {
     case 1: delta_update_kernel<1><<<grid, kDeltaWarps * 32, 0, s>>>(a); break;
     case 2: delta_update_kernel<2><<<grid, kDeltaWarps * 32, 0, s>>>(a); break;

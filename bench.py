@@ -20,6 +20,10 @@ the total over all ranks divided by the slowest rank's time.  With --gpus
 N > 1 (torchrun) every rank decodes its own replicas: the path has no
 data-path exchange.
 
+`--config deltanet` times the other decode step instead: one token through
+one 64-head x 128x128 gated delta-rule state (45 states in rotation, 180 MiB),
+with the same timing rules and JSON keys.
+
 The JSON line also carries: the latency of one isolated step after a 256 MiB
 L2 flush; the roofline of the layer kernel (algorithmic bytes per launch /
 measured time per launch vs the measured HBM copy bandwidth); an

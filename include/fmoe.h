@@ -16,7 +16,9 @@
  * (weight = nibble * scale + bias, evaluated as fma(nibble, scale*x, bias*x):
  * [P1] "Técnicas innovadoras" item 2, [P2] "FMA-optimierter Dequant-Kernel");
  * and a fused end step that adds the weighted expert outputs, the residual and
- * the sigmoid-gated shared expert ([P2] "Metal-Compute-Shader").
+ * the sigmoid-gated shared expert ([P2] "Metal-Compute-Shader").  Beside it,
+ * the gated delta-rule update of the model's linear-attention state
+ * (fmoe_delta_update; [P2] "Accelerate-BLAS für lineare Aufmerksamkeit").
  *
  * Conventions for every entry point
  *   - Tensor pointers are DEVICE pointers owned by the caller; the library

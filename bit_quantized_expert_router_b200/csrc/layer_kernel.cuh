@@ -1,4 +1,4 @@
-// The single-token MoE layer as one persistent, cooperative kernel.
+// The single-token MoE layer as one persistent kernel.
 //
 // What it computes (the Flash-MoE pages): a router GEMV over the experts, then
 // softmax, top-K and renormalised weights ("Flash-MoE: Ausführen eines
@@ -8,22 +8,24 @@
 // out = residual + sum_k w_k y_k + sigmoid(w_sg . x) * y_shared (same section,
 // "MoE-Kombination + Rest + Sigmoid-Gate").
 //
-// How it runs on B200.  One CTA per SM, every CTA co-resident (cooperative
-// launch).  Three phases:
+// How it runs on B200.  One CTA per SM, every CTA co-resident (one CTA fits
+// per SM and the grid is the SM count; a programmatic dependent launch by
+// default, so that its weight-only set-up overlaps the previous kernel's end,
+// or a cooperative launch).  Three phases:
 //   A  router rows and the shared expert's gate/up rows (need nothing);
 //   B  the routed experts' gate/up rows (need the routing decision);
 //   C  the down projections of every expert over each CTA's own contiguous
 //      block of output rows, then the combine (need all SwiGLU activations).
 // Units of phases A and B are dealt round-robin over all warps of the grid.
 //
-// Hand-offs.  Each router warp stores its logit and counts it with one
-// release add on a grid counter.  Every CTA then takes the routing decision
-// with all of its warps: one warp polls until every router row is counted and
-// copies the logits into shared memory, each warp selects the top K of its
-// slice, and one warp merges the candidates (two CTA barriers).  "All
-// activations written" is a second counter that every CTA bumps once and
-// polls once.  Every wait is time-limited: on expiry the kernel sets a status
-// bit and carries on instead of hanging.
+// Hand-offs.  Each router warp publishes its logit as one 64-bit word tagged
+// with this launch's number (the workspace's epoch + 1).  Every CTA then
+// takes the routing decision with all of its warps: each lane polls the words
+// of its warp's slice of the logits until they carry the tag, each warp
+// selects the top K of its slice, and the candidates are ranked (CTA
+// barriers between the steps).  "All activations written" is a counter that
+// every CTA bumps once and polls once.  Every wait is time-limited: on expiry
+// the kernel sets a status bit and carries on instead of hanging.
 //
 // Data movement.  Each warp streams its gate/up units through a private ring
 // of shared-memory stages filled by cp.async.bulk copies that complete on an
@@ -760,9 +762,9 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   // this workspace left, plus one).
   const unsigned ptag = (router_warp && lane == 0) ? ld_relaxed_gpu(&a.bar[0]) + 1u : 0u;
 
-  // x and the router rows are the critical path to the routing decision, so
-  // they are the only traffic of the first microseconds; the shared expert's
-  // gate/up rows follow once x is staged.
+  // x and the router rows are the critical path to the routing decision; the
+  // shared expert's gate/up rows are requested once x is staged (by a router
+  // warp once its dot product is done).
   int issued = 0;
   if (!mbar_wait_bounded(&cs.x_bar, 0, a.timeout_ns) && lane == 0) set_status(kStatusCopyTimeout);
   FMOE_TRACE_WARP(16);
@@ -786,7 +788,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   }
   const float* xu = sm.vec + a.xu_off;
   if (router_warp) {
-    // ---- Phase A, router rows: published, then counted once per CTA ---------
+    // ---- Phase A, router rows: each logit published as one tagged word ------
     for (int j = 0; j < plan.router.count; ++j) {
       const int e = plan.router.first + j * GW;
       float l;

@@ -59,14 +59,15 @@ def test_single_rank_is_identity():
     assert bench.whole_job_rate(10, 1, 1000.0) == pytest.approx(10.0)
 
 
+@pytest.mark.parametrize("config,unit", [("tiny", "decodes/s"), ("deltanet", "updates/s")])
 @pytest.mark.parametrize("rank", [0, 1])
-def test_reference_arm_prints_on_rank_zero_only(rank):
+def test_reference_arm_prints_on_rank_zero_only(rank, config, unit):
     import json
     import subprocess
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank))
-    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--config", "tiny",
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--config", config,
                         "--steps", "1", "--warmup", "3"], capture_output=True, text=True, env=env, timeout=300,
                        cwd=root)
     assert r.returncode == 0, r.stderr
@@ -75,5 +76,5 @@ def test_reference_arm_prints_on_rank_zero_only(rank):
         assert lines == []
     else:
         d = json.loads(lines[-1])
-        assert d["impl"] == "reference" and d["unit"] == "decodes/s" and d["value"] > 0
+        assert d["impl"] == "reference" and d["unit"] == unit and d["value"] > 0
         assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0

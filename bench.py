@@ -192,8 +192,21 @@ class ClockSampler:
 # CPU oracle leg (reference arm and cpu_baseline)
 # ---------------------------------------------------------------------------
 
-def oracle_sample(cfg, budget_s: float, max_tokens: int = 1000) -> dict:
-    """Time the oracle (as it stands) on a bounded sample of the same workload."""
+REF_WARMUP_S = 30.0   # the reference arm's warm-up stops after this much host time
+REF_BUDGET_S = 120.0  # and its timed steps after this much
+
+
+def host_cores() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    except Exception:
+        return 1
+
+
+def oracle_prepare(cfg):
+    """Draw the oracle's inputs for the layer workload once (untimed input
+    preparation) and return decode(t): one single-token decode of pool token t."""
     import oracle as O
     h, i, e, k = cfg["hidden"], cfg["inter"], cfg["experts"], cfg["top_k"]
     w_router = S.router_bf16(SEED, 0, e, h)
@@ -203,65 +216,90 @@ def oracle_sample(cfg, budget_s: float, max_tokens: int = 1000) -> dict:
         return O.assemble_blob(S.expert_parts(SEED, 0, ex, h, i, bits), h, i, bits)
 
     shared = blob(S.SHARED_EXPERT_ID, cfg["shared_bits"])
-    xs = S.token_x(SEED, 0, 0, POOL, h)
-    res = S.token_residual(SEED, 0, 0, POOL, h)
-    # expert blobs are input preparation, drawn before the clock starts
+    n_tok = min(POOL, 8)
+    xs = S.token_x(SEED, 0, 0, n_tok, h)
+    res = S.token_residual(SEED, 0, 0, n_tok, h)
     pre = {}
-    for t in range(min(POOL, 8)):
+    for t in range(n_tok):
         for ex in O.route(w_router, w_sg, xs[t], k)["idx"]:
             if int(ex) not in pre:
                 pre[int(ex)] = blob(int(ex), cfg["bits"])
-    n = 0
-    t0 = time.perf_counter()
-    while True:
-        t = n % min(POOL, 8)
+
+    def decode(t):
+        t %= n_tok
         O.layer_decode(w_router, w_sg, lambda ex: pre[ex], shared, xs[t], res[t], k, h, i, cfg["bits"],
                        cfg["shared_bits"])
+    return decode
+
+
+def delta_oracle_prepare(cfg):
+    """The same for the delta-rule workload: decode(t) is one token's update."""
+    import oracle as O
+    H, dk, dv = cfg["heads"], cfg["dk"], cfg["dv"]
+    box = {"state": S.delta_state(SEED, 0, H, dv, dk)}
+    toks = [S.delta_tokens(SEED, 0, j, 1, H, dk, dv) for j in range(8)]
+
+    def decode(t):
+        tk = toks[t % len(toks)]
+        box["state"], _ = O.delta_update(box["state"], tk["q"], tk["k"], tk["v"], tk["alpha"], tk["beta"])
+    return decode
+
+
+def time_oracle(decode, max_steps: int, budget_s: float):
+    """Run decode(0), decode(1), ... until max_steps or budget_s; (steps, seconds)."""
+    n = 0
+    t0 = time.perf_counter()
+    while n < max_steps:
+        decode(n)
         n += 1
-        el = time.perf_counter() - t0
-        if el >= budget_s or n >= max_tokens:
+        if time.perf_counter() - t0 >= budget_s:
             break
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    except Exception:
-        cores = 1
-    return dict(value=n / el, unit=UNIT, cores=cores, kind="oracle", seconds=el, tokens=n,
-                sample=f"{n} single-token decodes of the {cfg['workload']} layer (fp64 numpy oracle, "
-                       f"expert blobs pre-drawn), {el:.1f} s")
+    return n, time.perf_counter() - t0
+
+
+def oracle_sample(cfg, budget_s: float) -> dict:
+    """Time the oracle (as it stands) on a bounded sample of the same workload."""
+    delta = cfg.get("kind") == "deltanet"
+    decode = (delta_oracle_prepare if delta else oracle_prepare)(cfg)
+    n, el = time_oracle(decode, 1 << 30, budget_s)
+    what = (f"one-token updates of the {cfg['workload']} state" if delta else
+            f"single-token decodes of the {cfg['workload']} layer (fp64 numpy oracle, expert blobs pre-drawn)")
+    return dict(value=n / el, unit="updates/s" if delta else UNIT, cores=host_cores(), kind="oracle", seconds=el,
+                tokens=n, sample=f"{n} {what}, {el:.1f} s")
 
 
 def run_reference(args, cfg, rank, world):
+    """The reference arm: the CPU oracle as it stands, on rank 0 only.  Its
+    inputs are drawn once; W warm-up steps (at most REF_WARMUP_S of host time)
+    and then up to K timed steps, stopping after REF_BUDGET_S so that the run
+    ends within a few minutes whatever K is; the rate is taken over the steps
+    that ran, and the line says how many."""
     if rank != 0:
         return
-    steps, warm = args.steps, args.warmup
-    # bounded: the whole reference run stays within a few minutes
-    per_step_budget = max(0.5, min(20.0, 120.0 / max(1, steps + warm)))
-    for _ in range(warm):
-        oracle_sample(cfg, per_step_budget * 0.2, max_tokens=1)
-    t_total, n_total = 0.0, 0
-    last = None
-    for _ in range(steps):
-        r = oracle_sample(cfg, per_step_budget, max_tokens=2)
-        t_total += r["seconds"]
-        n_total += r["tokens"]
-        last = r
+    delta = cfg.get("kind") == "deltanet"
+    decode = (delta_oracle_prepare if delta else oracle_prepare)(cfg)
+    time_oracle(decode, args.warmup, REF_WARMUP_S)
+    n, el = time_oracle(decode, args.steps, REF_BUDGET_S)
     lps = cfg.get("layers_per_step", 1)
     tt = cfg.get("tokens", 1)
     metric, unit = METRIC, UNIT
-    if lps > 1:
+    if delta:
+        metric, unit = DELTA_METRIC, "updates/s"
+    elif lps > 1:
         metric, unit = f"decode steps/s through {lps} MoE layers (batch 1)", "steps/s"
     elif tt > 1:
         metric, unit = f"token decodes/s through one MoE layer ({tt}-token batches)", "tokens/s"
-    value = n_total / t_total / lps
+    value = n / el / lps  # one oracle step is one token through one layer (or one state update)
+    what = "one-token state updates" if delta else "single-token single-layer decodes"
+    sample = (f"{n} {what} timed of the {args.steps} steps asked (at most {REF_BUDGET_S:.0f} s of host time), "
+              f"{el:.1f} s" + (f"; steps/s = decodes/s / {lps}" if lps > 1 else ""))
     line = {
-        "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": steps,
-        "warmup": warm, "ms_per_step": 1000.0 * t_total / n_total * lps, "higher_is_better": True, "scaling": "weak",
+        "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 / value, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {**{k: v for k, v in cfg.items()}, "batch": 1, "parallelism": "host cores"},
-        "cpu_baseline": {"value": value, "unit": unit, "cores": last["cores"], "kind": "oracle",
-                         "sample": f"{n_total} single-layer decodes over {steps} steps"
-                                   + (f"; steps/s = decodes/s / {lps}" if lps > 1 else "")},
+        "config": {**cfg, "batch": 1, "parallelism": "host cores"},
+        "steps_timed": n,
+        "cpu_baseline": {"value": value, "unit": unit, "cores": host_cores(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -512,56 +550,6 @@ def delta_bytes(cfg) -> int:
     return 4 * (2 * H * dv * dk + 2 * H * dk + 2 * H * dv + 2 * H)
 
 
-def delta_oracle_sample(cfg, budget_s: float, max_steps: int = 100000) -> dict:
-    """Time the oracle (as it stands) on state updates of the same shape."""
-    import oracle as O
-    H, dk, dv = cfg["heads"], cfg["dk"], cfg["dv"]
-    st = S.delta_state(SEED, 0, H, dv, dk)
-    toks = [S.delta_tokens(SEED, 0, j, 1, H, dk, dv) for j in range(8)]
-    n = 0
-    t0 = time.perf_counter()
-    while True:
-        tk = toks[n % len(toks)]
-        st, _ = O.delta_update(st, tk["q"], tk["k"], tk["v"], tk["alpha"], tk["beta"])
-        n += 1
-        el = time.perf_counter() - t0
-        if el >= budget_s or n >= max_steps:
-            break
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    except Exception:
-        cores = 1
-    return dict(value=n / el, unit="updates/s", cores=cores, kind="oracle", seconds=el, tokens=n,
-                sample=f"{n} one-token updates of the {cfg['workload']} state (fp64 numpy oracle), {el:.1f} s")
-
-
-def run_reference_delta(args, cfg, rank, world):
-    if rank != 0:
-        return
-    steps, warm = args.steps, args.warmup
-    per_step_budget = max(0.05, min(5.0, 60.0 / max(1, steps + warm)))
-    for _ in range(warm):
-        delta_oracle_sample(cfg, per_step_budget * 0.2, max_steps=1)
-    t_total, n_total, last = 0.0, 0, None
-    for _ in range(steps):
-        r = delta_oracle_sample(cfg, per_step_budget, max_steps=4)
-        t_total += r["seconds"]
-        n_total += r["tokens"]
-        last = r
-    value = n_total / t_total
-    line = {
-        "impl": "reference", "metric": DELTA_METRIC, "value": value, "unit": "updates/s", "n_gpus": world,
-        "steps": steps, "warmup": warm, "ms_per_step": 1000.0 * t_total / n_total, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {**cfg, "batch": 1, "parallelism": "host cores"},
-        "cpu_baseline": {"value": value, "unit": "updates/s", "cores": last["cores"], "kind": "oracle",
-                         "sample": f"{n_total} one-token state updates over {steps} steps"},
-        "e2e": {"value": value, "unit": "updates/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }
-    print(json.dumps(line), flush=True)
-
-
 def run_delta(args, cfg, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -703,7 +691,7 @@ def run_delta(args, cfg, rank, world, local_rank):
             "device_status": status,
         }
         if not args.no_cpu_baseline:
-            cb = delta_oracle_sample(cfg, args.cpu_seconds)
+            cb = oracle_sample(cfg, args.cpu_seconds)
             cb.pop("seconds", None)
             cb.pop("tokens", None)
             line["cpu_baseline"] = cb
@@ -733,7 +721,7 @@ def main():
     delta = cfg.get("kind") == "deltanet"
     if args.impl == "reference":
         if rank == 0:
-            (run_reference_delta if delta else run_reference)(args, cfg, rank, world)
+            run_reference(args, cfg, rank, world)
         return
     if world > 1:
         import datetime

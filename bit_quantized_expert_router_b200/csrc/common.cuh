@@ -73,7 +73,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
-// ---- bulk copies (no tensor map, no multicast) --------------------------------
+// ---- bulk copies (no tensor map; each copy lands in this CTA only) ------------
 // Order this thread's earlier generic-proxy shared-memory accesses before
 // subsequent async-proxy (bulk copy) writes.
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -38,3 +38,23 @@ def test_router_and_tokens():
     x = S.token_x(3, 0, 0, 2, 512)
     assert x.dtype == np.float32 and x.shape == (2, 512) and abs(x.std() - 1) < 0.1
     assert not np.array_equal(S.token_x(3, 0, 0, 1, 512, redraw=1), x[:1])
+
+
+def test_delta_inputs_seeded_and_shaped():
+    """The delta-rule inputs: deterministic per (seed, layer, step), the stated
+    shapes and distributions (unit keys, gates in their ranges)."""
+    a = S.delta_tokens(7, 2, 3, 4, 5, 128, 96)
+    b = S.delta_tokens(7, 2, 3, 4, 5, 128, 96)
+    c = S.delta_tokens(7, 2, 4, 4, 5, 128, 96)
+    for n in a:
+        assert a[n].dtype == np.float32 and np.array_equal(a[n], b[n])
+        assert not np.array_equal(a[n], c[n])
+    assert a["q"].shape == a["k"].shape == (4, 5, 128) and a["v"].shape == (4, 5, 96)
+    assert a["alpha"].shape == a["beta"].shape == (4, 5)
+    np.testing.assert_allclose(np.linalg.norm(a["k"].astype(np.float64), axis=-1), 1.0, rtol=1e-6)
+    assert (a["alpha"] >= 0.9).all() and (a["alpha"] <= 1.0).all()
+    assert (a["beta"] >= 0.0).all() and (a["beta"] <= 1.0).all()
+    st = S.delta_state(7, 2, 5, 96, 128)
+    assert st.shape == (5, 96, 128) and st.dtype == np.float32
+    assert np.array_equal(st, S.delta_state(7, 2, 5, 96, 128))
+    assert abs(float(st.std()) - 0.1) < 0.005

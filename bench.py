@@ -236,12 +236,12 @@ def delta_oracle_prepare(cfg):
     """The same for the delta-rule workload: decode(t) is one token's update."""
     import oracle as O
     H, dk, dv = cfg["heads"], cfg["dk"], cfg["dv"]
-    box = {"state": S.delta_state(SEED, 0, H, dv, dk)}
+    cur = {"state": S.delta_state(SEED, 0, H, dv, dk)}
     toks = [S.delta_tokens(SEED, 0, j, 1, H, dk, dv) for j in range(8)]
 
     def decode(t):
         tk = toks[t % len(toks)]
-        box["state"], _ = O.delta_update(box["state"], tk["q"], tk["k"], tk["v"], tk["alpha"], tk["beta"])
+        cur["state"], _ = O.delta_update(cur["state"], tk["q"], tk["k"], tk["v"], tk["alpha"], tk["beta"])
     return decode
 
 

@@ -11,6 +11,7 @@ import ctypes
 import os
 from dataclasses import dataclass
 
+import numpy as np
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -26,6 +27,7 @@ EXPORTED = [
     "fmoe_route", "fmoe_expert_workspace_bytes", "fmoe_expert_forward", "fmoe_workspace_bytes",
     "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status", "fmoe_strerror", "fmoe_last_cuda_error",
     "fmoe_layer_decode_noalloc", "fmoe_set_wait_limit_ns", "fmoe_set_dependent_launch", "fmoe_delta_update",
+    "fmoe_cache_create", "fmoe_cache_destroy", "fmoe_cache_lookup", "fmoe_cache_stats", "fmoe_cache_reset",
 ]
 
 
@@ -81,6 +83,12 @@ def lib() -> ctypes.CDLL:
     L.fmoe_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong)]
     L.fmoe_set_dependent_launch.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
     L.fmoe_delta_update.argtypes = [vp] * 7 + [i, i, i, i, vp]
+    L.fmoe_cache_create.argtypes = [i, ctypes.POINTER(vp)]
+    L.fmoe_cache_destroy.argtypes = [vp]
+    L.fmoe_cache_lookup.argtypes = [vp, i, vp, i, vp, vp, ctypes.POINTER(i)]
+    u64p = ctypes.POINTER(ctypes.c_uint64)
+    L.fmoe_cache_stats.argtypes = [vp, u64p, u64p, u64p]
+    L.fmoe_cache_reset.argtypes = [vp]
     L.fmoe_last_cuda_error.argtypes = []
     L.fmoe_last_cuda_error.restype = i
     L.fmoe_strerror.argtypes = [i]
@@ -309,6 +317,42 @@ def delta_update(state: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch
                                    beta.data_ptr(), o.data_ptr(), heads, dk, dv, T, _stream(stream)),
            "fmoe_delta_update")
     return o
+
+
+class ExpertCache:
+    """Host directory of a device expert cache of n_slots slots (see
+    fmoe_cache_lookup in include/fmoe.h): which selected experts are in a
+    slot and which slot each miss goes to (least recently used)."""
+
+    def __init__(self, n_slots: int):
+        h = ctypes.c_void_p()
+        _check(lib().fmoe_cache_create(int(n_slots), ctypes.byref(h)), "fmoe_cache_create")
+        self._h = h
+        self.n_slots = int(n_slots)
+
+    def lookup(self, layer: int, idx) -> tuple[np.ndarray, np.ndarray]:
+        """(slots, misses) for the experts idx selected in `layer`."""
+        idx = np.ascontiguousarray(np.asarray(idx, dtype=np.int32).reshape(-1))
+        slot = np.empty_like(idx)
+        miss = np.empty_like(idx)
+        n = ctypes.c_int(0)
+        _check(lib().fmoe_cache_lookup(self._h, int(layer), idx.ctypes.data, idx.size, slot.ctypes.data,
+                                       miss.ctypes.data, ctypes.byref(n)), "fmoe_cache_lookup")
+        return slot, miss
+
+    def stats(self) -> dict:
+        v = [ctypes.c_uint64(0) for _ in range(3)]
+        _check(lib().fmoe_cache_stats(self._h, *(ctypes.byref(x) for x in v)), "fmoe_cache_stats")
+        return {"hits": v[0].value, "misses": v[1].value, "evictions": v[2].value}
+
+    def reset(self) -> None:
+        _check(lib().fmoe_cache_reset(self._h), "fmoe_cache_reset")
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value and _lib is not None:
+            _lib.fmoe_cache_destroy(h)
+            self._h = None
 
 
 def set_dependent_launch(enable: bool) -> bool:

@@ -6,6 +6,7 @@
 
 #include "../../include/fmoe.h"
 #include "deltanet.cuh"
+#include "expert_cache.h"
 #include "shared_tc.cuh"
 
 using namespace fmoe;
@@ -718,6 +719,57 @@ int fmoe_delta_update(float* state, const float* q, const float* k, const float*
     default: delta_update_kernel<4><<<grid, kDeltaWarps * 32, 0, s>>>(a); break;
   }
   if (cudaError_t e = cudaGetLastError()) return cuda_fail(e);
+  return FMOE_OK;
+}
+
+struct fmoe_expert_cache_s {
+  fmoe::ExpertCache c;
+  explicit fmoe_expert_cache_s(int n) : c(n) {}
+};
+
+int fmoe_cache_create(int n_slots, fmoe_expert_cache** cache_out) {
+  if (!cache_out || n_slots < 1 || n_slots > FMOE_CACHE_MAX_SLOTS) return FMOE_EINVAL;
+  *cache_out = nullptr;
+  try {
+    *cache_out = new fmoe_expert_cache_s(n_slots);
+  } catch (...) {
+    return FMOE_ENOMEM;
+  }
+  return FMOE_OK;
+}
+
+int fmoe_cache_destroy(fmoe_expert_cache* cache) {
+  delete cache;
+  return FMOE_OK;
+}
+
+int fmoe_cache_lookup(fmoe_expert_cache* cache, int layer, const int32_t* idx, int K, int32_t* slot_out,
+                      int32_t* miss_out, int* n_miss_out) {
+  if (!cache || !idx || !slot_out || !miss_out || layer < 0 || K < 1 || K > cache->c.n_slots()) return FMOE_EINVAL;
+  for (int k = 0; k < K; ++k)
+    if (idx[k] < 0) return FMOE_EINVAL;
+  try {
+    cache->c.lookup(layer, idx, K, slot_out, miss_out);
+  } catch (...) {
+    return FMOE_ENOMEM;
+  }
+  if (n_miss_out) {
+    int n = 0;
+    for (int k = 0; k < K; ++k) n += miss_out[k];
+    *n_miss_out = n;
+  }
+  return FMOE_OK;
+}
+
+int fmoe_cache_stats(const fmoe_expert_cache* cache, uint64_t* hits, uint64_t* misses, uint64_t* evictions) {
+  if (!cache) return FMOE_EINVAL;
+  cache->c.stats(hits, misses, evictions);
+  return FMOE_OK;
+}
+
+int fmoe_cache_reset(fmoe_expert_cache* cache) {
+  if (!cache) return FMOE_EINVAL;
+  cache->c.reset();
   return FMOE_OK;
 }
 

@@ -261,6 +261,47 @@ int fmoe_set_wait_limit_ns(unsigned long long limit_ns, unsigned long long* prev
 int fmoe_delta_update(float* state, const float* q, const float* k, const float* v, const float* alpha,
                       const float* beta, float* o, int heads, int dk, int dv, int T, fmoe_stream_t stream);
 
+/* ---- Expert cache directory (host side of streaming non-resident experts) ---- */
+
+#define FMOE_CACHE_MAX_SLOTS (1 << 20)
+
+/* The pages read each layer's K selected experts from the SSD on demand and
+ * let the operating system's page cache, a least-recently-used cache, hold
+ * them (~71 % hits: [P1] "Técnicas innovadoras" §1, [P2]
+ * "SSD-Experten-Streaming", [P3] "Trust the OS").  The B200 analogue keeps
+ * the experts in pinned host memory and a pool of n_slots device slots (one
+ * expert blob each) as the cache.  This opaque directory decides, per layer
+ * call, which selected experts are already in a slot and which slot each miss
+ * goes to: never-used slots first (lowest index first), then the least
+ * recently used slot over all layers.  It is host-only: it moves no data and
+ * makes no CUDA call (copying a miss's blob into its slot is the caller's).
+ * Not thread-safe: one directory per thread, or the caller's lock. */
+typedef struct fmoe_expert_cache_s fmoe_expert_cache;
+
+/* A directory of n_slots slots, all free.  1 <= n_slots <=
+ * FMOE_CACHE_MAX_SLOTS; *cache_out is set (NULL on error).  Errors:
+ * FMOE_EINVAL, FMOE_ENOMEM. */
+int fmoe_cache_create(int n_slots, fmoe_expert_cache** cache_out);
+
+/* Free a directory (NULL is accepted).  Returns FMOE_OK. */
+int fmoe_cache_destroy(fmoe_expert_cache* cache);
+
+/* For the K experts idx[0..K) selected in `layer` (host arrays): slot_out[k]
+ * is the expert's slot and miss_out[k] is 1 when its blob must be copied in
+ * (0 when it is there already); *n_miss_out (optional) counts the misses.
+ * The touched entries become the most recently used, in k order; an expert
+ * listed twice takes one slot (its second listing is a hit).  Requires
+ * layer >= 0, idx[k] >= 0 and 1 <= K <= n_slots (so that no slot of this call
+ * is evicted by it).  Errors: FMOE_EINVAL, FMOE_ENOMEM. */
+int fmoe_cache_lookup(fmoe_expert_cache* cache, int layer, const int32_t* idx, int K, int32_t* slot_out,
+                      int32_t* miss_out, int* n_miss_out);
+
+/* Running totals since creation or the last reset (each pointer optional). */
+int fmoe_cache_stats(const fmoe_expert_cache* cache, uint64_t* hits, uint64_t* misses, uint64_t* evictions);
+
+/* Empty the directory (all slots free) and zero the totals. */
+int fmoe_cache_reset(fmoe_expert_cache* cache);
+
 /* How the single-token layer kernel (fmoe_layer_decode with T = 1,
  * fmoe_layer_decode_noalloc with T = 1, fmoe_expert_forward) is launched,
  * process-wide, for the calls made after this one.

@@ -5,6 +5,7 @@ is written next to this file so that it travels with the source tree.
 """
 from __future__ import annotations
 
+import hashlib
 import os
 import subprocess
 import sys
@@ -23,18 +24,34 @@ ENGINE_DEPS = [os.path.join(HERE, "csrc", f) for f in
 ENGINE_SO = os.path.join(HERE, "libfmoe.so")
 
 
-def _stale(target: str, sources: list[str]) -> bool:
-    if not os.path.exists(target):
+def build_key(sources: list[str], cmd: list[str]) -> str:
+    """Hash of the sources' bytes and the compiler command: a library is rebuilt
+    whenever this differs from the key stored beside it (file times are not
+    trusted: a copied tree can carry a stale library with a fresh time)."""
+    h = hashlib.sha256()
+    for c in cmd:
+        h.update(c.encode() + b"\0")
+    for s in sources:
+        h.update(os.path.basename(s).encode() + b"\0")
+        with open(s, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def _stale(target: str, key: str) -> bool:
+    try:
+        with open(target + ".key") as f:
+            return not os.path.exists(target) or f.read().strip() != key
+    except OSError:
         return True
-    t = os.path.getmtime(target)
-    return any(os.path.getmtime(s) > t for s in sources)
 
 
 def compile_so(src: str, out: str, deps: list[str], extra: list[str] | None = None,
                force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale(out, [src] + deps):
-        return out
     cmd = [NVCC, *ARCH, *FLAGS, *(extra or []), src, "-o", out + ".tmp"]
+    key = build_key([src] + deps, cmd)
+    if not force and not _stale(out, key):
+        return out
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -43,6 +60,9 @@ def compile_so(src: str, out: str, deps: list[str], extra: list[str] | None = No
     if verbose:
         sys.stderr.write(r.stderr)
     os.replace(out + ".tmp", out)
+    with open(out + ".key.tmp", "w") as f:
+        f.write(key + "\n")
+    os.replace(out + ".key.tmp", out + ".key")
     return out
 
 

@@ -554,6 +554,43 @@ int fmoe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream_t stream) {
   return FMOE_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Every host-side check of a layer decode call except those of the workspace
+// (shapes, pointers, alignment, the stream's device); on success the current
+// device and its info.  Nothing is enqueued.
+int check_layer_call(const fmoe_layer* L, const float* x, const float* residual, const float* out, int T,
+                     fmoe_stream_t stream, int* dev_out, DevInfo** info_out) {
+  if (!L || !x || !out || !L->w_router || !L->experts) return FMOE_EINVAL;
+  const int H = L->hidden, I = L->inter, E = L->n_experts, K = L->top_k;
+  if (!shape_ok(H, I) || !bits_ok(L->bits) || (L->shared && !bits_ok(L->shared_bits)) ||
+      L->group != FMOE_GROUP || E < 1 || E > FMOE_MAX_EXPERTS || K < 1 || K > FMOE_MAX_TOPK || K > E ||
+      T < 1 || T > FMOE_MAX_TOKENS || (K + 1) * I > 10240)
+    return FMOE_EINVAL;
+  if (L->expert_stride < (int64_t)fmoe_expert_bytes(H, I, L->bits) || L->expert_stride % 256)
+    return FMOE_EINVAL;
+  if (!aligned(L->experts, 256) || (L->shared && !aligned(L->shared, 256)) || !aligned(L->w_router, 16) ||
+      (L->w_sgate && !aligned(L->w_sgate, 16)) || !aligned(x, 16) || !aligned(out, 16) ||
+      (residual && !aligned(residual, 16)) || x == out)
+    return FMOE_EINVAL;
+  if (L->norm_weight && (!aligned(L->norm_weight, 16) || !(L->norm_eps >= 0.f) || !(L->norm_eps < INFINITY)))
+    return FMOE_EINVAL;
+  int dev;
+  DevInfo* info;
+  if (int rc = dev_info(&dev, &info)) return rc;
+  if (int rc = check_stream(stream, dev)) return rc;
+  if (E + 1 > (kWarps / 2) * info->sms) return FMOE_EINVAL;  // router rows must leave staging warps
+  *dev_out = dev;
+  *info_out = info;
+  return FMOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual, float* out, int T,
                       void* ws, size_t ws_bytes, int32_t* idx_out_opt, float* w_out_opt,
                       fmoe_stream_t stream) {
@@ -634,12 +671,15 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
 int fmoe_layer_decode_noalloc(const fmoe_layer* L, const float* x, const float* residual, float* out, int T,
                               int32_t* idx_out_opt, float* w_out_opt, fmoe_stream_t stream) {
   if (!L) return FMOE_EINVAL;
+  if (T != 1) return FMOE_EINVAL;  // single-token decodes only (a grouped workspace never fits the scratch)
   const size_t need = fmoe_workspace_bytes(L, T);
   if (need == 0) return FMOE_EINVAL;
   if (need > kNoallocScratchBytes) return FMOE_ENOMEM;  // layer too large for the fixed scratch
+  // Every check of the decode itself comes first: a call that is rejected
+  // enqueues nothing (not even the clearing of the scratch below).
   int dev = 0;
-  if (cudaError_t e = cudaGetDevice(&dev)) return cuda_fail(e);
-  if (dev < 0 || dev >= 64) return FMOE_EINVAL;
+  DevInfo* info = nullptr;
+  if (int rc = check_layer_call(L, x, residual, out, T, stream, &dev, &info)) return rc;
   void* ws = nullptr;
   if (int rc = noalloc_scratch(dev, &ws)) return rc;
   // The scratch keeps whatever the previous call left: clear the counters and

@@ -198,7 +198,10 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
  * device allocator of their own.  The Flash-MoE pages have no counterpart:
  * this is an interface convenience of this library.
  *   Arguments, outputs and errors are those of fmoe_layer_decode, minus the
- *   workspace.  The workspace comes from one fixed 32 KiB array in device
+ *   workspace, for single-token decodes only: T must be 1 (FMOE_EINVAL
+ *   otherwise; a grouped decode's workspace is far larger than the array).
+ *   Every argument is checked before anything is enqueued, so a rejected
+ *   call leaves the array untouched.  The workspace comes from one fixed 32 KiB array in device
  *   memory that every GPU which loads the library keeps until the process
  *   exits; a layer whose fmoe_workspace_bytes() exceeds 32 KiB is rejected
  *   with FMOE_ENOMEM (the full-size layer of the pages, 512 experts, top-4,

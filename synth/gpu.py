@@ -9,6 +9,7 @@ layer's arithmetic.
 from __future__ import annotations
 
 import ctypes
+import hashlib
 import os
 import subprocess
 
@@ -26,13 +27,29 @@ _lib = None
 
 
 def build(force: bool = False) -> str:
-    if force or not os.path.exists(SO) or os.path.getmtime(SO) < os.path.getmtime(SRC):
-        cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-Xcompiler",
-               "-fPIC", "-shared", SRC, "-o", SO + ".tmp"]
+    """Compile synth.cu in-tree; rebuilt whenever the hash of its source and
+    command differs from the one stored beside the library."""
+    cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-Xcompiler",
+           "-fPIC", "-shared", SRC, "-o", SO + ".tmp"]
+    h = hashlib.sha256()
+    for c in cmd:
+        h.update(c.encode() + b"\0")
+    with open(SRC, "rb") as f:
+        h.update(f.read())
+    key = h.hexdigest()
+    try:
+        with open(SO + ".key") as f:
+            stale = f.read().strip() != key or not os.path.exists(SO)
+    except OSError:
+        stale = True
+    if force or stale:
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed for {SRC}:\n{r.stdout}\n{r.stderr}")
         os.replace(SO + ".tmp", SO)
+        with open(SO + ".key.tmp", "w") as f:
+            f.write(key + "\n")
+        os.replace(SO + ".key.tmp", SO + ".key")
     return SO
 
 

@@ -439,6 +439,127 @@ def pin_quantizer(O):
         assert np.max(np.abs(m - ref)) < 0.02 * 8 / 15
 
 
+def load_bf16_golden():
+    rows = []
+    with open(os.path.join(GOLDEN, "bf16_rounding.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                a, b = line.split()[:2]
+                rows.append((int(a, 16), int(b, 16)))
+    return rows
+
+
+def _bf16_nearest_even(u32: int) -> int:
+    """bf16 pattern nearest to the finite fp32 pattern u32 by exact comparison
+    of the two neighbouring bf16 values (ties to the even mantissa)."""
+    x = Fraction(float(np.array([u32], dtype=np.uint32).view(np.float32)[0]))
+    lo = u32 >> 16  # the bf16 pattern of the same sign toward zero
+    hi = lo + 1     # the next bf16 pattern away from zero
+    d_lo = abs(x - bf16_exact(lo))
+    d_hi = abs(bf16_exact(hi) - x) if (hi & 0x7FFF) < 0x7F80 else None
+    if d_hi is None or d_lo < d_hi:
+        return lo
+    if d_hi < d_lo:
+        return hi
+    return lo if lo % 2 == 0 else hi
+
+
+def pin_bf16_rne(O):
+    """fp32 -> bf16 is round to nearest, ties to even: hand-worked bit patterns
+    (ties both ways, just above and below a tie, a carry into the exponent,
+    subnormals; tests/golden/bf16_rounding.txt) and, on random finite values,
+    the nearest bf16 neighbour found by exact rational comparison."""
+    gold = load_bf16_golden()
+    assert len(gold) >= 16
+    src = np.array([a for a, _ in gold], dtype=np.uint32).view(np.float32)
+    got = O.f32_to_bf16_bits(src)
+    for (a, want), g in zip(gold, got.tolist()):
+        assert g == want, (hex(a), hex(g), hex(want))
+    rng = np.random.default_rng(22)
+    u = rng.integers(0, 2**32, size=3000, dtype=np.uint64).astype(np.uint32)
+    u = u[(u & 0x7F800000) < 0x7F000000]  # finite, clear of bf16 overflow
+    # every exact tie pattern of these exponents too
+    u = np.concatenate([u, (u & np.uint32(0xFFFF0000)) | np.uint32(0x8000)])
+    got = O.f32_to_bf16_bits(u.view(np.float32))
+    for a, g in zip(u.tolist(), got.tolist()):
+        assert g == _bf16_nearest_even(a), hex(a)
+
+
+def load_quantizer_ties():
+    groups = []
+    with open(os.path.join(GOLDEN, "quantizer_ties.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = line.split()
+            if parts[0] == "group":
+                groups.append((int(parts[1]), int(parts[2], 16), [], []))
+            else:
+                groups[-1][2].append(int(parts[0], 16))
+                groups[-1][3].append(int(parts[1]))
+    return groups
+
+
+def pin_quantizer_ties(O):
+    """Groups whose fp32 quotient (w - bias) / s is an exact half only after
+    the fp32 subtraction rounds: the hand-worked codes (round half to even on
+    the fp32 quotient, tests/golden/quantizer_ties.txt) separate the stated
+    fp32 op order from an fp64 division and from rounding halves up."""
+    groups = load_quantizer_ties()
+    assert [g[0] for g in groups] == [4, 2]
+    for bits, sbw, wbits, codes in groups:
+        assert len(wbits) == 64
+        w = np.array(wbits, dtype=np.uint32).view(np.float32).reshape(1, 64)
+        got_codes, got_sb = O.quantize_matrix(w, bits)
+        assert int(got_sb[0, 0]) == sbw, (bits, hex(int(got_sb[0, 0])))
+        words = [int(v) for v in got_codes[0]]
+        per = 32 // bits
+        dec = [code_from_bitstring(words[k // per], bits, k % per) for k in range(64)]
+        assert dec == codes, (bits, dec, codes)
+    # on every quotient: the fp32 subtraction, the fp32 division and ties to
+    # even, evaluated one element at a time with Python floats narrowed to fp32
+    rng = np.random.default_rng(23)
+    f32 = lambda v: float(np.float32(v))
+    for bits in (4, 2):
+        qmax = (1 << bits) - 1
+        w = (rng.standard_normal((4, 128)) * 0.02).astype(np.float32)
+        got_codes, got_sb = O.quantize_matrix(w, bits)
+        for r in range(4):
+            for gi in range(2):
+                grp = [float(v) for v in w[r, gi * 64:(gi + 1) * 64]]
+                sbw = int(got_sb[r, gi])
+                s = float(bf16_exact(sbw & 0xFFFF))
+                b = float(bf16_exact(sbw >> 16))
+                for j, v in enumerate(grp):
+                    quot = f32(f32(v - b) / s)
+                    want = min(max(round(quot), 0), qmax)  # Python round: ties to even
+                    k = gi * 64 + j
+                    got = code_from_bitstring(int(got_codes[r, k // (32 // bits)]), bits, k % (32 // bits))
+                    assert got == want, (bits, r, k, quot)
+
+
+def pin_near_tie_gap(O):
+    """The near-tie screen is the smallest gap between adjacent values among
+    the k + 1 largest logits (descending order), ties giving 0."""
+    # top-5 of (9, 7, 5, 3, 3 - 2^-7, -4): gaps 2, 2, 2, 2^-7
+    assert O.top5_min_gap(np.array([3.0, 9.0, -4.0, 5.0, 3.0 - 2.0**-7, 7.0]), 4) == 2.0**-7
+    # a small gap just outside the k + 1 largest does not count
+    assert O.top5_min_gap(np.array([10.0, 8.0, 6.0, 4.0, 2.0, 2.0 - 2.0**-10]), 4) == 2.0
+    # an exact tie among the largest
+    assert O.top5_min_gap(np.array([1.0, 5.0, 5.0, 0.0, -1.0]), 4) == 0.0
+    # k = 1 looks at the two largest only
+    assert O.top5_min_gap(np.array([0.0, 4.0, 3.5, 3.4]), 1) == 0.5
+    # against a plain sort on random vectors
+    rng = np.random.default_rng(24)
+    for _ in range(50):
+        v = rng.standard_normal(40)
+        k = int(rng.integers(1, 8))
+        top = sorted(v.tolist(), reverse=True)[: k + 1]
+        assert O.top5_min_gap(v, k) == min(a - b for a, b in zip(top, top[1:]))
+
+
 def pin_rms_norm(O):
     """RMS normalisation against closed forms (eps = 0 unless stated)."""
     one = np.full(8, 0x3F80, dtype=np.uint16)  # bf16 1.0
@@ -549,4 +670,5 @@ def pin_delta_rule(O):
 
 ALL_PINS = [pin_expert_size, pin_packing_golden, pin_fma_identity_exact, pin_constant_codes,
             pin_one_hot, pin_permutation_expert, pin_dense_bruteforce, pin_activations,
-            pin_routing, pin_layer, pin_quantizer, pin_rms_norm, pin_delta_rule]
+            pin_routing, pin_layer, pin_quantizer, pin_rms_norm, pin_delta_rule, pin_bf16_rne,
+            pin_quantizer_ties, pin_near_tie_gap]

@@ -78,6 +78,25 @@ def test_matches_the_rule_on_random_routing(n_slots, K, layers, experts):
     assert len(set(m.od.values())) == len(m.od) <= n_slots
 
 
+def test_matches_the_rule_at_scale():
+    """Many slots, layers and evictions: the directory's fixed-size index
+    (probe runs, entries removed from the middle of a run) keeps agreeing
+    with the plain model."""
+    n_slots, K, layers, experts = 1000, 4, 40, 512
+    rng = np.random.default_rng(77)
+    pop = 1.0 / np.arange(1, experts + 1) ** 0.9
+    pop /= pop.sum()
+    c, m = F.ExpertCache(n_slots), ModelLRU(n_slots)
+    for step in range(6000):
+        layer = step % layers
+        idx = rng.choice(experts, size=K, replace=False, p=pop)
+        got_s, got_m = c.lookup(layer, idx)
+        want_s, want_m = m.lookup(layer, idx)
+        assert got_s.tolist() == want_s and got_m.tolist() == want_m, step
+    assert m.evictions > 10000
+    assert c.stats() == {"hits": m.hits, "misses": m.misses, "evictions": m.evictions}
+
+
 def test_inclusion_more_slots_never_hit_less():
     rng = np.random.default_rng(5)
     seq = [(s % 4, rng.choice(64, size=4, replace=False)) for s in range(600)]

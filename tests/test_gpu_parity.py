@@ -84,6 +84,32 @@ def test_quantize_bit_exact(F, hidden, inter, bits):
     assert np.array_equal(blob.cpu().numpy(), want)
 
 
+@pytest.mark.parametrize("bits", [4, 2])
+def test_quantize_exact_half_quotients(F, bits):
+    """Groups whose fp32 quotient is an exact half only after the fp32
+    subtraction rounds (the hand-worked fixture of the oracle's pins): the
+    device quantiser gives the fixture's codes, bit for bit."""
+    from tests import oracle_pins as P
+    (grp,) = [g for g in P.load_quantizer_ties() if g[0] == bits]
+    row = np.array(grp[2], dtype=np.uint32).view(np.float32)
+    H, I = 128, 64
+    wg = S.dense_matrix(4, 1, I, H)
+    wu = S.dense_matrix(4, 2, I, H)
+    wd = S.dense_matrix(4, 3, H, I)
+    wg[5, 64:128] = row  # gate row 5, group 1
+    wd[7, 0:64] = row    # down row 7, group 0
+    blob = F.quantize_expert(*(torch.from_numpy(m).to(dev()) for m in (wg, wu, wd)), bits)
+    want = O.quantize_expert(wg, wu, wd, bits)
+    got = blob.cpu().numpy()
+    assert np.array_equal(got, want)
+    parts = O.split_blob(got, H, I, bits)
+    for name, r, g in (("gate", 5, 1), ("down", 7, 0)):
+        codes, sb = parts[name]
+        assert int(sb[r, g]) == grp[1]
+        q = O.unpack_codes(codes, bits)[r, g * 64:(g + 1) * 64]
+        assert q.tolist() == grp[3]
+
+
 # ---------------------------------------------------------------------------
 # Router
 # ---------------------------------------------------------------------------
@@ -412,6 +438,8 @@ def run_grouped_case(F, SG, shape, T, seed=31, layer=0, with_shared=True, with_s
         assert gi[k].tolist() == r["idx"].tolist(), f"token {k}"
         C.assert_close(gw[k], r["w"], f"token {k} w", max_abs=1e-6, rel_l2=1e-6)
         C.assert_close(got[k], r["out"], f"{shape.name} T={T} token {k}")
+        # the layer's own contribution, undiluted by the O(1) residual
+        C.assert_close(got[k] - res[k], r["out"] - res[k], f"{shape.name} T={T} token {k} (out - residual)")
     return L, x, res, got
 
 

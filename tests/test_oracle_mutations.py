@@ -177,6 +177,50 @@ def _delta_variant(order):
     return fn
 
 
+def _bf16_truncate(f):
+    u = np.ascontiguousarray(f, dtype=np.float32).view(np.uint32)
+    return (u >> np.uint32(16)).astype(np.uint16)
+
+
+def _bf16_half_up(f):
+    u = np.ascontiguousarray(f, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return ((u + np.uint64(0x8000)) >> np.uint64(16)).astype(np.uint16)
+
+
+def _quantize_variant(kind):
+    """The stated quantiser with one slip: an fp64 quotient, or halves rounded up."""
+    def fn(w, bits):
+        w = np.ascontiguousarray(w, dtype=np.float32)
+        n, kdim = w.shape
+        g = w.reshape(n, kdim // 64, 64)
+        mn, mx = g.min(-1), g.max(-1)
+        s32 = (mx - mn).astype(np.float32) / np.float32((1 << bits) - 1)
+        sbits = O.f32_to_bf16_bits(s32)
+        bbits = O.f32_to_bf16_bits(mn)
+        s_f = (sbits.astype(np.uint32) << 16).view(np.float32)
+        b_f = (bbits.astype(np.uint32) << 16).view(np.float32)
+        safe = np.where(s_f == 0, np.float32(1), s_f)
+        if kind == "fp64_quotient":
+            ratio = (g.astype(np.float64) - b_f[..., None].astype(np.float64)) / safe[..., None].astype(np.float64)
+            q = np.rint(ratio)
+        else:  # half_up
+            ratio = ((g - b_f[..., None]).astype(np.float32) / safe[..., None]).astype(np.float32)
+            q = np.floor(ratio + np.float32(0.5))
+        q = np.clip(q, 0, (1 << bits) - 1)
+        q = np.where((s_f == 0)[..., None], 0, q).astype(np.uint32)
+        return O.pack_codes(q.reshape(n, kdim), bits), sbits.astype(np.uint32) | (bbits.astype(np.uint32) << 16)
+    return fn
+
+
+def _gap_never_near(logits, k=4):
+    return np.inf
+
+
+def _gap_top_k_only(logits, k=4):
+    s = np.sort(np.asarray(logits, dtype=np.float64))[::-1][:k]
+    return float(np.min(s[:-1] - s[1:])) if s.size > 1 else np.inf
+
+
 ORIG_ROUTE = O.route
 ORIG_LAYER = O.layer_decode
 ORIG_QUANT = O.quantize_matrix
@@ -208,6 +252,12 @@ MUTANTS = {
     "delta_no_beta": ("delta_update", _delta_variant("no_beta")),
     "delta_transposed_outer": ("delta_update", _delta_variant("transposed_outer")),
     "delta_readout_before_update": ("delta_update", _delta_variant("readout_before_update")),
+    "bf16_truncation": ("f32_to_bf16_bits", _bf16_truncate),
+    "bf16_round_half_up": ("f32_to_bf16_bits", _bf16_half_up),
+    "quantizer_fp64_quotient": ("quantize_matrix", _quantize_variant("fp64_quotient")),
+    "quantizer_round_half_up": ("quantize_matrix", _quantize_variant("half_up")),
+    "near_tie_gap_never_near": ("top5_min_gap", _gap_never_near),
+    "near_tie_gap_top_k_only": ("top5_min_gap", _gap_top_k_only),
 }
 
 

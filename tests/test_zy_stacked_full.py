@@ -111,5 +111,7 @@ def test_stacked_40_layers_64_steps(F):
             continue  # the selection may legitimately differ from the oracle's
         r = C.oracle_layer(SEED, l, shape, x, x, norm_w=norms[l], norm_eps=EPS)
         C.assert_close(outs[step, l], r["out"], f"stacked layer {l} step {step}")
+        # the residual is the layer input: check the layer's own contribution too
+        C.assert_close(outs[step, l] - x, r["out"] - x, f"stacked layer {l} step {step} (out - residual)")
     del layers, ws
     torch.cuda.empty_cache()

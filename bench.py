@@ -106,7 +106,7 @@ def peaks():
 
 # Device sources the single-token layer kernel is compiled from (its DRAM
 # traffic depends on nothing else).
-LAYER_KERNEL_SOURCES = ("common.cuh", "dequant.cuh", "layer_kernel.cuh")
+LAYER_KERNEL_SOURCES = ("common.cuh", "dequant.cuh", "routing.cuh", "decode_kernel.cuh")
 
 
 def source_hash() -> str:
@@ -447,6 +447,57 @@ def run_fmoe(args, cfg, rank, world, local_rank):
     lat_us = [1000.0 * a.elapsed_time(b) for a, b in lat]
     del flush
 
+    # The expert path alone: the same decodes with the routing given (the
+    # selected experts' blobs, weights and gate passed in; no router rows, no
+    # top-K), through fmoe_experts_decode, from graphs of GSTEPS calls.
+    expert_path = None
+    if LPS == 1 and TT == 1:
+        routes = []
+        idx = torch.empty(1, k, dtype=torch.int32, device=dev)
+        wk = torch.empty(1, k, dtype=torch.float32, device=dev)
+        for j in range(NL * 4):
+            layers[j % NL].decode(xs[j % POOL], rs[j % POOL], out=out[j % POOL], idx_out=idx, w_out=wk,
+                                  ws=ws[j % NL])
+            routes.append((idx.cpu().numpy()[0].tolist(), wk.cpu().numpy()[0].tolist()))
+        stride = layers[0].experts.stride(0)
+
+        def expert_step(j):
+            l = j % NL
+            ix, wv = routes[j % len(routes)]
+            base = layers[l].experts.data_ptr()
+            F.experts_decode(layers[l], [base + e * stride for e in ix], wv, 0.5, xs[j % POOL], rs[j % POOL],
+                             out=out[j % POOL], ws=ws[l])
+
+        def capture_e(first, n):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for j in range(first, first + n):
+                    expert_step(j)
+            return g
+
+        for j in range(3):
+            expert_step(j)
+        ge = capture_e(0, GSTEPS)
+        ge.replay()
+        torch.cuda.synchronize()
+        reps = max(1, K // GSTEPS)
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(reps):
+            ge.replay()
+        c1.record(stream)
+        torch.cuda.synchronize()
+        ep_us = 1000.0 * c0.elapsed_time(c1) / (reps * GSTEPS)
+        ab_e = algorithmic_bytes(cfg)
+        ep_bytes = ab_e["experts"] + ab_e["vectors"]
+        pk, _ = peaks()
+        expert_path = {"us_per_decode": ep_us, "decodes_per_s": 1e6 / ep_us,
+                       "bytes_per_decode": ep_bytes, "gbs": ep_bytes / (ep_us * 1e-6) / 1e9,
+                       "frac_of_hbm": ep_bytes / (ep_us * 1e-6) / 1e9 / pk,
+                       "note": "fmoe_experts_decode: the routed and shared experts' gate/up, SwiGLU, down and "
+                               "the combine with the routing given (no router GEMV or top-K), same rotation"}
+        del ge
+
     # End to end through the same call with host buffers: pinned host -> device
     # copy of x and residual, decode, device -> host copy of out, every step.
     xh = torch.from_numpy(S.token_x(SEED + rank, 0, 1, POOL * TT, h).reshape(shape)).pin_memory()
@@ -521,7 +572,7 @@ def run_fmoe(args, cfg, rank, world, local_rank):
             "expert_frac_of_hbm": ab["experts"] / avg_launch_s / 1e9 / peak,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": profiled_traffic(args.config),
-                         "kernel": (f"layer_kernel<{cfg['bits']},{cfg['shared_bits']}>" if TT == 1 else
+                         "kernel": (f"decode_kernel<{cfg['bits']},{cfg['shared_bits']}>" if TT == 1 else
                                     "grouped decode step (router, prep, gate/up, stage, down launches)"),
                          "algorithmic_bytes_per_launch": ab["total"]},
             "layer_decodes_per_s": whole_job_rate(K, world, total_ms_max),
@@ -530,6 +581,7 @@ def run_fmoe(args, cfg, rank, world, local_rank):
                     "h2d_bytes_per_step": (2 if LPS == 1 else 1) * TT * h * 4, "d2h_bytes_per_step": TT * h * 4},
             "gpu_launches": K * (1 if TT == 1 else 5),
             **({"distinct_routed_experts_per_step": distinct} if distinct is not None else {}),
+            **({"expert_path": expert_path} if expert_path is not None else {}),
             "clocks": clk,
             "device_status": status,
         }

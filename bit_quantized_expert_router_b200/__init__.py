@@ -28,6 +28,7 @@ EXPORTED = [
     "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status", "fmoe_strerror", "fmoe_last_cuda_error",
     "fmoe_layer_decode_noalloc", "fmoe_set_wait_limit_ns", "fmoe_set_dependent_launch", "fmoe_delta_update",
     "fmoe_cache_create", "fmoe_cache_destroy", "fmoe_cache_lookup", "fmoe_cache_stats", "fmoe_cache_reset",
+    "fmoe_experts_decode",
 ]
 
 
@@ -79,6 +80,8 @@ def lib() -> ctypes.CDLL:
     L.fmoe_workspace_init.argtypes = [vp, sz, vp]
     L.fmoe_layer_decode.argtypes = [ctypes.POINTER(FmoeLayerC), vp, vp, vp, i, vp, sz, vp, vp, vp]
     L.fmoe_layer_decode_noalloc.argtypes = [ctypes.POINTER(FmoeLayerC), vp, vp, vp, i, vp, vp, vp]
+    L.fmoe_experts_decode.argtypes = [ctypes.POINTER(FmoeLayerC), ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_float),
+                                      ctypes.c_float, vp, vp, vp, vp, sz, vp]
     L.fmoe_get_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
     L.fmoe_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong)]
     L.fmoe_set_dependent_launch.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
@@ -94,7 +97,8 @@ def lib() -> ctypes.CDLL:
     L.fmoe_strerror.argtypes = [i]
     L.fmoe_strerror.restype = ctypes.c_char_p
     for name in ("fmoe_blob_offsets", "fmoe_quantize_expert", "fmoe_route", "fmoe_expert_forward",
-                 "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status", "fmoe_layer_decode_noalloc"):
+                 "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status", "fmoe_layer_decode_noalloc",
+                 "fmoe_experts_decode"):
         getattr(L, name).restype = i
     _lib = L
     return L
@@ -272,6 +276,33 @@ class Layer:
                                        ws.data_ptr(), ws.numel(), _ptr(idx_out), _ptr(w_out), _stream(stream)),
                "fmoe_layer_decode")
         return out
+
+
+def experts_decode(layer: "Layer", blobs, weights, shared_gate: float, x: torch.Tensor,
+                   residual: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                   ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The layer's expert path for one token with the routing given: blobs are
+    the top_k routed experts' device addresses (ints or uint8 tensors, e.g.
+    expert-cache slots), weights their combine weights, shared_gate the
+    shared expert's factor.  out = residual + sum_k w_k E_k(x) + g E_shared(x)."""
+    _dev_tensor(x, torch.float32, "x")
+    x1 = x.view(layer.hidden)
+    if residual is not None:
+        _dev_tensor(residual, torch.float32, "residual")
+    if out is None:
+        out = torch.empty_like(x1)
+    if ws is None:
+        ws = layer.workspace(1)
+    K = layer.top_k
+    ptrs = [b if isinstance(b, int) else b.data_ptr() for b in blobs]
+    if len(ptrs) != K or len(weights) != K:
+        raise ValueError(f"experts_decode: need {K} blobs and weights")
+    pa = (ctypes.c_void_p * K)(*ptrs)
+    wa = (ctypes.c_float * K)(*[float(w) for w in weights])
+    _check(lib().fmoe_experts_decode(ctypes.byref(layer.c), pa, wa, ctypes.c_float(float(shared_gate)),
+                                     x1.data_ptr(), _ptr(residual), out.data_ptr(), ws.data_ptr(), ws.numel(),
+                                     _stream(stream)), "fmoe_experts_decode")
+    return out
 
 
 def layer_decode_noalloc(layer: "Layer", x: torch.Tensor, residual: torch.Tensor | None = None,

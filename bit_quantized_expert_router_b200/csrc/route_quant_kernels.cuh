@@ -1,6 +1,6 @@
 // Stand-alone router (T tokens) and the offline quantiser.
 #pragma once
-#include "layer_kernel.cuh"
+#include "routing.cuh"
 
 namespace fmoe {
 

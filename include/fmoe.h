@@ -186,10 +186,38 @@ int fmoe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream_t stream);
  * fp32 rounding).  Limits: as fmoe_route and fmoe_expert_forward, plus
  * (top_k + 1) * inter <= 10240.  Errors: FMOE_EINVAL, FMOE_ENOMEM, FMOE_ECUDA.
  * Kernel-side problems (a time-limited wait that ran out) are reported by
- * fmoe_get_status(). */
+ * fmoe_get_status(); for T = 1 the kernel then also writes quiet NaN to the
+ * out rows that depend on what was missing (and -1 / NaN to idx_out_opt /
+ * w_out_opt when the routing itself was affected), so no result built on a
+ * missing value looks plausible. */
 int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual, float* out, int T,
                       void* ws, size_t ws_bytes, int32_t* idx_out_opt, float* w_out_opt,
                       fmoe_stream_t stream);
+
+/* The expert path of fmoe_layer_decode for one token with the routing given
+ * instead of computed: out = residual + sum_k w_k * E_k(x) + shared_gate *
+ * E_shared(x) ([P2] "Metal-Compute-Shader": the dequantised expert GEMVs, the
+ * fused SwiGLU and the combine with the residual and the shared expert's
+ * gate).  It serves experts that do not live in the layer's expert table:
+ * the pages read each token's K selected experts from the SSD into memory
+ * after routing ([P2] "SSD-Experten-Streaming"), and here a caller that
+ * keeps experts in host memory routes with fmoe_route, copies the misses
+ * into device slots (fmoe_cache_lookup) and decodes from the slots.
+ *   L: shapes, code widths, the shared expert and the optional input norm
+ *   (w_router, w_sgate, experts, expert_stride and n_experts are ignored;
+ *   top_k is the number of routed experts).
+ *   expert_blobs: HOST array of top_k device pointers, each a packed expert
+ *   of L's shape and routed code width, 256-byte aligned (the same blob may
+ *   appear twice).  expert_weights: HOST array of top_k combine weights (not
+ *   renormalised here).  shared_gate: the shared expert's factor (1 for an
+ *   ungated shared expert; ignored without a shared expert).
+ *   x, residual, out, ws, ws_bytes: as fmoe_layer_decode with T = 1
+ *   (ws_bytes >= fmoe_workspace_bytes(L, 1)).
+ * Errors: FMOE_EINVAL, FMOE_ENOMEM, FMOE_ECUDA; kernel-side problems as
+ * fmoe_layer_decode. */
+int fmoe_experts_decode(const fmoe_layer* L, const void* const* expert_blobs, const float* expert_weights,
+                        float shared_gate, const float* x, const float* residual, float* out, void* ws,
+                        size_t ws_bytes, fmoe_stream_t stream);
 
 /* fmoe_layer_decode without a caller-provided workspace, for callers that
  * cannot allocate device memory: code that runs where an allocator must not be
@@ -201,15 +229,16 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
  *   workspace, for single-token decodes only: T must be 1 (FMOE_EINVAL
  *   otherwise; a grouped decode's workspace is far larger than the array).
  *   Every argument is checked before anything is enqueued, so a rejected
- *   call leaves the array untouched.  The workspace comes from one fixed 32 KiB array in device
- *   memory that every GPU which loads the library keeps until the process
- *   exits; a layer whose fmoe_workspace_bytes() exceeds 32 KiB is rejected
- *   with FMOE_ENOMEM (the full-size layer of the pages, 512 experts, top-4,
- *   intermediate 1024, needs about 29 KiB).
+ *   call leaves the array untouched.  The workspace comes from one fixed
+ *   96 KiB array in device memory that every GPU which loads the library
+ *   keeps until the process exits; a layer whose fmoe_workspace_bytes()
+ *   exceeds 96 KiB is rejected with FMOE_ENOMEM (a single-token workspace is
+ *   88.5 KiB for every layer the library accepts).
  *   The first call on a device looks the array's device address up (a
  *   synchronous runtime query); make that first call before capturing a
  *   stream into a graph.  Every call clears the array's hand-off counters on
- *   `stream` before the layer kernel runs.
+ *   `stream` before the layer kernel runs (the launch epoch and the tagged
+ *   words carry over from call to call, as in any workspace).
  *   All calls on a device share the one array: calls that may overlap on the
  *   GPU (different streams without ordering between them) race and give wrong
  *   results.  Nothing is allocated or freed by this call. */

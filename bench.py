@@ -106,7 +106,7 @@ def peaks():
 
 # Device sources the single-token layer kernel is compiled from (its DRAM
 # traffic depends on nothing else).
-LAYER_KERNEL_SOURCES = ("common.cuh", "dequant.cuh", "routing.cuh", "decode_kernel.cuh")
+LAYER_KERNEL_SOURCES = ("common.cuh", "dequant.cuh", "layer_kernel.cuh")
 
 
 def source_hash() -> str:
@@ -572,7 +572,7 @@ def run_fmoe(args, cfg, rank, world, local_rank):
             "expert_frac_of_hbm": ab["experts"] / avg_launch_s / 1e9 / peak,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": profiled_traffic(args.config),
-                         "kernel": (f"decode_kernel<{cfg['bits']},{cfg['shared_bits']}>" if TT == 1 else
+                         "kernel": (f"layer_kernel<{cfg['bits']},{cfg['shared_bits']}>" if TT == 1 else
                                     "grouped decode step (router, prep, gate/up, stage, down launches)"),
                          "algorithmic_bytes_per_launch": ab["total"]},
             "layer_decodes_per_s": whole_job_rate(K, world, total_ms_max),

@@ -7,7 +7,6 @@
 #include "../../include/fmoe.h"
 #include "deltanet.cuh"
 #include "expert_cache.h"
-#include "decode_kernel.cuh"
 #include "shared_tc.cuh"
 
 using namespace fmoe;
@@ -21,12 +20,10 @@ std::atomic<unsigned long long> g_wait_limit_ns{kTimeoutNs};
 std::atomic<int> g_dependent_launch{1};
 constexpr size_t kCounterBytes = 256;
 // Every workspace starts with the counters, then the single-token decode's
-// tagged router logits and tagged activations, both sized for the largest
-// layer (so that no other use of a workspace, whatever its layer's shape,
-// ever writes these bytes).
+// tagged router logits (sized for the most experts, so that no other use of a
+// workspace, whatever its layer's shape, ever writes these bytes).
 constexpr size_t kTagBytes = (kTagWords * 8 + 255) / 256 * 256;
-constexpr size_t kActBytes = (size_t)kMaxActWords * 8;
-constexpr size_t kHeaderBytes = kCounterBytes + kTagBytes + kActBytes;
+constexpr size_t kHeaderBytes = kCounterBytes + kTagBytes;
 constexpr int kMaxNst = 4;
 
 struct DevInfo {
@@ -39,11 +36,11 @@ struct DevInfo {
   int grouped_max_smem = 0;  // dynamic shared memory left by the grouped kernels' static arrays
 };
 
-using DecodeFn = void (*)(DecodeArgs);
+using LayerFn = void (*)(LayerArgs);
 // The instantiation for (routed bits, shared bits), and its index 0..3.
-DecodeFn decode_fn(int br, int bs) {
-  if (br == 4) return bs == 4 ? decode_kernel<4, 4> : decode_kernel<4, 2>;
-  return bs == 4 ? decode_kernel<2, 4> : decode_kernel<2, 2>;
+LayerFn layer_fn(int br, int bs) {
+  if (br == 4) return bs == 4 ? layer_kernel<4, 4> : layer_kernel<4, 2>;
+  return bs == 4 ? layer_kernel<2, 4> : layer_kernel<2, 2>;
 }
 int layer_fn_index(int br, int bs) { return (br == 4 ? 0 : 2) + (bs == 4 ? 0 : 1); }
 DevInfo g_dev[64];
@@ -72,7 +69,7 @@ int dev_info(int* dev_out, DevInfo** info) {
     for (int br : {4, 2})
       for (int bs : {4, 2}) {
         cudaFuncAttributes fa;
-        if ((e = cudaFuncGetAttributes(&fa, decode_fn(br, bs))) != cudaSuccess) return cuda_fail(e);
+        if ((e = cudaFuncGetAttributes(&fa, layer_fn(br, bs))) != cudaSuccess) return cuda_fail(e);
         static_smem = std::max(static_smem, (int)fa.sharedSizeBytes);
       }
     d.max_smem = optin - static_smem;
@@ -111,57 +108,57 @@ bool shape_ok(int h, int i) {
 bool bits_ok(int b) { return b == 2 || b == 4; }
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Fill the grid-dependent fields of a decode launch (unit offsets, work-list
-// maxima and the dynamic shared-memory layout of decode_kernel) for G CTAs;
-// returns the dynamic shared memory the launch needs, or 0 if it exceeds
-// max_smem.
-size_t plan_decode(DecodeArgs& a, int G, int max_smem) {
-  const int nv = a.H / 32, P = (nv + 31) / 32;
-  const int nvi = a.I / 32, Pd = (nvi + 31) / 32;
-  const int n_sh = a.has_shared ? a.I : 0, n_ro = a.K * a.I;
-  const int n_slots = a.K + (a.has_shared ? 1 : 0);
-  // the router rows, then the shared units, then the routed units continue
-  // one round-robin over the CTAs
-  a.off_sh = a.n_router % G;
-  a.off_ro = (a.n_router + n_sh) % G;
-  a.max_units = (n_sh + G - 1) / G + (n_ro + G - 1) / G;
-  a.max_rrows = (a.n_router + G - 1) / G;
-  a.max_drows = (a.H + G - 1) / G;
-  size_t off = round_up((size_t)a.H * 4, 16);  // x, normalised in place when the layer has a norm
-  a.sm_norm = (int)off;
-  off += a.norm_w ? round_up((size_t)a.H * 2, 16) : 0;
-  a.sm_abuf = (int)off;
-  a.sm_abuf_stride = (int)round_up((size_t)a.I * 4 + (size_t)nvi * 8, 16);
-  off += 2 * (size_t)a.sm_abuf_stride;
-  a.sm_upart = (int)off;
-  off += round_up((size_t)std::max(a.max_units, 1) * P * 8, 16);
-  a.sm_ucnt = (int)off;
-  off += round_up((size_t)std::max(a.max_units, 1) * 4, 16);
-  a.sm_rpart = (int)off;
-  off += round_up((size_t)std::max(a.max_rrows, 1) * P * 4, 16);
-  a.sm_rcnt = (int)off;
-  off += round_up((size_t)std::max(a.max_rrows, 1) * 4, 16);
-  a.sm_ysp = (int)off;
-  off += round_up((size_t)std::max(n_slots, 1) * a.max_drows * Pd * 4, 16);
-  for (int r = 0; r < 2; ++r) {
-    const BlobOff o = blob_offsets(a.H, a.I, r == 0 ? a.bits_r : a.bits_s);
-    long long* d = r == 0 ? a.off_r : a.off_s;
-    d[0] = o.gc;
-    d[1] = o.gsb;
-    d[2] = o.uc;
-    d[3] = o.usb;
-    d[4] = o.dc;
-    d[5] = o.dsb;
+// Shared-memory plan of the layer kernel (see carve_smem in layer_kernel.cuh).
+struct Plan {
+  int nst, stage_bytes, nst_c, c_stage_bytes, xs4_off, xs2_off, xu_off, vec_floats, sf_floats, ys_stride;
+  size_t smem;
+};
+
+bool plan_layer(int H, int I, int K, bool has_shared, int bits_r, int bits_s, int G, int n_router, int max_smem,
+                Plan* p) {
+  const int n_slots = K + (has_shared ? 1 : 0);
+  bool use4 = false, use2 = false;
+  int stage = 0, cstage = 0;
+  auto use_bits = [&](int b) {
+    if (b == 4) use4 = true; else use2 = true;
+    const int cb = H * b / 8;
+    const int cap = ((H / 16 + 15) & ~15) + 16;
+    stage = std::max(stage, 2 * cb + 2 * cap);
+    cstage = std::max(cstage, kRC * (I * b / 8 + I / 16));
+  };
+  if (K > 0) use_bits(bits_r);
+  if (has_shared) use_bits(bits_s);
+  cstage = (int)round_up(cstage, 128);
+  stage = (int)round_up(std::max(stage, cstage), 128);
+  int off = 0;
+  p->xu_off = off;  // x, copied in by one bulk copy
+  off += H;
+  p->xs4_off = -1;
+  p->xs2_off = -1;
+  if (use4) { p->xs4_off = off; off += H; }
+  if (use2) { p->xs2_off = off; off += H; }
+  p->vec_floats = (int)round_up((size_t)std::max(off, n_slots * I), 32);
+  p->sf_floats = (int)round_up((size_t)std::max((use4 ? H / 32 : 0) + (use2 ? H / 64 : 0), n_slots * I / 32), 16);
+  const int nq = H / kRC;
+  p->ys_stride = kRC * ((nq + G - 1) / G);
+  p->stage_bytes = stage;
+  const size_t fixed = (size_t)p->vec_floats * 4 + (size_t)p->sf_floats * 8 +
+                       round_up((size_t)n_slots * p->ys_stride * 4, 16);
+  p->c_stage_bytes = cstage;
+  for (int nst = kMaxNst; nst >= 1; --nst) {
+    const size_t total = (size_t)kWarps * nst * stage + fixed + (size_t)kWarps * (nst + kMaxNstC) * 8;
+    if (total <= (size_t)max_smem) {
+      p->nst = nst;
+      p->nst_c = std::min(kMaxNstC, nst * stage / cstage);
+      p->smem = total;
+      return true;
+    }
   }
-  return off <= (size_t)max_smem ? off : 0;
+  return false;
 }
 
-// Point a decode launch at a workspace (counters, tagged logits, tagged activations).
-void set_workspace(DecodeArgs& a, void* ws) {
-  char* w8 = static_cast<char*>(ws);
-  a.bar = reinterpret_cast<unsigned*>(w8);
-  a.tlog = reinterpret_cast<unsigned long long*>(w8 + kCounterBytes);
-  a.tact = reinterpret_cast<unsigned long long*>(w8 + kCounterBytes + kTagBytes);
+size_t layer_ws_bytes(int I, int K) {
+  return kHeaderBytes + round_up((size_t)(K + 1) * I * 4, 256);
 }
 
 // Workspace of the grouped (T >= 2) decode, byte offsets (every section 256-B aligned).
@@ -340,29 +337,47 @@ int launch_grouped(const fmoe_layer* L, const float* x, const float* residual, f
   return FMOE_OK;
 }
 
-int launch_decode(const DecodeArgs& args, size_t smem, DevInfo* info, cudaStream_t s) {
-  const DecodeFn fn = decode_fn(args.bits_r, args.bits_s);
+// Fill the grid-shape-dependent fields and the blob section offsets.
+void set_offsets(LayerArgs& a, int G) {
+  const int GW = G * kWarps;
+  const int n_static = a.shared ? a.I : 0;
+  a.off_a = a.n_router % GW;
+  a.off_b = (int)(((long long)a.n_router + n_static) % GW);
+  for (int r = 0; r < 2; ++r) {
+    const BlobOff o = blob_offsets(a.H, a.I, r == 0 ? a.bits_r : a.bits_s);
+    long long* d = r == 0 ? a.off_r : a.off_s;
+    d[0] = o.gc;
+    d[1] = o.gsb;
+    d[2] = o.uc;
+    d[3] = o.usb;
+    d[4] = o.dc;
+    d[5] = o.dsb;
+  }
+}
+
+int launch_layer(const LayerArgs& args, const Plan& pl, DevInfo* info, cudaStream_t s) {
+  const LayerFn fn = layer_fn(args.bits_r, args.bits_s);
   const int fi = layer_fn_index(args.bits_r, args.bits_s);
   if (!info->layer_attr_set[fi]) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, info->max_smem);
     if (e != cudaSuccess) return cuda_fail(e);
     info->layer_attr_set[fi] = true;
   }
-  DecodeArgs a = args;
+  LayerArgs a = args;
   if (!g_dependent_launch.load(std::memory_order_relaxed)) {
     void* kargs[] = {&a};
-    cudaError_t e = cudaLaunchCooperativeKernel((const void*)fn, dim3(info->sms), dim3(kThreads), kargs, smem, s);
+    cudaError_t e = cudaLaunchCooperativeKernel((const void*)fn, dim3(info->sms), dim3(kThreads), kargs, pl.smem, s);
     return e == cudaSuccess ? FMOE_OK : cuda_fail(e);
   }
   // Programmatic dependent launch: this grid's CTAs may start while the
   // previous kernel on the stream finishes (the kernel waits for it before
   // its first dependent access).  A plain launch gives no co-residency
   // guarantee, so it is only made when one CTA fits on every SM; the grid
-  // is then resident once the previous grid has left (the grid-wide waits
-  // are bounded either way).
+  // is then resident once the previous grid has left (the grid barriers are
+  // bounded waits either way).
   if (info->layer_occupancy[fi] < 0) {
     int n = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kThreads, info->max_smem);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kThreads, pl.smem);
     if (e != cudaSuccess) return cuda_fail(e);
     info->layer_occupancy[fi] = n;
   }
@@ -370,7 +385,7 @@ int launch_decode(const DecodeArgs& args, size_t smem, DevInfo* info, cudaStream
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(info->sms);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -384,7 +399,7 @@ int launch_decode(const DecodeArgs& args, size_t smem, DevInfo* info, cudaStream
 // Fixed scratch for fmoe_layer_decode_noalloc: callers that cannot allocate
 // device memory themselves get the decode's workspace from this file-scope
 // array, which every GPU that loads the library keeps until the process exits.
-constexpr size_t kNoallocScratchBytes = 96 << 10;
+constexpr size_t kNoallocScratchBytes = 32 << 10;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
 // Device address of g_noalloc_scratch per device, looked up once per device
@@ -480,7 +495,7 @@ int fmoe_route(const uint16_t* w_router, const uint16_t* w_sgate, const float* x
 
 size_t fmoe_expert_workspace_bytes(int hidden, int inter) {
   if (!shape_ok(hidden, inter)) return 0;
-  return kHeaderBytes;
+  return kHeaderBytes + round_up((size_t)inter * 4, 256);
 }
 
 int fmoe_expert_forward(const void* blob, int hidden, int inter, int bits, const float* x, float* y,
@@ -493,27 +508,44 @@ int fmoe_expert_forward(const void* blob, int hidden, int inter, int bits, const
   DevInfo* info;
   if (int rc = dev_info(&dev, &info)) return rc;
   if (int rc = check_stream(stream, dev)) return rc;
-  DecodeArgs a;
+  Plan pl;
+  if (!plan_layer(hidden, inter, 0, true, bits, bits, info->sms, 0, info->max_smem, &pl)) return FMOE_EINVAL;
+  LayerArgs a;
   std::memset(&a, 0, sizeof(a));
   a.shared = static_cast<const char*>(blob);
-  a.has_shared = 1;
   a.x = x;
   a.out = y;
+  char* w8 = static_cast<char*>(ws);
+  a.bar = reinterpret_cast<unsigned*>(w8);
+  a.act = reinterpret_cast<float*>(w8 + kHeaderBytes);
   a.H = hidden;
   a.I = inter;
+  a.E = 0;
+  a.K = 0;
   a.bits_r = bits;
   a.bits_s = bits;
+  a.n_router = 0;
+  a.n_slots = 1;
+  a.nst = pl.nst;
+  a.stage_bytes = pl.stage_bytes;
+  a.xs4_off = pl.xs4_off;
+  a.xs2_off = pl.xs2_off;
+  a.xu_off = pl.xu_off;
+  a.vec_floats = pl.vec_floats;
+  a.sf_floats = pl.sf_floats;
+  a.ys_stride = pl.ys_stride;
+  a.nst_c = pl.nst_c;
+  a.c_stage_bytes = pl.c_stage_bytes;
   a.timeout_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
-  set_workspace(a, ws);
-  const size_t smem = plan_decode(a, info->sms, info->max_smem);
-  if (!smem) return FMOE_EINVAL;
-  return launch_decode(a, smem, info, reinterpret_cast<cudaStream_t>(stream));
+  set_offsets(a, info->sms);
+  return launch_layer(a, pl, info, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t fmoe_workspace_bytes(const fmoe_layer* L, int T) {
   if (!L || T < 1 || T > FMOE_MAX_TOKENS) return 0;
-  if (T == 1) return kHeaderBytes;
-  return grouped_layout(L->n_experts, L->hidden, L->inter, L->top_k, T).total;
+  const size_t single = layer_ws_bytes(L->inter, L->top_k);
+  if (T == 1) return single;
+  return std::max(single, grouped_layout(L->n_experts, L->hidden, L->inter, L->top_k, T).total);
 }
 
 int fmoe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream_t stream) {
@@ -535,8 +567,7 @@ int check_layer_args(const fmoe_layer* L, const float* x, const float* residual,
   if (!routed_given && (!L->w_router || !L->experts)) return FMOE_EINVAL;
   const int H = L->hidden, I = L->inter, E = L->n_experts, K = L->top_k;
   if (!shape_ok(H, I) || !bits_ok(L->bits) || (L->shared && !bits_ok(L->shared_bits)) ||
-      L->group != FMOE_GROUP || K < 1 || K > FMOE_MAX_TOPK || T < 1 || T > FMOE_MAX_TOKENS ||
-      (K + 1) * I > kMaxActWords)
+      L->group != FMOE_GROUP || K < 1 || K > FMOE_MAX_TOPK || T < 1 || T > FMOE_MAX_TOKENS || (K + 1) * I > 10240)
     return FMOE_EINVAL;
   if (!routed_given) {
     if (E < 1 || E > FMOE_MAX_EXPERTS || K > E) return FMOE_EINVAL;
@@ -559,33 +590,53 @@ int device_for(fmoe_stream_t stream, int* dev_out, DevInfo** info_out) {
   return check_stream(stream, *dev_out);
 }
 
-// The single-token decode launch of a checked layer call (routing computed
-// from the layer's router, or given).
-DecodeArgs layer_args(const fmoe_layer* L, const float* x, const float* residual, float* out, void* ws) {
-  DecodeArgs a;
-  std::memset(&a, 0, sizeof(a));
+
+// The single-token kernel's arguments for a checked layer call; with
+// `routed_given` there are no router rows (the routing comes from the
+// caller).  Returns false if the layer does not fit the kernel's plan.
+bool layer_args(const fmoe_layer* L, void* ws, DevInfo* info, bool routed_given, LayerArgs* out_a, Plan* pl) {
+  const int H = L->hidden, I = L->inter, E = L->n_experts, K = L->top_k;
   const bool has_shared = L->shared != nullptr;
-  a.w_router = L->w_router;
-  a.w_sgate = L->w_sgate;
+  const int n_router = routed_given ? 0 : E + (L->w_sgate ? 1 : 0);
+  if (!plan_layer(H, I, K, has_shared, L->bits, has_shared ? L->shared_bits : L->bits, info->sms, n_router,
+                  info->max_smem, pl))
+    return false;
+  LayerArgs& a = *out_a;
+  std::memset(&a, 0, sizeof(a));
+  a.w_router = routed_given ? nullptr : L->w_router;
+  a.w_sgate = routed_given ? nullptr : L->w_sgate;
   a.experts = static_cast<const char*>(L->experts);
   a.expert_stride = L->expert_stride;
   a.shared = static_cast<const char*>(L->shared);
-  a.has_shared = has_shared ? 1 : 0;
-  a.x = x;
-  a.residual = residual;
-  a.out = out;
-  a.norm_w = L->norm_weight;
-  a.norm_eps = L->norm_eps;
-  a.H = L->hidden;
-  a.I = L->inter;
-  a.E = L->n_experts;
-  a.K = L->top_k;
+  char* w8 = static_cast<char*>(ws);
+  a.bar = reinterpret_cast<unsigned*>(w8);
+  a.tlog = reinterpret_cast<unsigned long long*>(w8 + kCounterBytes);
+  a.act = reinterpret_cast<float*>(w8 + kHeaderBytes);
+  a.H = H;
+  a.I = I;
+  a.E = routed_given ? 0 : E;
+  a.K = K;
   a.bits_r = L->bits;
   a.bits_s = has_shared ? L->shared_bits : L->bits;
-  a.n_router = L->n_experts + (L->w_sgate ? 1 : 0);
+  a.n_router = n_router;
+  a.n_slots = K + (has_shared ? 1 : 0);
+  a.nst = pl->nst;
+  a.stage_bytes = pl->stage_bytes;
+  a.xs4_off = pl->xs4_off;
+  a.xs2_off = pl->xs2_off;
+  a.xu_off = pl->xu_off;
+  a.vec_floats = pl->vec_floats;
+  a.sf_floats = pl->sf_floats;
+  a.ys_stride = pl->ys_stride;
+  a.nst_c = pl->nst_c;
+  a.c_stage_bytes = pl->c_stage_bytes;
   a.timeout_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
-  set_workspace(a, ws);
-  return a;
+  a.norm_w = L->norm_weight;
+  a.norm_eps = L->norm_eps;
+  // A router warp's row (2H bytes) fits in its ring: copy it there at entry.
+  a.router_smem = (long long)pl->nst * pl->stage_bytes >= 2LL * H ? 1 : 0;
+  set_offsets(a, info->sms);
+  return true;
 }
 
 }  // namespace
@@ -601,14 +652,19 @@ int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual
   int dev;
   DevInfo* info;
   if (int rc = device_for(stream, &dev, &info)) return rc;
+  if (L->n_experts + 1 > (kWarps / 2) * info->sms) return FMOE_EINVAL;  // router rows must leave staging warps
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (T > 1) return launch_grouped(L, x, residual, out, T, ws, idx_out_opt, w_out_opt, info, s);
-  DecodeArgs a = layer_args(L, x, residual, out, ws);
+  LayerArgs a;
+  Plan pl;
+  if (!layer_args(L, ws, info, false, &a, &pl)) return FMOE_EINVAL;
+  a.x = x;
+  a.residual = residual;
+  a.out = out;
   a.idx_out = idx_out_opt;
   a.w_out = w_out_opt;
-  const size_t smem = plan_decode(a, info->sms, info->max_smem);
-  if (!smem) return FMOE_EINVAL;
-  return launch_decode(a, smem, info, s);
+  a.sg_out = nullptr;
+  return launch_layer(a, pl, info, s);
 }
 
 int fmoe_experts_decode(const fmoe_layer* L, const void* const* expert_blobs, const float* expert_weights,
@@ -622,20 +678,19 @@ int fmoe_experts_decode(const fmoe_layer* L, const void* const* expert_blobs, co
   int dev;
   DevInfo* info;
   if (int rc = device_for(stream, &dev, &info)) return rc;
-  DecodeArgs a = layer_args(L, x, residual, out, ws);
-  a.w_router = nullptr;
-  a.w_sgate = nullptr;
-  a.n_router = 0;
-  a.E = 0;
+  LayerArgs a;
+  Plan pl;
+  if (!layer_args(L, ws, info, true, &a, &pl)) return FMOE_EINVAL;
   a.fixed_route = 1;
   for (int k = 0; k < L->top_k; ++k) {
     a.fixed_blob[k] = static_cast<const char*>(expert_blobs[k]);
     a.fixed_w[k] = expert_weights[k];
   }
   a.fixed_sg = shared_gate;
-  const size_t smem = plan_decode(a, info->sms, info->max_smem);
-  if (!smem) return FMOE_EINVAL;
-  return launch_decode(a, smem, info, reinterpret_cast<cudaStream_t>(stream));
+  a.x = x;
+  a.residual = residual;
+  a.out = out;
+  return launch_layer(a, pl, info, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int fmoe_layer_decode_noalloc(const fmoe_layer* L, const float* x, const float* residual, float* out, int T,
@@ -651,14 +706,13 @@ int fmoe_layer_decode_noalloc(const fmoe_layer* L, const float* x, const float* 
   int dev = 0;
   DevInfo* info = nullptr;
   if (int rc = device_for(stream, &dev, &info)) return rc;
+  if (L->n_experts + 1 > (kWarps / 2) * info->sms) return FMOE_EINVAL;  // router rows must leave staging warps
   void* ws = nullptr;
   if (int rc = noalloc_scratch(dev, &ws)) return rc;
-  // The scratch keeps whatever the previous call left.  The launch epoch and
-  // the tagged words must carry over (a word left by an earlier call carries
-  // an earlier epoch's tag, never the next one's), so only the counters that
-  // must start at zero are cleared; the rest is written before it is read.
-  if (cudaError_t e = cudaMemsetAsync(static_cast<char*>(ws) + 4, 0, kCounterBytes - 4,
-                                      reinterpret_cast<cudaStream_t>(stream)))
+  // The scratch keeps whatever the previous call left: clear the counters and
+  // the tagged logits (epoch 0, no word tagged), as a fresh workspace has them;
+  // the rest is written before it is read.
+  if (cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes, reinterpret_cast<cudaStream_t>(stream)))
     return cuda_fail(e);
   return fmoe_layer_decode(L, x, residual, out, T, ws, kNoallocScratchBytes, idx_out_opt, w_out_opt, stream);
 }

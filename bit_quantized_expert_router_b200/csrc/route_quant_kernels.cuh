@@ -1,6 +1,6 @@
 // Stand-alone router (T tokens) and the offline quantiser.
 #pragma once
-#include "routing.cuh"
+#include "layer_kernel.cuh"
 
 namespace fmoe {
 

@@ -187,8 +187,9 @@ int fmoe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream_t stream);
  * (top_k + 1) * inter <= 10240.  Errors: FMOE_EINVAL, FMOE_ENOMEM, FMOE_ECUDA.
  * Kernel-side problems (a time-limited wait that ran out) are reported by
  * fmoe_get_status(); for T = 1 the kernel then also writes quiet NaN to the
- * out rows that depend on what was missing (and -1 / NaN to idx_out_opt /
- * w_out_opt when the routing itself was affected), so no result built on a
+ * out rows of every CTA whose wait ran out, hands NaN on to the rest through
+ * any value it still publishes, and writes -1 / NaN to idx_out_opt /
+ * w_out_opt when the routing itself was affected, so no result built on a
  * missing value looks plausible. */
 int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual, float* out, int T,
                       void* ws, size_t ws_bytes, int32_t* idx_out_opt, float* w_out_opt,
@@ -230,15 +231,14 @@ int fmoe_experts_decode(const fmoe_layer* L, const void* const* expert_blobs, co
  *   otherwise; a grouped decode's workspace is far larger than the array).
  *   Every argument is checked before anything is enqueued, so a rejected
  *   call leaves the array untouched.  The workspace comes from one fixed
- *   96 KiB array in device memory that every GPU which loads the library
+ *   32 KiB array in device memory that every GPU which loads the library
  *   keeps until the process exits; a layer whose fmoe_workspace_bytes()
- *   exceeds 96 KiB is rejected with FMOE_ENOMEM (a single-token workspace is
- *   88.5 KiB for every layer the library accepts).
+ *   exceeds 32 KiB is rejected with FMOE_ENOMEM (the full-size layer of the
+ *   pages, 512 experts, top-4, intermediate 1024, needs about 29 KiB).
  *   The first call on a device looks the array's device address up (a
  *   synchronous runtime query); make that first call before capturing a
- *   stream into a graph.  Every call clears the array's hand-off counters on
- *   `stream` before the layer kernel runs (the launch epoch and the tagged
- *   words carry over from call to call, as in any workspace).
+ *   stream into a graph.  Every call clears the array's hand-off counters and
+ *   tagged words on `stream` before the layer kernel runs.
  *   All calls on a device share the one array: calls that may overlap on the
  *   GPU (different streams without ordering between them) race and give wrong
  *   results.  Nothing is allocated or freed by this call. */

@@ -1,16 +1,14 @@
 """Failure detection on the GPU without a fault: a time-limited wait that runs out.
 
-The single-token decode's CTAs hand router logits and activations to one
-another as words tagged with the launch's number, derived from the launch
-epoch kept in the caller's workspace.  Here the epoch is left at a value that
-is not a valid epoch (as if the workspace had not been zeroed), so no tagged
-word can ever match, with a short wait limit.  Every wait for a tagged word
-must run out, the kernel must end on its own, report through the status word
-and write NaN (never plausible numbers) to every output that depended on the
-missing words, the context must stay usable, and the next launch on the same
-workspace must be correct again (the kernel's last CTA restarts the epoch and
-clears the tagged words on its way out).  Both launch modes (programmatic
-dependent and cooperative) are covered.
+The layer kernel's CTAs hand off through counters in the caller's workspace.
+Here the activation hand-off counter is left at a value no launch can bring
+to its target (as if the workspace had not been zeroed), with a short wait
+limit.  Every wait on it must run out, the kernel must end on its own and
+report through the status word, the context must stay usable, and the next
+launch on the same workspace must be correct again (the kernel's last CTA
+resets the counter on its way out).  A CTA whose wait ran out writes NaN to its
+output rows, so the result of the starved launch is not plausible numbers.
+Both launch modes (programmatic dependent and cooperative) are covered.
 """
 import numpy as np
 import pytest
@@ -46,15 +44,15 @@ def test_wait_limit_bounds(F):
 
 
 @pytest.mark.parametrize("dependent", [True, False], ids=["dependent_launch", "cooperative_launch"])
-def test_unmatchable_tags_time_out_and_recover(F, dependent):
+def test_unreachable_counter_times_out_and_recovers(F, dependent):
     prev_mode = F.set_dependent_launch(dependent)
     try:
-        unmatchable_tags_case(F)
+        unreachable_counter_case(F)
     finally:
         F.set_dependent_launch(prev_mode)
 
 
-def unmatchable_tags_case(F):
+def unreachable_counter_case(F):
     import synth.gpu as SG
     shape, seed, layer = C.TINY, 21, 0
     dev = torch.device("cuda:0")
@@ -68,24 +66,21 @@ def unmatchable_tags_case(F):
     xd, rd = torch.from_numpy(x).to(dev), torch.from_numpy(res).to(dev)
     ws = L.workspace(1)
     assert F.get_status() == 0
-    L.decode(xd, rd, ws=ws)  # a normal launch first: the tagged words hold real values
-    assert F.get_status() == 0
 
     prev = F.set_wait_limit_ns(20_000_000)  # 20 ms
     try:
         counters = ws[:12].view(torch.int32)
-        counters[0:1].fill_(-1024)  # launch epoch 0xFFFFFC00: not a valid epoch, no tag can match
-        idx = torch.zeros(1, shape.top_k, dtype=torch.int32, device=dev)
-        w = torch.zeros(1, shape.top_k, dtype=torch.float32, device=dev)
-        out = L.decode(xd, rd, ws=ws, idx_out=idx, w_out=w)
+        epoch = int(counters[0])
+        counters[1:2].fill_(-1024)  # hand-off counter 0xFFFFFC00: above any grid size, never "reached"
+        out = L.decode(xd, rd, ws=ws)
         bits = F.get_status()  # synchronises: the launch ended on its own
         assert bits & STATUS_GRID_BARRIER_TIMEOUT, f"status bits {bits:#x}"
         assert F.get_status() == 0  # read-and-clear
-        # nothing plausible came out: every row depended on the routing
+        # every CTA waited in vain at the hand-off: every output row is NaN
         assert torch.isnan(out).all()
-        assert (idx == -1).all() and torch.isnan(w).all()
-        # the last CTA restarted the epoch and put the ticket back to zero
-        assert counters.cpu().tolist() == [0, 0, 0]
+        # the last CTA advanced the launch epoch and put both hand-off
+        # counters back to zero
+        assert counters.cpu().tolist() == [epoch + 1, 0, 0]
     finally:
         F.set_wait_limit_ns(prev)
 

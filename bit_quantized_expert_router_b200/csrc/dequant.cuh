@@ -96,15 +96,60 @@ __device__ __forceinline__ int code_bitpos_t(int n) {
 // back in memory (the routed experts' activations) can be staged in one call;
 // input s's vectors are then columns s*(n_s/CPV) ... of one [F4][NV] array.
 //
+// Stage float4 j of vector v (q = v*F4 + j < total, else only the shuffles)
+// from its four inputs `val`.  The F4 lanes of a vector are consecutive lanes
+// of one warp and combine their max and sum with shuffles, so the whole warp
+// calls this together.
+template <int BITS>
+__device__ __forceinline__ void stage_f4(float4 val, int q, int total, int NV, float4* xs, float2* sf) {
+  constexpr int CPV = 128 / BITS, CPW = 32 / BITS, F4 = CPV / 4;
+  const bool on = q < total;
+  const int v = q / F4, j = q % F4;
+  float mx = fmaxf(fmaxf(fabsf(val.x), fabsf(val.y)), fmaxf(fabsf(val.z), fabsf(val.w)));
+  float sum = (val.x + val.y) + (val.z + val.w);
+#pragma unroll
+  for (int o = 1; o < F4; o <<= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  }
+  // max|x| * 2^S < 2^125; S in [22, 249] keeps 2^(149 - S) and 2^(S - p) finite.
+  int S = 109;
+  if (mx > 0.f) {
+    int e;
+    frexpf(mx, &e);  // mx < 2^e
+    S = 125 - e;
+    S = S < 22 ? 22 : (S > 249 ? 249 : S);
+  }
+  const float* in = &val.x;
+  float4 o;
+  float* out = &o.x;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    int e = S - code_bitpos_t<BITS>((4 * j + c) % CPW);  // in [0, 249]
+    float t = in[c];
+    if (e > 126) {
+      t *= pow2f(126);
+      e -= 126;
+    }
+    out[c] = t * pow2f(e);
+  }
+  if (on) {
+    xs[j * NV + v] = o;
+    if (j == 0) {
+      const int fe = 149 - S;  // in [-100, 127]
+      sf[v] = make_float2(sum, pow2f(fe));
+    }
+  }
+}
+
 // All threads of the CTA call this; thread q of each pass handles float4 j of
-// vector v (q = v*F4 + j), and the F4 lanes of a vector combine their max and
-// sum with shuffles, so a pass costs one 16-byte load per thread.  With
+// vector v (q = v*F4 + j), so a pass costs one 16-byte load per thread.  With
 // kGlobal, src is global memory read through L2 (other CTAs of the grid may
 // have written it); otherwise src is this CTA's shared memory.
 template <int BITS, bool kGlobal>
 __device__ inline void stage_inputs(const float* __restrict__ src, int n, float4* xs, float2* sf, int tid,
                                     int nthreads) {
-  constexpr int CPV = 128 / BITS, CPW = 32 / BITS, F4 = CPV / 4;
+  constexpr int CPV = 128 / BITS, F4 = CPV / 4;
   // passes whose loads are all issued before any is used: global sources need
   // the loads in flight together; from shared memory one pass at a time keeps
   // this code (run once per launch, from a cold instruction cache) short
@@ -124,46 +169,72 @@ __device__ inline void stage_inputs(const float* __restrict__ src, int n, float4
     for (int b = 0; b < kBatch; ++b) {
       const int base = base0 + b * nthreads;
       if (base >= total) break;  // warp-uniform
-      const int q = base + lane;
-      const bool on = q < total;
-      const int v = q / F4, j = q % F4;
-      float mx = fmaxf(fmaxf(fabsf(val[b].x), fabsf(val[b].y)), fmaxf(fabsf(val[b].z), fabsf(val[b].w)));
-      float sum = (val[b].x + val[b].y) + (val[b].z + val[b].w);
-#pragma unroll
-      for (int o = 1; o < F4; o <<= 1) {
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      }
-      // max|x| * 2^S < 2^125; S in [22, 249] keeps 2^(149 - S) and 2^(S - p) finite.
-      int S = 109;
-      if (mx > 0.f) {
-        int e;
-        frexpf(mx, &e);  // mx < 2^e
-        S = 125 - e;
-        S = S < 22 ? 22 : (S > 249 ? 249 : S);
-      }
-      const float* in = &val[b].x;
-      float4 o;
-      float* out = &o.x;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        int e = S - code_bitpos_t<BITS>((4 * j + c) % CPW);  // in [0, 249]
-        float t = in[c];
-        if (e > 126) {
-          t *= pow2f(126);
-          e -= 126;
-        }
-        out[c] = t * pow2f(e);
-      }
-      if (on) {
-        xs[j * NV + v] = o;
-        if (j == 0) {
-          const int fe = 149 - S;  // in [-100, 127]
-          sf[v] = make_float2(sum, pow2f(fe));
-        }
-      }
+      stage_f4<BITS>(val[b], base + lane, total, NV, xs, sf);
     }
   }
+}
+
+// stage_inputs from a tagged source written by other CTAs of the running
+// grid: word k is {tag (high 32 bits), fp32 bits of input k}.  Each thread
+// issues the loads of all its float4s (two 16-byte loads each) at once, then
+// re-reads those whose four words do not all carry `tag` yet, until they do
+// or limit_ns has passed since the first re-read; then the warp stages them.
+// Returns false if the wait ran out (the values staged are then whatever was
+// read; the caller poisons its results).
+template <int BITS>
+__device__ inline bool stage_tagged(const unsigned long long* src, int n, float4* xs, float2* sf, int tid,
+                                    int nthreads, unsigned tag, uint64_t limit_ns) {
+  constexpr int CPV = 128 / BITS, F4 = CPV / 4;
+  constexpr int kBatch = 4;
+  const int NV = n / CPV, total = NV * F4;
+  const int lane = tid & 31;
+  bool ok = true;
+  for (int base0 = tid - lane; base0 < total; base0 += kBatch * nthreads) {
+    unsigned long long w[kBatch][4];
+    unsigned pend = 0;
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int q = base0 + b * nthreads + lane;
+      w[b][0] = w[b][1] = w[b][2] = w[b][3] = 0ull;
+      if (q < total) {
+        ld_relaxed_gpu_v2u64(src + 4 * (long long)q, w[b][0], w[b][1]);
+        ld_relaxed_gpu_v2u64(src + 4 * (long long)q + 2, w[b][2], w[b][3]);
+        pend |= 1u << b;
+      }
+    }
+    uint64_t t0 = 0;
+    while (true) {
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b)
+        if ((pend >> b & 1u) && (unsigned)(w[b][0] >> 32) == tag && (unsigned)(w[b][1] >> 32) == tag &&
+            (unsigned)(w[b][2] >> 32) == tag && (unsigned)(w[b][3] >> 32) == tag)
+          pend &= ~(1u << b);
+      if (!pend) break;
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > limit_ns) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b)
+        if (pend >> b & 1u) {
+          const long long q = base0 + b * nthreads + lane;
+          ld_relaxed_gpu_v2u64(src + 4 * q, w[b][0], w[b][1]);
+          ld_relaxed_gpu_v2u64(src + 4 * q + 2, w[b][2], w[b][3]);
+        }
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int base = base0 + b * nthreads;
+      if (base >= total) break;  // warp-uniform
+      const float4 val = make_float4(__uint_as_float((unsigned)w[b][0]), __uint_as_float((unsigned)w[b][1]),
+                                     __uint_as_float((unsigned)w[b][2]), __uint_as_float((unsigned)w[b][3]));
+      stage_f4<BITS>(val, base + lane, total, NV, xs, sf);
+    }
+  }
+  return ok;
 }
 
 }  // namespace fmoe

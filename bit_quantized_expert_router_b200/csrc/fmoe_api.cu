@@ -20,10 +20,12 @@ std::atomic<unsigned long long> g_wait_limit_ns{kTimeoutNs};
 std::atomic<int> g_dependent_launch{1};
 constexpr size_t kCounterBytes = 256;
 // Every workspace starts with the counters, then the single-token decode's
-// tagged router logits (sized for the most experts, so that no other use of a
-// workspace, whatever its layer's shape, ever writes these bytes).
+// tagged router logits and tagged activations (each sized for the largest
+// layer, so that no other use of a workspace, whatever its layer's shape,
+// ever writes these bytes).
 constexpr size_t kTagBytes = (kTagWords * 8 + 255) / 256 * 256;
-constexpr size_t kHeaderBytes = kCounterBytes + kTagBytes;
+constexpr size_t kActTagBytes = (kActWords * 8 + 255) / 256 * 256;
+constexpr size_t kHeaderBytes = kCounterBytes + kTagBytes + kActTagBytes;
 constexpr int kMaxNst = 4;
 
 struct DevInfo {
@@ -157,9 +159,8 @@ bool plan_layer(int H, int I, int K, bool has_shared, int bits_r, int bits_s, in
   return false;
 }
 
-size_t layer_ws_bytes(int I, int K) {
-  return kHeaderBytes + round_up((size_t)(K + 1) * I * 4, 256);
-}
+// The single-token decode uses the header alone ((K + 1) * I <= kActWords).
+size_t layer_ws_bytes() { return kHeaderBytes; }
 
 // Workspace of the grouped (T >= 2) decode, byte offsets (every section 256-B aligned).
 struct GroupedLayout {
@@ -399,7 +400,8 @@ int launch_layer(const LayerArgs& args, const Plan& pl, DevInfo* info, cudaStrea
 // Fixed scratch for fmoe_layer_decode_noalloc: callers that cannot allocate
 // device memory themselves get the decode's workspace from this file-scope
 // array, which every GPU that loads the library keeps until the process exits.
-constexpr size_t kNoallocScratchBytes = 32 << 10;
+constexpr size_t kNoallocScratchBytes = 128 << 10;
+static_assert(kHeaderBytes <= kNoallocScratchBytes, "the scratch holds a single-token workspace");
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
 // Device address of g_noalloc_scratch per device, looked up once per device
@@ -495,7 +497,7 @@ int fmoe_route(const uint16_t* w_router, const uint16_t* w_sgate, const float* x
 
 size_t fmoe_expert_workspace_bytes(int hidden, int inter) {
   if (!shape_ok(hidden, inter)) return 0;
-  return kHeaderBytes + round_up((size_t)inter * 4, 256);
+  return kHeaderBytes;  // inter <= 8192 < kActWords tagged activations
 }
 
 int fmoe_expert_forward(const void* blob, int hidden, int inter, int bits, const float* x, float* y,
@@ -517,7 +519,7 @@ int fmoe_expert_forward(const void* blob, int hidden, int inter, int bits, const
   a.out = y;
   char* w8 = static_cast<char*>(ws);
   a.bar = reinterpret_cast<unsigned*>(w8);
-  a.act = reinterpret_cast<float*>(w8 + kHeaderBytes);
+  a.tact = reinterpret_cast<unsigned long long*>(w8 + kCounterBytes + kTagBytes);
   a.H = hidden;
   a.I = inter;
   a.E = 0;
@@ -543,7 +545,7 @@ int fmoe_expert_forward(const void* blob, int hidden, int inter, int bits, const
 
 size_t fmoe_workspace_bytes(const fmoe_layer* L, int T) {
   if (!L || T < 1 || T > FMOE_MAX_TOKENS) return 0;
-  const size_t single = layer_ws_bytes(L->inter, L->top_k);
+  const size_t single = layer_ws_bytes();
   if (T == 1) return single;
   return std::max(single, grouped_layout(L->n_experts, L->hidden, L->inter, L->top_k, T).total);
 }
@@ -567,7 +569,7 @@ int check_layer_args(const fmoe_layer* L, const float* x, const float* residual,
   if (!routed_given && (!L->w_router || !L->experts)) return FMOE_EINVAL;
   const int H = L->hidden, I = L->inter, E = L->n_experts, K = L->top_k;
   if (!shape_ok(H, I) || !bits_ok(L->bits) || (L->shared && !bits_ok(L->shared_bits)) ||
-      L->group != FMOE_GROUP || K < 1 || K > FMOE_MAX_TOPK || T < 1 || T > FMOE_MAX_TOKENS || (K + 1) * I > 10240)
+      L->group != FMOE_GROUP || K < 1 || K > FMOE_MAX_TOPK || T < 1 || T > FMOE_MAX_TOKENS || (K + 1) * I > kActWords)
     return FMOE_EINVAL;
   if (!routed_given) {
     if (E < 1 || E > FMOE_MAX_EXPERTS || K > E) return FMOE_EINVAL;
@@ -611,7 +613,7 @@ bool layer_args(const fmoe_layer* L, void* ws, DevInfo* info, bool routed_given,
   char* w8 = static_cast<char*>(ws);
   a.bar = reinterpret_cast<unsigned*>(w8);
   a.tlog = reinterpret_cast<unsigned long long*>(w8 + kCounterBytes);
-  a.act = reinterpret_cast<float*>(w8 + kHeaderBytes);
+  a.tact = reinterpret_cast<unsigned long long*>(w8 + kCounterBytes + kTagBytes);
   a.H = H;
   a.I = I;
   a.E = routed_given ? 0 : E;
@@ -710,8 +712,7 @@ int fmoe_layer_decode_noalloc(const fmoe_layer* L, const float* x, const float* 
   void* ws = nullptr;
   if (int rc = noalloc_scratch(dev, &ws)) return rc;
   // The scratch keeps whatever the previous call left: clear the counters and
-  // the tagged logits (epoch 0, no word tagged), as a fresh workspace has them;
-  // the rest is written before it is read.
+  // the tagged words (epoch 0, no word tagged), as a fresh workspace has them.
   if (cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes, reinterpret_cast<cudaStream_t>(stream)))
     return cuda_fail(e);
   return fmoe_layer_decode(L, x, residual, out, T, ws, kNoallocScratchBytes, idx_out_opt, w_out_opt, stream);

@@ -18,13 +18,15 @@
 //      block of output rows, then the combine (need all SwiGLU activations).
 // Units of phases A and B are dealt round-robin over all warps of the grid.
 //
-// Hand-offs.  Each router warp publishes its logit as one 64-bit word tagged
-// with this launch's number (the workspace's epoch + 1).  Every CTA then
-// takes the routing decision with all of its warps: each lane polls the words
-// of its warp's slice of the logits until they carry the tag, each warp
-// selects the top K of its slice, and the candidates are ranked (CTA
-// barriers between the steps).  "All activations written" is a counter that
-// every CTA bumps once and polls once.  Every wait is time-limited: on expiry
+// Hand-offs.  Each router warp publishes its logit, and each gate/up warp its
+// SwiGLU activation, as one 64-bit word tagged with this launch's number (the
+// workspace's epoch + 1); a reader polls a word until it carries the tag, so
+// no grid-wide barrier is needed.  Every CTA takes the routing decision with
+// all of its warps: each lane polls the words of its warp's slice of the
+// logits, each warp selects the top K of its slice, and the candidates are
+// ranked (CTA barriers between the steps).  For the down projections every
+// CTA polls and stages all activations in one pass.  Every wait is
+// time-limited: on expiry
 // the kernel sets a status bit and carries on instead of hanging, and the CTA
 // that waited in vain writes and hands on NaN from then on (its activations,
 // its output rows, the routing outputs), so no result built on a missing value
@@ -50,6 +52,12 @@ constexpr int kMaxTopK = 8;
 constexpr int kMaxSlots = kMaxTopK + 1;
 constexpr int kMaxExperts = 1024; // top-K is one warp with 32 logits per lane
 constexpr int kTagWords = kMaxExperts + 1;  // tagged-logit words of a workspace (routers and the gate)
+constexpr int kActWords = 10240;            // tagged-activation words of a workspace ((K + 1) * I at most)
+// Launch epochs run 0 .. kEpochWrap; a launch's tag is its epoch + 1, so tags
+// run 1 .. kEpochWrap + 1 and 0 never matches.  An epoch with the top bit set
+// is a workspace that was not zeroed (or was overwritten): its launch tags
+// nothing (tag 0), so every tagged wait runs out instead of accepting words.
+constexpr unsigned kEpochWrap = 0x7FFFFFFEu;
 constexpr int kMaxNstC = 8;       // most down-item stages a warp keeps in flight
 
 // Optional phase trace (compile with -DFMOE_TRACE_BUILD): thread 0 of every CTA
@@ -79,8 +87,9 @@ struct LayerArgs {
   // workspace [n_router] tagged logits: word e = (tag << 32) | bits of logit e,
   // tag = this launch's epoch + 1 (written by the router warps only)
   unsigned long long* tlog;
-  float* act;                // workspace [n_slots][I]
-  unsigned* bar;             // workspace: [0] launch epoch, [1] CTAs past gate/up, [2] done ticket
+  // workspace [n_slots][I] tagged activations, same word format as tlog
+  unsigned long long* tact;
+  unsigned* bar;             // workspace: [0] launch epoch, [1] unused (zero), [2] done ticket
   int* idx_out;              // optional [K]
   float* w_out;              // optional [K]
   float* sg_out;             // optional [1]
@@ -182,6 +191,7 @@ struct CtaShared {
   unsigned long long param_touch;  // see the kernel's set-up
   float red[kWarps];               // per-warp partial sums (input norm)
   int c_prefetch;          // warps past their gate/up work (the first prefetches down rows)
+  int last;                // this CTA took the last done ticket
   int idx[kMaxTopK];
   float w[kMaxTopK];
   float sg;
@@ -512,31 +522,21 @@ __device__ __forceinline__ void wait_failed(CtaShared& cs, unsigned status_bit) 
   cs.poison = 1;
 }
 
-// Wait until *ctr >= target (one thread), for at most limit_ns.
-__device__ __forceinline__ bool counter_reached(unsigned v, unsigned target) {
-  // Counts never exceed the grid size; a value with the top bit set is a
-  // workspace that was not zeroed (or was overwritten), never "reached", so
-  // the wait runs out and reports instead of passing on garbage.
-  return v >= target && v < 0x80000000u;
-}
-
-__device__ __forceinline__ bool grid_wait(const unsigned* ctr, unsigned target, uint64_t limit_ns) {
-  if (counter_reached(ld_acquire_gpu(ctr), target)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (!counter_reached(ld_acquire_gpu(ctr), target)) {
-    FMOE_SPIN(1);
-    __nanosleep(64);
-    if (globaltimer_ns() - t0 > limit_ns) return false;
-  }
-  return true;
+// The tag of this launch: the workspace's epoch + 1, or 0 (never matched) for
+// an epoch that no launch leaves (a workspace that was not zeroed).
+__device__ __forceinline__ unsigned launch_tag(const unsigned* epoch) {
+  const unsigned e = ld_relaxed_gpu(epoch);
+  return e <= kEpochWrap ? e + 1u : 0u;
 }
 
 // Top-K rounds over keys held by a warp, NK per lane, each with its expert
 // index (empty slots: key 0): per round the largest key wins and, among equal
-// keys, the lowest expert index; only the winner lane rescans.  Lane kk < k
-// ends with the kk-th winner's key and index.
+// keys, the lowest expert index; only the winner lane rescans.  A winner's key
+// and index are both dropped, so a slice with fewer than k nonzero keys (a
+// logit that never arrived) still yields distinct entries.  Lane kk < k ends
+// with the kk-th winner's key and index.
 template <int NK>
-__device__ __forceinline__ void warp_select(uint32_t (&key)[NK], const uint32_t (&eix)[NK], int k, int lane,
+__device__ __forceinline__ void warp_select(uint32_t (&key)[NK], uint32_t (&eix)[NK], int k, int lane,
                                             uint32_t& out_key, uint32_t& out_idx) {
   uint32_t mk = key[0], mx = eix[0];
   int mp = 0;
@@ -549,10 +549,13 @@ __device__ __forceinline__ void warp_select(uint32_t (&key)[NK], const uint32_t 
   for (int kk = 0; kk < k; ++kk) {
     const uint32_t h = __reduce_max_sync(0xffffffffu, mk);
     const uint32_t e = __reduce_min_sync(0xffffffffu, mk == h ? mx : 0xffffffffu);
-    if (mk == h && mx == e) {  // the winner drops its key and rescans
+    if (mk == h && mx == e) {  // the winner drops its entry and rescans
 #pragma unroll
       for (int i = 0; i < NK; ++i)
-        if (i == mp) key[i] = 0u;
+        if (i == mp) {
+          key[i] = 0u;
+          eix[i] = 0xffffffffu;
+        }
       mk = key[0];
       mx = eix[0];
       mp = 0;
@@ -574,29 +577,30 @@ __device__ __forceinline__ void warp_select(uint32_t (&key)[NK], const uint32_t 
 // selects the top k of its slice into the candidates.  The tag check replaces
 // a grid barrier: a word is this launch's logit or it is not read.
 template <int NKW>
-__device__ __forceinline__ float slice_topk(const LayerArgs& a, unsigned tag, int warp, int lane, CtaShared& cs) {
+__device__ __forceinline__ float slice_topk(const unsigned long long* tlog, int E, int K, bool gated,
+                                            uint64_t timeout_ns, unsigned tag, int warp, int lane, CtaShared& cs) {
   uint32_t key[NKW], eix[NKW];
   unsigned pend = 0;
 #pragma unroll
   for (int i = 0; i < NKW; ++i) {
     const int e = (warp * NKW + i) * 32 + lane;
     key[i] = 0u;
-    eix[i] = e < a.E ? (uint32_t)e : 0xffffffffu;
-    if (e < a.E) pend |= 1u << i;
+    eix[i] = e < E ? (uint32_t)e : 0xffffffffu;
+    if (e < E) pend |= 1u << i;
   }
-  if (warp == 0 && lane == 0 && a.n_router > a.E) pend |= 1u << NKW;
+  if (warp == 0 && lane == 0 && gated) pend |= 1u << NKW;
   float gate_logit = 0.f;
   uint64_t t0 = 0;
   while (pend) {
     unsigned long long v[NKW + 1];
 #pragma unroll
     for (int i = 0; i <= NKW; ++i) {
-      const int e = i < NKW ? (warp * NKW + i) * 32 + lane : a.E;
-      v[i] = (pend >> i & 1u) ? ld_relaxed_gpu_u64(a.tlog + e) : 0ull;
+      const int e = i < NKW ? (warp * NKW + i) * 32 + lane : E;
+      v[i] = (pend >> i & 1u) ? ld_relaxed_gpu_u64(tlog + e) : 0ull;
     }
 #pragma unroll
     for (int i = 0; i <= NKW; ++i) {
-      if ((pend >> i & 1u) && (unsigned)(v[i] >> 32) == tag) {
+      if ((pend >> i & 1u) && tag != 0u && (unsigned)(v[i] >> 32) == tag) {
         const float l = __uint_as_float((unsigned)v[i]);
         if (i < NKW) key[i] = order_bits(l); else gate_logit = l;
         pend &= ~(1u << i);
@@ -607,17 +611,17 @@ __device__ __forceinline__ float slice_topk(const LayerArgs& a, unsigned tag, in
     const uint64_t now = globaltimer_ns();
     if (t0 == 0) {
       t0 = now;
-    } else if (now - t0 > a.timeout_ns) {
+    } else if (now - t0 > timeout_ns) {
       wait_failed(cs, kStatusGridBarrierTimeout);
       break;
     }
   }
   FMOE_TRACE_WARP(17);
   uint32_t hk, hi;
-  warp_select<NKW>(key, eix, a.K, lane, hk, hi);
-  if (lane < a.K) {
-    cs.cand_key[warp * a.K + lane] = hk;
-    cs.cand_idx[warp * a.K + lane] = hi;
+  warp_select<NKW>(key, eix, K, lane, hk, hi);
+  if (lane < K) {
+    cs.cand_key[warp * K + lane] = hk;
+    cs.cand_idx[warp * K + lane] = hi;
   }
   return gate_logit;
 }
@@ -628,21 +632,34 @@ __device__ __forceinline__ float slice_topk(const LayerArgs& a, unsigned tag, in
 //   published; after a CTA barrier the candidates are ranked in parallel (the
 //   global top K is among them, ties included); after a second barrier warp 0
 //   computes the weights, and a third publishes the decision to the CTA.
-__device__ __noinline__ void cta_routing(const LayerArgs& a, CtaShared& cs, int warp, int lane) {
-  const unsigned tag = ld_relaxed_gpu(&a.bar[0]) + 1u;
+// Kept out of line (measured faster than inlined into the kernel).
+__device__ __noinline__ void cta_routing(const LayerArgs& a, CtaShared& cs, int warp, int lane, unsigned tag) {
+  // Every parameter used here, read once up front: the loads overlap the wait
+  // for the logits, and no later store can make the compiler read them again.
+  const unsigned long long* const tlog = a.tlog;
+  const int E = a.E, K = a.K;
+  const bool gated = a.n_router > a.E;
+  const uint64_t timeout_ns = a.timeout_ns;
+  const char* const experts = a.experts;
+  const long long expert_stride = a.expert_stride;
+  int* const idx_out = a.idx_out;
+  float* const w_out = a.w_out;
+  float* const sg_out = a.sg_out;
   float gate_logit;
-  if (a.E <= kWarps * 32)
-    gate_logit = slice_topk<1>(a, tag, warp, lane, cs);
+  if (E <= kWarps * 32)
+    gate_logit = slice_topk<1>(tlog, E, K, gated, timeout_ns, tag, warp, lane, cs);
   else
-    gate_logit = slice_topk<kMaxExperts / (kWarps * 32)>(a, tag, warp, lane, cs);
+    gate_logit = slice_topk<kMaxExperts / (kWarps * 32)>(tlog, E, K, gated, timeout_ns, tag, warp, lane, cs);
   FMOE_TRACE_WARP(14);
   __syncthreads();
+  FMOE_TRACE_WARP(9);
   // Stage 2: each candidate's rank among the nc candidates (larger key first,
-  // then lower expert index) is counted by P threads over nc_pad / P
-  // candidates each and summed over those P lanes; the K candidates of rank
-  // < K are the decision, written in rank order.
+  // then lower expert index, then lower candidate position, a total order, so
+  // the ranks are 0 .. nc-1 even among empty candidates) is counted by P
+  // threads over nc_pad / P candidates each and summed over those P lanes;
+  // the K candidates of rank < K are the decision, written in rank order.
   {
-    const int nc = kWarps * a.K;
+    const int nc = kWarps * K;
     int nc_pad = kWarps;
     while (nc_pad < nc) nc_pad <<= 1;  // 16 .. 128
     // P threads per candidate (consecutive lanes, a power of two dividing 32),
@@ -654,36 +671,38 @@ __device__ __noinline__ void cta_routing(const LayerArgs& a, CtaShared& cs, int 
     int rank = 0;
     for (int j = part * per; j < part * per + per && j < nc; ++j) {
       const uint32_t k2 = cs.cand_key[j], i2 = cs.cand_idx[j];
-      rank += (k2 > ck) || (k2 == ck && i2 < ci);
+      rank += (k2 > ck) || (k2 == ck && (i2 < ci || (i2 == ci && j < c)));
     }
     for (int o = P >> 1; o > 0; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
-    if (part == 0 && c < nc && rank < a.K) {
+    if (part == 0 && c < nc && rank < K) {
       cs.sel_key[rank] = ck;
-      cs.idx[rank] = ci < (uint32_t)a.E ? (int)ci : 0;  // (always in range)
+      cs.idx[rank] = ci < (uint32_t)E ? (int)ci : 0;  // (always in range)
     }
   }
+  FMOE_TRACE_WARP(23);
   __syncthreads();
   if (warp == 0) {
     // w_k = exp(l_k - l_0) / sum_j exp(l_j - l_0): softmax restricted to the
     // selected experts, equal to softmax-then-renormalise.
-    const float val = lane < a.K ? from_order_bits(cs.sel_key[lane]) : 0.f;
+    const float val = lane < K ? from_order_bits(cs.sel_key[lane]) : 0.f;
     const float l0 = __shfl_sync(0xffffffffu, val, 0);
-    const float ex = (lane < a.K) ? expf(val - l0) : 0.f;
+    const float ex = (lane < K) ? expf(val - l0) : 0.f;
     const float ssum = warp_sum(ex);
     const bool poisoned = cs.poison != 0;  // (a logit never arrived: no plausible routing)
-    if (lane < a.K) {
+    if (lane < K) {
       const int idx = cs.idx[lane];
       const float w = poisoned ? quiet_nan() : ex / ssum;
       cs.w[lane] = w;
-      cs.blob[lane] = a.experts + (long long)idx * a.expert_stride;
+      cs.blob[lane] = experts + (long long)idx * expert_stride;
       if (blockIdx.x == 0) {
-        if (a.idx_out) a.idx_out[lane] = poisoned ? -1 : idx;
-        if (a.w_out) a.w_out[lane] = w;
+        if (idx_out) idx_out[lane] = poisoned ? -1 : idx;
+        if (w_out) w_out[lane] = w;
       }
     }
     if (lane == 0) {
-      cs.sg = poisoned ? quiet_nan() : (a.w_sgate ? sigmoidf_(gate_logit) : 1.0f);
-      if (blockIdx.x == 0 && a.sg_out) *a.sg_out = cs.sg;
+      const float sg = poisoned ? quiet_nan() : (gated ? sigmoidf_(gate_logit) : 1.0f);
+      cs.sg = sg;
+      if (blockIdx.x == 0 && sg_out) *sg_out = sg;
     }
     FMOE_TRACE_WARP(10);
   }
@@ -736,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     {
       unsigned long long t = (uintptr_t)a.w_router ^ (uintptr_t)a.w_sgate ^ (uintptr_t)a.experts ^
                              (unsigned long long)a.expert_stride ^ (uintptr_t)a.shared ^ (uintptr_t)a.x ^
-                             (uintptr_t)a.residual ^ (uintptr_t)a.out ^ (uintptr_t)a.tlog ^ (uintptr_t)a.act ^
+                             (uintptr_t)a.residual ^ (uintptr_t)a.out ^ (uintptr_t)a.tlog ^ (uintptr_t)a.tact ^
                              (uintptr_t)a.bar ^ (uintptr_t)a.idx_out ^ (uintptr_t)a.w_out ^ (uintptr_t)a.sg_out ^
                              a.timeout_ns;
       t += (unsigned)(a.H ^ a.I ^ a.E ^ a.K ^ a.bits_r ^ a.bits_s ^ a.n_router ^ a.n_slots ^ a.off_a ^ a.off_b ^
@@ -785,9 +804,9 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   grid_dep_wait();
   FMOE_TRACE(24);
   if (tid == 0) bulk_g2s(sm.vec + a.xu_off, a.x, a.H * 4, &cs.x_bar);
-  // The tag of this launch's router logits (the epoch the previous launch on
-  // this workspace left, plus one).
-  const unsigned ptag = (router_warp && lane == 0) ? ld_relaxed_gpu(&a.bar[0]) + 1u : 0u;
+  // The tag of this launch's published words (the epoch the previous launch
+  // on this workspace left, plus one).
+  const unsigned tag = launch_tag(&a.bar[0]);
 
   // x and the router rows are the critical path to the routing decision; the
   // shared expert's gate/up rows are requested once x is staged (by a router
@@ -828,7 +847,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
         l = router_dot(router_row_ptr(e), xu, a.H, lane);
       }
       if (lane == 0) {
-        st_relaxed_gpu_u64(a.tlog + e, ((unsigned long long)ptag << 32) | __float_as_uint(l));
+        st_relaxed_gpu_u64(a.tlog + e, ((unsigned long long)tag << 32) | __float_as_uint(l));
         FMOE_TRACE_WARP(22);
       }
     }
@@ -867,7 +886,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   }
   issued = __shfl_sync(0xffffffffu, issued, 0);
   // Every warp of the CTA takes part in the routing decision (layer mode).
-  if (layer_mode) cta_routing(a, cs, warp, lane);
+  if (layer_mode) cta_routing(a, cs, warp, lane, tag);
   if (!mbar_wait_bounded(&cs.staged_bar, 0, a.timeout_ns) && lane == 0) wait_failed(cs, kStatusCtaWaitTimeout);
   FMOE_TRACE(1);
 
@@ -907,7 +926,10 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
       pair_dot<BR>(stage, a.H, sbo_g, sbo_u, BR == 4 ? xs4 : xs2, BR == 4 ? sf4 : sf2, lane, g, u);
     else
       pair_dot<BS>(stage, a.H, sbo_g, sbo_u, BS == 4 ? xs4 : xs2, BS == 4 ? sf4 : sf2, lane, g, u);
-    if (lane == 0) a.act[(long long)slot * a.I + row] = cs.poison ? quiet_nan() : g * sigmoidf_(g) * u;
+    if (lane == 0) {
+      const float act = cs.poison ? quiet_nan() : g * sigmoidf_(g) * u;
+      st_relaxed_gpu_u64(a.tact + (long long)slot * a.I + row, ((unsigned long long)tag << 32) | __float_as_uint(act));
+    }
     __syncwarp();
   }
 
@@ -937,32 +959,30 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     }
   issued_c = __shfl_sync(0xffffffffu, issued_c, 0);
 
-  // ---- Hand-off: every activation of the grid is written --------------------
+  // ---- Hand-off: poll and stage every activation of the grid ----------------
+  // (the staged activations overwrite the staged x: every warp of the CTA is
+  // past its gate/up work first).  With one code width every slot (back to
+  // back in the workspace) is staged in one pass, as one [F4][n_slots*I/CPV]
+  // array; otherwise the K routed experts in one pass and the shared expert in
+  // a second, its own [F4][I/CPV] array at sm.vec + K * I.  Slot s's scale
+  // pairs start at sm.sf + s * I / CPV either way.
   FMOE_TRACE_WARP(4);
   __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    red_release_gpu_add(&a.bar[1], 1);
-    if (!grid_wait(&a.bar[1], G, a.timeout_ns)) wait_failed(cs, kStatusGridBarrierTimeout);
-  }
   FMOE_TRACE(5);
-  __syncthreads();
-
-  // Stage the activations.  With one code width every slot (back to back in
-  // the workspace) is staged in one pass, as one [F4][n_slots*I/CPV] array;
-  // otherwise the K routed experts in one pass and the shared expert in a
-  // second, its own [F4][I/CPV] array at sm.vec + K * I.  Slot s's scale pairs
-  // start at sm.sf + s * I / CPV either way.
   if (plan.nq > 0) {
+    bool ok = true;
     if (BR == BS) {
-      stage_inputs<BR, true>(a.act, a.n_slots * a.I, reinterpret_cast<float4*>(sm.vec), sm.sf, tid, kThreads);
+      ok = stage_tagged<BR>(a.tact, a.n_slots * a.I, reinterpret_cast<float4*>(sm.vec), sm.sf, tid, kThreads, tag,
+                            a.timeout_ns);
     } else {
       if (a.K > 0)
-        stage_inputs<BR, true>(a.act, a.K * a.I, reinterpret_cast<float4*>(sm.vec), sm.sf, tid, kThreads);
+        ok = stage_tagged<BR>(a.tact, a.K * a.I, reinterpret_cast<float4*>(sm.vec), sm.sf, tid, kThreads, tag,
+                              a.timeout_ns);
       if (a.n_slots > a.K)
-        stage_inputs<BS, true>(a.act + (long long)a.K * a.I, a.I, reinterpret_cast<float4*>(sm.vec + a.K * a.I),
-                               sm.sf + a.K * a.I * BR / 128, tid, kThreads);
+        ok &= stage_tagged<BS>(a.tact + (long long)a.K * a.I, a.I, reinterpret_cast<float4*>(sm.vec + a.K * a.I),
+                               sm.sf + a.K * a.I * BR / 128, tid, kThreads, tag, a.timeout_ns);
     }
+    if (!ok) wait_failed(cs, kStatusGridBarrierTimeout);
   }
   FMOE_TRACE(6);
   __syncthreads();
@@ -1016,20 +1036,23 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   // ---- Done: the last CTA advances the epoch and resets the counters -------
   __syncthreads();
   FMOE_TRACE(8);
-  if (tid == 0) {
-    const unsigned t = atomicAdd(&a.bar[2], 1u);
-    if (t + 1 == (unsigned)G) {
-      // Every CTA is past its last use of the epoch.  Tags run 1 .. 2^32 - 1
-      // (epoch + 1); before the epoch would reach 2^32 - 1 the tagged words are
-      // cleared (tag 0 never matches) and it restarts at 0, so no word left by
-      // an earlier launch ever carries a later launch's tag.
-      unsigned ep = ld_relaxed_gpu(&a.bar[0]) + 1u;
-      if (ep == 0xFFFFFFFFu) {
-        if (a.tlog)
-          for (int e = 0; e < kTagWords; ++e) st_relaxed_gpu_u64(a.tlog + e, 0ull);
-        ep = 0u;
-      }
-      atomicExch(&a.bar[0], ep);
+  if (tid == 0) cs.last = atomicAdd(&a.bar[2], 1u) + 1u == (unsigned)G;
+  __syncthreads();
+  if (cs.last) {
+    // Every CTA is past its last use of the epoch.  Before the epoch would
+    // pass kEpochWrap (or when it is not a valid epoch) every tagged word is
+    // cleared (tag 0 never matches) and it restarts at 0, so no word left by
+    // an earlier launch ever carries a later launch's tag.
+    const unsigned ep = ld_relaxed_gpu(&a.bar[0]);
+    const bool wrap = ep >= kEpochWrap;
+    if (wrap) {
+      if (a.tlog)
+        for (int e = tid; e < kTagWords; e += kThreads) st_relaxed_gpu_u64(a.tlog + e, 0ull);
+      for (int e = tid; e < kActWords; e += kThreads) st_relaxed_gpu_u64(a.tact + e, 0ull);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      atomicExch(&a.bar[0], wrap ? 0u : ep + 1u);
       atomicExch(&a.bar[1], 0u);
       atomicExch(&a.bar[2], 0u);
       __threadfence();

@@ -177,6 +177,10 @@ int fmoe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream_t stream);
  *   of the routing decision.
  *   ws: workspace of ws_bytes >= fmoe_workspace_bytes(L, T), zero-filled
  *   before its first use; calls sharing a workspace must be stream-ordered.
+ *   For T = 1 the workspace carries the launch epoch and the router logits
+ *   and SwiGLU activations as words tagged with it; a workspace whose epoch
+ *   is not one a launch leaves (not zero-filled) makes every wait of the next
+ *   launch run out (reported, NaN results), after which it is usable again.
  * The whole layer runs on the GPU; the routing decision never returns to the
  * host.  T = 1 runs one persistent kernel.  T >= 2 groups the tokens by
  * expert: every distinct selected expert's weights are read once per call and
@@ -231,10 +235,10 @@ int fmoe_experts_decode(const fmoe_layer* L, const void* const* expert_blobs, co
  *   otherwise; a grouped decode's workspace is far larger than the array).
  *   Every argument is checked before anything is enqueued, so a rejected
  *   call leaves the array untouched.  The workspace comes from one fixed
- *   32 KiB array in device memory that every GPU which loads the library
- *   keeps until the process exits; a layer whose fmoe_workspace_bytes()
- *   exceeds 32 KiB is rejected with FMOE_ENOMEM (the full-size layer of the
- *   pages, 512 experts, top-4, intermediate 1024, needs about 29 KiB).
+ *   128 KiB array in device memory that every GPU which loads the library
+ *   keeps until the process exits; every layer that fmoe_layer_decode
+ *   accepts fits it (a single-token workspace is 90,624 bytes whatever the
+ *   shape), and FMOE_ENOMEM would report one that did not.
  *   The first call on a device looks the array's device address up (a
  *   synchronous runtime query); make that first call before capturing a
  *   stream into a graph.  Every call clears the array's hand-off counters and

@@ -1,14 +1,16 @@
 """Failure detection on the GPU without a fault: a time-limited wait that runs out.
 
-The layer kernel's CTAs hand off through counters in the caller's workspace.
-Here the activation hand-off counter is left at a value no launch can bring
-to its target (as if the workspace had not been zeroed), with a short wait
-limit.  Every wait on it must run out, the kernel must end on its own and
-report through the status word, the context must stay usable, and the next
+The layer kernel's CTAs hand off through words in the caller's workspace
+tagged with the launch's epoch + 1.  Here the epoch is left at a value no
+launch leaves behind (top bit set, as if the workspace had not been zeroed),
+with a short wait limit: such a launch tags nothing, so every tagged wait (the
+router logits, the activations) must run out.  The kernel must end on its own
+and report through the status word, the context must stay usable, and the next
 launch on the same workspace must be correct again (the kernel's last CTA
-resets the counter on its way out).  A CTA whose wait ran out writes NaN to its
-output rows, so the result of the starved launch is not plausible numbers.
-Both launch modes (programmatic dependent and cooperative) are covered.
+restarts the epoch at 0 and clears the tagged words on its way out).  A CTA
+whose wait ran out writes NaN to its output rows, so the result of the starved
+launch is not plausible numbers.  Both launch modes (programmatic dependent and
+cooperative) are covered.
 """
 import numpy as np
 import pytest
@@ -44,15 +46,15 @@ def test_wait_limit_bounds(F):
 
 
 @pytest.mark.parametrize("dependent", [True, False], ids=["dependent_launch", "cooperative_launch"])
-def test_unreachable_counter_times_out_and_recovers(F, dependent):
+def test_invalid_epoch_times_out_and_recovers(F, dependent):
     prev_mode = F.set_dependent_launch(dependent)
     try:
-        unreachable_counter_case(F)
+        invalid_epoch_case(F)
     finally:
         F.set_dependent_launch(prev_mode)
 
 
-def unreachable_counter_case(F):
+def invalid_epoch_case(F):
     import synth.gpu as SG
     shape, seed, layer = C.TINY, 21, 0
     dev = torch.device("cuda:0")
@@ -70,17 +72,21 @@ def unreachable_counter_case(F):
     prev = F.set_wait_limit_ns(20_000_000)  # 20 ms
     try:
         counters = ws[:12].view(torch.int32)
-        epoch = int(counters[0])
-        counters[1:2].fill_(-1024)  # hand-off counter 0xFFFFFC00: above any grid size, never "reached"
+        counters[0:1].fill_(-1024)  # epoch 0xFFFFFC00: no launch leaves it, so this one tags nothing
+        tagged = ws[256:256 + (1025 * 8 + 255) // 256 * 256 + 10240 * 8]
+        tagged.fill_(0x5A)  # stale words (their tags never match either)
         out = L.decode(xd, rd, ws=ws)
         bits = F.get_status()  # synchronises: the launch ended on its own
         assert bits & STATUS_GRID_BARRIER_TIMEOUT, f"status bits {bits:#x}"
         assert F.get_status() == 0  # read-and-clear
-        # every CTA waited in vain at the hand-off: every output row is NaN
+        # every CTA waited in vain for the logits: every output row is NaN
         assert torch.isnan(out).all()
-        # the last CTA advanced the launch epoch and put both hand-off
-        # counters back to zero
-        assert counters.cpu().tolist() == [epoch + 1, 0, 0]
+        # the last CTA restarted the epoch at 0, reset the counters and
+        # cleared every tagged word
+        assert counters.cpu().tolist() == [0, 0, 0]
+        tlog_words = tagged[:1025 * 8].cpu()  # (the rest of its 256-byte block is padding, never read)
+        tact_words = tagged[(1025 * 8 + 255) // 256 * 256:].cpu()
+        assert (tlog_words == 0).all() and (tact_words == 0).all()
     finally:
         F.set_wait_limit_ns(prev)
 

@@ -363,11 +363,11 @@ def test_dependent_launch_matches_cooperative(F, SG, shape):
 
 
 def test_routing_epoch_wraps(F, SG):
-    """The router logits are published as words tagged with the workspace's
-    launch epoch + 1.  Started two launches before the epoch would reach
-    2^32 - 1, three decodes must all be right: the second clears the tagged
-    words and restarts the epoch at 0, so the third (tag 1) reads no stale
-    word."""
+    """The router logits and the activations are published as words tagged
+    with the workspace's launch epoch + 1.  Started two launches before the
+    epoch would pass 0x7FFFFFFE, three decodes must all be right: the second
+    clears the tagged words and restarts the epoch at 0, so the third (tag 1)
+    reads no stale word."""
     shape, seed = C.FULL4, 23
     L, _ = make_gpu_layer(F, SG, seed, 0, shape)
     H, K = shape.hidden, shape.top_k
@@ -376,16 +376,19 @@ def test_routing_epoch_wraps(F, SG):
     res = S.token_residual(seed, 0, 0, 3, H)
     ws = L.workspace(1)
     epoch = ws[:4].view(torch.int32)
-    epoch.fill_(-3)  # 0xFFFFFFFD
-    expect_epoch = [-2, 0, 1]  # 0xFFFFFFFE, then the wrap to 0
+    epoch.fill_(0x7FFFFFFD)
+    expect_epoch = [0x7FFFFFFE, 0, 1]  # then the wrap to 0
+    n_tagged = (1025 * 8 + 255) // 256 * 256 // 8 + 10240
     for i in range(3):
         idx = torch.empty(1, K, dtype=torch.int32, device=dev())
         out = L.decode(torch.from_numpy(xs[i]).to(dev()), torch.from_numpy(res[i]).to(dev()), idx_out=idx, ws=ws)
         assert F.get_status() == 0
         assert int(epoch.cpu()[0]) == expect_epoch[i], f"decode {i}"
+        tags = ws[256:256 + n_tagged * 8].view(torch.int64).cpu().numpy()
         if i == 1:  # the wrap cleared every tagged word
-            tags = ws[256:256 + 1025 * 8].view(torch.int64).cpu().numpy()
             assert (tags == 0).all()
+        else:  # this launch's words carry its tag
+            assert ((tags >> 32) == expect_epoch[i]).sum() == shape.n_experts + 1 + (K + 1) * shape.inter
         r = C.oracle_layer(seed, 0, shape, xs[i], res[i])
         assert idx.cpu().numpy()[0].tolist() == r["idx"].tolist(), f"decode {i}"
         C.assert_close(out.cpu().numpy()[0], r["out"], f"decode {i} across the epoch wrap")

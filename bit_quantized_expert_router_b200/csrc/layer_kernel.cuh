@@ -12,7 +12,8 @@
 // per SM and the grid is the SM count; a programmatic dependent launch by
 // default, so that its weight-only set-up overlaps the previous kernel's end,
 // or a cooperative launch).  Three phases:
-//   A  router rows and the shared expert's gate/up rows (need nothing);
+//   A  router rows (each split over several warps of its CTA) and the shared
+//      expert's gate/up rows (need nothing);
 //   B  the routed experts' gate/up rows (need the routing decision);
 //   C  the down projections of every expert over each CTA's own contiguous
 //      block of output rows, then the combine (need all SwiGLU activations).
@@ -141,11 +142,13 @@ __device__ __forceinline__ Smem carve_smem(const LayerArgs& a, char* base) {
 }
 
 // ---------------------------------------------------------------------------
-// Work assignment.  Phases A and B: unit u of a phase whose numbering starts at
-// offset `off` goes to grid-warp slot (u + off) mod GW; slot s is warp s / G of
-// CTA s mod G, so consecutive units land on consecutive CTAs.  Phase C: CTA c
-// owns output-row quads [c*nq/G, (c+1)*nq/G) and its warps take the items
-// (slot, quad) of that block round-robin.
+// Work assignment.  Router rows: CTA c takes rows c, c + G, c + 2G, ...,
+// each split into segments over several of its warps (RouterPart).  Gate/up
+// units of phases A and B: unit u of a phase whose numbering starts at offset
+// `off` goes to grid-warp slot (u + off) mod GW; slot s is warp s / G of CTA
+// s mod G, so consecutive units land on consecutive CTAs.  Phase C: CTA c owns
+// output-row quads [c*nq/G, (c+1)*nq/G) and its warps take the items (slot,
+// quad) of that block round-robin.
 // ---------------------------------------------------------------------------
 struct PhaseList {
   int first, count;
@@ -160,17 +163,39 @@ __device__ __forceinline__ PhaseList phase_list(int n_units, int off, int gslot,
 }
 
 struct WarpPlan {
-  PhaseList router, a, b;
+  PhaseList a, b;
   int q0, nq;      // this CTA's quad block
   int c_count;     // phase-C items of this warp
   int n_loads;     // ring loads: a.count + b.count + c_count
 };
 
+// This warp's router segment: the CTA's nr rows are each split into wpr
+// segments of H / wpr inputs (wpr the largest power of two with nr * wpr <=
+// kWarps and H / wpr a multiple of 8); warp w < nr * wpr takes segment w % wpr
+// of row cta + (w / wpr) * G.
+struct RouterPart {
+  int nr, wpr;   // rows of this CTA, warps per row
+  bool on;       // this warp has a segment
+  int row;       // its router row (E: the shared gate's row)
+  int seg0, n;   // its first input and length
+};
+
+__device__ __forceinline__ RouterPart router_part(int n_router, int H, int cta, int warp, int G) {
+  RouterPart r;
+  r.nr = n_router > cta ? (n_router - cta + G - 1) / G : 0;
+  r.wpr = 1;
+  while (r.nr > 0 && 2 * r.wpr * r.nr <= kWarps && (H / (2 * r.wpr)) % 8 == 0) r.wpr *= 2;
+  r.on = warp < r.nr * r.wpr;
+  r.row = cta + (warp / r.wpr) * G;
+  r.n = H / r.wpr;
+  r.seg0 = (warp % r.wpr) * r.n;
+  return r;
+}
+
 __device__ __forceinline__ WarpPlan make_plan(const LayerArgs& a, int cta, int warp, int G) {
   const int GW = G * kWarps;
   const int gslot = warp * G + cta;
   WarpPlan p;
-  p.router = phase_list(a.n_router, 0, gslot, GW);
   p.a = phase_list(a.shared != nullptr ? a.I : 0, a.off_a, gslot, GW);
   p.b = phase_list(a.K * a.I, a.off_b, gslot, GW);
   const int nq_all = a.H / kRC;  // <= 2048, so cta * nq_all fits in 32 bits
@@ -185,6 +210,7 @@ __device__ __forceinline__ WarpPlan make_plan(const LayerArgs& a, int cta, int w
 // Per-CTA shared state (static shared memory).
 struct CtaShared {
   int poison;           // a wait of this CTA ran out: what it hands on or writes is NaN
+  float rpart[kWarps];  // router segment dot products, by warp
   uint64_t x_bar;       // completes once x is in shared memory
   uint64_t staged_bar;  // completes once x is staged in the decode layouts
   uint64_t rbar[kWarps];  // router warp w's row is in its ring (router_smem)
@@ -192,13 +218,11 @@ struct CtaShared {
   float red[kWarps];               // per-warp partial sums (input norm)
   int c_prefetch;          // warps past their gate/up work (the first prefetches down rows)
   int last;                // this CTA took the last done ticket
-  int idx[kMaxTopK];
   float w[kMaxTopK];
   float sg;
   const char* blob[kMaxSlots];  // blob of each slot (routed ones once the routing is known)
   uint32_t cand_key[kWarps * kMaxTopK];  // per-warp top-K candidates (order-preserving keys)
   uint32_t cand_idx[kWarps * kMaxTopK];  // and their expert indices
-  uint32_t sel_key[kMaxTopK];            // the selected keys, in rank order
 };
 
 
@@ -629,9 +653,9 @@ __device__ __forceinline__ float slice_topk(const unsigned long long* tlog, int 
 // The routing decision of this CTA, computed by all of its warps together;
 // every warp calls this once, before it computes any unit (layer mode).
 //   Each warp takes the top K of its slice of the logits as they are
-//   published; after a CTA barrier the candidates are ranked in parallel (the
-//   global top K is among them, ties included); after a second barrier warp 0
-//   computes the weights, and a third publishes the decision to the CTA.
+//   published; after a CTA barrier warp 0 selects the top K of the candidates
+//   and computes the weights, and a second barrier publishes the decision to
+//   the CTA.
 // Kept out of line (measured faster than inlined into the kernel).
 __device__ __noinline__ void cta_routing(const LayerArgs& a, CtaShared& cs, int warp, int lane, unsigned tag) {
   // Every parameter used here, read once up front: the loads overlap the wait
@@ -653,44 +677,30 @@ __device__ __noinline__ void cta_routing(const LayerArgs& a, CtaShared& cs, int 
   FMOE_TRACE_WARP(14);
   __syncthreads();
   FMOE_TRACE_WARP(9);
-  // Stage 2: each candidate's rank among the nc candidates (larger key first,
-  // then lower expert index, then lower candidate position, a total order, so
-  // the ranks are 0 .. nc-1 even among empty candidates) is counted by P
-  // threads over nc_pad / P candidates each and summed over those P lanes;
-  // the K candidates of rank < K are the decision, written in rank order.
-  {
-    const int nc = kWarps * K;
-    int nc_pad = kWarps;
-    while (nc_pad < nc) nc_pad <<= 1;  // 16 .. 128
-    // P threads per candidate (consecutive lanes, a power of two dividing 32),
-    // each comparing against nc_pad / P >= 1 candidates
-    const int P = min(kThreads / nc_pad, nc_pad);
-    const int tid = warp * 32 + lane;
-    const int c = tid / P, part = tid - c * P, per = nc_pad / P;
-    const uint32_t ck = c < nc ? cs.cand_key[c] : 0u, ci = c < nc ? cs.cand_idx[c] : 0xffffffffu;
-    int rank = 0;
-    for (int j = part * per; j < part * per + per && j < nc; ++j) {
-      const uint32_t k2 = cs.cand_key[j], i2 = cs.cand_idx[j];
-      rank += (k2 > ck) || (k2 == ck && (i2 < ci || (i2 == ci && j < c)));
-    }
-    for (int o = P >> 1; o > 0; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
-    if (part == 0 && c < nc && rank < K) {
-      cs.sel_key[rank] = ck;
-      cs.idx[rank] = ci < (uint32_t)E ? (int)ci : 0;  // (always in range)
-    }
-  }
-  FMOE_TRACE_WARP(23);
-  __syncthreads();
   if (warp == 0) {
+    // Stage 2: warp 0 selects the top K of the kWarps * K candidates (the
+    // global top K is among them, ties included) with the same rounds, up to
+    // four candidates per lane; lane kk < K ends with the kk-th.
+    const int nc = kWarps * K;
+    uint32_t ckey[kMaxTopK * kWarps / 32], cidx[kMaxTopK * kWarps / 32];
+#pragma unroll
+    for (int i = 0; i < kMaxTopK * kWarps / 32; ++i) {
+      const int c = i * 32 + lane;
+      ckey[i] = c < nc ? cs.cand_key[c] : 0u;
+      cidx[i] = c < nc ? cs.cand_idx[c] : 0xffffffffu;
+    }
+    uint32_t hk, hi;
+    warp_select<kMaxTopK * kWarps / 32>(ckey, cidx, K, lane, hk, hi);
+    FMOE_TRACE_WARP(23);
     // w_k = exp(l_k - l_0) / sum_j exp(l_j - l_0): softmax restricted to the
     // selected experts, equal to softmax-then-renormalise.
-    const float val = lane < K ? from_order_bits(cs.sel_key[lane]) : 0.f;
+    const float val = lane < K ? from_order_bits(hk) : 0.f;
     const float l0 = __shfl_sync(0xffffffffu, val, 0);
     const float ex = (lane < K) ? expf(val - l0) : 0.f;
     const float ssum = warp_sum(ex);
     const bool poisoned = cs.poison != 0;  // (a logit never arrived: no plausible routing)
     if (lane < K) {
-      const int idx = cs.idx[lane];
+      const int idx = hi < (uint32_t)E ? (int)hi : 0;  // (always in range)
       const float w = poisoned ? quiet_nan() : ex / ssum;
       cs.w[lane] = w;
       cs.blob[lane] = experts + (long long)idx * expert_stride;
@@ -733,9 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   uint64_t* my_bars = sm.bars + warp * (a.nst + kMaxNstC);
   uint64_t* my_bars_c = my_bars + a.nst;
   const bool layer_mode = a.n_router > 0;
-  const bool router_warp = plan.router.count > 0;
-  // Router rows go to warps w with w*G + cta < n_router, i.e. the first ones.
-  const int n_router_warps = min(kWarps, max(0, (a.n_router - (int)blockIdx.x + G - 1) / G));
+  const RouterPart rp = router_part(a.n_router, a.H, blockIdx.x, warp, G);
   FMOE_TRACE(0);
   // The next layer decode on the stream may be scheduled now: its CTAs take
   // the SMs this grid's CTAs leave, and do their weight-only set-up while
@@ -746,7 +754,7 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   auto router_row_ptr = [&](int e) { return (e < a.E) ? a.w_router + (long long)e * a.H : a.w_sgate; };
   if (tid == 0) {
     mbar_init(&cs.x_bar, 1);
-    mbar_init(&cs.staged_bar, kWarps - n_router_warps);
+    mbar_init(&cs.staged_bar, kWarps);
     cs.sg = 1.0f;
     cs.c_prefetch = 0;
     cs.poison = 0;
@@ -783,16 +791,15 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     if (a.norm_w) bulk_g2s(sm.vec + (a.xs4_off >= 0 ? a.xs4_off : a.xs2_off), a.norm_w, a.H * 2, &cs.x_bar);
   }
   if (lane == 0) {
-    if (a.router_smem && plan.router.count == 1) {
-      // The router row is the first thing this warp needs after x: bring it
-      // into the warp's (still unused) ring now, alongside x.
+    if (rp.on && a.router_smem) {
+      // The router segment is the first thing this warp needs after x: bring
+      // it into the warp's (still unused) ring now, alongside x.
       mbar_init(&cs.rbar[warp], 1);
       fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&cs.rbar[warp], a.H * 2);
-      bulk_g2s(my_ring, router_row_ptr(plan.router.first), a.H * 2, &cs.rbar[warp]);
-    } else {
-      for (int j = 0; j < plan.router.count; ++j)
-        bulk_prefetch_l2(router_row_ptr(plan.router.first + j * GW), a.H * 2);
+      mbar_arrive_expect_tx(&cs.rbar[warp], rp.n * 2);
+      bulk_g2s(my_ring, router_row_ptr(rp.row) + rp.seg0, rp.n * 2, &cs.rbar[warp]);
+    } else if (rp.on) {
+      bulk_prefetch_l2(router_row_ptr(rp.row) + rp.seg0, rp.n * 2);
     }
     for (int s = 0; s < a.nst + kMaxNstC; ++s) mbar_init(&my_bars[s], 1);
     fence_proxy_async_smem();
@@ -809,8 +816,8 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   const unsigned tag = launch_tag(&a.bar[0]);
 
   // x and the router rows are the critical path to the routing decision; the
-  // shared expert's gate/up rows are requested once x is staged (by a router
-  // warp once its dot product is done).
+  // shared expert's gate/up rows are requested once the router segments are
+  // done with the rings, then every warp stages x.
   int issued = 0;
   if (!mbar_wait_bounded(&cs.x_bar, 0, a.timeout_ns) && lane == 0) wait_failed(cs, kStatusCopyTimeout);
   FMOE_TRACE_WARP(16);
@@ -833,56 +840,55 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     __syncthreads();
   }
   const float* xu = sm.vec + a.xu_off;
-  if (router_warp) {
-    // ---- Phase A, router rows: each logit published as one tagged word ------
-    for (int j = 0; j < plan.router.count; ++j) {
-      const int e = plan.router.first + j * GW;
+  if (rp.nr > 0) {  // (uniform over the CTA)
+    // ---- Phase A, router rows: segment dot products, then each row's sum
+    // (fixed order) published as one tagged word ---------------------------------
+    if (rp.on) {
       float l;
-      if (a.router_smem && plan.router.count == 1) {
+      if (a.router_smem) {
         if (!mbar_wait_bounded(&cs.rbar[warp], 0, a.timeout_ns) && lane == 0) wait_failed(cs, kStatusCopyTimeout);
         FMOE_TRACE_WARP(20);
-        l = router_dot_smem(reinterpret_cast<const uint16_t*>(my_ring), xu, a.H, lane);
-        FMOE_TRACE_WARP(21);
+        l = router_dot_smem(reinterpret_cast<const uint16_t*>(my_ring), xu + rp.seg0, rp.n, lane);
       } else {
-        l = router_dot(router_row_ptr(e), xu, a.H, lane);
+        l = router_dot(router_row_ptr(rp.row) + rp.seg0, xu + rp.seg0, rp.n, lane);
       }
-      if (lane == 0) {
-        st_relaxed_gpu_u64(a.tlog + e, ((unsigned long long)tag << 32) | __float_as_uint(l));
-        FMOE_TRACE_WARP(22);
-      }
+      FMOE_TRACE_WARP(21);
+      if (lane == 0) cs.rpart[warp] = l;
+    }
+    __syncthreads();
+    if (rp.on && warp % rp.wpr == 0 && lane == 0) {
+      float l = cs.rpart[warp];
+      for (int q = 1; q < rp.wpr; ++q) l += cs.rpart[warp + q];
+      st_relaxed_gpu_u64(a.tlog + rp.row, ((unsigned long long)tag << 32) | __float_as_uint(cs.poison ? quiet_nan() : l));
+      FMOE_TRACE_WARP(22);
     }
     FMOE_TRACE_WARP(2);
-  } else {
-    // ---- Stage x into the decode layouts (the non-router warps) --------------
-    // At once, alongside the router dot products: the staging is what keeps
-    // these warps from polling for the logits.
-    const int t0 = tid - n_router_warps * 32, nt = kThreads - n_router_warps * 32;
-    if (BR == 4 || BS == 4)
-      stage_inputs<4, false>(xu, a.H, reinterpret_cast<float4*>(sm.vec + a.xs4_off), sm.sf, t0, nt);
-    if (BR == 2 || BS == 2)
-      stage_inputs<2, false>(xu, a.H, reinterpret_cast<float4*>(sm.vec + a.xs2_off),
-                             sm.sf + (a.xs4_off >= 0 ? a.H / 32 : 0), t0, nt);
-    __syncwarp();
-    FMOE_TRACE_WARP(18);
-    if (lane == 0) mbar_arrive(&cs.staged_bar);
-    if (warp == kWarps - 1 && lane == 0 && a.shared && plan.nq > 0) {
-      // the shared expert's down rows of this CTA are known from the start
-      const BlobOff o = blob_offsets(a.H, a.I, BS);
-      const int cb = codes_row_bytes(a.I, BS), sbr = sb_row_bytes(a.I);
-      const long long r0 = (long long)plan.q0 * kRC, nr = (long long)plan.nq * kRC;
-      bulk_prefetch_l2(a.shared + o.dc + r0 * cb, (uint32_t)(nr * cb));
-      bulk_prefetch_l2(a.shared + o.dsb + r0 * sbr, (uint32_t)(nr * sbr));
-    }
   }
-  // The shared expert's gate/up loads (no routing decision needed).  A
-  // router warp's ring held its router row: its reads come before the copies.
-  __syncwarp();
+  // The shared expert's gate/up loads (no routing decision needed).  A router
+  // warp's ring held its segment: its reads come before the copies.
   if (lane == 0) {
-    if (router_warp && a.router_smem) fence_proxy_async_smem();
+    if (rp.on && a.router_smem) fence_proxy_async_smem();
     while (issued < plan.a.count && issued < a.nst) {
       issue_load(a, plan, cs, issued, warp, my_ring + (size_t)issued * a.stage_bytes, &my_bars[issued], GW);
       ++issued;
     }
+  }
+  // ---- Stage x into the decode layouts (every warp) ---------------------------
+  if (BR == 4 || BS == 4)
+    stage_inputs<4, false>(xu, a.H, reinterpret_cast<float4*>(sm.vec + a.xs4_off), sm.sf, tid, kThreads);
+  if (BR == 2 || BS == 2)
+    stage_inputs<2, false>(xu, a.H, reinterpret_cast<float4*>(sm.vec + a.xs2_off),
+                           sm.sf + (a.xs4_off >= 0 ? a.H / 32 : 0), tid, kThreads);
+  __syncwarp();
+  FMOE_TRACE_WARP(18);
+  if (lane == 0) mbar_arrive(&cs.staged_bar);
+  if (warp == kWarps - 1 && lane == 0 && a.shared && plan.nq > 0) {
+    // the shared expert's down rows of this CTA are known from the start
+    const BlobOff o = blob_offsets(a.H, a.I, BS);
+    const int cb = codes_row_bytes(a.I, BS), sbr = sb_row_bytes(a.I);
+    const long long r0 = (long long)plan.q0 * kRC, nr = (long long)plan.nq * kRC;
+    bulk_prefetch_l2(a.shared + o.dc + r0 * cb, (uint32_t)(nr * cb));
+    bulk_prefetch_l2(a.shared + o.dsb + r0 * sbr, (uint32_t)(nr * sbr));
   }
   issued = __shfl_sync(0xffffffffu, issued, 0);
   // Every warp of the CTA takes part in the routing decision (layer mode).

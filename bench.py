@@ -65,6 +65,13 @@ CONFIGS = {
     # 64-head x 128x128 gated delta-rule state (45 such layers in rotation).
     "deltanet": dict(workload="gated_delta_h64_dk128_dv128", kind="deltanet", heads=64, dk=128, dv=128,
                      layers=45),
+    # Routed experts streamed from pinned host memory (the pages' SSD expert
+    # streaming): 2 full-size 4-bit layers whose 1024 routed experts (7.25 GB)
+    # stay on the host, device slot caches of several sizes, one token of an
+    # autoregressive stream (rho 0.9) decoded through both layers per step.
+    "stream": dict(workload="stream_2x_full_h4096_i1024_e512_k4_shared_4bit_host_experts", kind="stream",
+                   hidden=4096, inter=1024, experts=512, top_k=4, bits=4, shared_bits=4, stream_layers=2,
+                   slot_counts=[128, 512, 1024], default_slots=512, rho=0.9),
     # 16 tokens per step through the full-size 4-bit layer, grouped by expert.
     "batch16": dict(workload="batch16_full_h4096_i1024_e512_k4_shared_4bit", hidden=4096, inter=1024,
                     experts=512, top_k=4, bits=4, shared_bits=4, tokens=16),
@@ -292,10 +299,13 @@ def run_reference(args, cfg, rank, world):
     decode = (delta_oracle_prepare if delta else oracle_prepare)(cfg)
     time_oracle(decode, args.warmup, REF_WARMUP_S)
     n, el = time_oracle(decode, args.steps, REF_BUDGET_S)
-    lps = cfg.get("layers_per_step", 1)
+    lps = cfg.get("layers_per_step", cfg.get("stream_layers", 1))
     tt = cfg.get("tokens", 1)
     metric, unit = METRIC, UNIT
-    if delta:
+    if cfg.get("kind") == "stream":
+        metric, unit = (f"tokens/s through {lps} MoE layers with routed experts streamed from host memory "
+                        "(batch 1)"), "tokens/s"
+    elif delta:
         metric, unit = DELTA_METRIC, "updates/s"
     elif lps > 1:
         metric, unit = f"decode steps/s through {lps} MoE layers (batch 1)", "steps/s"
@@ -770,6 +780,141 @@ def run_delta(args, cfg, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# Routed experts streamed from host memory (config "stream")
+# ---------------------------------------------------------------------------
+
+STREAM_MAX_STEPS = 2000
+
+
+def run_stream(args, cfg, rank, world, local_rank):
+    """Tokens/s through a stack of layers whose routed experts live in pinned
+    host memory, per device slot count: each step copies the token in from
+    pinned host memory, decodes it through every layer with the streamer
+    (routing on the GPU, the decision to the host, one copy per missed expert
+    on a copy stream, the shared expert and the hits decoded meanwhile) and
+    reads the result back.  The hit rate and the host-to-device GB/s are those
+    of the timed steps (the warm-up steps fill the slots)."""
+    import torch
+
+    import bit_quantized_expert_router_b200 as F
+    import synth.gpu as SG
+    from bit_quantized_expert_router_b200 import build as B
+
+    if rank == 0 or not os.path.exists(F.LIB_PATH):
+        B.build_engine()
+        SG.build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    h, i, e, k = cfg["hidden"], cfg["inter"], cfg["experts"], cfg["top_k"]
+    NLS = cfg["stream_layers"]
+    layers, hosts = [], []
+    for l in range(NLS):
+        t = SG.make_layer(SEED + 1000 * rank, l, h, i, e, cfg["bits"], cfg["shared_bits"], F.blob_offsets,
+                          F.expert_bytes, dev)
+        stride = t["experts"].stride(0)
+        host = torch.empty(e, stride, dtype=torch.uint8, pin_memory=True)
+        host.copy_(t["experts"])
+        stub = torch.zeros(1, stride, dtype=torch.uint8, device=dev)
+        layers.append(F.Layer(t["w_router"], t["w_sgate"], stub, t["shared"], h, i, k, cfg["bits"],
+                              cfg["shared_bits"]))
+        hosts.append(host)
+        del t
+        torch.cuda.empty_cache()
+    steps = min(args.steps, STREAM_MAX_STEPS)
+    n_tok = args.warmup + steps
+    xs_host = torch.from_numpy(S.token_stream(SEED + rank, n_tok, h, cfg["rho"])).pin_memory()
+    out_host = torch.empty(h, dtype=torch.float32).pin_memory()
+    ws = layers[0].workspace(1)
+    stream = torch.cuda.current_stream()
+    copy_stream = torch.cuda.Stream()
+    xbuf = torch.empty(h, dtype=torch.float32, device=dev)
+    hbuf = [torch.empty(h, dtype=torch.float32, device=dev) for _ in range(2)]
+    blob = F.expert_bytes(h, i, cfg["bits"])
+    results = []
+    for n_slots in cfg["slot_counts"]:
+        slots = torch.empty(n_slots, hosts[0].shape[1], dtype=torch.uint8, device=dev)
+        st = F.Streamer(layers, hosts, slots)
+        launches = [0]
+
+        def step(j, count=False):
+            xbuf.copy_(xs_host[j], non_blocking=True)
+            src = xbuf
+            for l in range(NLS):
+                before = st.stats()["misses"] if count else 0
+                st.decode(l, src, src, out=hbuf[l % 2], ws=ws, copy_stream=copy_stream)
+                if count:
+                    # router + top-K, the hits/shared launch, and one more if anything was missed
+                    launches[0] += 3 + (st.stats()["misses"] > before)
+                src = hbuf[l % 2]
+            out_host.copy_(src, non_blocking=True)
+            stream.synchronize()
+
+        for j in range(args.warmup):
+            step(j)
+        s0 = st.stats()
+        torch.cuda.synchronize()
+        clocks = ClockSampler(local_rank)
+        clocks.start()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
+        for j in range(args.warmup, n_tok):
+            step(j, count=True)
+        ev1.record()
+        torch.cuda.synchronize()
+        clk = clocks.stop()
+        ms = ev0.elapsed_time(ev1)
+        s1 = st.stats()
+        hits, misses = s1["hits"] - s0["hits"], s1["misses"] - s0["misses"]
+        h2d = s1["h2d_bytes"] - s0["h2d_bytes"]
+        status = F.get_status()
+        (ms_max,) = max_over_ranks([ms], world, dev)
+        results.append({"slots": n_slots, "slot_gb": n_slots * hosts[0].shape[1] / 1e9,
+                        "hit_rate": hits / max(1, hits + misses), "misses_per_layer_decode": misses / (steps * NLS),
+                        "h2d_gbs": h2d / (ms / 1000.0) / 1e9, "tokens_per_s": whole_job_rate(steps, world, ms_max),
+                        "ms_per_token": ms_max / steps, "gpu_launches": launches[0], "clocks": clk,
+                        "h2d_bytes_per_step": h * 4 + h2d / steps,
+                        "device_status": status})
+        del st, slots
+        torch.cuda.empty_cache()
+    if rank == 0:
+        main_r = next(r for r in results if r["slots"] == cfg["default_slots"])
+        line = {
+            "impl": "fmoe", "metric": f"tokens/s through {NLS} MoE layers with routed experts streamed from host "
+                                      "memory (batch 1)",
+            "value": main_r["tokens_per_s"], "unit": "tokens/s", "n_gpus": world, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": main_r["ms_per_token"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {**cfg, "batch": 1, "group": 64, "slots": cfg["default_slots"],
+                       "expert_bytes": blob, "host_expert_gb": NLS * e * hosts[0].shape[1] / 1e9,
+                       "tokens": f"autoregressive stream, rho {cfg['rho']}, N(0,1) per element",
+                       "l2": "experts stream from host memory; the device slots and the layers' router and shared "
+                             "weights total far less than L2 per token only when they hit",
+                       "parallelism": f"replicas x{world}"},
+            "caches": results,
+            "e2e": {"value": main_r["tokens_per_s"], "unit": "tokens/s",
+                    "h2d_bytes_per_step": main_r["h2d_bytes_per_step"], "d2h_bytes_per_step": h * 4,
+                    "note": "the timed steps copy each token in from pinned host memory and its result back, "
+                            "and copy every missed expert from host memory: the value is end to end; "
+                            f"per step the input is {h * 4} B plus misses x {blob} B of experts"},
+            "gpu_launches": main_r["gpu_launches"],
+            "clocks": main_r["clocks"],
+            "device_status": max(r["device_status"] for r in results),
+        }
+        if not args.no_cpu_baseline:
+            cb = oracle_sample(cfg, args.cpu_seconds)
+            cb.pop("seconds", None)
+            cb.pop("tokens", None)
+            cb["value"] /= NLS
+            cb["unit"] = "tokens/s"
+            cb["sample"] += f"; tokens/s = decodes/s / {NLS} (experts resident in host memory, as here)"
+            line["cpu_baseline"] = cb
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -803,7 +948,10 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        (run_delta if delta else run_fmoe)(args, cfg, rank, world, local_rank)
+        if cfg.get("kind") == "stream":
+            run_stream(args, cfg, rank, world, local_rank)
+        else:
+            (run_delta if delta else run_fmoe)(args, cfg, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -28,7 +28,8 @@ EXPORTED = [
     "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status", "fmoe_strerror", "fmoe_last_cuda_error",
     "fmoe_layer_decode_noalloc", "fmoe_set_wait_limit_ns", "fmoe_set_dependent_launch", "fmoe_delta_update",
     "fmoe_cache_create", "fmoe_cache_destroy", "fmoe_cache_lookup", "fmoe_cache_stats", "fmoe_cache_reset",
-    "fmoe_experts_decode",
+    "fmoe_experts_decode", "fmoe_streamer_create", "fmoe_streamer_decode", "fmoe_streamer_stats",
+    "fmoe_streamer_destroy",
 ]
 
 
@@ -92,13 +93,18 @@ def lib() -> ctypes.CDLL:
     u64p = ctypes.POINTER(ctypes.c_uint64)
     L.fmoe_cache_stats.argtypes = [vp, u64p, u64p, u64p]
     L.fmoe_cache_reset.argtypes = [vp]
+    L.fmoe_streamer_create.argtypes = [ctypes.POINTER(FmoeLayerC), i, ctypes.POINTER(vp), vp, i, ctypes.POINTER(vp)]
+    L.fmoe_streamer_decode.argtypes = [vp, i, vp, vp, vp, vp, sz, vp, vp, vp, vp]
+    L.fmoe_streamer_stats.argtypes = [vp, u64p, u64p, u64p]
+    L.fmoe_streamer_destroy.argtypes = [vp]
     L.fmoe_last_cuda_error.argtypes = []
     L.fmoe_last_cuda_error.restype = i
     L.fmoe_strerror.argtypes = [i]
     L.fmoe_strerror.restype = ctypes.c_char_p
     for name in ("fmoe_blob_offsets", "fmoe_quantize_expert", "fmoe_route", "fmoe_expert_forward",
                  "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status", "fmoe_layer_decode_noalloc",
-                 "fmoe_experts_decode"):
+                 "fmoe_experts_decode", "fmoe_streamer_create", "fmoe_streamer_decode", "fmoe_streamer_stats",
+                 "fmoe_streamer_destroy"):
         getattr(L, name).restype = i
     _lib = L
     return L
@@ -383,6 +389,60 @@ class ExpertCache:
         h = getattr(self, "_h", None)
         if h is not None and h.value and _lib is not None:
             _lib.fmoe_cache_destroy(h)
+            self._h = None
+
+
+class Streamer:
+    """Routed experts streamed from page-locked host memory into n_slots device
+    slots (see fmoe_streamer_create in include/fmoe.h).  `layers`: Layer
+    objects of one shape (their `experts` tables are not used); `host_experts`:
+    per layer a pinned CPU uint8 tensor [n_experts, expert_stride]; `slots`: a
+    CUDA uint8 tensor [n_slots, expert_stride]."""
+
+    def __init__(self, layers, host_experts, slots: torch.Tensor):
+        if len(layers) != len(host_experts) or not layers:
+            raise ValueError("one host expert table per layer")
+        for h in host_experts:
+            if not isinstance(h, torch.Tensor) or h.is_cuda or not h.is_pinned() or h.dtype != torch.uint8:
+                raise ValueError("host_experts must be pinned CPU uint8 tensors")
+        _dev_tensor(slots, torch.uint8, "slots")
+        self.layers = list(layers)
+        self._keep = (list(host_experts), slots)
+        arr = (FmoeLayerC * len(layers))(*[L.c for L in layers])
+        hp = (ctypes.c_void_p * len(layers))(*[h.data_ptr() for h in host_experts])
+        h = ctypes.c_void_p()
+        _check(lib().fmoe_streamer_create(arr, len(layers), hp, slots.data_ptr(), slots.shape[0], ctypes.byref(h)),
+               "fmoe_streamer_create")
+        self._h = h
+
+    def decode(self, layer: int, x: torch.Tensor, residual: torch.Tensor | None = None,
+               out: torch.Tensor | None = None, ws: torch.Tensor | None = None, stream=None, copy_stream=None,
+               return_routing: bool = False):
+        L = self.layers[layer]
+        x = _dev_tensor(x, torch.float32, "x")
+        if out is None:
+            out = torch.empty_like(x)
+        if ws is None:
+            ws = L.workspace(1)
+        K = L.top_k
+        idx = np.empty(K, dtype=np.int32)
+        w = np.empty(K, dtype=np.float32)
+        cs = _stream(stream)
+        ks = cs if copy_stream is None else copy_stream.cuda_stream
+        _check(lib().fmoe_streamer_decode(self._h, int(layer), x.data_ptr(), _ptr(residual), out.data_ptr(),
+                                          ws.data_ptr(), ws.numel(), cs, ks, idx.ctypes.data, w.ctypes.data),
+               "fmoe_streamer_decode")
+        return (out, idx, w) if return_routing else out
+
+    def stats(self) -> dict:
+        v = [ctypes.c_uint64(0) for _ in range(3)]
+        _check(lib().fmoe_streamer_stats(self._h, *(ctypes.byref(x) for x in v)), "fmoe_streamer_stats")
+        return {"hits": v[0].value, "misses": v[1].value, "h2d_bytes": v[2].value}
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value and _lib is not None:
+            _lib.fmoe_streamer_destroy(h)
             self._h = None
 
 

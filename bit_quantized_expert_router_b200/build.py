@@ -19,7 +19,7 @@ FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared"]
 ENGINE_SRC = os.path.join(HERE, "csrc", "fmoe_api.cu")
 ENGINE_DEPS = [os.path.join(HERE, "csrc", f) for f in
                ("common.cuh", "dequant.cuh", "layer_kernel.cuh", "route_quant_kernels.cuh", "grouped_kernels.cuh", "tc.cuh", "shared_tc.cuh",
-                "deltanet.cuh", "expert_cache.h")] + \
+                "deltanet.cuh", "expert_cache.h", "streamer.cuh")] + \
               [os.path.join(ROOT, "include", "fmoe.h")]
 ENGINE_SO = os.path.join(HERE, "libfmoe.so")
 

@@ -3,6 +3,8 @@
 #include <atomic>
 #include <cstring>
 #include <mutex>
+#include <new>
+#include <vector>
 
 #include "../../include/fmoe.h"
 #include "deltanet.cuh"
@@ -563,9 +565,8 @@ namespace {
 // The argument checks of a layer decode call that need no device (shapes,
 // pointers, alignment).  With `routed_given` the layer's router and expert
 // table are not used (the caller passes the experts).
-int check_layer_args(const fmoe_layer* L, const float* x, const float* residual, const float* out, int T,
-                     bool routed_given) {
-  if (!L || !x || !out) return FMOE_EINVAL;
+int check_layer_shape(const fmoe_layer* L, int T, bool routed_given) {
+  if (!L) return FMOE_EINVAL;
   if (!routed_given && (!L->w_router || !L->experts)) return FMOE_EINVAL;
   const int H = L->hidden, I = L->inter, E = L->n_experts, K = L->top_k;
   if (!shape_ok(H, I) || !bits_ok(L->bits) || (L->shared && !bits_ok(L->shared_bits)) ||
@@ -578,11 +579,17 @@ int check_layer_args(const fmoe_layer* L, const float* x, const float* residual,
     if (!aligned(L->experts, 256) || !aligned(L->w_router, 16) || (L->w_sgate && !aligned(L->w_sgate, 16)))
       return FMOE_EINVAL;
   }
-  if ((L->shared && !aligned(L->shared, 256)) || !aligned(x, 16) || !aligned(out, 16) ||
-      (residual && !aligned(residual, 16)) || x == out)
-    return FMOE_EINVAL;
+  if (L->shared && !aligned(L->shared, 256)) return FMOE_EINVAL;
   if (L->norm_weight && (!aligned(L->norm_weight, 16) || !(L->norm_eps >= 0.f) || !(L->norm_eps < INFINITY)))
     return FMOE_EINVAL;
+  return FMOE_OK;
+}
+
+int check_layer_args(const fmoe_layer* L, const float* x, const float* residual, const float* out, int T,
+                     bool routed_given) {
+  if (!L || !x || !out) return FMOE_EINVAL;
+  if (int rc = check_layer_shape(L, T, routed_given)) return rc;
+  if (!aligned(x, 16) || !aligned(out, 16) || (residual && !aligned(residual, 16)) || x == out) return FMOE_EINVAL;
   return FMOE_OK;
 }
 
@@ -877,3 +884,5 @@ const char* fmoe_strerror(int code) {
 }
 
 }  // extern "C"
+
+#include "streamer.cuh"

@@ -874,9 +874,11 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
     }
   }
   // ---- Stage x into the decode layouts (every warp) ---------------------------
-  if (BR == 4 || BS == 4)
+  // (each width the launch uses: a given-routing launch without routed
+  // experts has no routed width, whatever its instantiation)
+  if ((BR == 4 || BS == 4) && a.xs4_off >= 0)
     stage_inputs<4, false>(xu, a.H, reinterpret_cast<float4*>(sm.vec + a.xs4_off), sm.sf, tid, kThreads);
-  if (BR == 2 || BS == 2)
+  if ((BR == 2 || BS == 2) && a.xs2_off >= 0)
     stage_inputs<2, false>(xu, a.H, reinterpret_cast<float4*>(sm.vec + a.xs2_off),
                            sm.sf + (a.xs4_off >= 0 ? a.H / 32 : 0), tid, kThreads);
   __syncwarp();

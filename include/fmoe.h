@@ -338,6 +338,60 @@ int fmoe_cache_stats(const fmoe_expert_cache* cache, uint64_t* hits, uint64_t* m
 /* Empty the directory (all slots free) and zero the totals. */
 int fmoe_cache_reset(fmoe_expert_cache* cache);
 
+/* ---- Routed experts streamed from host memory ------------------------------
+ * The B200 counterpart of the pages' expert streaming ([P2] "SSD-Experten-
+ * Streaming": only the K active experts of a layer are read, on demand, and
+ * the OS page cache keeps the recently used ones, an LRU with ~71 % hits;
+ * [P2] "Verzögerte GPU-Experten-Berechnung": the expert command is queued
+ * without waiting).  The routed experts of every layer stay in page-locked
+ * host memory; n_slots device slots hold the recently used ones (an
+ * fmoe_expert_cache directory over (layer, expert)).  Per layer and token,
+ * fmoe_streamer_decode:
+ *   1. runs the router GEMV and top-K on the GPU (as fmoe_route) and copies
+ *      the decision to the host, the one synchronisation of the call;
+ *   2. looks the K experts up in the directory and copies every miss from
+ *      host memory into its slot, one cudaMemcpyAsync each, on copy_stream;
+ *   3. meanwhile decodes the shared expert and the hits on stream
+ *      (out = residual + sum over hits + gated shared expert), then, once the
+ *      copies have landed, adds the misses with a second launch.
+ * It returns once these are queued; the result is that of fmoe_layer_decode
+ * within fp32 rounding (same routing, a different summation order). */
+typedef struct fmoe_streamer_s fmoe_streamer;
+
+/* layers[0..n_layers): w_router, w_sgate, shared, shapes and code widths as
+ * for fmoe_layer_decode, all with the same hidden, inter, n_experts, top_k,
+ * bits and expert_stride, no norm_weight (the router reads x as given); the
+ * `experts` field is ignored.  host_experts[l]: page-locked host memory
+ * (cudaHostAlloc, or registered), 256-byte aligned, holding layer l's
+ * n_experts blobs at expert_stride.  slots: device memory of n_slots *
+ * expert_stride bytes, 256-byte aligned, top_k <= n_slots <=
+ * FMOE_CACHE_MAX_SLOTS.  All stay owned by the caller and must outlive the
+ * streamer.  *out is set (NULL on error).  Errors: FMOE_EINVAL (also for
+ * host memory that is not page-locked), FMOE_ENOMEM, FMOE_ECUDA. */
+int fmoe_streamer_create(const fmoe_layer* layers, int n_layers, const void* const* host_experts, void* slots,
+                         int n_slots, fmoe_streamer** out);
+
+/* Decode one token through layer `layer` (see above).  x, residual, out, ws,
+ * ws_bytes: as fmoe_layer_decode with T = 1.  stream: the compute stream;
+ * copy_stream: the stream of the host-to-device copies (may equal stream:
+ * no overlap then).  Every decode of a streamer must use the same stream (a
+ * slot is overwritten only after the kernels that read it, which that stream
+ * orders).  The call synchronises `stream` once, so it cannot be captured
+ * into a graph.  idx_out_opt, w_out_opt: optional HOST arrays [top_k] that
+ * receive the routing decision.  Errors: FMOE_EINVAL, FMOE_ENOMEM,
+ * FMOE_ECUDA; kernel-side problems as fmoe_layer_decode. */
+int fmoe_streamer_decode(fmoe_streamer* s, int layer, const float* x, const float* residual, float* out, void* ws,
+                         size_t ws_bytes, fmoe_stream_t stream, fmoe_stream_t copy_stream, int32_t* idx_out_opt,
+                         float* w_out_opt);
+
+/* Running totals: expert hits and misses (the directory's) and bytes copied
+ * from host to device (each pointer optional). */
+int fmoe_streamer_stats(const fmoe_streamer* s, uint64_t* hits, uint64_t* misses, uint64_t* h2d_bytes);
+
+/* Free a streamer (NULL is accepted); the caller's memory is untouched.
+ * Returns FMOE_OK. */
+int fmoe_streamer_destroy(fmoe_streamer* s);
+
 /* How the single-token layer kernel (fmoe_layer_decode with T = 1,
  * fmoe_layer_decode_noalloc with T = 1, fmoe_expert_forward) is launched,
  * process-wide, for the calls made after this one.

@@ -188,6 +188,25 @@ def token_x(seed: int, layer: int, step: int, n_tokens: int, hidden: int,
     return g.standard_normal((n_tokens, hidden), dtype=np.float32)
 
 
+TAG_STREAM = 0x57E4
+
+
+def token_stream(seed: int, n_tokens: int, hidden: int, rho: float) -> np.ndarray:
+    """fp32 [T][H]: a first-order autoregressive token sequence, each row
+    N(0, 1) per element, consecutive rows correlated by rho
+    (x_t = rho x_{t-1} + sqrt(1 - rho^2) z_t), a stand-in for the temporal
+    locality of a decoded text (consecutive tokens tend to pick the same
+    experts)."""
+    g = _rng(seed, TAG_STREAM, n_tokens, hidden)
+    z = g.standard_normal((n_tokens, hidden), dtype=np.float32)
+    out = np.empty_like(z)
+    out[0] = z[0]
+    c = np.float32(np.sqrt(1.0 - rho * rho))
+    for t in range(1, n_tokens):
+        out[t] = np.float32(rho) * out[t - 1] + c * z[t]
+    return out
+
+
 def token_residual(seed: int, layer: int, step: int, n_tokens: int,
                    hidden: int) -> np.ndarray:
     g = _rng(seed, TAG_RES, layer, step)

@@ -118,6 +118,23 @@ def test_invalid_arguments_rejected_on_host(F):
     assert L.fmoe_layer_decode_noalloc(ctypes.byref(c), fake, None, fake * 2, 2, None, None, None) == F.FMOE_EINVAL
     assert L.fmoe_workspace_bytes(ctypes.byref(c), 0) == 0
     assert L.fmoe_route_workspace_bytes(17, 512) == 0
+    # the expert streamer checks its layers on the host before any CUDA call
+    def streamer(layers, hosts=None, slots=fake, n_slots=8):
+        arr = (F.FmoeLayerC * len(layers))(*layers)
+        hp = (ctypes.c_void_p * len(layers))(*(hosts or [fake] * len(layers)))
+        h = ctypes.c_void_p(123)
+        rc = L.fmoe_streamer_create(arr, len(layers), hp, slots, n_slots, ctypes.byref(h))
+        assert not h.value  # nothing is created on an error
+        return rc
+    assert streamer([c], n_slots=3) == F.FMOE_EINVAL  # fewer slots than top_k
+    assert streamer([c], slots=fake + 16) == F.FMOE_EINVAL  # slots off the 256-byte grid
+    assert streamer([c], hosts=[fake + 8]) == F.FMOE_EINVAL  # host blobs off the grid
+    assert streamer([F.FmoeLayerC(**{**base, "norm_weight": fake})]) == F.FMOE_EINVAL  # routing reads x as given
+    assert streamer([c, F.FmoeLayerC(**{**base, "inter": 512})]) == F.FMOE_EINVAL  # layers of different shapes
+    assert streamer([F.FmoeLayerC(**{**base, "expert_stride": 1000})]) == F.FMOE_EINVAL
+    assert L.fmoe_streamer_decode(None, 0, fake, None, fake * 2, fake, 1 << 20, None, None, None, None) \
+        == F.FMOE_EINVAL
+    assert L.fmoe_streamer_destroy(None) == F.FMOE_OK
     # delta-rule update: shapes, alignment and overlap are checked on the host.
     # The defaults are disjoint stand-ins (the 64 x 128 x 128 state spans 4 MiB
     # from 1 MiB; every other buffer lies beyond it); only variants with one

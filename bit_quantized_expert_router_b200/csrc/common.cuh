@@ -54,8 +54,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, ui
   return ok != 0;
 }
 #ifdef FMOE_TRACE_BUILD
-// Trace builds count wait-loop iterations: [0] mbarrier waits, [1] grid waits,
-// [2] routing polls.
+// Trace builds count wait-loop iterations: [0] mbarrier waits, [1] activation
+// polls, [2] routing polls.
 __device__ unsigned long long g_fmoe_spins[4];
 #define FMOE_SPIN(i) atomicAdd(&g_fmoe_spins[i], 1ull)
 #else

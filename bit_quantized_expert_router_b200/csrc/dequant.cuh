@@ -210,6 +210,7 @@ __device__ inline bool stage_tagged(const unsigned long long* src, int n, float4
             (unsigned)(w[b][2] >> 32) == tag && (unsigned)(w[b][3] >> 32) == tag)
           pend &= ~(1u << b);
       if (!pend) break;
+      FMOE_SPIN(1);
       const uint64_t now = globaltimer_ns();
       if (t0 == 0) {
         t0 = now;

@@ -857,10 +857,12 @@ int fmoe_set_dependent_launch(int enable, int* previous_opt) {
 
 #ifdef FMOE_TRACE_BUILD
 // Trace builds only: copy the phase timestamps of the last layer launch
-// ([1024][12] u64, ns) to host memory and clear them.
+// ([1024][kTraceCols] u64: SM cycles at the trace points, then globaltimer ns
+// at the dependency wait and at the end and the cycles at the end) to host
+// memory and clear them.
 int fmoe_trace_read(unsigned long long* host) {
   if (cudaError_t e = cudaMemcpyFromSymbol(host, g_fmoe_trace, sizeof(g_fmoe_trace))) return cuda_fail(e);
-  static unsigned long long zero[1024][kTracePoints];
+  static unsigned long long zero[1024][kTraceCols];
   if (cudaError_t e = cudaMemcpyToSymbol(g_fmoe_trace, zero, sizeof(zero))) return cuda_fail(e);
   return FMOE_OK;
 }

@@ -61,16 +61,18 @@ constexpr int kActWords = 10240;            // tagged-activation words of a work
 constexpr unsigned kEpochWrap = 0x7FFFFFFEu;
 constexpr int kMaxNstC = 8;       // most down-item stages a warp keeps in flight
 
-// Optional phase trace (compile with -DFMOE_TRACE_BUILD): thread 0 of every CTA
-// stores %globaltimer at fixed points of the kernel into g_fmoe_trace.
+// Optional phase trace (compile with -DFMOE_TRACE_BUILD): the SM cycle counter
+// at fixed points of the kernel, per CTA in shared memory (points marked per
+// warp keep the latest warp), copied to g_fmoe_trace[blockIdx] at the end, with
+// %globaltimer at the dependency wait and at the end to place and scale them.
 #ifdef FMOE_TRACE_BUILD
 constexpr int kTracePoints = 25;
-__device__ unsigned long long g_fmoe_trace[1024][kTracePoints];
+constexpr int kTraceCols = kTracePoints + 3;  // + globaltimer at point 24 and at the end, cycles at the end
+__device__ unsigned long long g_fmoe_trace[1024][kTraceCols];
 #define FMOE_TRACE(i) \
-  do { if (threadIdx.x == 0 && blockIdx.x < 1024) g_fmoe_trace[blockIdx.x][i] = globaltimer_ns(); } while (0)
+  do { if (threadIdx.x == 0) cs.trace[i] = clock64(); } while (0)
 #define FMOE_TRACE_WARP(i) \
-  do { if ((threadIdx.x & 31) == 0 && blockIdx.x < 1024) \
-    atomicMax(&g_fmoe_trace[blockIdx.x][i], (unsigned long long)globaltimer_ns()); } while (0)
+  do { if ((threadIdx.x & 31) == 0) atomicMax(&cs.trace[i], (unsigned long long)clock64()); } while (0)
 #else
 #define FMOE_TRACE(i) do { } while (0)
 #define FMOE_TRACE_WARP(i) do { } while (0)
@@ -209,6 +211,9 @@ __device__ __forceinline__ WarpPlan make_plan(const LayerArgs& a, int cta, int w
 
 // Per-CTA shared state (static shared memory).
 struct CtaShared {
+#ifdef FMOE_TRACE_BUILD
+  unsigned long long trace[kTraceCols];
+#endif
   int poison;           // a wait of this CTA ran out: what it hands on or writes is NaN
   float rpart[kWarps];  // router segment dot products, by warp
   uint64_t x_bar;       // completes once x is in shared memory
@@ -519,7 +524,6 @@ __device__ __noinline__ void warp_topk_n(const float* lg, int n, int k, int lane
       my_idx = (int)e;
     }
   }
-  FMOE_TRACE_WARP(14);
   // w_k = exp(l_k - l_0) / sum_j exp(l_j - l_0): softmax restricted to the
   // selected experts, equal to softmax-then-renormalise.
   const float l0 = __shfl_sync(0xffffffffu, my_val, 0);
@@ -744,6 +748,9 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   uint64_t* my_bars_c = my_bars + a.nst;
   const bool layer_mode = a.n_router > 0;
   const RouterPart rp = router_part(a.n_router, a.H, blockIdx.x, warp, G);
+#ifdef FMOE_TRACE_BUILD
+  if (tid < kTraceCols) cs.trace[tid] = 0;
+#endif
   FMOE_TRACE(0);
   // The next layer decode on the stream may be scheduled now: its CTAs take
   // the SMs this grid's CTAs leave, and do their weight-only set-up while
@@ -810,6 +817,9 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   // no access to them before it has completed.
   grid_dep_wait();
   FMOE_TRACE(24);
+#ifdef FMOE_TRACE_BUILD
+  if (tid == 0) cs.trace[kTracePoints] = globaltimer_ns();
+#endif
   if (tid == 0) bulk_g2s(sm.vec + a.xu_off, a.x, a.H * 4, &cs.x_bar);
   // The tag of this launch's published words (the epoch the previous launch
   // on this workspace left, plus one).
@@ -1066,6 +1076,13 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
       __threadfence();
     }
   }
+#ifdef FMOE_TRACE_BUILD
+  if (tid == 0 && blockIdx.x < 1024) {
+    cs.trace[kTracePoints + 2] = clock64();
+    cs.trace[kTracePoints + 1] = globaltimer_ns();
+    for (int i = 0; i < kTraceCols; ++i) g_fmoe_trace[blockIdx.x][i] = cs.trace[i];
+  }
+#endif
 }
 
 }  // namespace fmoe

@@ -150,10 +150,9 @@ template <int BITS, bool kGlobal>
 __device__ inline void stage_inputs(const float* __restrict__ src, int n, float4* xs, float2* sf, int tid,
                                     int nthreads) {
   constexpr int CPV = 128 / BITS, F4 = CPV / 4;
-  // passes whose loads are all issued before any is used: global sources need
-  // the loads in flight together; from shared memory one pass at a time keeps
-  // this code (run once per launch, from a cold instruction cache) short
-  constexpr int kBatch = kGlobal ? 4 : 1;
+  // passes whose loads are all issued before any is used (their latencies,
+  // and those of their shuffles, overlap)
+  constexpr int kBatch = kGlobal ? 4 : 2;
   const int NV = n / CPV, total = NV * F4;
   const int lane = tid & 31;
   for (int base0 = tid - lane; base0 < total; base0 += kBatch * nthreads) {

@@ -341,24 +341,48 @@ __device__ __forceinline__ float router_dot(const uint16_t* row, const float* xu
   return warp_sum(acc);
 }
 
-// The same dot product with the row in shared memory.
+// The same dot product with the row in shared memory: four 16-byte vectors
+// per lane in flight (their loads issued together), four accumulators.
 __device__ __forceinline__ float router_dot_smem(const uint16_t* row, const float* xu, int H, int lane) {
   const uint4* rv = reinterpret_cast<const uint4*>(row);
   const float4* xv = reinterpret_cast<const float4*>(xu);
-  float acc0 = 0.f, acc1 = 0.f;
-  for (int v = lane; v < H / 8; v += 32) {
+  const int nv = H / 8;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  int v = lane;
+  for (; v + 96 < nv; v += 128) {
+    uint4 w[4];
+    float4 xa[4], xb[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      w[j] = rv[v + 32 * j];
+      xa[j] = xv[2 * (v + 32 * j)];
+      xb[j] = xv[2 * (v + 32 * j) + 1];
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      acc[j] = fmaf(bf16_lo(w[j].x), xa[j].x, acc[j]);
+      acc[j] = fmaf(bf16_hi(w[j].x), xa[j].y, acc[j]);
+      acc[j] = fmaf(bf16_lo(w[j].y), xa[j].z, acc[j]);
+      acc[j] = fmaf(bf16_hi(w[j].y), xa[j].w, acc[j]);
+      acc[j] = fmaf(bf16_lo(w[j].z), xb[j].x, acc[j]);
+      acc[j] = fmaf(bf16_hi(w[j].z), xb[j].y, acc[j]);
+      acc[j] = fmaf(bf16_lo(w[j].w), xb[j].z, acc[j]);
+      acc[j] = fmaf(bf16_hi(w[j].w), xb[j].w, acc[j]);
+    }
+  }
+  for (; v < nv; v += 32) {
     const uint4 w = rv[v];
     const float4 xa = xv[2 * v], xb = xv[2 * v + 1];
-    acc0 = fmaf(bf16_lo(w.x), xa.x, acc0);
-    acc1 = fmaf(bf16_hi(w.x), xa.y, acc1);
-    acc0 = fmaf(bf16_lo(w.y), xa.z, acc0);
-    acc1 = fmaf(bf16_hi(w.y), xa.w, acc1);
-    acc0 = fmaf(bf16_lo(w.z), xb.x, acc0);
-    acc1 = fmaf(bf16_hi(w.z), xb.y, acc1);
-    acc0 = fmaf(bf16_lo(w.w), xb.z, acc0);
-    acc1 = fmaf(bf16_hi(w.w), xb.w, acc1);
+    acc[0] = fmaf(bf16_lo(w.x), xa.x, acc[0]);
+    acc[1] = fmaf(bf16_hi(w.x), xa.y, acc[1]);
+    acc[2] = fmaf(bf16_lo(w.y), xa.z, acc[2]);
+    acc[3] = fmaf(bf16_hi(w.y), xa.w, acc[3]);
+    acc[0] = fmaf(bf16_lo(w.z), xb.x, acc[0]);
+    acc[1] = fmaf(bf16_hi(w.z), xb.y, acc[1]);
+    acc[2] = fmaf(bf16_lo(w.w), xb.z, acc[2]);
+    acc[3] = fmaf(bf16_hi(w.w), xb.w, acc[3]);
   }
-  return warp_sum(acc0 + acc1);
+  return warp_sum((acc[0] + acc[1]) + (acc[2] + acc[3]));
 }
 
 // Gate and up rows of one expert (stage layout: gate codes | up codes | gate sb

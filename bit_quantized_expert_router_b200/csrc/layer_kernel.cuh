@@ -60,6 +60,7 @@ constexpr int kActWords = 10240;            // tagged-activation words of a work
 // nothing (tag 0), so every tagged wait runs out instead of accepting words.
 constexpr unsigned kEpochWrap = 0x7FFFFFFEu;
 constexpr int kMaxNstC = 8;       // most down-item stages a warp keeps in flight
+constexpr int kRouteWarps = 4;    // warps of a CTA that take the routing decision (the others stage x meanwhile)
 
 // Optional phase trace (compile with -DFMOE_TRACE_BUILD): the SM cycle counter
 // at fixed points of the kernel, per CTA in shared memory (points marked per
@@ -217,7 +218,6 @@ struct CtaShared {
   int poison;           // a wait of this CTA ran out: what it hands on or writes is NaN
   float rpart[kWarps];  // router segment dot products, by warp
   uint64_t x_bar;       // completes once x is in shared memory
-  uint64_t staged_bar;  // completes once x is staged in the decode layouts
   uint64_t rbar[kWarps];  // router warp w's row is in its ring (router_smem)
   unsigned long long param_touch;  // see the kernel's set-up
   float red[kWarps];               // per-warp partial sums (input norm)
@@ -622,8 +622,9 @@ __device__ __forceinline__ void warp_select(uint32_t (&key)[NK], uint32_t (&eix)
   }
 }
 
-// Stage 1 of the CTA's top-K.  Each lane holds NKW logits of its warp's slice
-// (NKW * 32 consecutive experts from w * NKW * 32) as order-preserving keys,
+// Stage 1 of the CTA's top-K (routing warps).  Each lane holds NKW logits of
+// its warp's slice (NKW * 32 consecutive experts from w * NKW * 32) as
+// order-preserving keys,
 // read from the tagged words as soon as they carry this launch's tag (warp 0's
 // lane 0 also reads the shared gate's logit, which it returns); the warp then
 // selects the top k of its slice into the candidates.  The tag check replaces
@@ -678,12 +679,12 @@ __device__ __forceinline__ float slice_topk(const unsigned long long* tlog, int 
   return gate_logit;
 }
 
-// The routing decision of this CTA, computed by all of its warps together;
-// every warp calls this once, before it computes any unit (layer mode).
-//   Each warp takes the top K of its slice of the logits as they are
-//   published; after a CTA barrier warp 0 selects the top K of the candidates
-//   and computes the weights, and a second barrier publishes the decision to
-//   the CTA.
+// The routing decision of this CTA, taken by its first kRouteWarps warps
+// while the others stage x (layer mode): each routing warp takes the top K of
+// its slice of the logits as they are published; after a barrier of the
+// routing warps, warp 0 selects the top K of their candidates and computes the
+// weights; the CTA barrier that follows (in the kernel) publishes the
+// decision to every warp.
 // Kept out of line (measured faster than inlined into the kernel).
 __device__ __noinline__ void cta_routing(const LayerArgs& a, CtaShared& cs, int warp, int lane, unsigned tag) {
   // Every parameter used here, read once up front: the loads overlap the wait
@@ -698,27 +699,24 @@ __device__ __noinline__ void cta_routing(const LayerArgs& a, CtaShared& cs, int 
   float* const w_out = a.w_out;
   float* const sg_out = a.sg_out;
   float gate_logit;
-  if (E <= kWarps * 32)
-    gate_logit = slice_topk<1>(tlog, E, K, gated, timeout_ns, tag, warp, lane, cs);
+  if (E <= kRouteWarps * 32 * 4)
+    gate_logit = slice_topk<4>(tlog, E, K, gated, timeout_ns, tag, warp, lane, cs);
   else
-    gate_logit = slice_topk<kMaxExperts / (kWarps * 32)>(tlog, E, K, gated, timeout_ns, tag, warp, lane, cs);
+    gate_logit = slice_topk<kMaxExperts / (kRouteWarps * 32)>(tlog, E, K, gated, timeout_ns, tag, warp, lane, cs);
   FMOE_TRACE_WARP(14);
-  __syncthreads();
+  // the routing warps' candidates are in shared memory
+  asm volatile("bar.sync 1, %0;" ::"r"(kRouteWarps * 32) : "memory");
   FMOE_TRACE_WARP(9);
   if (warp == 0) {
-    // Stage 2: warp 0 selects the top K of the kWarps * K candidates (the
-    // global top K is among them, ties included) with the same rounds, up to
-    // four candidates per lane; lane kk < K ends with the kk-th.
-    const int nc = kWarps * K;
-    uint32_t ckey[kMaxTopK * kWarps / 32], cidx[kMaxTopK * kWarps / 32];
-#pragma unroll
-    for (int i = 0; i < kMaxTopK * kWarps / 32; ++i) {
-      const int c = i * 32 + lane;
-      ckey[i] = c < nc ? cs.cand_key[c] : 0u;
-      cidx[i] = c < nc ? cs.cand_idx[c] : 0xffffffffu;
-    }
+    // Stage 2: warp 0 selects the top K of the kRouteWarps * K candidates
+    // (the global top K is among them, ties included) with the same rounds,
+    // one candidate per lane; lane kk < K ends with the kk-th.
+    const int nc = kRouteWarps * K;
+    uint32_t ckey[1], cidx[1];
+    ckey[0] = lane < nc ? cs.cand_key[lane] : 0u;
+    cidx[0] = lane < nc ? cs.cand_idx[lane] : 0xffffffffu;
     uint32_t hk, hi;
-    warp_select<kMaxTopK * kWarps / 32>(ckey, cidx, K, lane, hk, hi);
+    warp_select<1>(ckey, cidx, K, lane, hk, hi);
     FMOE_TRACE_WARP(23);
     // w_k = exp(l_k - l_0) / sum_j exp(l_j - l_0): softmax restricted to the
     // selected experts, equal to softmax-then-renormalise.
@@ -744,8 +742,6 @@ __device__ __noinline__ void cta_routing(const LayerArgs& a, CtaShared& cs, int 
     }
     FMOE_TRACE_WARP(10);
   }
-  __syncthreads();
-  FMOE_TRACE_WARP(3);
 }
 
 // Issue phase-C load i (>= a.count + b.count) into the re-carved ring (lane 0).
@@ -785,7 +781,6 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
   auto router_row_ptr = [&](int e) { return (e < a.E) ? a.w_router + (long long)e * a.H : a.w_sgate; };
   if (tid == 0) {
     mbar_init(&cs.x_bar, 1);
-    mbar_init(&cs.staged_bar, kWarps);
     cs.sg = 1.0f;
     cs.c_prefetch = 0;
     cs.poison = 0;
@@ -907,30 +902,36 @@ __global__ void __launch_bounds__(kThreads, 1) layer_kernel(const __grid_constan
       ++issued;
     }
   }
-  // ---- Stage x into the decode layouts (every warp) ---------------------------
-  // (each width the launch uses: a given-routing launch without routed
-  // experts has no routed width, whatever its instantiation)
-  if ((BR == 4 || BS == 4) && a.xs4_off >= 0)
-    stage_inputs<4, false>(xu, a.H, reinterpret_cast<float4*>(sm.vec + a.xs4_off), sm.sf, tid, kThreads);
-  if ((BR == 2 || BS == 2) && a.xs2_off >= 0)
-    stage_inputs<2, false>(xu, a.H, reinterpret_cast<float4*>(sm.vec + a.xs2_off),
-                           sm.sf + (a.xs4_off >= 0 ? a.H / 32 : 0), tid, kThreads);
-  __syncwarp();
-  FMOE_TRACE_WARP(18);
-  if (lane == 0) mbar_arrive(&cs.staged_bar);
-  if (warp == kWarps - 1 && lane == 0 && a.shared && plan.nq > 0) {
-    // the shared expert's down rows of this CTA are known from the start
-    const BlobOff o = blob_offsets(a.H, a.I, BS);
-    const int cb = codes_row_bytes(a.I, BS), sbr = sb_row_bytes(a.I);
-    const long long r0 = (long long)plan.q0 * kRC, nr = (long long)plan.nq * kRC;
-    bulk_prefetch_l2(a.shared + o.dc + r0 * cb, (uint32_t)(nr * cb));
-    bulk_prefetch_l2(a.shared + o.dsb + r0 * sbr, (uint32_t)(nr * sbr));
-  }
   issued = __shfl_sync(0xffffffffu, issued, 0);
-  // Every warp of the CTA takes part in the routing decision (layer mode).
-  if (layer_mode) cta_routing(a, cs, warp, lane, tag);
-  if (!mbar_wait_bounded(&cs.staged_bar, 0, a.timeout_ns) && lane == 0) wait_failed(cs, kStatusCtaWaitTimeout);
+  if (layer_mode && warp < kRouteWarps) {
+    // ---- Routing decision (the first kRouteWarps warps) ------------------------
+    cta_routing(a, cs, warp, lane, tag);
+  } else {
+    // ---- Stage x into the decode layouts (the other warps, meanwhile) ---------
+    // (each width the launch uses: a given-routing launch without routed
+    // experts has no routed width, whatever its instantiation)
+    const int w0 = layer_mode ? kRouteWarps * 32 : 0;
+    const int t0 = tid - w0, nt = kThreads - w0;
+    if ((BR == 4 || BS == 4) && a.xs4_off >= 0)
+      stage_inputs<4, false>(xu, a.H, reinterpret_cast<float4*>(sm.vec + a.xs4_off), sm.sf, t0, nt);
+    if ((BR == 2 || BS == 2) && a.xs2_off >= 0)
+      stage_inputs<2, false>(xu, a.H, reinterpret_cast<float4*>(sm.vec + a.xs2_off),
+                             sm.sf + (a.xs4_off >= 0 ? a.H / 32 : 0), t0, nt);
+    __syncwarp();
+    FMOE_TRACE_WARP(18);
+    if (warp == kWarps - 1 && lane == 0 && a.shared && plan.nq > 0) {
+      // the shared expert's down rows of this CTA are known from the start
+      const BlobOff o = blob_offsets(a.H, a.I, BS);
+      const int cb = codes_row_bytes(a.I, BS), sbr = sb_row_bytes(a.I);
+      const long long r0 = (long long)plan.q0 * kRC, nr = (long long)plan.nq * kRC;
+      bulk_prefetch_l2(a.shared + o.dc + r0 * cb, (uint32_t)(nr * cb));
+      bulk_prefetch_l2(a.shared + o.dsb + r0 * sbr, (uint32_t)(nr * sbr));
+    }
+  }
+  // the routing decision and the staged x reach every warp
+  __syncthreads();
   FMOE_TRACE(1);
+  FMOE_TRACE_WARP(3);
 
   // ---- Ring loop over phases A (static gate/up) and B (routed gate/up) ------
   const int n_gu = plan.a.count + plan.b.count;

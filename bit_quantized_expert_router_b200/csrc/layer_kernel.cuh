@@ -60,7 +60,7 @@ constexpr int kActWords = 10240;            // tagged-activation words of a work
 // nothing (tag 0), so every tagged wait runs out instead of accepting words.
 constexpr unsigned kEpochWrap = 0x7FFFFFFEu;
 constexpr int kMaxNstC = 8;       // most down-item stages a warp keeps in flight
-constexpr int kRouteWarps = 4;    // warps of a CTA that take the routing decision (the others stage x meanwhile)
+constexpr int kRouteWarps = 8;    // warps of a CTA that take the routing decision (the others stage x meanwhile)
 
 // Optional phase trace (compile with -DFMOE_TRACE_BUILD): the SM cycle counter
 // at fixed points of the kernel, per CTA in shared memory (points marked per
@@ -699,8 +699,8 @@ __device__ __noinline__ void cta_routing(const LayerArgs& a, CtaShared& cs, int 
   float* const w_out = a.w_out;
   float* const sg_out = a.sg_out;
   float gate_logit;
-  if (E <= kRouteWarps * 32 * 4)
-    gate_logit = slice_topk<4>(tlog, E, K, gated, timeout_ns, tag, warp, lane, cs);
+  if (E <= kRouteWarps * 32 * 2)
+    gate_logit = slice_topk<2>(tlog, E, K, gated, timeout_ns, tag, warp, lane, cs);
   else
     gate_logit = slice_topk<kMaxExperts / (kRouteWarps * 32)>(tlog, E, K, gated, timeout_ns, tag, warp, lane, cs);
   FMOE_TRACE_WARP(14);
@@ -709,14 +709,19 @@ __device__ __noinline__ void cta_routing(const LayerArgs& a, CtaShared& cs, int 
   FMOE_TRACE_WARP(9);
   if (warp == 0) {
     // Stage 2: warp 0 selects the top K of the kRouteWarps * K candidates
-    // (the global top K is among them, ties included) with the same rounds,
-    // one candidate per lane; lane kk < K ends with the kk-th.
+    // (the global top K is among them, ties included) with the same rounds;
+    // lane kk < K ends with the kk-th.
     const int nc = kRouteWarps * K;
-    uint32_t ckey[1], cidx[1];
-    ckey[0] = lane < nc ? cs.cand_key[lane] : 0u;
-    cidx[0] = lane < nc ? cs.cand_idx[lane] : 0xffffffffu;
+    constexpr int kC = (kRouteWarps * kMaxTopK + 31) / 32;
+    uint32_t ckey[kC], cidx[kC];
+#pragma unroll
+    for (int i = 0; i < kC; ++i) {
+      const int c = i * 32 + lane;
+      ckey[i] = c < nc ? cs.cand_key[c] : 0u;
+      cidx[i] = c < nc ? cs.cand_idx[c] : 0xffffffffu;
+    }
     uint32_t hk, hi;
-    warp_select<1>(ckey, cidx, K, lane, hk, hi);
+    warp_select<kC>(ckey, cidx, K, lane, hk, hi);
     FMOE_TRACE_WARP(23);
     // w_k = exp(l_k - l_0) / sum_j exp(l_j - l_0): softmax restricted to the
     // selected experts, equal to softmax-then-renormalise.

@@ -878,6 +878,50 @@ def run_stream(args, cfg, rank, world, local_rank):
                         "ms_per_token": ms_max / steps, "gpu_launches": launches[0], "clocks": clk,
                         "h2d_bytes_per_step": h * 4 + h2d / steps,
                         "device_status": status})
+        if n_slots == cfg["default_slots"]:
+            # Independent layer inputs (each layer its own token stream): each
+            # step decoded layer after layer, and with every layer prepared
+            # while the previous one decodes (its misses copied meanwhile).
+            xs_ind = [torch.from_numpy(S.token_stream(SEED + 17 * (l + 1) + rank, n_tok, h, cfg["rho"])).pin_memory()
+                      for l in range(NLS)]
+            xin = [torch.empty(h, dtype=torch.float32, device=dev) for _ in range(NLS)]
+            route_stream = torch.cuda.Stream()
+            indep = {}
+            for mode in ("one_step", "prepared_ahead"):
+                def istep(j):
+                    for l in range(NLS):
+                        xin[l].copy_(xs_ind[l][j], non_blocking=True)
+                    stream.synchronize()
+                    if mode == "one_step":
+                        for l in range(NLS):
+                            st.decode(l, xin[l], xin[l], out=hbuf[l % 2], ws=ws, copy_stream=copy_stream)
+                    else:
+                        # layer l + 1 is routed and its misses copied while layer l decodes
+                        st.prepare(0, xin[0], route_stream=route_stream, copy_stream=copy_stream)
+                        for l in range(NLS):
+                            st.finish(l, xin[l], xin[l], out=hbuf[l % 2], ws=ws)
+                            if l + 1 < NLS:
+                                st.prepare(l + 1, xin[l + 1], route_stream=route_stream, copy_stream=copy_stream)
+                    out_host.copy_(hbuf[(NLS - 1) % 2], non_blocking=True)
+                    stream.synchronize()
+                for j in range(args.warmup):
+                    istep(j)
+                q0 = st.stats()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for j in range(args.warmup, n_tok):
+                    istep(j)
+                e1.record()
+                torch.cuda.synchronize()
+                q1 = st.stats()
+                ims = e0.elapsed_time(e1)
+                hh, mm = q1["hits"] - q0["hits"], q1["misses"] - q0["misses"]
+                (ims_max,) = max_over_ranks([ims], world, dev)
+                indep[mode] = {"tokens_per_s": whole_job_rate(steps, world, ims_max), "ms_per_token": ims_max / steps,
+                               "hit_rate": hh / max(1, hh + mm),
+                               "h2d_gbs": (q1["h2d_bytes"] - q0["h2d_bytes"]) / (ims / 1000.0) / 1e9}
+            results[-1]["independent_layer_inputs"] = indep
         del st, slots
         torch.cuda.empty_cache()
     if rank == 0:

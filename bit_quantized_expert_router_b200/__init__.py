@@ -29,7 +29,7 @@ EXPORTED = [
     "fmoe_layer_decode_noalloc", "fmoe_set_wait_limit_ns", "fmoe_set_dependent_launch", "fmoe_delta_update",
     "fmoe_cache_create", "fmoe_cache_destroy", "fmoe_cache_lookup", "fmoe_cache_stats", "fmoe_cache_reset",
     "fmoe_experts_decode", "fmoe_streamer_create", "fmoe_streamer_decode", "fmoe_streamer_stats",
-    "fmoe_streamer_destroy",
+    "fmoe_streamer_destroy", "fmoe_streamer_prepare", "fmoe_streamer_finish",
 ]
 
 
@@ -95,6 +95,8 @@ def lib() -> ctypes.CDLL:
     L.fmoe_cache_reset.argtypes = [vp]
     L.fmoe_streamer_create.argtypes = [ctypes.POINTER(FmoeLayerC), i, ctypes.POINTER(vp), vp, i, ctypes.POINTER(vp)]
     L.fmoe_streamer_decode.argtypes = [vp, i, vp, vp, vp, vp, sz, vp, vp, vp, vp]
+    L.fmoe_streamer_prepare.argtypes = [vp, i, vp, vp, vp, vp, vp]
+    L.fmoe_streamer_finish.argtypes = [vp, i, vp, vp, vp, vp, sz, vp]
     L.fmoe_streamer_stats.argtypes = [vp, u64p, u64p, u64p]
     L.fmoe_streamer_destroy.argtypes = [vp]
     L.fmoe_last_cuda_error.argtypes = []
@@ -104,7 +106,7 @@ def lib() -> ctypes.CDLL:
     for name in ("fmoe_blob_offsets", "fmoe_quantize_expert", "fmoe_route", "fmoe_expert_forward",
                  "fmoe_workspace_init", "fmoe_layer_decode", "fmoe_get_status", "fmoe_layer_decode_noalloc",
                  "fmoe_experts_decode", "fmoe_streamer_create", "fmoe_streamer_decode", "fmoe_streamer_stats",
-                 "fmoe_streamer_destroy"):
+                 "fmoe_streamer_destroy", "fmoe_streamer_prepare", "fmoe_streamer_finish"):
         getattr(L, name).restype = i
     _lib = L
     return L
@@ -433,6 +435,32 @@ class Streamer:
                                           ws.data_ptr(), ws.numel(), cs, ks, idx.ctypes.data, w.ctypes.data),
                "fmoe_streamer_decode")
         return (out, idx, w) if return_routing else out
+
+    def prepare(self, layer: int, x: torch.Tensor, route_stream=None, copy_stream=None):
+        """Route x for `layer` and start its misses' copies; returns the
+        routing decision (host arrays idx, w)."""
+        L = self.layers[layer]
+        x = _dev_tensor(x, torch.float32, "x")
+        idx = np.empty(L.top_k, dtype=np.int32)
+        w = np.empty(L.top_k, dtype=np.float32)
+        rs = _stream(route_stream)
+        ks = rs if copy_stream is None else copy_stream.cuda_stream
+        _check(lib().fmoe_streamer_prepare(self._h, int(layer), x.data_ptr(), rs, ks, idx.ctypes.data, w.ctypes.data),
+               "fmoe_streamer_prepare")
+        return idx, w
+
+    def finish(self, layer: int, x: torch.Tensor, residual: torch.Tensor | None = None,
+               out: torch.Tensor | None = None, ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """Decode the oldest prepared layer (`layer`, with the same x)."""
+        L = self.layers[layer]
+        x = _dev_tensor(x, torch.float32, "x")
+        if out is None:
+            out = torch.empty_like(x)
+        if ws is None:
+            ws = L.workspace(1)
+        _check(lib().fmoe_streamer_finish(self._h, int(layer), x.data_ptr(), _ptr(residual), out.data_ptr(),
+                                          ws.data_ptr(), ws.numel(), _stream(stream)), "fmoe_streamer_finish")
+        return out
 
     def stats(self) -> dict:
         v = [ctypes.c_uint64(0) for _ in range(3)]

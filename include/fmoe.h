@@ -378,11 +378,33 @@ int fmoe_streamer_create(const fmoe_layer* layers, int n_layers, const void* con
  * slot is overwritten only after the kernels that read it, which that stream
  * orders).  The call synchronises `stream` once, so it cannot be captured
  * into a graph.  idx_out_opt, w_out_opt: optional HOST arrays [top_k] that
- * receive the routing decision.  Errors: FMOE_EINVAL, FMOE_ENOMEM,
+ * receive the routing decision.  No layer may be prepared and unfinished
+ * (see fmoe_streamer_prepare).  Errors: FMOE_EINVAL, FMOE_ENOMEM,
  * FMOE_ECUDA; kernel-side problems as fmoe_layer_decode. */
 int fmoe_streamer_decode(fmoe_streamer* s, int layer, const float* x, const float* residual, float* out, void* ws,
                          size_t ws_bytes, fmoe_stream_t stream, fmoe_stream_t copy_stream, int32_t* idx_out_opt,
                          float* w_out_opt);
+
+/* fmoe_streamer_decode in two halves, for callers that know the next layer's
+ * input before this layer's decode is done (independent layer inputs): a
+ * layer prepared while the previous one decodes copies its misses during
+ * that decode ([P2] "Verzögerte GPU-Experten-Berechnung": the host prepares
+ * the next layer while the GPU computes).
+ * fmoe_streamer_prepare: steps 1 and 2 for `layer` and its input x (device,
+ * ready on route_stream): the routing kernels on route_stream, the decision
+ * to the host (synchronises route_stream), the directory lookup and the
+ * misses' copies on copy_stream, each after the last decode that read its
+ * slot.  At most two layers may be prepared and not yet finished, and a
+ * second one needs n_slots >= 2 * top_k (so that it cannot evict the first
+ * one's experts).  idx_out_opt, w_out_opt: optional HOST arrays [top_k].
+ * fmoe_streamer_finish: step 3 for the oldest prepared layer (`layer` must
+ * be it; x the same input), on stream; it returns once the launches are
+ * queued.  Use one copy stream for all calls of a streamer.  Errors:
+ * FMOE_EINVAL (including a call out of order), FMOE_ENOMEM, FMOE_ECUDA. */
+int fmoe_streamer_prepare(fmoe_streamer* s, int layer, const float* x, fmoe_stream_t route_stream,
+                          fmoe_stream_t copy_stream, int32_t* idx_out_opt, float* w_out_opt);
+int fmoe_streamer_finish(fmoe_streamer* s, int layer, const float* x, const float* residual, float* out, void* ws,
+                         size_t ws_bytes, fmoe_stream_t stream);
 
 /* Running totals: expert hits and misses (the directory's) and bytes copied
  * from host to device (each pointer optional). */

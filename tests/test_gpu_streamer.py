@@ -127,3 +127,56 @@ def test_streamer_rejects_pageable_host_memory(F):
     h = ctypes.c_void_p()
     assert F.lib().fmoe_streamer_create(arr, 1, hp, slots.data_ptr(), 4, ctypes.byref(h)) == F.FMOE_EINVAL
     assert not h.value
+
+
+def test_streamer_prepared_ahead_matches_oracle_and_serial(F):
+    """Layers with independent inputs, each prepared while the previous one
+    decodes (its misses copied during that decode): every output matches the
+    oracle, the hit/miss sequence and the outputs equal the one-step decode's
+    in the same order, and calls out of order are refused."""
+    shape = C.Shape("stream_h512_i128_e12_k4", 512, 128, 12, 4, 4)
+    seed, n_layers, n_tokens = 67, 2, 6
+    layers, hosts = make_streamed_layers(F, shape, seed, n_layers, True)
+    stride = hosts[0].shape[1]
+    H = shape.hidden
+    inputs = []
+    for t in range(n_tokens):
+        for l in range(n_layers):
+            wr = S.router_bf16(seed, l, shape.n_experts, H)
+            x = C.parity_x(seed, l, t, wr, shape.top_k, H)[0]
+            inputs.append((l, torch.from_numpy(x).to(dev()), x))
+    n_slots = 2 * shape.top_k  # the least a prepared-ahead layer needs
+    piped = F.Streamer(layers, hosts, torch.zeros(n_slots, stride, dtype=torch.uint8, device=dev()))
+    serial = F.Streamer(layers, hosts, torch.zeros(n_slots, stride, dtype=torch.uint8, device=dev()))
+    copy_a, copy_b, route_s = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ws = layers[0].workspace(1)
+    outs = [torch.empty(H, device=dev()) for _ in inputs]
+    routes = [None] * len(inputs)
+    l0, xd0, _ = inputs[0]
+    routes[0] = piped.prepare(l0, xd0, route_stream=route_s, copy_stream=copy_a)
+    for i, (l, xd, _) in enumerate(inputs):
+        if i + 1 < len(inputs):
+            ln, xn, _ = inputs[i + 1]
+            routes[i + 1] = piped.prepare(ln, xn, route_stream=route_s, copy_stream=copy_a)
+            # a third layer may not be prepared while two are pending
+            with pytest.raises(F.FmoeError):
+                piped.prepare(ln, xn, route_stream=route_s, copy_stream=copy_a)
+        piped.finish(l, xd, out=outs[i], ws=ws)
+    torch.cuda.synchronize()
+    assert F.get_status() == 0
+    for i, (l, xd, x) in enumerate(inputs):
+        r = C.oracle_layer(seed, l, shape, x, np.zeros(H, dtype=np.float32))
+        assert routes[i][0].tolist() == r["idx"].tolist()
+        C.assert_close(outs[i].cpu().numpy(), r["out"], f"prepared-ahead input {i}")
+        ys = serial.decode(l, xd, copy_stream=copy_b)
+        assert torch.equal(ys, outs[i]), f"input {i}: prepared-ahead and one-step decodes differ"
+    assert piped.stats() == serial.stats()
+    # finishing a layer that is not the oldest prepared one is refused
+    piped.prepare(0, inputs[0][1], route_stream=route_s, copy_stream=copy_a)
+    with pytest.raises(F.FmoeError):
+        piped.finish(1, inputs[1][1], ws=ws)
+    with pytest.raises(F.FmoeError):  # and so is a one-step decode while a layer is prepared
+        piped.decode(1, inputs[1][1], copy_stream=copy_a)
+    piped.finish(0, inputs[0][1], ws=ws)
+    torch.cuda.synchronize()
+    assert F.get_status() == 0

@@ -167,7 +167,7 @@ size_t layer_ws_bytes() { return kHeaderBytes; }
 // Workspace of the grouped (T >= 2) decode, byte offsets (every section 256-B aligned).
 struct GroupedLayout {
   size_t logits, meta, slot_expert, slot_pair0, pair_token, pair_slot, pair_nk, tok_pair, tok_w, tok_sg;
-  size_t xs_r, sf_r, xs_s, sf_s, gu_part, as, sfa, y_part, sh_gu, sh_y, xn, total;
+  size_t sched, xs_r, sf_r, xs_s, sf_s, gu_part, as, sfa, y_part, sh_gu, sh_y, xn, total;
 };
 
 GroupedLayout grouped_layout(int E, int H, int I, int K, int T) {
@@ -189,6 +189,7 @@ GroupedLayout grouped_layout(int E, int H, int I, int K, int T) {
   g.tok_pair = take((size_t)T * (K + 1) * 4);
   g.tok_w = take((size_t)T * K * 4);
   g.tok_sg = take((size_t)T * 4);
+  g.sched = take((size_t)2 * kSchedInts * 4);
   g.xs_r = take((size_t)T * H * 4);
   g.sf_r = take((size_t)T * (H / 32) * 8);
   g.xs_s = take((size_t)T * H * 4);
@@ -228,6 +229,7 @@ int launch_grouped(const fmoe_layer* L, const float* x, const float* residual, f
   const bool has_shared = L->shared != nullptr;
   const int br = L->bits, bs = has_shared ? L->shared_bits : L->bits;
   const GroupedLayout gl = grouped_layout(E, H, I, K, T);
+  if (G > kMaxSchedCtas) return FMOE_EINVAL;  // (more SMs than the unit schedule holds CTAs)
   char* w8 = static_cast<char*>(ws);
   GroupArgs a;
   std::memset(&a, 0, sizeof(a));
@@ -250,6 +252,7 @@ int launch_grouped(const fmoe_layer* L, const float* x, const float* residual, f
   a.tb.tok_pair = reinterpret_cast<int*>(w8 + gl.tok_pair);
   a.tb.tok_w = reinterpret_cast<float*>(w8 + gl.tok_w);
   a.tb.tok_sg = reinterpret_cast<float*>(w8 + gl.tok_sg);
+  a.tb.sched = reinterpret_cast<int*>(w8 + gl.sched);
   a.xs_r = reinterpret_cast<float4*>(w8 + gl.xs_r);
   a.sf_r = reinterpret_cast<float2*>(w8 + gl.sf_r);
   const bool separate = has_shared && bs != br;
@@ -274,6 +277,7 @@ int launch_grouped(const fmoe_layer* L, const float* x, const float* residual, f
   a.E = E;
   a.K = K;
   a.T = T;
+  a.grid = G;
   a.bits_r = br;
   a.bits_s = bs;
   a.has_sgate = L->w_sgate != nullptr;

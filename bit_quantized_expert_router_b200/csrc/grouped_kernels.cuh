@@ -43,6 +43,13 @@ constexpr int kMaxChunks = 8;              // input chunks per slot, at most
 constexpr int kChunkBudget = 32 << 10;     // bytes of staged inputs of one (slot, chunk)
 constexpr int kUnitCostBase = 2;           // unit cost = chunk length * (kUnitCostBase + tokens)
 constexpr int kRouterRows = 4;             // router rows per CTA
+constexpr int kMaxSchedCtas = 1024;        // CTAs of the gate/up and down grids, at most
+// Unit schedule of one grid (gate/up or down), ints: every slot's input
+// chunks and inputs per chunk, every slot's first unit (and the total), every
+// CTA's first unit (and the total).
+constexpr int kSchedNk = 0, kSchedCl = kMaxPairs + 1, kSchedUbase = 2 * (kMaxPairs + 1);
+constexpr int kSchedRange = kSchedUbase + kMaxPairs + 2;
+constexpr int kSchedInts = kSchedRange + kMaxSchedCtas + 1;
 
 // Chunks the n_in inputs of a slot with n_tok tokens are split into: the
 // fewest (a divisor of n_in / 64, at most kMaxChunks) that keep n_tok chunks of
@@ -69,6 +76,7 @@ struct GroupTables {
   int* tok_pair;     // [T][K + 1] pair of (t, k); column K: the shared pair (-1 if none)
   float* tok_w;      // [T][K]
   float* tok_sg;     // [T]
+  int* sched;        // [2][kSchedInts] unit schedules of the gate/up (0) and down (1) grids
 };
 
 struct GroupArgs {
@@ -95,6 +103,7 @@ struct GroupArgs {
   float* sh_gu;     // tensor-core shared expert: [2][H/512][16][I] gate/up partials
   float* sh_y;      // [I/512][16][H] down partials
   int H, I, E, K, T, bits_r, bits_s;
+  int grid;         // CTAs of the gate/up and down grids
   int has_sgate;
   int shared_tc;    // the shared expert runs on the tensor cores (not as a slot)
   int nst, stage_bytes;      // gate/up ring
@@ -212,6 +221,65 @@ __global__ void __launch_bounds__(kNormThreads) rms_norm_tokens_kernel(const flo
 }
 
 // ---------------------------------------------------------------------------
+// Unit schedules of the gate/up (q = 0: kin = H inputs, ru = I row units per
+// chunk) and down (q = 1: kin = I, ru = H / kRC) grids.  The units of slot s
+// are its input chunks x ru row units, chunk-major; slot after slot in slot
+// order.  A unit costs (kin / chunks) * (kUnitCostBase + tokens of the slot)
+// (bytes read plus per-token work); CTA b of G takes the units whose cost
+// intervals start in [total * b / G, total * (b + 1) / G).  Computed once by
+// all threads of the grouping CTA: per-slot values in parallel, prefix sums by
+// one thread per slot, each CTA's first unit by one thread per CTA.
+// ---------------------------------------------------------------------------
+__device__ __noinline__ void schedule_units(const GroupArgs& a) {
+  __shared__ long long s_cost[2][kMaxPairs + 2];  // cost of slot s, then cost before slot s
+  __shared__ int s_units[2][kMaxPairs + 2];       // units of slot s, then units before slot s
+  __shared__ int s_n[kMaxPairs + 1];
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int ns = a.tb.meta[0], G = a.grid;
+  for (int i = tid; i < 2 * ns; i += nt) {
+    const int q = i / ns, s = i - q * ns;
+    const int kin = q ? a.I : a.H, ru = q ? a.H / kRC : a.I;
+    const int n = a.tb.slot_pair0[s + 1] - a.tb.slot_pair0[s];
+    const int nk = input_chunks(n, kin);
+    if (q == 0) s_n[s] = n;
+    a.tb.sched[q * kSchedInts + kSchedNk + s] = nk;
+    a.tb.sched[q * kSchedInts + kSchedCl + s] = kin / nk;
+    s_units[q][s] = nk * ru;
+    s_cost[q][s] = (long long)ru * kin * (kUnitCostBase + n);
+  }
+  __syncthreads();
+  long long cb = 0;
+  int ub = 0;
+  const int q0 = tid / (ns + 1), s0 = tid - q0 * (ns + 1);
+  if (tid < 2 * (ns + 1)) {  // sums over the slots before s0
+    for (int j = 0; j < s0; ++j) {
+      cb += s_cost[q0][j];
+      ub += s_units[q0][j];
+    }
+    a.tb.sched[q0 * kSchedInts + kSchedUbase + s0] = ub;
+  }
+  __syncthreads();
+  if (tid < 2 * (ns + 1)) {
+    s_cost[q0][s0] = cb;
+    s_units[q0][s0] = ub;
+  }
+  __syncthreads();
+  for (int i = tid; i < 2 * (G + 1); i += nt) {
+    const int q = i / (G + 1), b = i - q * (G + 1);
+    const long long target = s_cost[q][ns] * b / G;
+    int u = s_units[q][ns];  // first unit whose cost interval starts at or after target
+    for (int s = 0; s < ns; ++s) {
+      if (target < s_cost[q][s + 1]) {
+        const long long uc = (long long)a.tb.sched[q * kSchedInts + kSchedCl + s] * (kUnitCostBase + s_n[s]);
+        u = s_units[q][s] + (int)((target - s_cost[q][s] + uc - 1) / uc);
+        break;
+      }
+    }
+    a.tb.sched[q * kSchedInts + kSchedRange + b] = u;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // prep: top-K per token, grouping, input staging
 // ---------------------------------------------------------------------------
 // CTA `b` of the prep step (0 <= b <= T): b = 0 routes and groups, b > 0
@@ -305,6 +373,8 @@ __device__ __noinline__ void prep_cta(const GroupArgs& a, int b) {
     a.tb.meta[0] = ns;
     a.tb.meta[1] = np;
   }
+  __syncthreads();  // (the tables above are read back by this CTA's threads)
+  schedule_units(a);
 }
 
 template <int BR, int BS>
@@ -320,56 +390,47 @@ struct CtaSched {
   int ns;
   int* pair0;   // [ns + 1]
   int* expert;  // [ns]
-  int* nk;      // [ns]
+  int* nk;      // [ns] input chunks
+  int* cl;      // [ns] inputs per chunk
   int* ubase;   // [ns + 1] units before slot s
+  int* ptok;    // [pairs] token of each pair
   int u0, u1;   // this CTA's units
 };
 
-// Load the slot tables and cut this CTA's range; all threads call it.
-__device__ inline void cta_sched(const GroupArgs& a, int kin, int ru, CtaSched& cs, int* s_pair0, int* s_expert,
-                                 int* s_nk, int* s_ubase, int* s_range) {
+// Shared-memory copies of the slot tables, declared by each grid's kernel.
+struct SchedSmem {
+  int pair0[kMaxPairs + 2], expert[kMaxPairs + 1], nk[kMaxPairs + 1], cl[kMaxPairs + 1], ubase[kMaxPairs + 2];
+  int ptok[kMaxPairs];
+  int range[2];
+};
+
+// Load the slot tables and this CTA's unit range of grid q (0 gate/up, 1
+// down) from the schedule the grouping step computed; all threads call it.
+__device__ inline void cta_sched(const GroupArgs& a, int q, CtaSched& cs, SchedSmem& sm) {
   const int tid = threadIdx.x;
-  const int ns = a.tb.meta[0];
+  const int ns = a.tb.meta[0], np = a.tb.meta[1];
+  const int* t = a.tb.sched + q * kSchedInts;
   for (int s = tid; s <= ns; s += blockDim.x) {
-    s_pair0[s] = a.tb.slot_pair0[s];
-    if (s < ns) s_expert[s] = a.tb.slot_expert[s];
-  }
-  __syncthreads();
-  if (tid == 0) {
-    long long total = 0;
-    int ub = 0;
-    for (int s = 0; s < ns; ++s) {
-      const int n = s_pair0[s + 1] - s_pair0[s];
-      s_nk[s] = input_chunks(n, kin);
-      s_ubase[s] = ub;
-      ub += s_nk[s] * ru;
-      total += (long long)ru * kin * (kUnitCostBase + n);
+    sm.pair0[s] = a.tb.slot_pair0[s];
+    sm.ubase[s] = t[kSchedUbase + s];
+    if (s < ns) {
+      sm.expert[s] = a.tb.slot_expert[s];
+      sm.nk[s] = t[kSchedNk + s];
+      sm.cl[s] = t[kSchedCl + s];
     }
-    s_ubase[ns] = ub;
-    // first unit whose cost interval starts at or after `target`
-    auto first_unit = [&](long long target) {
-      long long cc = 0;
-      for (int s = 0; s < ns; ++s) {
-        const int n = s_pair0[s + 1] - s_pair0[s];
-        const long long uc = (long long)(kin / s_nk[s]) * (kUnitCostBase + n);
-        const long long span = uc * s_nk[s] * ru;
-        if (target < cc + span) return s_ubase[s] + (int)((target - cc + uc - 1) / uc);
-        cc += span;
-      }
-      return s_ubase[ns];
-    };
-    const long long G = gridDim.x, b = blockIdx.x;
-    s_range[0] = first_unit(total * b / G);
-    s_range[1] = first_unit(total * (b + 1) / G);
   }
+  for (int p = tid; p < np; p += blockDim.x) sm.ptok[p] = a.tb.pair_token[p];
+  if (tid < 2) sm.range[tid] = t[kSchedRange + blockIdx.x + tid];
   __syncthreads();
   cs.ns = ns;
-  cs.pair0 = s_pair0;
-  cs.expert = s_expert;
-  cs.nk = s_nk;
-  cs.ubase = s_ubase;
-  cs.u0 = s_range[0];
-  cs.u1 = s_range[1];
+  cs.pair0 = sm.pair0;
+  cs.expert = sm.expert;
+  cs.nk = sm.nk;
+  cs.cl = sm.cl;
+  cs.ubase = sm.ubase;
+  cs.ptok = sm.ptok;
+  cs.u0 = sm.range[0];
+  cs.u1 = sm.range[1];
 }
 
 // (slot, chunk, row unit) of unit u; `s` is a cursor that only moves forward.
@@ -607,95 +668,113 @@ __device__ __forceinline__ void down_dot_chunk2(const char* stA, const char* stB
 // ---------------------------------------------------------------------------
 // gate/up
 // ---------------------------------------------------------------------------
+// Ring position of a warp's unit: stage index and the phase parity its
+// mbarrier completes with; advanced one unit at a time (no divisions).
+struct RingPos {
+  int idx;
+  uint32_t ph;
+};
+__device__ __forceinline__ void ring_next(RingPos& r, int n) {
+  if (++r.idx == n) {
+    r.idx = 0;
+    r.ph ^= 1u;
+  }
+}
+
 template <int BR, int BS>
 __global__ void __launch_bounds__(kThreads, 1) grouped_gateup_kernel(const __grid_constant__ GroupArgs a) {
   extern __shared__ __align__(128) char smem_raw[];
-  __shared__ int s_pair0[kMaxPairs + 2], s_expert[kMaxPairs + 1], s_nk[kMaxPairs + 1], s_ubase[kMaxPairs + 2];
-  __shared__ int s_range[2];
+  __shared__ SchedSmem ss;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  char* my_ring = smem_raw + (size_t)warp * a.nst * a.stage_bytes;
-  uint64_t* my_bars = reinterpret_cast<uint64_t*>(smem_raw + (size_t)kWarps * a.nst * a.stage_bytes) + warp * a.nst;
+  const int nst = a.nst, stage_bytes = a.stage_bytes;
+  char* my_ring = smem_raw + (size_t)warp * nst * stage_bytes;
+  uint64_t* my_bars = reinterpret_cast<uint64_t*>(smem_raw + (size_t)kWarps * nst * stage_bytes) + warp * nst;
   if (lane == 0) {
-    for (int s = 0; s < a.nst; ++s) mbar_init(&my_bars[s], 1);
+    for (int s = 0; s < nst; ++s) mbar_init(&my_bars[s], 1);
     fence_proxy_async_smem();
   }
   CtaSched cs;
-  cta_sched(a, a.H, a.I, cs, s_pair0, s_expert, s_nk, s_ubase, s_range);  // includes __syncthreads
+  cta_sched(a, 0, cs, ss);  // includes __syncthreads
   // this warp's units: cs.u0 + warp + i * kWarps
   const int n = cs.u1 - cs.u0 > warp ? (cs.u1 - cs.u0 - warp - 1) / kWarps + 1 : 0;
-  const int sbr = sb_row_bytes(a.H), cap = sb_superset_cap(a.H);
+  const int H = a.H, I = a.I;
+  const int sbr = sb_row_bytes(H), cap = sb_superset_cap(H);
+  // Section offsets of both code widths; the up section's scale/bias words lie
+  // a multiple of 16 bytes after the gate section's (code and scale/bias
+  // sections are whole multiples of 16 bytes), so a row chunk's gate and up
+  // scale/bias copies share their alignment and length.
+  const long long gc_r = a.off_r[0], gsb_r = a.off_r[1], uc_r = a.off_r[2], usb_r = a.off_r[3];
+  const long long gc_s = a.off_s[0], gsb_s = a.off_s[1], uc_s = a.off_s[2], usb_s = a.off_s[3];
 
-  UnitCursor ki = cursor_at(cs, a.I, cs.u0 + warp);  // next unit to issue
-  auto issue = [&](int i) {  // lane 0; units are issued in order
+  UnitCursor ki = cursor_at(cs, I, cs.u0 + warp);  // next unit to issue
+  int ri = 0;                                       // its ring stage
+  auto issue = [&]() {  // lane 0; units are issued in order
     const int s = ki.s, c = ki.c, row = ki.r;
-    cursor_step(cs, a.I, ki);
+    cursor_step(cs, I, ki);
     const int e = cs.expert[s];
-    const int bits = e >= 0 ? BR : BS;
-    const char* blob = e >= 0 ? a.experts + (long long)e * a.expert_stride : a.shared;
-    const long long* o = e >= 0 ? a.off_r : a.off_s;
-    const int cl = a.H / cs.nk[s];  // inputs per chunk
-    const int cb = cl * bits / 8;
-    const long long code0 = (long long)row * (a.H * bits / 8) + (long long)c * cb;
-    const long long gs0 = o[1] + (long long)row * sbr + c * (cl / 16), us0 = o[3] + (long long)row * sbr + c * (cl / 16);
-    const long long ga = gs0 & ~15LL, ua = us0 & ~15LL;
-    const int glen = (int)(((gs0 + cl / 16 + 15) & ~15LL) - ga);
-    const int ulen = (int)(((us0 + cl / 16 + 15) & ~15LL) - ua);
-    char* stage = my_ring + (size_t)(i % a.nst) * a.stage_bytes;
-    uint64_t* bar = &my_bars[i % a.nst];
-    mbar_arrive_expect_tx(bar, 2 * cb + glen + ulen);
-    bulk_g2s(stage, blob + o[0] + code0, cb, bar);
-    bulk_g2s(stage + cb, blob + o[2] + code0, cb, bar);
-    bulk_g2s(stage + 2 * cb, blob + ga, glen, bar);
-    bulk_g2s(stage + 2 * cb + cap, blob + ua, ulen, bar);
+    const bool routed = e >= 0;
+    const char* blob = routed ? a.experts + (long long)e * a.expert_stride : a.shared;
+    const int cl = cs.cl[s];
+    const int cb = routed ? cl * BR / 8 : cl * BS / 8;
+    const int rowb = routed ? H * BR / 8 : H * BS / 8;
+    const long long code0 = (long long)row * rowb + c * cb;
+    const long long gs0 = (routed ? gsb_r : gsb_s) + (long long)row * sbr + ((c * cl) >> 4);
+    const long long ga = gs0 & ~15LL;
+    const int len = (((int)gs0 & 15) + (cl >> 4) + 15) & ~15;
+    char* stage = my_ring + ri * stage_bytes;
+    uint64_t* bar = &my_bars[ri];
+    if (++ri == nst) ri = 0;
+    mbar_arrive_expect_tx(bar, 2 * cb + 2 * len);
+    bulk_g2s(stage, blob + (routed ? gc_r : gc_s) + code0, cb, bar);
+    bulk_g2s(stage + cb, blob + (routed ? uc_r : uc_s) + code0, cb, bar);
+    bulk_g2s(stage + 2 * cb, blob + ga, len, bar);
+    bulk_g2s(stage + 2 * cb + cap, blob + ga + (routed ? usb_r - gsb_r : usb_s - gsb_s), len, bar);
   };
   if (lane == 0)
-    for (int i = 0; i < n && i < a.nst; ++i) issue(i);
+    for (int i = 0; i < n && i < nst; ++i) issue();
 
-  UnitCursor kc = cursor_at(cs, a.I, cs.u0 + warp);  // unit being computed
+  UnitCursor kc = cursor_at(cs, I, cs.u0 + warp);  // unit being computed
+  RingPos rc{0, 0u};                                // its ring stage
   for (int i = 0; i < n;) {
     // Two consecutive units of the same slot and input chunk are computed in
     // one pass (each input load then serves four rows).
     UnitCursor kn = kc;
-    cursor_step(cs, a.I, kn);
-    const bool two = a.nst >= 2 && i + 1 < n && kn.s == kc.s && kn.c == kc.c;
-    const char* stage = my_ring + (size_t)(i % a.nst) * a.stage_bytes;
-    const char* stage2 = my_ring + (size_t)((i + 1) % a.nst) * a.stage_bytes;
-    if (!mbar_wait_bounded(&my_bars[i % a.nst], (i / a.nst) & 1, a.timeout_ns) && lane == 0)
-      set_status(kStatusCopyTimeout);
-    if (two && !mbar_wait_bounded(&my_bars[(i + 1) % a.nst], ((i + 1) / a.nst) & 1, a.timeout_ns) && lane == 0)
+    cursor_step(cs, I, kn);
+    const bool two = nst >= 2 && i + 1 < n && kn.s == kc.s && kn.c == kc.c;
+    RingPos r2 = rc;
+    ring_next(r2, nst);
+    const char* stage = my_ring + rc.idx * stage_bytes;
+    const char* stage2 = my_ring + r2.idx * stage_bytes;
+    if (!mbar_wait_bounded(&my_bars[rc.idx], rc.ph, a.timeout_ns) && lane == 0) set_status(kStatusCopyTimeout);
+    if (two && !mbar_wait_bounded(&my_bars[r2.idx], r2.ph, a.timeout_ns) && lane == 0)
       set_status(kStatusCopyTimeout);
     const int s = kc.s, c = kc.c, row = kc.r, row2 = kn.r;
     const bool routed = cs.expert[s] >= 0;
-    const int cl = a.H / cs.nk[s];
-    const long long* o = routed ? a.off_r : a.off_s;
-    const int sbo_g = (int)((o[1] + (long long)row * sbr + c * (cl / 16)) & 15);
-    const int sbo_u = (int)((o[3] + (long long)row * sbr + c * (cl / 16)) & 15);
-    const int sbo_g2 = (int)((o[1] + (long long)row2 * sbr + c * (cl / 16)) & 15);
-    const int sbo_u2 = (int)((o[3] + (long long)row2 * sbr + c * (cl / 16)) & 15);
+    const int cl = cs.cl[s];
+    const int sb_c = (int)(routed ? gsb_r : gsb_s) + ((c * cl) >> 4);
+    const int sbo = (sb_c + row * sbr) & 15, sbo2 = (sb_c + row2 * sbr) & 15;
     for (int p = cs.pair0[s]; p < cs.pair0[s + 1]; ++p) {
-      const int t = a.tb.pair_token[p];
+      const int t = cs.ptok[p];
       float g, up;
-      float2* dst = a.gu_part + ((long long)p * kMaxChunks + c) * a.I;
+      float2* dst = a.gu_part + ((long long)p * kMaxChunks + c) * I;
       if (routed || BR == BS) {
         constexpr int CPV = 128 / BR;
-        const float4* xs = a.xs_r + (long long)t * (a.H / 4);
-        const float2* sf = a.sf_r + (long long)t * (a.H / CPV);
+        const float4* xs = a.xs_r + (long long)t * (H / 4);
+        const float2* sf = a.sf_r + (long long)t * (H / CPV);
         if (two)
-          gu_dot_chunk2<BR>(stage, stage2, cl / CPV, cl * BR / 8, cap, sbo_g, sbo_u, sbo_g2, sbo_u2, xs, a.H / CPV,
+          gu_dot_chunk2<BR>(stage, stage2, cl / CPV, cl * BR / 8, cap, sbo, sbo, sbo2, sbo2, xs, H / CPV,
                             c * (cl / CPV), sf, lane, g, up);
         else
-          gu_dot_chunk<BR>(stage, cl / CPV, cl * BR / 8, cap, sbo_g, sbo_u, xs, a.H / CPV, c * (cl / CPV), sf, lane,
-                           g, up);
+          gu_dot_chunk<BR>(stage, cl / CPV, cl * BR / 8, cap, sbo, sbo, xs, H / CPV, c * (cl / CPV), sf, lane, g, up);
       } else {
         constexpr int CPV = 128 / BS;
-        const float4* xs = a.xs_s + (long long)t * (a.H / 4);
-        const float2* sf = a.sf_s + (long long)t * (a.H / CPV);
+        const float4* xs = a.xs_s + (long long)t * (H / 4);
+        const float2* sf = a.sf_s + (long long)t * (H / CPV);
         if (two)
-          gu_dot_chunk2<BS>(stage, stage2, cl / CPV, cl * BS / 8, cap, sbo_g, sbo_u, sbo_g2, sbo_u2, xs, a.H / CPV,
+          gu_dot_chunk2<BS>(stage, stage2, cl / CPV, cl * BS / 8, cap, sbo, sbo, sbo2, sbo2, xs, H / CPV,
                             c * (cl / CPV), sf, lane, g, up);
         else
-          gu_dot_chunk<BS>(stage, cl / CPV, cl * BS / 8, cap, sbo_g, sbo_u, xs, a.H / CPV, c * (cl / CPV), sf, lane,
-                           g, up);
+          gu_dot_chunk<BS>(stage, cl / CPV, cl * BS / 8, cap, sbo, sbo, xs, H / CPV, c * (cl / CPV), sf, lane, g, up);
       }
       if (lane == 0) dst[row] = make_float2(g, up);
       if (two && lane == 16) dst[row2] = make_float2(g, up);
@@ -703,12 +782,16 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gateup_kernel(const __gri
     __syncwarp();
     if (lane == 0) {
       fence_proxy_async_smem();
-      if (i + a.nst < n) issue(i + a.nst);
-      if (two && i + 1 + a.nst < n) issue(i + 1 + a.nst);
+      if (i + nst < n) issue();
+      if (two && i + 1 + nst < n) issue();
     }
     i += two ? 2 : 1;
     kc = kn;
-    if (two) cursor_step(cs, a.I, kc);
+    rc = r2;
+    if (two) {
+      cursor_step(cs, I, kc);
+      ring_next(rc, nst);
+    }
   }
 }
 
@@ -750,107 +833,114 @@ __global__ void __launch_bounds__(kStageThreads) grouped_stage_act_kernel(const 
 template <int BR, int BS>
 __global__ void __launch_bounds__(kThreads, 1) grouped_down_kernel(const __grid_constant__ GroupArgs a) {
   extern __shared__ __align__(128) char smem_raw[];
-  __shared__ int s_pair0[kMaxPairs + 2], s_expert[kMaxPairs + 1], s_nk[kMaxPairs + 1], s_ubase[kMaxPairs + 2];
-  __shared__ int s_range[2];
+  __shared__ SchedSmem ss;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  char* my_ring = smem_raw + (size_t)warp * a.nst_c * a.c_stage_bytes;
-  uint64_t* my_bars =
-      reinterpret_cast<uint64_t*>(smem_raw + (size_t)kWarps * a.nst_c * a.c_stage_bytes) + warp * a.nst_c;
+  const int nst = a.nst_c, stage_bytes = a.c_stage_bytes;
+  char* my_ring = smem_raw + (size_t)warp * nst * stage_bytes;
+  uint64_t* my_bars = reinterpret_cast<uint64_t*>(smem_raw + (size_t)kWarps * nst * stage_bytes) + warp * nst;
   if (lane == 0) {
-    for (int s = 0; s < a.nst_c; ++s) mbar_init(&my_bars[s], 1);
+    for (int s = 0; s < nst; ++s) mbar_init(&my_bars[s], 1);
     fence_proxy_async_smem();
   }
-  const int nq = a.H / kRC;
+  const int H = a.H, I = a.I, nq = H / kRC;
   CtaSched cs;
-  cta_sched(a, a.I, nq, cs, s_pair0, s_expert, s_nk, s_ubase, s_range);
+  cta_sched(a, 1, cs, ss);
   const int n = cs.u1 - cs.u0 > warp ? (cs.u1 - cs.u0 - warp - 1) / kWarps + 1 : 0;
-  const int sbr = sb_row_bytes(a.I);  // bytes of one row's scale/bias words
+  const int sbr = sb_row_bytes(I);  // bytes of one row's scale/bias words
+  const long long dc_r = a.off_r[4], dsb_r = a.off_r[5], dc_s = a.off_s[4], dsb_s = a.off_s[5];
 
   UnitCursor ki = cursor_at(cs, nq, cs.u0 + warp);  // next unit to issue
-  auto issue = [&](int i) {  // lane 0; units are issued in order
+  int ri = 0;                                        // its ring stage
+  auto issue = [&]() {  // lane 0; units are issued in order
     const int s = ki.s, c = ki.c, q = ki.r;
     cursor_step(cs, nq, ki);
     const int e = cs.expert[s];
-    const int bits = e >= 0 ? BR : BS;
-    const char* blob = e >= 0 ? a.experts + (long long)e * a.expert_stride : a.shared;
-    const long long* o = e >= 0 ? a.off_r : a.off_s;
-    const int cl = a.I / cs.nk[s];
-    const int cb = cl * bits / 8, rowb = a.I * bits / 8;
-    const long long r0 = (long long)q * kRC;
-    char* stage = my_ring + (size_t)(i % a.nst_c) * a.c_stage_bytes;
-    uint64_t* bar = &my_bars[i % a.nst_c];
+    const bool routed = e >= 0;
+    const char* blob = routed ? a.experts + (long long)e * a.expert_stride : a.shared;
+    const int cl = cs.cl[s];
+    const int cb = routed ? cl * BR / 8 : cl * BS / 8;
+    const int rowb = routed ? I * BR / 8 : I * BS / 8;
+    const int r0 = q * kRC;
+    char* stage = my_ring + ri * stage_bytes;
+    uint64_t* bar = &my_bars[ri];
+    if (++ri == nst) ri = 0;
     // kRC code row chunks, then one copy covering the rows' scale/bias chunks
-    const long long sb0 = o[5] + r0 * sbr + c * (cl / 16);
+    const long long sb0 = (routed ? dsb_r : dsb_s) + (long long)r0 * sbr + ((c * cl) >> 4);
     const long long sba = sb0 & ~15LL;
-    const int sblen = (int)(((sb0 + (kRC - 1) * sbr + cl / 16 + 15) & ~15LL) - sba);
+    const int sblen = (((int)sb0 & 15) + (kRC - 1) * sbr + (cl >> 4) + 15) & ~15;
     mbar_arrive_expect_tx(bar, kRC * cb + sblen);
-    if (cs.nk[s] == 1) {
-      bulk_g2s(stage, blob + o[4] + r0 * rowb, kRC * cb, bar);
+    const char* codes = blob + (routed ? dc_r : dc_s) + (long long)r0 * rowb + c * cb;
+    if (cb == rowb) {
+      bulk_g2s(stage, codes, kRC * cb, bar);
     } else {
 #pragma unroll
-      for (int j = 0; j < kRC; ++j) bulk_g2s(stage + j * cb, blob + o[4] + (r0 + j) * rowb + (long long)c * cb, cb, bar);
+      for (int j = 0; j < kRC; ++j) bulk_g2s(stage + j * cb, codes + j * rowb, cb, bar);
     }
     bulk_g2s(stage + kRC * cb, blob + sba, sblen, bar);
   };
   if (lane == 0)
-    for (int i = 0; i < n && i < a.nst_c; ++i) issue(i);
+    for (int i = 0; i < n && i < nst; ++i) issue();
 
   UnitCursor kc = cursor_at(cs, nq, cs.u0 + warp);  // unit being computed
+  RingPos rc{0, 0u};                                 // its ring stage
   for (int i = 0; i < n;) {
     // Two consecutive units of the same slot and input chunk are computed in
     // one pass (each activation load then serves 2 * kRC rows).
     UnitCursor kn = kc;
     cursor_step(cs, nq, kn);
-    const bool two = a.nst_c >= 2 && i + 1 < n && kn.s == kc.s && kn.c == kc.c;
-    const char* stage = my_ring + (size_t)(i % a.nst_c) * a.c_stage_bytes;
-    const char* stage2 = my_ring + (size_t)((i + 1) % a.nst_c) * a.c_stage_bytes;
-    if (!mbar_wait_bounded(&my_bars[i % a.nst_c], (i / a.nst_c) & 1, a.timeout_ns) && lane == 0)
-      set_status(kStatusCopyTimeout);
-    if (two && !mbar_wait_bounded(&my_bars[(i + 1) % a.nst_c], ((i + 1) / a.nst_c) & 1, a.timeout_ns) && lane == 0)
+    const bool two = nst >= 2 && i + 1 < n && kn.s == kc.s && kn.c == kc.c;
+    RingPos r2 = rc;
+    ring_next(r2, nst);
+    const char* stage = my_ring + rc.idx * stage_bytes;
+    const char* stage2 = my_ring + r2.idx * stage_bytes;
+    if (!mbar_wait_bounded(&my_bars[rc.idx], rc.ph, a.timeout_ns) && lane == 0) set_status(kStatusCopyTimeout);
+    if (two && !mbar_wait_bounded(&my_bars[r2.idx], r2.ph, a.timeout_ns) && lane == 0)
       set_status(kStatusCopyTimeout);
     const int s = kc.s, c = kc.c, q = kc.r, q2 = kn.r;
     const bool routed = cs.expert[s] >= 0;
-    const int cl = a.I / cs.nk[s];
-    const long long sbbase = (routed ? a.off_r : a.off_s)[5] + c * (cl / 16);
-    const long long sb0 = sbbase + (long long)q * kRC * sbr, sb2 = sbbase + (long long)q2 * kRC * sbr;
-    const int bits = routed ? BR : BS;
-    const int cb = cl * bits / 8;
-    const uint32_t* sbw = reinterpret_cast<const uint32_t*>(stage + kRC * cb + (sb0 & 15));
-    const uint32_t* sbw2 = reinterpret_cast<const uint32_t*>(stage2 + kRC * cb + (sb2 & 15));
+    const int cl = cs.cl[s];
+    const int sb_c = (int)(routed ? dsb_r : dsb_s) + ((c * cl) >> 4);
+    const int cb = routed ? cl * BR / 8 : cl * BS / 8;
+    const uint32_t* sbw = reinterpret_cast<const uint32_t*>(stage + kRC * cb + ((sb_c + q * kRC * sbr) & 15));
+    const uint32_t* sbw2 = reinterpret_cast<const uint32_t*>(stage2 + kRC * cb + ((sb_c + q2 * kRC * sbr) & 15));
     for (int p = cs.pair0[s]; p < cs.pair0[s + 1]; ++p) {
       float y[kRC], y2 = 0.f;
-      const float4* as = a.as + (long long)p * (a.I / 4);
-      const float2* sf = a.sfa + (long long)p * (a.I / 32);
+      const float4* as = a.as + (long long)p * (I / 4);
+      const float2* sf = a.sfa + (long long)p * (I / 32);
       if (routed || BR == BS) {
         constexpr int CPV = 128 / BR;
         if (two)
-          down_dot_chunk2<BR>(stage, stage2, cl / CPV, cb, sbw, sbw2, sbr / 4, as, a.I / CPV, c * (cl / CPV), sf, lane,
+          down_dot_chunk2<BR>(stage, stage2, cl / CPV, cb, sbw, sbw2, sbr / 4, as, I / CPV, c * (cl / CPV), sf, lane,
                               y[0], y2);
         else
-          down_dot_chunk<BR>(stage, cl / CPV, cb, sbw, sbr / 4, as, a.I / CPV, c * (cl / CPV), sf, lane, y);
+          down_dot_chunk<BR>(stage, cl / CPV, cb, sbw, sbr / 4, as, I / CPV, c * (cl / CPV), sf, lane, y);
       } else {
         constexpr int CPV = 128 / BS;
         if (two)
-          down_dot_chunk2<BS>(stage, stage2, cl / CPV, cb, sbw, sbw2, sbr / 4, as, a.I / CPV, c * (cl / CPV), sf, lane,
+          down_dot_chunk2<BS>(stage, stage2, cl / CPV, cb, sbw, sbw2, sbr / 4, as, I / CPV, c * (cl / CPV), sf, lane,
                               y[0], y2);
         else
-          down_dot_chunk<BS>(stage, cl / CPV, cb, sbw, sbr / 4, as, a.I / CPV, c * (cl / CPV), sf, lane, y);
+          down_dot_chunk<BS>(stage, cl / CPV, cb, sbw, sbr / 4, as, I / CPV, c * (cl / CPV), sf, lane, y);
       }
-      float* dst = a.y_part + ((long long)p * kMaxChunks + c) * a.H + (lane >> 3);
+      float* dst = a.y_part + ((long long)p * kMaxChunks + c) * H + (lane >> 3);
       if ((lane & 7) == 0) {
-        dst[(long long)q * kRC] = y[0];
-        if (two) dst[(long long)q2 * kRC] = y2;
+        dst[q * kRC] = y[0];
+        if (two) dst[q2 * kRC] = y2;
       }
     }
     __syncwarp();
     if (lane == 0) {
       fence_proxy_async_smem();
-      if (i + a.nst_c < n) issue(i + a.nst_c);
-      if (two && i + 1 + a.nst_c < n) issue(i + 1 + a.nst_c);
+      if (i + nst < n) issue();
+      if (two && i + 1 + nst < n) issue();
     }
     i += two ? 2 : 1;
     kc = kn;
-    if (two) cursor_step(cs, nq, kc);
+    rc = r2;
+    if (two) {
+      cursor_step(cs, nq, kc);
+      ring_next(rc, nst);
+    }
   }
 }
 

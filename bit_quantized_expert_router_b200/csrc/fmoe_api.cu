@@ -323,24 +323,42 @@ int launch_grouped(const fmoe_layer* L, const float* x, const float* residual, f
         return cuda_fail(e);
     info->grouped_attr_set[fi] = true;
   }
-  if (L->norm_weight)
-    rms_norm_tokens_kernel<<<T, kNormThreads, 0, s>>>(x_in, L->norm_weight, L->norm_eps, H, xn);
+  // Every step is a programmatic dependent launch (when enabled): its CTAs
+  // may start while the previous kernel ends and wait for it in the kernel.
+  cudaError_t e = cudaSuccess;
+  auto launch = [&](auto f, dim3 grid, int threads, size_t smem, auto... args) {
+    if (e != cudaSuccess) return;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    if (g_dependent_launch.load(std::memory_order_relaxed)) {
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+    }
+    e = cudaLaunchKernelEx(&cfg, f, args...);
+  };
+  if (L->norm_weight) launch(rms_norm_tokens_kernel, dim3(T), kNormThreads, 0, x_in, L->norm_weight, L->norm_eps, H, xn);
   const int rows = E + (L->w_sgate ? 1 : 0);
   const int router_ctas = (rows + kRouterRows - 1) / kRouterRows;
   if (a.shared_tc) {
     const int n_gu = 2 * (I / kTcRows) * (H / kTcK), n_down = (H / kTcRows) * (I / kTcK);
-    tc1<<<std::max(router_ctas, n_gu), kThreads, kTcSmemBytes, s>>>(a);
-    tc2<<<1 + T + n_down, kThreads, kTcSmemBytes, s>>>(a);
+    launch(tc1, dim3(std::max(router_ctas, n_gu)), kThreads, kTcSmemBytes, a);
+    launch(tc2, dim3(1 + T + n_down), kThreads, kTcSmemBytes, a);
   } else {
-    router_tokens_kernel<<<router_ctas, kThreads, 0, s>>>(L->w_router, L->w_sgate, x, T, H, E,
-                                                         const_cast<float*>(a.logits));
-    fns.prep<<<1 + T, kThreads, 0, s>>>(a);
+    launch(router_tokens_kernel, dim3(router_ctas), kThreads, 0, L->w_router, L->w_sgate, x, T, H, E,
+           const_cast<float*>(a.logits));
+    launch(fns.prep, dim3(1 + T), kThreads, 0, a);
   }
-  fns.gateup<<<G, kThreads, smem_gu, s>>>(a);
-  fns.stage<<<T * K + T, kStageThreads, (size_t)I * 4, s>>>(a);
-  fns.down<<<G, kThreads, smem_d, s>>>(a);
-  grouped_combine_kernel<<<dim3((H / 4 + kCombineThreads - 1) / kCombineThreads, T), kCombineThreads, 0, s>>>(a);
-  if (cudaError_t e = cudaGetLastError()) return cuda_fail(e);
+  launch(fns.gateup, dim3(G), kThreads, smem_gu, a);
+  launch(fns.stage, dim3(T * K + T), kStageThreads, (size_t)I * 4, a);
+  launch(fns.down, dim3(G), kThreads, smem_d, a);
+  launch(grouped_combine_kernel, dim3((H / 4 + kCombineThreads - 1) / kCombineThreads, T), kCombineThreads, 0, a);
+  if (e != cudaSuccess) return cuda_fail(e);
   return FMOE_OK;
 }
 

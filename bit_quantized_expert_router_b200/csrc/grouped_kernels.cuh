@@ -193,6 +193,8 @@ __global__ void __launch_bounds__(kThreads) router_tokens_kernel(const uint16_t*
                                                                  const uint16_t* __restrict__ w_sgate,
                                                                  const float* __restrict__ x, int T, int H, int E,
                                                                  float* __restrict__ logits) {
+  grid_dep_wait();  // (programmatic dependent launch: the previous kernel's writes are visible from here)
+  grid_dep_launch_dependents();
   router_rows_tokens(w_router, w_sgate, x, T, H, E, blockIdx.x * kRouterRows, logits);
 }
 
@@ -204,6 +206,8 @@ constexpr int kNormThreads = 256;
 __global__ void __launch_bounds__(kNormThreads) rms_norm_tokens_kernel(const float* __restrict__ x,
                                                                        const uint16_t* __restrict__ w, float eps,
                                                                        int H, float* __restrict__ xn) {
+  grid_dep_wait();  // (programmatic dependent launch: the previous kernel's writes are visible from here)
+  grid_dep_launch_dependents();
   __shared__ float red[kNormThreads / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float* xt = x + (long long)blockIdx.x * H;
@@ -379,6 +383,8 @@ __device__ __noinline__ void prep_cta(const GroupArgs& a, int b) {
 
 template <int BR, int BS>
 __global__ void __launch_bounds__(kThreads) grouped_prep_kernel(const __grid_constant__ GroupArgs a) {
+  grid_dep_wait();  // (programmatic dependent launch: the previous kernel's writes are visible from here)
+  grid_dep_launch_dependents();
   prep_cta<BR, BS>(a, blockIdx.x);
 }
 
@@ -694,6 +700,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gateup_kernel(const __gri
     fence_proxy_async_smem();
   }
   CtaSched cs;
+  grid_dep_wait();  // (programmatic dependent launch: the previous kernel's writes are visible from here)
+  grid_dep_launch_dependents();
   cta_sched(a, 0, cs, ss);  // includes __syncthreads
   // this warp's units: cs.u0 + warp + i * kWarps
   const int n = cs.u1 - cs.u0 > warp ? (cs.u1 - cs.u0 - warp - 1) / kWarps + 1 : 0;
@@ -804,6 +812,8 @@ constexpr int kStageThreads = 256;
 template <int BR, int BS>
 __global__ void __launch_bounds__(kStageThreads) grouped_stage_act_kernel(const __grid_constant__ GroupArgs a) {
   extern __shared__ __align__(16) float act[];  // [I]
+  grid_dep_wait();  // (programmatic dependent launch: the previous kernel's writes are visible from here)
+  grid_dep_launch_dependents();
   const int p = blockIdx.x;
   if (p >= a.tb.meta[1]) return;
   const int nk = a.tb.pair_nk[p] & 0xFF;
@@ -844,6 +854,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_down_kernel(const __grid_
   }
   const int H = a.H, I = a.I, nq = H / kRC;
   CtaSched cs;
+  grid_dep_wait();  // (programmatic dependent launch: the previous kernel's writes are visible from here)
+  grid_dep_launch_dependents();
   cta_sched(a, 1, cs, ss);
   const int n = cs.u1 - cs.u0 > warp ? (cs.u1 - cs.u0 - warp - 1) / kWarps + 1 : 0;
   const int sbr = sb_row_bytes(I);  // bytes of one row's scale/bias words
@@ -951,6 +963,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_down_kernel(const __grid_
 constexpr int kCombineThreads = 256;
 
 __global__ void __launch_bounds__(kCombineThreads) grouped_combine_kernel(const __grid_constant__ GroupArgs a) {
+  grid_dep_wait();  // (programmatic dependent launch: the previous kernel's writes are visible from here)
+  grid_dep_launch_dependents();
   __shared__ int s_pair[kMaxTopK + 1], s_nk[kMaxTopK + 1];
   __shared__ float s_w[kMaxTopK + 1];
   const int t = blockIdx.y, K = a.K;

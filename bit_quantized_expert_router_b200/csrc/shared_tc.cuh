@@ -221,6 +221,8 @@ __device__ __forceinline__ char* align1024(char* p) {
 template <int BS>
 __global__ void __launch_bounds__(kThreads, 1) router_shared_gu_kernel(const __grid_constant__ GroupArgs a) {
   extern __shared__ __align__(128) char smem_raw[];  // (aligned to 1024 below)
+  grid_dep_wait();  // (programmatic dependent launch: the previous kernel's writes are visible from here)
+  grid_dep_launch_dependents();
   char* sbase = align1024(smem_raw);
   const int b = blockIdx.x;
   const int rows = a.E + (a.w_sgate ? 1 : 0);
@@ -253,6 +255,8 @@ __global__ void __launch_bounds__(kThreads, 1) router_shared_gu_kernel(const __g
 template <int BR, int BS>
 __global__ void __launch_bounds__(kThreads, 1) prep_shared_down_kernel(const __grid_constant__ GroupArgs a) {
   extern __shared__ __align__(128) char smem_raw[];  // (aligned to 1024 below)
+  grid_dep_wait();  // (programmatic dependent launch: the previous kernel's writes are visible from here)
+  grid_dep_launch_dependents();
   const int b = blockIdx.x;
   if (b <= a.T) {
     prep_cta<BR, BS>(a, b);

@@ -429,6 +429,11 @@ int fmoe_streamer_destroy(fmoe_streamer* s);
  *     fmoe_set_wait_limit_ns) instead of results.
  *   0: cooperative launch, all CTAs resident by the driver's guarantee, no
  *     overlap with the previous kernel.
+ * The same setting governs the kernels of the grouped decode
+ * (fmoe_layer_decode with T >= 2): with 1 each of them is a programmatic
+ * dependent launch that waits for the previous kernel before its first
+ * access of device memory (no grid barriers, so no residency condition);
+ * with 0 they are plain launches.
  * Outputs are bit-identical either way.  enable must be 0 or 1, else
  * FMOE_EINVAL and nothing changes; the previous setting is stored in
  * *previous_opt when non-NULL.  The pages have no counterpart: launch

@@ -477,7 +477,8 @@ class Streamer:
 def set_dependent_launch(enable: bool) -> bool:
     """Launch the single-token layer kernel as a programmatic dependent launch
     (True, the default: it overlaps the previous kernel's end) or as a
-    cooperative launch (False); returns the previous setting."""
+    cooperative launch (False); the grouped decode's kernels follow the same
+    switch (dependent or plain launches).  Returns the previous setting."""
     prev = ctypes.c_int(0)
     rc = lib().fmoe_set_dependent_launch(1 if enable else 0, ctypes.byref(prev))
     if rc != FMOE_OK:

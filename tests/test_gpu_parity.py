@@ -521,6 +521,67 @@ def test_grouped_deterministic_and_graph_replay(F, SG):
     del g
 
 
+def test_grouped_dependent_and_plain_launches_agree(F, SG):
+    """Two layers decoded back to back on 6 tokens (the second reads the
+    first's output as input and residual) with one shared workspace, as
+    programmatic dependent launches and as plain launches, eagerly and from
+    a graph: outputs, indices and weights are bit-identical, and layer 0
+    agrees with the oracle."""
+    shape, T, seed = C.FULL4, 6, 37
+    layers = [make_gpu_layer(F, SG, seed, l, shape)[0] for l in range(2)]
+    H, K = shape.hidden, shape.top_k
+    x = C.parity_x(seed, 0, 0, S.router_bf16(seed, 0, shape.n_experts, H), K, H, T)
+    res = S.token_residual(seed, 0, 0, T, H)
+    xd, rd = torch.from_numpy(x).to(dev()), torch.from_numpy(res).to(dev())
+    ws = layers[0].workspace(T)
+
+    def chain(hs, idx, w):
+        layers[0].decode(xd, rd, out=hs[0], idx_out=idx[0], w_out=w[0], ws=ws)
+        layers[1].decode(hs[0], hs[0], out=hs[1], idx_out=idx[1], w_out=w[1], ws=ws)
+
+    def bufs():
+        return (torch.full((2, T, H), float("nan"), device=dev()),
+                torch.full((2, T, K), -1, dtype=torch.int32, device=dev()),
+                torch.full((2, T, K), float("nan"), device=dev()))
+
+    runs = {}
+    prev = F.set_dependent_launch(True)
+    try:
+        for mode in (True, False):
+            F.set_dependent_launch(mode)
+            eager = bufs()
+            for _ in range(2):
+                chain(*eager)
+            torch.cuda.synchronize()
+            assert F.get_status() == 0
+            graphed = bufs()
+            stream = torch.cuda.Stream()
+            stream.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(stream):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    chain(*graphed)
+                for _ in range(2):
+                    g.replay()
+            torch.cuda.synchronize()
+            assert F.get_status() == 0
+            del g
+            runs[mode] = (eager, graphed)
+    finally:
+        F.set_dependent_launch(prev)
+    ref = runs[True][0]
+    for mode, (eager, graphed) in runs.items():
+        for a, b in zip(ref, eager):
+            assert torch.equal(a, b), f"dependent={mode} eager"
+        for a, b in zip(ref, graphed):
+            assert torch.equal(a, b), f"dependent={mode} graph"
+    got, gi = ref[0][0].cpu().numpy(), ref[1][0].cpu().numpy()
+    for k in range(T):
+        r = C.oracle_layer(seed, 0, shape, x[k], res[k])
+        assert gi[k].tolist() == r["idx"].tolist(), f"token {k}"
+        C.assert_close(got[k], r["out"], f"token {k}")
+
+
 @pytest.mark.parametrize("T", [1, 6])
 def test_layer_exact_ties_pick_lowest_indices(F, SG, T):
     """Every router row equal: all logits tie exactly, and the decision is the

@@ -753,9 +753,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gateup_kernel(const __gri
     ring_next(r2, nst);
     const char* stage = my_ring + rc.idx * stage_bytes;
     const char* stage2 = my_ring + r2.idx * stage_bytes;
-    if (!mbar_wait_bounded(&my_bars[rc.idx], rc.ph, a.timeout_ns) && lane == 0) set_status(kStatusCopyTimeout);
-    if (two && !mbar_wait_bounded(&my_bars[r2.idx], r2.ph, a.timeout_ns) && lane == 0)
-      set_status(kStatusCopyTimeout);
+    // A copy that did not arrive in time makes its unit's results NaN (the
+    // decision is the whole warp's), which reaches every token using them.
+    const bool ok1 = __all_sync(0xffffffffu, mbar_wait_bounded(&my_bars[rc.idx], rc.ph, a.timeout_ns));
+    const bool ok2 = !two || __all_sync(0xffffffffu, mbar_wait_bounded(&my_bars[r2.idx], r2.ph, a.timeout_ns));
+    if (!(ok1 && ok2) && lane == 0) set_status(kStatusCopyTimeout);
     const int s = kc.s, c = kc.c, row = kc.r, row2 = kn.r;
     const bool routed = cs.expert[s] >= 0;
     const int cl = cs.cl[s];
@@ -784,8 +786,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gateup_kernel(const __gri
         else
           gu_dot_chunk<BS>(stage, cl / CPV, cl * BS / 8, cap, sbo, sbo, xs, H / CPV, c * (cl / CPV), sf, lane, g, up);
       }
-      if (lane == 0) dst[row] = make_float2(g, up);
-      if (two && lane == 16) dst[row2] = make_float2(g, up);
+      if (lane == 0) dst[row] = ok1 ? make_float2(g, up) : make_float2(quiet_nan(), quiet_nan());
+      if (two && lane == 16) dst[row2] = ok2 ? make_float2(g, up) : make_float2(quiet_nan(), quiet_nan());
     }
     __syncwarp();
     if (lane == 0) {
@@ -905,9 +907,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_down_kernel(const __grid_
     ring_next(r2, nst);
     const char* stage = my_ring + rc.idx * stage_bytes;
     const char* stage2 = my_ring + r2.idx * stage_bytes;
-    if (!mbar_wait_bounded(&my_bars[rc.idx], rc.ph, a.timeout_ns) && lane == 0) set_status(kStatusCopyTimeout);
-    if (two && !mbar_wait_bounded(&my_bars[r2.idx], r2.ph, a.timeout_ns) && lane == 0)
-      set_status(kStatusCopyTimeout);
+    // A copy that did not arrive in time makes its unit's results NaN (the
+    // decision is the whole warp's), which reaches every token using them.
+    const bool ok1 = __all_sync(0xffffffffu, mbar_wait_bounded(&my_bars[rc.idx], rc.ph, a.timeout_ns));
+    const bool ok2 = !two || __all_sync(0xffffffffu, mbar_wait_bounded(&my_bars[r2.idx], r2.ph, a.timeout_ns));
+    if (!(ok1 && ok2) && lane == 0) set_status(kStatusCopyTimeout);
     const int s = kc.s, c = kc.c, q = kc.r, q2 = kn.r;
     const bool routed = cs.expert[s] >= 0;
     const int cl = cs.cl[s];
@@ -936,8 +940,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_down_kernel(const __grid_
       }
       float* dst = a.y_part + ((long long)p * kMaxChunks + c) * H + (lane >> 3);
       if ((lane & 7) == 0) {
-        dst[q * kRC] = y[0];
-        if (two) dst[q2 * kRC] = y2;
+        dst[q * kRC] = ok1 ? y[0] : quiet_nan();
+        if (two) dst[q2 * kRC] = ok2 ? y2 : quiet_nan();
       }
     }
     __syncwarp();

@@ -177,7 +177,7 @@ __device__ __noinline__ void tc_tile(char* sbase, const char* __restrict__ codes
     const uint4 s0 = __ldg(sp), s1 = __ldg(sp + 1);
     sbv[0] = s0.x; sbv[1] = s0.y; sbv[2] = s0.z; sbv[3] = s0.w;
     sbv[4] = s1.x; sbv[5] = s1.y; sbv[6] = s1.z; sbv[7] = s1.w;
-    done = mbar_wait_bounded(bar, 0, timeout_ns);
+    done = __all_sync(0xffffffffu, mbar_wait_bounded(bar, 0, timeout_ns));
     if (!done && lane == 0) set_status(kStatusMmaTimeout);
     tc_fence_after_sync();
     float acc[kMaxTokens];
@@ -194,9 +194,10 @@ __device__ __noinline__ void tc_tile(char* sbase, const char* __restrict__ codes
         acc[t] = fmaf(sc, __uint_as_float(d[t]) + __uint_as_float(d[kMaxTokens + t]),
                       fmaf(bi, xsum[g * kMaxTokens + t], acc[t]));
     }
+    // results of MMAs not known complete are NaN (they reach every token)
 #pragma unroll
     for (int t = 0; t < kMaxTokens; ++t)
-      if (t < T) out[(long long)t * ldo + r0 + r] = acc[t];
+      if (t < T) out[(long long)t * ldo + r0 + r] = done ? acc[t] : quiet_nan();
   }
   // TMEM is freed only once the MMAs are known complete (a second bounded
   // wait if the first one ran out).

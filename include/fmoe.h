@@ -193,8 +193,10 @@ int fmoe_workspace_init(void* ws, size_t ws_bytes, fmoe_stream_t stream);
  * fmoe_get_status(); for T = 1 the kernel then also writes quiet NaN to the
  * out rows of every CTA whose wait ran out, hands NaN on to the rest through
  * any value it still publishes, and writes -1 / NaN to idx_out_opt /
- * w_out_opt when the routing itself was affected, so no result built on a
- * missing value looks plausible. */
+ * w_out_opt when the routing itself was affected; for T >= 2 every unit of
+ * work whose weight copy or tensor-core result did not arrive in time yields
+ * NaN, which reaches the out rows of each token that uses it.  So no result
+ * built on a missing value looks plausible. */
 int fmoe_layer_decode(const fmoe_layer* L, const float* x, const float* residual, float* out, int T,
                       void* ws, size_t ws_bytes, int32_t* idx_out_opt, float* w_out_opt,
                       fmoe_stream_t stream);

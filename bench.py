@@ -583,13 +583,15 @@ def run_fmoe(args, cfg, rank, world, local_rank):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": profiled_traffic(args.config),
                          "kernel": (f"layer_kernel<{cfg['bits']},{cfg['shared_bits']}>" if TT == 1 else
-                                    "grouped decode step (router, prep, gate/up, stage, down launches)"),
+                                    "grouped decode step (router + shared gate/up, prep + shared down, routed "
+                                    "gate/up, activation staging, routed down, combine launches)"),
                          "algorithmic_bytes_per_launch": ab["total"]},
             "layer_decodes_per_s": whole_job_rate(K, world, total_ms_max),
             "sustained_gbs": world * K * ab["total"] / (total_ms_max / 1000.0) / 1e9,
             "e2e": {"value": whole_job_rate(K * TT / LPS, world, e2e_ms_max), "unit": unit,
                     "h2d_bytes_per_step": (2 if LPS == 1 else 1) * TT * h * 4, "d2h_bytes_per_step": TT * h * 4},
-            "gpu_launches": K * (1 if TT == 1 else 5),
+            # a grouped step is six launches (see the kernel entry above)
+            "gpu_launches": K * (1 if TT == 1 else 6),
             **({"distinct_routed_experts_per_step": distinct} if distinct is not None else {}),
             **({"expert_path": expert_path} if expert_path is not None else {}),
             "clocks": clk,
